@@ -1,0 +1,252 @@
+"""Seeded synthetic inputs for the QSA forward pass.
+
+This module only draws random tensors and plants needles.  It holds none of
+the method's arithmetic (no pooling, rotary encoding, scoring, selection or
+attention), so the oracle side and the CUDA side can both consume what it
+produces without sharing any of the method's code.
+
+Workloads mirror the shapes the pages describe for Qwen3.8-Flash-Next's QSA
+layers (Miles docs "Qwen3.8-Flash-Next", section 1: 24 heads, 2 query groups,
+kv-channels 256, rotary 0.25 at base 1e7; design report, QSA item: r=4, a
+4-head indexer, budget 2048 tokens):
+
+  tiny_fp32     1 sequence, 256 tokens, indexer dim 64, budget 64 tokens, fp32
+  prefill_8k    2 sequences x 8192 tokens, bf16, 4 needles per 1024 queries
+  prefill_128k  1 sequence x 131072 tokens, bf16, a needle every 8192 positions
+  decode_256k   32 sequences x 1 decode query against a 262144-token cache
+  mixed_1m      8 decode queries at 1048576-token context plus one 4096-query
+                prefill chunk at [942080, 946176) of a 90%-cached sequence
+
+Distributions: q, k, v, indexer q and indexer k ~ N(0, 1) drawn in fp32 and
+rounded once to the I/O dtype; head weights w ~ U(0, 1) in fp32.
+
+Needles ("key = scaled copy of query"): for a target query t* of cache slot s
+and a block b* < floor(t*/r), the r indexer-key rows of b* are set to
+alpha * u, u = sum_h w[t*,h] * q_idx[t*,h] with the rotary dims zeroed (so the
+block's position encoding leaves it unchanged), and the main K rows of b* in
+every group are set to beta * q[t*, head 0].  alpha = beta = 1.
+"""
+from __future__ import annotations
+
+import dataclasses
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Tuple
+
+import torch
+
+
+@dataclass(frozen=True)
+class Shape:
+    n_heads: int = 24
+    n_groups: int = 2
+    head_dim: int = 256
+    idx_heads: int = 4
+    idx_dim: int = 128
+    r: int = 4
+    budget_tokens: int = 2048
+    rope_fraction: float = 0.25
+    rope_base: float = 1e7
+    dtype: str = "bf16"           # "bf16" or "f32": I/O dtype of q, k, v, indexer q/k, k^, o
+
+    @property
+    def rope_dims(self) -> int:
+        d = int(self.idx_dim * self.rope_fraction)
+        return d - (d % 2)
+
+    @property
+    def budget_blocks(self) -> int:
+        return self.budget_tokens // self.r
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+
+@dataclass(frozen=True)
+class Segment:
+    """A run of consecutive query tokens of one cached sequence."""
+    slot: int        # cache slot of the sequence
+    pos0: int        # absolute position of the first query token
+    q_len: int       # number of query tokens (positions pos0 .. pos0+q_len-1)
+
+
+@dataclass
+class Workload:
+    name: str
+    shape: Shape
+    segments: List[Segment]
+    n_slots: int
+    n_cap: int                         # cache capacity per slot (tokens)
+    fill: List[int]                    # tokens present in each slot's cache
+    cached_blocks: List[int]           # k^ blocks already pooled before the step
+    needles: List[Tuple[int, int, int]] = field(default_factory=list)  # (slot, t*, b*)
+    seed: int = 0
+
+    @property
+    def n_tokens(self) -> int:
+        return sum(s.q_len for s in self.segments)
+
+    def token_offsets(self) -> List[int]:
+        out, acc = [], 0
+        for s in self.segments:
+            out.append(acc)
+            acc += s.q_len
+        return out
+
+    def token_positions(self) -> torch.Tensor:
+        return torch.cat([torch.arange(s.pos0, s.pos0 + s.q_len, dtype=torch.int64)
+                          for s in self.segments])
+
+    def token_slots(self) -> torch.Tensor:
+        return torch.cat([torch.full((s.q_len,), s.slot, dtype=torch.int64) for s in self.segments])
+
+
+def _needles_per_window(rng: torch.Generator, slot: int, lo: int, hi: int, per_1k: int,
+                        r: int) -> List[Tuple[int, int, int]]:
+    out = []
+    for w0 in range(lo, hi, 1024):
+        w1 = min(hi, w0 + 1024)
+        for _ in range(per_1k):
+            t = int(torch.randint(max(w0, r), w1, (1,), generator=rng)) if w1 > max(w0, r) else None
+            if t is None:
+                continue
+            b = int(torch.randint(0, t // r, (1,), generator=rng))
+            out.append((slot, t, b))
+    return out
+
+
+def _distinct_blocks(rng: torch.Generator, nblk: int, k: int) -> List[int]:
+    picks: List[int] = []
+    while len(picks) < k:
+        b = int(torch.randint(0, nblk, (1,), generator=rng))
+        if b not in picks:
+            picks.append(b)
+    return picks
+
+
+def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
+    """Return one of the named workloads (see module docstring).
+
+    Keyword overrides allow reduced sizes of the same recipe for parity tests:
+    n (prefill length), n_seqs, ctx (decode context), chunk (prefill chunk
+    length), chunk_pos0, n_decode.
+    """
+    rng = torch.Generator().manual_seed(1000 + (seed if seed is not None else 0))
+    if name == "tiny_fp32":
+        sh = Shape(idx_dim=64, budget_tokens=64, dtype="f32")
+        n = over.get("n", 256)
+        wl = Workload(name, sh, [Segment(0, 0, n)], 1, n, [n], [0], [], seed or 0)
+        return wl
+    if name == "prefill_8k":
+        sh = Shape(**over.get("shape", {}))
+        n = over.get("n", 8192)
+        n_seqs = over.get("n_seqs", 2)
+        segs = [Segment(s, 0, n) for s in range(n_seqs)]
+        needles = []
+        for s in range(n_seqs):
+            needles += _needles_per_window(rng, s, 0, n, 4, sh.r)
+        return Workload(name, sh, segs, n_seqs, n, [n] * n_seqs, [0] * n_seqs, needles,
+                        seed if seed is not None else 1)
+    if name == "prefill_128k":
+        sh = Shape()
+        n = over.get("n", 131072)
+        every = over.get("every", 8192)
+        needles = []
+        for i in range(n // every):
+            t = every * i + every - 1
+            b = int(torch.randint(0, t // sh.r, (1,), generator=rng))
+            needles.append((0, t, b))
+        return Workload(name, sh, [Segment(0, 0, n)], 1, n, [n], [0], needles,
+                        seed if seed is not None else 2)
+    if name == "decode_256k":
+        sh = Shape()
+        ctx = over.get("ctx", 262144)
+        n_seqs = over.get("n_seqs", 32)
+        segs = [Segment(s, ctx - 1, 1) for s in range(n_seqs)]
+        needles = []
+        for s in range(n_seqs):
+            t = ctx - 1
+            for b in _distinct_blocks(rng, t // sh.r, 8):
+                needles.append((s, t, b))
+        # the decode token completes block (ctx-1)//r; earlier blocks are cached
+        cached = [(ctx - 1) // sh.r] * n_seqs
+        return Workload(name, sh, segs, n_seqs, ctx, [ctx] * n_seqs, cached, needles,
+                        seed if seed is not None else 3)
+    if name == "mixed_1m":
+        sh = Shape()
+        ctx = over.get("ctx", 1 << 20)
+        n_dec = over.get("n_decode", 8)
+        chunk = over.get("chunk", 4096)
+        pos0 = over.get("chunk_pos0", 942080)
+        segs = [Segment(s, ctx - 1, 1) for s in range(n_dec)]
+        segs.append(Segment(n_dec, pos0, chunk))
+        needles = []
+        for s in range(n_dec):
+            for b in _distinct_blocks(rng, (ctx - 1) // sh.r, 8):
+                needles.append((s, ctx - 1, b))
+        needles += _needles_per_window(rng, n_dec, pos0, pos0 + chunk, 4, sh.r)
+        fill = [ctx] * n_dec + [pos0 + chunk]
+        cached = [(ctx - 1) // sh.r] * n_dec + [pos0 // sh.r]
+        return Workload(name, sh, segs, n_dec + 1, ctx, fill, cached, needles,
+                        seed if seed is not None else 4)
+    raise KeyError(name)
+
+
+def _randn(shape, gen, device, dtype, chunk_elems=1 << 28):
+    """N(0,1) drawn in fp32 and rounded once to dtype, generated in pieces."""
+    out = torch.empty(shape, dtype=dtype, device=device)
+    flat = out.view(-1)
+    for i in range(0, flat.numel(), chunk_elems):
+        n = min(chunk_elems, flat.numel() - i)
+        flat[i:i + n] = torch.randn(n, generator=gen, device=device, dtype=torch.float32).to(dtype)
+    return out
+
+
+def make_inputs(wl: Workload, device="cpu") -> Dict[str, torch.Tensor]:
+    """Draw every input tensor of the workload on `device` (seeded).
+
+    Returns token-major query tensors (q [T,H,D], q_idx [T,Hi,dI], w [T,Hi])
+    and slot-major caches (k_idx [S,N,dI], k and v [S,G,N,D]).  Cache rows
+    beyond a slot's fill are zero.
+    """
+    sh = wl.shape
+    dt = sh.torch_dtype
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev).manual_seed(wl.seed)
+    T = wl.n_tokens
+    q = _randn((T, sh.n_heads, sh.head_dim), gen, dev, dt)
+    q_idx = _randn((T, sh.idx_heads, sh.idx_dim), gen, dev, dt)
+    w = torch.rand((T, sh.idx_heads), generator=gen, device=dev, dtype=torch.float32)
+    k_idx = torch.zeros((wl.n_slots, wl.n_cap, sh.idx_dim), dtype=dt, device=dev)
+    k = torch.zeros((wl.n_slots, sh.n_groups, wl.n_cap, sh.head_dim), dtype=dt, device=dev)
+    v = torch.zeros_like(k)
+    for s in range(wl.n_slots):
+        f = wl.fill[s]
+        k_idx[s, :f] = _randn((f, sh.idx_dim), gen, dev, dt)
+        for g in range(sh.n_groups):
+            k[s, g, :f] = _randn((f, sh.head_dim), gen, dev, dt)
+            v[s, g, :f] = _randn((f, sh.head_dim), gen, dev, dt)
+    # needles
+    offs = wl.token_offsets()
+    rho = sh.rope_dims
+    for (slot, t, b) in wl.needles:
+        tok = None
+        for si, seg in enumerate(wl.segments):
+            if seg.slot == slot and seg.pos0 <= t < seg.pos0 + seg.q_len:
+                tok = offs[si] + (t - seg.pos0)
+        if tok is None:
+            continue
+        u = (w[tok].unsqueeze(1) * q_idx[tok].float()).sum(0)
+        u[:rho] = 0
+        k_idx[slot, b * sh.r:(b + 1) * sh.r] = u.to(dt)
+        for g in range(sh.n_groups):
+            k[slot, g, b * sh.r:(b + 1) * sh.r] = q[tok, 0]
+    return {"q": q, "q_idx": q_idx, "w": w, "k_idx": k_idx, "k": k, "v": v}
+
+
+def describe(wl: Workload) -> dict:
+    d = dataclasses.asdict(wl)
+    d["n_tokens"] = wl.n_tokens
+    d.pop("needles")
+    d["n_needles"] = len(wl.needles)
+    return d
