@@ -1,0 +1,498 @@
+#!/usr/bin/env python
+"""Benchmark of the QSA forward pass on B200 (one JSON line on rank 0).
+
+A step is one qsa_forward over the workload's batch: pooling of the blocks
+the batch completes, indexer scores, top-k selection and sparse attention.
+Default workload: 128K-token prefill (1 sequence x 131072 tokens, bf16, 24
+heads / 2 KV groups, head dim 256, 4-head indexer of dim 128, r = 4, budget
+2048 tokens, needles every 8192 positions).  The 1M-context mixed decode
+step (8 decode queries at 1048576 tokens plus a 4096-query chunk of a
+90%-cached sequence) is measured in the same run and reported under
+"decode_1m".
+
+Inputs are synthetic (seeded, N(0,1) with planted needles) and resident in
+HBM before the timed region; L2 is flushed (a 256 MiB write, outside the
+timed events) before every timed step.  Times are CUDA events on the
+launching stream, max over ranks.  With torchrun and N > 1 every rank runs
+an independent replica of the workload on its own GPU (the method has no
+cross-GPU exchange): scaling is weak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qsa|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import block_sparse_attention_22_b200 as qsa  # noqa: E402
+from block_sparse_attention_22_b200 import synth  # noqa: E402
+
+METRIC = "QSA fwd tokens/s (prefill 128K, decode 1M ctx); % of HBM/tensor roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples of this process's GPU during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.target = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.target = None
+
+    def start(self):
+        if self.target is None:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.target, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload set-up
+class Prepared:
+    """Device-resident inputs, caches, outputs and workspace of one workload."""
+
+    def __init__(self, wl: synth.Workload):
+        self.wl = wl
+        sh = wl.shape
+        self.sh = sh
+        self.x = synth.make_inputs(wl, device="cuda")
+        self.cfg = qsa.make_config(sh)
+        self.khat = torch.zeros((wl.n_slots, wl.n_cap // sh.r, sh.idx_dim), dtype=sh.torch_dtype, device="cuda")
+        self.cache = qsa.make_cache(self.x["k_idx"], self.khat, self.x["k"], self.x["v"])
+        slots = [s for s in range(wl.n_slots) if wl.cached_blocks[s] > 0]
+        if slots:   # the cached prefix: pooled by earlier steps, not part of this step
+            qsa.qsa_compress_keys(self.cfg, self.cache, slots, [0] * len(slots),
+                                  [wl.cached_blocks[s] for s in slots])
+        self.segl = [(off, s.q_len, s.pos0, s.slot) for off, s in zip(wl.token_offsets(), wl.segments)]
+        self.segs = qsa.make_segments(self.segl)
+        T = self.T = wl.n_tokens
+        self.o = torch.empty((T, sh.n_heads, sh.head_dim), dtype=sh.torch_dtype, device="cuda")
+        self.lse = torch.empty((T, sh.n_heads), dtype=torch.float32, device="cuda")
+        self.sel = torch.empty((T, sh.budget_blocks), dtype=torch.int32, device="cuda")
+        self.nsel = torch.empty((T,), dtype=torch.int32, device="cuda")
+        self.ld = max(4, math.ceil(max((p + n - 1) // sh.r for _, n, p, _ in self.segl) / 4) * 4)
+        self.ws = torch.empty(max(1, qsa.workspace_size(self.cfg, self.segs, T, qsa.QSA_OP_FORWARD)),
+                              dtype=torch.uint8, device="cuda")
+        self.scores = torch.empty((T, self.ld), dtype=torch.float32, device="cuda")
+        self.ws_sel = torch.empty(max(1, qsa.workspace_size(self.cfg, self.segs, T, qsa.QSA_OP_SELECT)),
+                                  dtype=torch.uint8, device="cuda")
+        self.ws_attn = torch.empty(max(1, qsa.workspace_size(self.cfg, self.segs, T, qsa.QSA_OP_ATTN)),
+                                   dtype=torch.uint8, device="cuda")
+        self.ranges = [(s.slot, s.pos0 // sh.r, (s.pos0 + s.q_len) // sh.r) for s in wl.segments]
+
+    def forward(self):
+        x = self.x
+        qsa.qsa_forward(self.cfg, self.cache, self.segs, self.T, x["q"], x["q_idx"], x["w"], self.o, self.lse,
+                        self.sel, self.nsel, self.ws)
+
+    # the same four calls qsa_forward makes, one public entry point each
+    def stage(self, i):
+        x = self.x
+        if i == 0:
+            qsa.qsa_compress_keys(self.cfg, self.cache, [r[0] for r in self.ranges], [r[1] for r in self.ranges],
+                                  [r[2] for r in self.ranges])
+        elif i == 1:
+            qsa.qsa_index_scores(self.cfg, self.cache, self.segs, self.T, x["q_idx"], x["w"], self.scores, self.ld)
+        elif i == 2:
+            qsa.qsa_select_topk(self.cfg, self.segs, self.T, self.scores, self.ld, self.sel, self.nsel, self.ws_sel)
+        else:
+            qsa.qsa_sparse_attn_fwd(self.cfg, self.cache, self.segs, self.T, x["q"], self.sel, self.nsel, self.o,
+                                    self.lse, self.ws_attn)
+
+    # ---------------------------------------------------------------- algorithmic work
+    def work(self):
+        """Algorithmic bytes / flops of each stage for this batch (what QSA must touch)."""
+        sh, wl = self.sh, self.wl
+        pos = wl.token_positions().double()
+        bt = torch.floor(pos / sh.r)
+        nsel = torch.clamp(bt + 1, max=sh.budget_blocks)
+        el = 2 if sh.dtype == "bf16" else 4
+        D, H, G, DI, HI = sh.head_dim, sh.n_heads, sh.n_groups, sh.idx_dim, sh.idx_heads
+        n_new_blocks = sum(b1 - b0 for _, b0, b1 in self.ranges)
+        comp_bytes = n_new_blocks * (sh.r + 1) * DI * el
+        cand = bt.sum().item()
+        idx_flops = 2.0 * HI * DI * cand
+        # scores: k^ rows read once per 64-query tile (L2-resident for prefill) + score writes
+        idx_bytes = cand * 4 + self.T * HI * (DI * el + 4)
+        if self.T <= 64:   # decode: every query streams its whole k^ prefix from HBM
+            idx_bytes += cand * DI * el
+        sel_bytes = cand * 4 + self.T * (sh.budget_blocks + 1) * 4
+        gathered = float((nsel * sh.r).sum().item()) * G * D * el * 2
+        attn_bytes = gathered + self.T * H * D * el * 2 + self.T * H * 4 + self.T * (sh.budget_blocks + 1) * 4
+        attn_flops = 4.0 * H * D * float((nsel * sh.r).sum().item())
+        return dict(compress=dict(bytes=comp_bytes), index=dict(bytes=idx_bytes, flops=idx_flops),
+                    select=dict(bytes=sel_bytes), attn=dict(bytes=attn_bytes, flops=attn_flops,
+                                                            gathered_bytes=gathered))
+
+
+def timed(prep: Prepared, steps: int, warmup: int, flush: torch.Tensor, staged: bool):
+    """Device time of `steps` steps (ms each), L2 flushed before every step."""
+    st = torch.cuda.current_stream()
+    n_ev = 5 if staged else 2
+    for _ in range(warmup):
+        flush.zero_()
+        if staged:
+            for i in range(4):
+                prep.stage(i)
+        else:
+            prep.forward()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
+    launches0 = qsa.launch_count()
+    for s in range(steps):
+        flush.zero_()
+        evs[s][0].record(st)
+        if staged:
+            for i in range(4):
+                prep.stage(i)
+                evs[s][i + 1].record(st)
+        else:
+            prep.forward()
+            evs[s][1].record(st)
+    torch.cuda.synchronize()
+    launches = qsa.launch_count() - launches0
+    per = [[evs[s][i].elapsed_time(evs[s][i + 1]) for i in range(n_ev - 1)] for s in range(steps)]
+    return per, launches
+
+
+def e2e_prefill(prep: Prepared, steps: int, warmup: int):
+    """qsa_forward with the step's inputs copied from pinned host memory and the
+    output read back, all inside the timed region."""
+    x = prep.x
+    slot = prep.wl.segments[0].slot
+    fill = prep.wl.fill[slot]
+    host = {"q": x["q"], "q_idx": x["q_idx"], "w": x["w"], "k_idx": x["k_idx"][slot, :fill],
+            "k": x["k"][slot, :, :fill], "v": x["v"][slot, :, :fill]}
+    host = {k: v.cpu().pin_memory() for k, v in host.items()}
+    o_host = torch.empty(prep.o.shape, dtype=prep.o.dtype).pin_memory()
+    lse_host = torch.empty(prep.lse.shape, dtype=prep.lse.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * lse_host.element_size()
+    st = torch.cuda.current_stream()
+
+    def one():
+        x["q"].copy_(host["q"], non_blocking=True)
+        x["q_idx"].copy_(host["q_idx"], non_blocking=True)
+        x["w"].copy_(host["w"], non_blocking=True)
+        x["k_idx"][slot, :fill].copy_(host["k_idx"], non_blocking=True)
+        x["k"][slot, :, :fill].copy_(host["k"], non_blocking=True)
+        x["v"][slot, :, :fill].copy_(host["v"], non_blocking=True)
+        prep.forward()
+        o_host.copy_(prep.o, non_blocking=True)
+        lse_host.copy_(prep.lse, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        one()
+    e1.record(st)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(wl: synth.Workload, x, target_s: float = 10.0):
+    """Time the CPU oracle on a stratified sample of the workload's queries and
+    extrapolate to the whole batch (per-query work grows linearly with the
+    position, so evenly spaced positions give an unbiased mean).  Returns
+    (tokens/s, threads, description)."""
+    import oracle
+    sh = wl.shape
+    cfg = oracle.config_from_shape(sh)
+    threads = len(os.sched_getaffinity(0))
+    pos_all = wl.token_positions().numpy()
+    slots_all = wl.token_slots().numpy()
+    f = lambda t: t.float().cpu().numpy()
+    # per slot: pooled-key cost once (all blocks the queries need), then queries
+    total_s, n_done, desc = 0.0, 0, []
+    seg_rows = {}
+    for off, s in zip(wl.token_offsets(), wl.segments):
+        seg_rows.setdefault(s.slot, []).extend(range(off, off + s.q_len))
+    budget_per_slot = target_s / max(1, len(seg_rows))
+    est_total = 0.0
+    for slot, rows in seg_rows.items():
+        fill = wl.fill[slot]
+        k_idx = f(x["k_idx"][slot, :fill])
+        k = f(x["k"][slot, :, :fill])
+        v = f(x["v"][slot, :, :fill])
+        rows = np.array(rows)
+        nb_new = sum((s.pos0 + s.q_len) // sh.r - s.pos0 // sh.r for s in wl.segments if s.slot == slot)
+        t0 = time.perf_counter()
+        oracle.compress_keys(cfg, k_idx, 0, max(1, nb_new))     # the blocks this step pools
+        t_comp = time.perf_counter() - t0
+        # calibrate with a few queries, then size the sample to the budget
+        n_cal = min(len(rows), max(2, threads))
+        pick = rows[np.linspace(0, len(rows) - 1, n_cal).astype(int)]
+        t0 = time.perf_counter()
+        oracle.forward(cfg, f(x["q"][pick]), f(x["q_idx"][pick]), f(x["w"][pick]), pos_all[pick], k_idx, k, v)
+        t_cal = time.perf_counter() - t0
+        n_s = int(min(len(rows), max(n_cal, n_cal * budget_per_slot / max(t_cal, 1e-3))))
+        pick = rows[np.linspace(0, len(rows) - 1, n_s).astype(int)]
+        t0 = time.perf_counter()
+        oracle.forward(cfg, f(x["q"][pick]), f(x["q_idx"][pick]), f(x["w"][pick]), pos_all[pick], k_idx, k, v)
+        t_s = time.perf_counter() - t0
+        # oracle.forward also pools every block up to max(pick); remove that part once
+        t0 = time.perf_counter()
+        oracle.compress_keys(cfg, k_idx, 0, int(pos_all[pick].max()) // sh.r)
+        t_pool_all = time.perf_counter() - t0
+        per_query = max(t_s - t_pool_all, 1e-9) / n_s
+        est_total += t_comp + per_query * len(rows)
+        total_s += t_s + t_comp
+        n_done += n_s
+        desc.append(f"slot {slot}: {n_s} of {len(rows)} queries at evenly spaced positions")
+    tokens = wl.n_tokens
+    return tokens / est_total, threads, "; ".join(desc) + f"; {total_s:.1f} s of oracle wall time, " \
+        f"extrapolated by query count (pooling of the step's new blocks timed in full)"
+
+
+# ------------------------------------------------------------------ main
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank
+
+
+def max_over_ranks(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def measure(prep: Prepared, steps, warmup, ws, flush, peaks, clocks=None):
+    barrier(ws)
+    if clocks:
+        clocks.start()
+    per, launches = timed(prep, steps, warmup, flush, staged=False)
+    if clocks:
+        clk = clocks.stop()
+    else:
+        clk = None
+    barrier(ws)
+    fused_ms = sum(p[0] for p in per) / steps
+    fused_ms = max_over_ranks(fused_ms, ws)
+    per_s, launches_s = timed(prep, steps, max(1, warmup // 2), flush, staged=True)
+    barrier(ws)
+    stage_ms = [sum(p[i] for p in per_s) / steps for i in range(4)]
+    work = prep.work()
+    names = ["compress", "index", "select", "attn"]
+    stages = {}
+    for n, ms in zip(names, stage_ms):
+        d = {"ms": ms}
+        if "bytes" in work[n]:
+            d["gbs"] = work[n]["bytes"] / (ms * 1e-3) / 1e9
+            d["hbm_frac"] = d["gbs"] / peaks["hbm_gbs"]
+        if "flops" in work[n]:
+            d["tflops"] = work[n]["flops"] / (ms * 1e-3) / 1e12
+            d["tensor_frac"] = d["tflops"] / peaks["bf16_tflops"]
+        stages[n] = d
+    return dict(fused_ms=fused_ms, stage_ms=stage_ms, stages=stages, work=work, launches=launches,
+                clocks=clk)
+
+
+def traffic_record(kernel: str, workload: str):
+    """dram bytes per launch recorded from an ncu capture of the current kernel build, if any."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        rec = json.load(open(p)).get(f"{kernel}:{workload}")
+        return rec.get("dram_bytes_per_launch") if rec else None
+    except Exception:
+        return None
+
+
+def run_reference(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = synth.make_workload(args.workload)
+    x = synth.make_inputs(wl, device="cuda" if torch.cuda.is_available() else "cpu")
+    vals = []
+    desc = ""
+    threads = 0
+    for i in range(args.warmup + args.steps):
+        v, threads, desc = oracle_sample(wl, x, target_s=args.cpu_seconds / max(1, args.steps + args.warmup))
+        if i >= args.warmup:
+            vals.append(v)
+    val = statistics.mean(vals)
+    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": wl.n_tokens / val * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": args.workload, "tokens_per_step": wl.n_tokens},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["qsa", "reference"], default="qsa")
+    ap.add_argument("--workload", default="prefill_128k")
+    ap.add_argument("--decode-workload", default="mixed_1m", help="'none' to skip")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    ws, rank = dist_setup()
+    peaks = load_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    wl = synth.make_workload(args.workload)
+    prep = Prepared(wl)
+    clocks = ClockSampler(torch.cuda.current_device())
+    m = measure(prep, args.steps, args.warmup, ws, flush, peaks, clocks)
+    tokens = wl.n_tokens
+    value = ws * tokens / (m["fused_ms"] * 1e-3)
+
+    work = m["work"]
+    attn_ms = m["stage_ms"][3]
+    achieved = work["attn"]["bytes"] / (attn_ms * 1e-3) / 1e9
+    roofline = {"kernel": "sparse attention (attn stage)", "bound": "hbm", "achieved": achieved,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": traffic_record("attn", args.workload), "peak_source": peaks["source"],
+                "bytes_per_launch": work["attn"]["bytes"]}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = e2e_prefill(prep, args.steps, args.warmup)
+        e2e_ms = max_over_ranks(e2e_ms, ws)
+        e2e = {"value": ws * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        v, threads, desc = oracle_sample(wl, prep.x, args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
+    del prep
+    torch.cuda.empty_cache()
+
+    decode = None
+    if args.decode_workload != "none":
+        wl2 = synth.make_workload(args.decode_workload)
+        prep2 = Prepared(wl2)
+        m2 = measure(prep2, args.steps, args.warmup, ws, flush, peaks)
+        w2 = m2["work"]
+        dec_tokens = sum(s.q_len for s in wl2.segments)
+        decode = {"workload": args.decode_workload, "ms_per_step": m2["fused_ms"],
+                  "tokens_per_step": dec_tokens, "tokens_per_s": ws * dec_tokens / (m2["fused_ms"] * 1e-3),
+                  "stages": m2["stages"], "gpu_launches": m2["launches"]}
+        tot_bytes = sum(w2[k]["bytes"] for k in ("compress", "index", "select", "attn"))
+        decode["hbm_roofline"] = {"bytes_per_step": tot_bytes,
+                                  "achieved_gbs": tot_bytes / (sum(m2["stage_ms"]) * 1e-3) / 1e9}
+        decode["hbm_roofline"]["frac"] = decode["hbm_roofline"]["achieved_gbs"] / peaks["hbm_gbs"]
+        del prep2
+        torch.cuda.empty_cache()
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": m["fused_ms"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": wl.shape.dtype, "data": "synthetic",
+                "config": {"workload": args.workload, "batch": len(wl.segments), "seq_len": wl.segments[0].q_len,
+                           "budget_tokens": wl.shape.budget_tokens, "heads": wl.shape.n_heads,
+                           "kv_groups": wl.shape.n_groups, "head_dim": wl.shape.head_dim,
+                           "idx_heads": wl.shape.idx_heads, "idx_dim": wl.shape.idx_dim,
+                           "parallelism": f"replicas x{ws}", "l2": "flushed before every timed step"},
+                "roofline": roofline, "stages": m["stages"], "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": m["launches"], "clocks": m["clocks"], "decode_1m": decode}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,525 @@
+// qsa_api.cu -- the C ABI of libqsa.so (declared in include/qsa.h).
+//
+// Host side only: validates arguments (before anything is enqueued), splits
+// the segment list into launch-sized tables, picks kernels by I/O dtype and
+// enqueues them on the caller's stream.  It never allocates, never
+// synchronises (except qsa_device_status, a diagnostic) and keeps no state
+// beyond per-function attribute set-up.
+//
+// One translation unit: every kernel file is included here.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "qsa_internal.cuh"
+#include "compress.cuh"
+#include "index_simt.cuh"
+#include "topk.cuh"
+#include "attn_simt.cuh"
+
+#define QSA_API extern "C" __attribute__((visibility("default")))
+
+namespace qsa {
+namespace {
+
+constexpr int kNumSms = 148;
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int rope_dims_of(const qsa_config_t* c) {
+  int d = (int)floor((double)c->idx_dim * (double)c->rope_fraction);
+  return d - (d & 1);
+}
+
+qsa_status_t check_cfg(const qsa_config_t* c) {
+  if (!c) return QSA_ERR_INVALID_ARG;
+  if (c->r <= 0 || c->budget_tokens <= 0 || c->n_q_heads <= 0 || c->n_kv_groups <= 0 ||
+      c->head_dim <= 0 || c->idx_heads <= 0 || c->idx_dim <= 0)
+    return QSA_ERR_INVALID_ARG;
+  if (c->budget_tokens % c->r != 0 || c->n_q_heads % c->n_kv_groups != 0) return QSA_ERR_INVALID_ARG;
+  if (!(c->rope_fraction >= 0.f && c->rope_fraction <= 1.f) || !(c->rope_base > 0.0))
+    return QSA_ERR_INVALID_ARG;
+  if (c->dtype != QSA_DTYPE_F32 && c->dtype != QSA_DTYPE_BF16) return QSA_ERR_INVALID_ARG;
+  if (c->r != 4 || c->head_dim != kHeadDim || c->idx_heads != 4 ||
+      (c->idx_dim != 64 && c->idx_dim != 128))
+    return QSA_ERR_UNSUPPORTED;
+  if (c->n_q_heads / c->n_kv_groups > kMaxHpg) return QSA_ERR_UNSUPPORTED;
+  if (c->budget_tokens / c->r > kMaxBudgetBlocks) return QSA_ERR_UNSUPPORTED;
+  if (rope_dims_of(c) / 2 > kMaxRopeHalf) return QSA_ERR_UNSUPPORTED;
+  return QSA_OK;
+}
+
+qsa_status_t check_cache(const qsa_config_t* c, const qsa_cache_t* k) {
+  if (!k || k->n_slots <= 0 || k->n_cap <= 0 || k->n_cap % c->r != 0) return QSA_ERR_INVALID_ARG;
+  if (k->n_cap > ((int64_t)1 << 31) - 1) return QSA_ERR_UNSUPPORTED;
+  return QSA_OK;
+}
+
+qsa_status_t check_segments(const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                            const qsa_cache_t* cache, int64_t n_cap_if_no_cache) {
+  if (n_segs < 0 || n_tokens < 0 || (n_segs > 0 && !segs)) return QSA_ERR_INVALID_ARG;
+  const int64_t n_cap = cache ? cache->n_cap : n_cap_if_no_cache;
+  for (int i = 0; i < n_segs; ++i) {
+    const qsa_segment_t& s = segs[i];
+    if (s.q_len < 0 || s.q_offset < 0 || s.pos0 < 0) return QSA_ERR_INVALID_ARG;
+    if ((int64_t)s.q_offset + s.q_len > n_tokens) return QSA_ERR_INVALID_ARG;
+    if (n_cap > 0 && (int64_t)s.pos0 + s.q_len > n_cap) return QSA_ERR_INVALID_ARG;
+    if (cache && (s.slot < 0 || s.slot >= cache->n_slots)) return QSA_ERR_INVALID_ARG;
+  }
+  return QSA_OK;
+}
+
+Geo make_geo(const qsa_config_t* c, const qsa_cache_t* k) {
+  Geo g;
+  memset(&g, 0, sizeof g);
+  g.r = c->r;
+  g.S = c->budget_tokens / c->r;
+  g.H = c->n_q_heads;
+  g.G = c->n_kv_groups;
+  g.hpg = c->n_q_heads / c->n_kv_groups;
+  g.HI = c->idx_heads;
+  g.DI = c->idx_dim;
+  const int rd = rope_dims_of(c);
+  g.rope_half = rd / 2;
+  g.scale = c->softmax_scale > 0.f ? c->softmax_scale : (float)(1.0 / sqrt((double)c->head_dim));
+  g.n_slots = k ? k->n_slots : 0;
+  g.n_cap = k ? k->n_cap : 0;
+  for (int i = 0; i < g.rope_half; ++i) g.theta[i] = pow(c->rope_base, -(2.0 * (double)i) / (double)rd);
+  return g;
+}
+
+int64_t seg_max_blocks(const qsa_segment_t* segs, int n, int r) {
+  int64_t m = 0;
+  for (int i = 0; i < n; ++i)
+    if (segs[i].q_len > 0) m = std::max<int64_t>(m, ((int64_t)segs[i].pos0 + segs[i].q_len - 1) / r);
+  return m;
+}
+
+int64_t seg_rows(const qsa_segment_t* segs, int n) {
+  int64_t t = 0;
+  for (int i = 0; i < n; ++i) t += std::max(0, segs[i].q_len);
+  return t;
+}
+
+// Calls launch(table) for batches of at most kMaxSegs non-empty segments;
+// items(seg) gives each segment's work-item count.
+template <typename Items, typename Launch>
+qsa_status_t for_each_table(const qsa_segment_t* segs, int n_segs, Items items, Launch launch) {
+  SegTable st;
+  memset(&st, 0, sizeof st);
+  auto flush = [&]() -> qsa_status_t {
+    if (st.n == 0 || st.item0[st.n] == 0) {
+      st.n = 0;
+      return QSA_OK;
+    }
+    cudaError_t e = launch(st);
+    st.n = 0;
+    return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+  };
+  for (int i = 0; i < n_segs; ++i) {
+    const qsa_segment_t& s = segs[i];
+    if (s.q_len <= 0) continue;
+    const int64_t it = items(s);
+    if (st.n > 0 && ((int64_t)st.item0[st.n] + it > INT32_MAX / 2)) {
+      qsa_status_t r = flush();
+      if (r != QSA_OK) return r;
+    }
+    st.q_offset[st.n] = s.q_offset;
+    st.q_len[st.n] = s.q_len;
+    st.pos0[st.n] = s.pos0;
+    st.slot[st.n] = s.slot;
+    if (st.n == 0) st.item0[0] = 0;
+    st.item0[st.n + 1] = st.item0[st.n] + (int32_t)it;
+    st.n++;
+    if (st.n == kMaxSegs) {
+      qsa_status_t r = flush();
+      if (r != QSA_OK) return r;
+    }
+  }
+  return flush();
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ selection plan
+struct TopkPlan {
+  int chunk;
+  int max_ch;      // chunks per row in the workspace (1: no split rows)
+  size_t ws;
+};
+
+TopkPlan topk_plan(const Geo& g, const qsa_segment_t* segs, int n) {
+  TopkPlan p{topk::kChunkLarge, 1, 0};
+  const int64_t nblk = seg_max_blocks(segs, n, g.r);
+  const int64_t rows = seg_rows(segs, n);
+  if (nblk + 1 <= g.S) return p;
+  if (rows * cdiv(nblk, topk::kChunkLarge) < 2 * kNumSms) p.chunk = topk::kChunkSmall;
+  if (cdiv(nblk, p.chunk) > 32) p.chunk = (int)std::min<int64_t>(topk::kChunkLarge, cdiv(nblk, 32));
+  p.max_ch = (int)cdiv(nblk, p.chunk);
+  if (p.max_ch > 1) {
+    int64_t T = 0;
+    for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
+    const size_t K = (size_t)(g.S - 1);
+    p.ws = align_up((size_t)T * p.max_ch * K * 4, 256) * 2 + align_up((size_t)T * p.max_ch * 4, 256);
+  }
+  return p;
+}
+
+// ------------------------------------------------------------------ attention plan
+struct AttnPlan {
+  int n_split;
+  int blocks_per_split;
+  size_t ws;
+};
+
+AttnPlan attn_plan(const Geo& g, const qsa_segment_t* segs, int n) {
+  int64_t T = 0;
+  for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
+  const int64_t units = seg_rows(segs, n) * g.G;
+  AttnPlan p{1, g.S, 0};
+  const int gran = simt_attn::KC / 4;
+  if (units > 0 && units < 2 * kNumSms) {
+    int ns = (int)std::min<int64_t>(cdiv(2 * kNumSms, units), cdiv(g.S, gran));
+    p.blocks_per_split = (int)(cdiv(cdiv(g.S, ns), gran) * gran);
+    p.n_split = (int)cdiv(g.S, p.blocks_per_split);
+  }
+  if (p.n_split > 1)
+    p.ws = align_up((size_t)T * g.G * p.n_split * g.hpg * kHeadDim * 4, 256) +
+           align_up((size_t)T * g.G * p.n_split * g.hpg * 2 * 4, 256);
+  return p;
+}
+
+// ------------------------------------------------------------------ stage launchers
+qsa_status_t run_compress(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
+                          const int32_t* slots, const int64_t* b0, const int64_t* b1, int n,
+                          cudaStream_t st) {
+  RangeTable rt;
+  memset(&rt, 0, sizeof rt);
+  auto flush = [&]() -> qsa_status_t {
+    if (rt.n == 0) return QSA_OK;
+    cudaError_t e = c->dtype == QSA_DTYPE_BF16
+                        ? launch_compress<__nv_bfloat16>(g, rt, cache->k_idx, cache->khat, st)
+                        : launch_compress<float>(g, rt, cache->k_idx, cache->khat, st);
+    rt.n = 0;
+    return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+  };
+  for (int i = 0; i < n; ++i) {
+    if (b1[i] <= b0[i]) continue;
+    rt.slot[rt.n] = slots[i];
+    rt.b0[rt.n] = b0[i];
+    if (rt.n == 0) rt.item0[0] = 0;
+    rt.item0[rt.n + 1] = rt.item0[rt.n] + (b1[i] - b0[i]);
+    if (++rt.n == kMaxSegs) {
+      qsa_status_t r = flush();
+      if (r != QSA_OK) return r;
+    }
+  }
+  return flush();
+}
+
+qsa_status_t run_index(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
+                       const qsa_segment_t* segs, int n, const void* q_idx, const float* w,
+                       float* scores, int64_t ld, cudaStream_t st) {
+  const bool bf = c->dtype == QSA_DTYPE_BF16;
+  size_t smem = sizeof(float) * (simt_index::QT * g.HI * g.DI + simt_index::QT * g.HI);
+  if (smem > 48 * 1024) {
+    cudaFuncSetAttribute(index_scores_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(index_scores_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  }
+  return for_each_table(
+      segs, n, [&](const qsa_segment_t& s) { return (int64_t)simt_index_items(s.q_len, s.pos0, g.r); },
+      [&](const SegTable& t) {
+        return bf ? launch_index_simt<__nv_bfloat16>(g, t, q_idx, w, cache->khat, scores, ld, st)
+                  : launch_index_simt<float>(g, t, q_idx, w, cache->khat, scores, ld, st);
+      });
+}
+
+qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const float* scores,
+                        int64_t ld, int32_t* sel, int32_t* nsel, void* ws, size_t ws_bytes,
+                        cudaStream_t st) {
+  const TopkPlan p = topk_plan(g, segs, n);
+  if (p.ws > 0 && (!ws || ws_bytes < p.ws)) return QSA_ERR_WORKSPACE;
+  TopkArgs a;
+  memset(&a, 0, sizeof a);
+  a.scores = scores;
+  a.ld = ld;
+  a.sel = sel;
+  a.nsel = nsel;
+  a.chunk = p.chunk;
+  a.max_ch = p.max_ch;
+  if (p.max_ch > 1) {
+    int64_t T = 0;
+    for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
+    const size_t K = (size_t)(g.S - 1);
+    char* base = (char*)ws;
+    a.cand_key = (uint32_t*)base;
+    base += align_up((size_t)T * p.max_ch * K * 4, 256);
+    a.cand_idx = (int32_t*)base;
+    base += align_up((size_t)T * p.max_ch * K * 4, 256);
+    a.cand_cnt = (int32_t*)base;
+  }
+  const size_t smem_c = topk_chunk_smem(p.chunk);
+  cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
+  const int64_t nblk = seg_max_blocks(segs, n, g.r);
+  (void)nblk;
+  qsa_status_t r = for_each_table(
+      segs, n,
+      [&](const qsa_segment_t& s) {
+        const int64_t nb = ((int64_t)s.pos0 + s.q_len - 1) / g.r;
+        return (int64_t)s.q_len * std::max<int64_t>(1, cdiv(nb, p.chunk));
+      },
+      [&](const SegTable& t) {
+        count_launch();
+        topk_chunk_kernel<<<t.item0[t.n], topk::THREADS, smem_c, st>>>(g, t, a);
+        return cudaGetLastError();
+      });
+  if (r != QSA_OK || p.max_ch <= 1) return r;
+  const size_t smem_m = topk_merge_smem(p.max_ch, g.S - 1);
+  cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_m);
+  return for_each_table(
+      segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
+      [&](const SegTable& t) {
+        count_launch();
+        topk_merge_kernel<<<t.item0[t.n], topk::THREADS, smem_m, st>>>(g, t, a);
+        return cudaGetLastError();
+      });
+}
+
+qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
+                      const qsa_segment_t* segs, int n, const void* q, const int32_t* sel,
+                      const int32_t* nsel, void* o, float* lse, void* ws, size_t ws_bytes,
+                      cudaStream_t st) {
+  const bool bf = c->dtype == QSA_DTYPE_BF16;
+  const AttnPlan p = attn_plan(g, segs, n);
+  if (p.ws > 0 && (!ws || ws_bytes < p.ws)) return QSA_ERR_WORKSPACE;
+  AttnArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = q;
+  a.k = cache->k;
+  a.v = cache->v;
+  a.sel = sel;
+  a.nsel = nsel;
+  a.o = o;
+  a.lse = lse;
+  a.n_split = p.n_split;
+  a.blocks_per_split = p.blocks_per_split;
+  if (p.n_split > 1) {
+    int64_t T = 0;
+    for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
+    a.part_o = (float*)ws;
+    a.part_ml = (float*)((char*)ws + align_up((size_t)T * g.G * p.n_split * g.hpg * kHeadDim * 4, 256));
+  }
+  const size_t smem = attn_simt_smem();
+  cudaFuncSetAttribute(attn_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  qsa_status_t r = for_each_table(
+      segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len * g.G * p.n_split; },
+      [&](const SegTable& t) {
+        if (bf) { count_launch(); attn_simt_kernel<__nv_bfloat16><<<t.item0[t.n], simt_attn::THREADS, smem, st>>>(g, t, a); }
+        else { count_launch(); attn_simt_kernel<float><<<t.item0[t.n], simt_attn::THREADS, smem, st>>>(g, t, a); }
+        return cudaGetLastError();
+      });
+  if (r != QSA_OK || p.n_split == 1) return r;
+  return for_each_table(
+      segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
+      [&](const SegTable& t) {
+        const int64_t total = (int64_t)t.item0[t.n] * g.H * kHeadDim;
+        const unsigned blocks = (unsigned)std::min<int64_t>(cdiv(total, 256), kNumSms * 32);
+        if (bf) { count_launch(); attn_combine_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(g, t, a); }
+        else { count_launch(); attn_combine_kernel<float><<<blocks, 256, 0, st>>>(g, t, a); }
+        return cudaGetLastError();
+      });
+}
+
+// ------------------------------------------------------------------ forward workspace
+struct FwdLayout {
+  int64_t ld;
+  size_t scores, sel, nsel, topk, attn, total;
+};
+
+FwdLayout fwd_layout(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens) {
+  FwdLayout L;
+  L.ld = std::max<int64_t>(4, cdiv(seg_max_blocks(segs, n, g.r), 4) * 4);
+  size_t off = 0;
+  L.scores = off;
+  off += align_up((size_t)n_tokens * L.ld * 4, 256);
+  L.sel = off;
+  off += align_up((size_t)n_tokens * g.S * 4, 256);
+  L.nsel = off;
+  off += align_up((size_t)n_tokens * 4, 256);
+  L.topk = off;
+  off += align_up(topk_plan(g, segs, n).ws, 256);
+  L.attn = off;
+  off += align_up(attn_plan(g, segs, n).ws, 256);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+}  // namespace qsa
+
+using namespace qsa;
+
+QSA_API qsa_status_t qsa_compress_keys(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                       const int32_t* slots, const int64_t* blk_begin,
+                                       const int64_t* blk_end, int32_t n_ranges, void* stream) {
+  qsa_status_t s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if ((s = check_cache(cfg, cache)) != QSA_OK) return s;
+  if (n_ranges < 0 || (n_ranges > 0 && (!slots || !blk_begin || !blk_end))) return QSA_ERR_INVALID_ARG;
+  if (n_ranges == 0) return QSA_OK;
+  if (!cache->k_idx || !cache->khat || !aligned16(cache->k_idx) || !aligned16(cache->khat))
+    return QSA_ERR_INVALID_ARG;
+  for (int i = 0; i < n_ranges; ++i) {
+    if (slots[i] < 0 || slots[i] >= cache->n_slots) return QSA_ERR_INVALID_ARG;
+    if (blk_begin[i] < 0 || blk_end[i] < blk_begin[i] || blk_end[i] > cache->n_cap / cfg->r)
+      return QSA_ERR_INVALID_ARG;
+  }
+  const Geo g = make_geo(cfg, cache);
+  return run_compress(g, cfg, cache, slots, blk_begin, blk_end, n_ranges, (cudaStream_t)stream);
+}
+
+QSA_API qsa_status_t qsa_index_scores(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                      const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                                      const void* q_idx, const float* w, float* scores,
+                                      int64_t ld_scores, void* stream) {
+  qsa_status_t s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if ((s = check_cache(cfg, cache)) != QSA_OK) return s;
+  if ((s = check_segments(segs, n_segs, n_tokens, cache, 0)) != QSA_OK) return s;
+  if (seg_rows(segs, n_segs) == 0) return QSA_OK;
+  if (!q_idx || !w || !scores || !cache->khat || !aligned16(q_idx) || !aligned16(cache->khat) ||
+      !aligned16(w) || !aligned16(scores))
+    return QSA_ERR_INVALID_ARG;
+  if (ld_scores < std::max<int64_t>(1, seg_max_blocks(segs, n_segs, cfg->r))) return QSA_ERR_INVALID_ARG;
+  const Geo g = make_geo(cfg, cache);
+  return run_index(g, cfg, cache, segs, n_segs, q_idx, w, scores, ld_scores, (cudaStream_t)stream);
+}
+
+QSA_API qsa_status_t qsa_select_topk(const qsa_config_t* cfg, const qsa_segment_t* segs,
+                                     int32_t n_segs, int32_t n_tokens, const float* scores,
+                                     int64_t ld_scores, int32_t* sel, int32_t* nsel, void* workspace,
+                                     size_t ws_bytes, void* stream) {
+  qsa_status_t s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if ((s = check_segments(segs, n_segs, n_tokens, nullptr, 0)) != QSA_OK) return s;
+  if (seg_rows(segs, n_segs) == 0) return QSA_OK;
+  if (!scores || !sel || !nsel || !aligned16(sel)) return QSA_ERR_INVALID_ARG;
+  const int64_t nblk = seg_max_blocks(segs, n_segs, cfg->r);
+  if (ld_scores < std::max<int64_t>(1, nblk)) return QSA_ERR_INVALID_ARG;
+  if (nblk > (int64_t)topk::kChunkLarge * 32) return QSA_ERR_UNSUPPORTED;
+  const Geo g = make_geo(cfg, nullptr);
+  return run_select(g, segs, n_segs, scores, ld_scores, sel, nsel, workspace, ws_bytes,
+                    (cudaStream_t)stream);
+}
+
+QSA_API qsa_status_t qsa_sparse_attn_fwd(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                         const qsa_segment_t* segs, int32_t n_segs,
+                                         int32_t n_tokens, const void* q, const int32_t* sel,
+                                         const int32_t* nsel, void* o, float* lse, void* workspace,
+                                         size_t ws_bytes, void* stream) {
+  qsa_status_t s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if ((s = check_cache(cfg, cache)) != QSA_OK) return s;
+  if ((s = check_segments(segs, n_segs, n_tokens, cache, 0)) != QSA_OK) return s;
+  if (seg_rows(segs, n_segs) == 0) return QSA_OK;
+  if (!q || !sel || !nsel || !o || !cache->k || !cache->v || !aligned16(q) || !aligned16(o) ||
+      !aligned16(cache->k) || !aligned16(cache->v) || !aligned16(sel))
+    return QSA_ERR_INVALID_ARG;
+  const Geo g = make_geo(cfg, cache);
+  return run_attn(g, cfg, cache, segs, n_segs, q, sel, nsel, o, lse, workspace, ws_bytes,
+                  (cudaStream_t)stream);
+}
+
+QSA_API size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* segs,
+                                  int32_t n_segs, int32_t n_tokens, qsa_op_t op) {
+  if (check_cfg(cfg) != QSA_OK || check_segments(segs, n_segs, n_tokens, nullptr, 0) != QSA_OK)
+    return SIZE_MAX;
+  const Geo g = make_geo(cfg, nullptr);
+  switch (op) {
+    case QSA_OP_COMPRESS:
+    case QSA_OP_INDEX: return 0;
+    case QSA_OP_SELECT: return topk_plan(g, segs, n_segs).ws;
+    case QSA_OP_ATTN: return attn_plan(g, segs, n_segs).ws;
+    case QSA_OP_FORWARD: return fwd_layout(g, segs, n_segs, n_tokens).total;
+  }
+  return SIZE_MAX;
+}
+
+QSA_API qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                 const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                                 const void* q, const void* q_idx, const float* w, void* o,
+                                 float* lse, int32_t* sel, int32_t* nsel, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  qsa_status_t s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if ((s = check_cache(cfg, cache)) != QSA_OK) return s;
+  if ((s = check_segments(segs, n_segs, n_tokens, cache, 0)) != QSA_OK) return s;
+  if (seg_rows(segs, n_segs) == 0) return QSA_OK;
+  if (!q || !q_idx || !w || !o || !cache->k || !cache->v || !cache->k_idx || !cache->khat)
+    return QSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(q_idx) || !aligned16(w) || !aligned16(o) || !aligned16(cache->k) ||
+      !aligned16(cache->v) || !aligned16(cache->k_idx) || !aligned16(cache->khat))
+    return QSA_ERR_INVALID_ARG;
+  if ((sel == nullptr) != (nsel == nullptr) || (sel && !aligned16(sel))) return QSA_ERR_INVALID_ARG;
+  const int64_t nblk = seg_max_blocks(segs, n_segs, cfg->r);
+  if (nblk > (int64_t)topk::kChunkLarge * 32) return QSA_ERR_UNSUPPORTED;
+  const Geo g = make_geo(cfg, cache);
+  const FwdLayout L = fwd_layout(g, segs, n_segs, n_tokens);
+  if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return QSA_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  float* scores = (float*)(ws + L.scores);
+  if (!sel) {
+    sel = (int32_t*)(ws + L.sel);
+    nsel = (int32_t*)(ws + L.nsel);
+  }
+  // 1. pool the blocks each segment completes
+  std::vector<int32_t> slots;
+  std::vector<int64_t> b0, b1;
+  for (int i = 0; i < n_segs; ++i) {
+    if (segs[i].q_len <= 0) continue;
+    slots.push_back(segs[i].slot);
+    b0.push_back(segs[i].pos0 / cfg->r);
+    b1.push_back(((int64_t)segs[i].pos0 + segs[i].q_len) / cfg->r);
+  }
+  s = run_compress(g, cfg, cache, slots.data(), b0.data(), b1.data(), (int)slots.size(), st);
+  if (s != QSA_OK) return s;
+  // 2. indexer scores, 3. selection, 4. attention
+  if ((s = run_index(g, cfg, cache, segs, n_segs, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
+  if ((s = run_select(g, segs, n_segs, scores, L.ld, sel, nsel, ws + L.topk, L.attn - L.topk, st)) != QSA_OK)
+    return s;
+  return run_attn(g, cfg, cache, segs, n_segs, q, sel, nsel, o, lse, ws + L.attn, L.total - L.attn, st);
+}
+
+QSA_API qsa_status_t qsa_device_status(void* stream) {
+  unsigned int h = 0, zero = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyFromSymbolAsync(&h, g_qsa_device_error, sizeof h, 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return QSA_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(g_qsa_device_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return QSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QSA_ERR_CUDA;
+  if (h == kErrWaitTimeout) return QSA_ERR_TIMEOUT;
+  if (h != kErrNone) return QSA_ERR_CUDA;
+  return QSA_OK;
+}
+
+QSA_API const char* qsa_status_string(qsa_status_t status) {
+  switch (status) {
+    case QSA_OK: return "ok";
+    case QSA_ERR_INVALID_ARG: return "invalid argument";
+    case QSA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QSA_ERR_CUDA: return "CUDA error";
+    case QSA_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+QSA_API int32_t qsa_version(void) { return 100; }
+
+QSA_API int64_t qsa_launch_count(void) { return (int64_t)launch_counter().load(); }

@@ -1,0 +1,126 @@
+// qsa_internal.cuh -- types and device helpers shared by the QSA kernels.
+//
+// The library is one translation unit (qsa_api.cu includes every kernel
+// file), so file-scope device state such as the error word has one instance
+// per device.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/qsa.h"
+
+namespace qsa {
+
+constexpr int kMaxSegs = 128;     // segments per launch: the table travels as a kernel parameter
+constexpr int kHeadDim = 256;     // main attention head dim (Miles docs section 1: kv-channels 256)
+constexpr int kMaxHpg = 16;       // query heads per KV group handled by one tile
+constexpr int kMaxBudgetBlocks = 512;
+constexpr int kMaxRopeHalf = 64;
+
+// Layer geometry, passed by value to every kernel.
+struct Geo {
+  int32_t r;          // tokens per micro-block
+  int32_t S;          // budget in blocks
+  int32_t H;          // query heads
+  int32_t G;          // KV groups
+  int32_t hpg;        // heads per group
+  int32_t HI;         // indexer heads
+  int32_t DI;         // indexer dim
+  int32_t rope_half;  // rotated dims / 2
+  float scale;        // softmax scale
+  int32_t n_slots;
+  int64_t n_cap;      // tokens per cache slot
+  double theta[kMaxRopeHalf];  // rope_base^(-2i/rope_dims), formed on the host in fp64
+};
+
+// Segment table of one launch, with a prefix sum of the work items each
+// segment contributes (the kernel maps blockIdx to a segment by bisection).
+struct SegTable {
+  int32_t n;
+  int32_t q_offset[kMaxSegs];
+  int32_t q_len[kMaxSegs];
+  int32_t pos0[kMaxSegs];
+  int32_t slot[kMaxSegs];
+  int32_t item0[kMaxSegs + 1];
+};
+
+__device__ __forceinline__ int find_segment(const SegTable& st, int item) {
+  int lo = 0, hi = st.n - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (st.item0[mid] <= item) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// ---------------------------------------------------------------- dtype traits
+template <typename T> struct IO;
+template <> struct IO<float> {
+  static __device__ __forceinline__ float to_f(float x) { return x; }
+  static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+template <> struct IO<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// ---------------------------------------------------------------- rotary encoding
+// cos/sin of the angle pos*theta_i: the angle is formed in fp64 and the result
+// rounded to fp32, so positions up to 2^20 keep full fp32 accuracy.
+__device__ __forceinline__ void rope_cs(const Geo& g, int64_t pos, int i, float& c, float& s) {
+  double a = (double)pos * g.theta[i];
+  double sd, cd;
+  sincos(a, &sd, &cd);
+  c = (float)cd;
+  s = (float)sd;
+}
+
+// One rotate-half pair (x_i, x_{i+half}) at angle (c, s), fp32 with every
+// product rounded separately (no contraction into FMA).
+__device__ __forceinline__ void rope_pair(float a, float b, float c, float s, float& oa, float& ob) {
+  oa = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
+  ob = __fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s));
+}
+
+// ---------------------------------------------------------------- status word
+// Written by bounded device-side waits that gave up; read by qsa_device_status().
+static __device__ unsigned int g_qsa_device_error;
+
+enum : unsigned int { kErrNone = 0, kErrWaitTimeout = 1, kErrBadIndex = 2 };
+
+__device__ __forceinline__ void report_error(unsigned int code) {
+  atomicCAS(&g_qsa_device_error, 0u, code);
+}
+
+// Cache row of token `j_in_block` of kept block `b`, or -1 when b is not a
+// block of the cache (a caller-supplied selection out of range: reported and
+// skipped, never dereferenced).
+__device__ __forceinline__ int64_t block_row(int32_t b, int j_in_block, const Geo& g) {
+  if (b < 0 || (int64_t)b >= g.n_cap / g.r) {
+    if (b != -1) report_error(kErrBadIndex);
+    return -1;
+  }
+  return (int64_t)b * g.r + j_in_block;
+}
+
+// Host-side count of kernels this library has launched (qsa_launch_count).
+inline std::atomic<long long>& launch_counter() {
+  static std::atomic<long long> n{0};
+  return n;
+}
+inline void count_launch() { launch_counter().fetch_add(1, std::memory_order_relaxed); }
+
+// ---------------------------------------------------------------- misc
+__host__ __device__ __forceinline__ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// fp32 score -> uint32 key whose unsigned order is the float order (-0 -> +0).
+__device__ __forceinline__ uint32_t score_key(float s) {
+  uint32_t u = __float_as_uint(s == 0.0f ? 0.0f : s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+}  // namespace qsa

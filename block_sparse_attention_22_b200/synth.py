@@ -135,7 +135,7 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
     if name == "tiny_fp32":
         sh = Shape(idx_dim=64, budget_tokens=64, dtype="f32")
         n = over.get("n", 256)
-        wl = Workload(name, sh, [Segment(0, 0, n)], 1, n, [n], [0], [], seed or 0)
+        wl = Workload(name, sh, [Segment(0, 0, n)], 1, _round_cap(n, sh.r), [n], [0], [], seed or 0)
         return wl
     if name == "prefill_8k":
         sh = Shape(**over.get("shape", {}))
@@ -145,7 +145,7 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
         needles = []
         for s in range(n_seqs):
             needles += _needles_per_window(rng, s, 0, n, 4, sh.r)
-        return Workload(name, sh, segs, n_seqs, n, [n] * n_seqs, [0] * n_seqs, needles,
+        return Workload(name, sh, segs, n_seqs, _round_cap(n, sh.r), [n] * n_seqs, [0] * n_seqs, needles,
                         seed if seed is not None else 1)
     if name == "prefill_128k":
         sh = Shape()
@@ -156,7 +156,7 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
             t = every * i + every - 1
             b = int(torch.randint(0, t // sh.r, (1,), generator=rng))
             needles.append((0, t, b))
-        return Workload(name, sh, [Segment(0, 0, n)], 1, n, [n], [0], needles,
+        return Workload(name, sh, [Segment(0, 0, n)], 1, _round_cap(n, sh.r), [n], [0], needles,
                         seed if seed is not None else 2)
     if name == "decode_256k":
         sh = Shape()
@@ -170,7 +170,7 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
                 needles.append((s, t, b))
         # the decode token completes block (ctx-1)//r; earlier blocks are cached
         cached = [(ctx - 1) // sh.r] * n_seqs
-        return Workload(name, sh, segs, n_seqs, ctx, [ctx] * n_seqs, cached, needles,
+        return Workload(name, sh, segs, n_seqs, _round_cap(ctx, sh.r), [ctx] * n_seqs, cached, needles,
                         seed if seed is not None else 3)
     if name == "mixed_1m":
         sh = Shape()
@@ -187,9 +187,13 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
         needles += _needles_per_window(rng, n_dec, pos0, pos0 + chunk, 4, sh.r)
         fill = [ctx] * n_dec + [pos0 + chunk]
         cached = [(ctx - 1) // sh.r] * n_dec + [pos0 // sh.r]
-        return Workload(name, sh, segs, n_dec + 1, ctx, fill, cached, needles,
+        return Workload(name, sh, segs, n_dec + 1, _round_cap(max(ctx, pos0 + chunk), sh.r), fill, cached, needles,
                         seed if seed is not None else 4)
     raise KeyError(name)
+
+
+def _round_cap(n: int, r: int) -> int:
+    return (n + r - 1) // r * r
 
 
 def _randn(shape, gen, device, dtype, chunk_elems=1 << 28):

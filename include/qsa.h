@@ -1,0 +1,225 @@
+/*
+ * qsa.h -- C ABI of libqsa.so: the forward pass of Qwen Sparse Attention (QSA)
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method (web pages on Qwen3.8-Flash-Next):
+ *   - design report summary "Qwen3.8-Next architecture design report"
+ *     (macin.top, on "On the Design of Qwen3.8-Next Architecture"), section
+ *     "Four architecture components", item 2 "Qwen Sparse Attention (QSA)":
+ *     the indexer works on micro-blocks of r=4 tokens; the keys of a block are
+ *     averaged and then position-encoded; scoring costs O(n^2/r); the indexer
+ *     has 4 query heads sharing one key (MQA); each query keeps K=2048 tokens.
+ *   - Miles docs "Qwen3.8-Flash-Next", section 1 "Model Introduction": each
+ *     QSA layer derives its own indexer queries and compressed keys, scores
+ *     them and keeps a budget of key tokens per query; attention then reads
+ *     only those tokens; selection rows are built outside the attention kernel
+ *     so that it needs no causal or segment logic; 24 heads, 2 query groups,
+ *     kv-channels 256, rotary base 1e7 at rotary percent 0.25.
+ *   - tahou.com article on the Qwen3.8-Flash-Next release, section "GDN+QSA":
+ *     a lightweight indexer groups the sequence into micro-blocks, scores
+ *     their importance, and attention runs on the most relevant regions only.
+ *
+ * Readings fixed here where the pages are silent:
+ *   score       s(t,b) = sum_h w[t,h] * max(0, q~[t,h] . k^[b]) over the
+ *               idx_heads indexer heads (the DeepSeek-DSA form), no extra scale;
+ *   block key   k^[b] = RoPE_{r*b}( (1/r) sum_{j<r} k_idx[r*b+j] ), computed in
+ *               fp32 in that order and stored in the I/O dtype (bf16 RNE);
+ *   query       q~[t,h] = RoPE_t(q_idx[t,h]) stored in the I/O dtype;
+ *   RoPE        partial: the first rope_dims = floor(idx_dim*rope_fraction)
+ *               (even) dims rotate in rotate-half pairs (i, i+rope_dims/2),
+ *               theta_i = rope_base^(-2i/rope_dims), angle formed in fp64;
+ *   candidates  blocks b < b_t = floor(t/r) (all complete);
+ *   selection   if b_t+1 <= S = budget_tokens/r, blocks 0..b_t; otherwise the
+ *               own block b_t plus the S-1 best candidates under the order
+ *               (score descending, block index ascending; -0 equals +0);
+ *   attention   token j is attended iff floor(j/r) is selected and j <= t;
+ *               head h reads KV group floor(h / (n_q_heads/n_kv_groups));
+ *               softmax scale 1/sqrt(head_dim) unless given.
+ *
+ * Conventions shared by every call:
+ *   - The caller owns every buffer.  The library never allocates, never
+ *     synchronises the stream and keeps no pointer after a call returns.
+ *   - "device" pointers are CUDA global memory of the current device,
+ *     16-byte aligned, densely packed in the layouts given (innermost last).
+ *     "host" pointers are read during the call only.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *     All work is enqueued on it in order; a call returns before it runs.
+ *   - Host-checkable errors return QSA_ERR_INVALID_ARG / QSA_ERR_UNSUPPORTED /
+ *     QSA_ERR_WORKSPACE before anything is enqueued.  A failed launch returns
+ *     QSA_ERR_CUDA.  Device-side faults of bounded waits are reported by
+ *     qsa_device_status().  A call with no query tokens is a no-op (QSA_OK).
+ *   - Supported shapes: r == 4, head_dim == 256, n_q_heads/n_kv_groups <= 16,
+ *     idx_heads == 4, idx_dim in {64, 128}, budget_tokens a multiple of r with
+ *     budget_tokens/r <= 512.
+ *
+ * Token batch.  A call processes T query tokens given as segments: segment i
+ * holds q_len consecutive positions pos0 .. pos0+q_len-1 of the sequence in
+ * cache slot `slot`, stored at token rows q_offset .. q_offset+q_len-1 of
+ * every token-major array (q, q_idx, w, o, lse, sel, nsel, score rows).
+ * Prefill, a prefill chunk over a cached prefix, and decode (q_len = 1) are
+ * all segments.  The cache must already hold every token <= pos0+q_len-1.
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1,  /* bad pointer, size, layout or segment; nothing enqueued */
+  QSA_ERR_UNSUPPORTED = 2,  /* valid configuration the kernels do not implement      */
+  QSA_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than qsa_workspace_size()     */
+  QSA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed             */
+  QSA_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (qsa_device_status)  */
+} qsa_status_t;
+
+typedef enum { QSA_DTYPE_F32 = 0, QSA_DTYPE_BF16 = 1 } qsa_dtype_t;
+
+/* Per-layer constants (Miles docs section 1; design report QSA item). */
+typedef struct {
+  int32_t r;              /* tokens per micro-block: 4                               */
+  int32_t budget_tokens;  /* kept tokens per query: 2048 (multiple of r)             */
+  int32_t n_q_heads;      /* attention query heads: 24                               */
+  int32_t n_kv_groups;    /* KV groups: 2                                            */
+  int32_t head_dim;       /* 256                                                     */
+  int32_t idx_heads;      /* indexer query heads: 4                                  */
+  int32_t idx_dim;        /* indexer head dim: 64 or 128                             */
+  float rope_fraction;    /* rotated share of idx_dim: 0.25                          */
+  double rope_base;       /* 1e7                                                     */
+  float softmax_scale;    /* <= 0 selects 1/sqrt(head_dim)                           */
+  qsa_dtype_t dtype;      /* I/O dtype of q, q_idx, k_idx, k^, K, V and o            */
+} qsa_config_t;
+
+/* One run of consecutive query tokens of one cached sequence. */
+typedef struct {
+  int32_t q_offset;       /* first token row in the token-major arrays               */
+  int32_t q_len;          /* number of query tokens (>= 0)                           */
+  int32_t pos0;           /* absolute position of the first query token (>= 0)       */
+  int32_t slot;           /* cache slot of the sequence, in [0, n_slots)             */
+} qsa_segment_t;
+
+/* Per-sequence caches (device memory, caller-owned).  n_cap tokens per slot. */
+typedef struct {
+  const void* k_idx;      /* [n_slots][n_cap][idx_dim]            indexer keys        */
+  void* khat;             /* [n_slots][n_cap/r][idx_dim]          pooled block keys   */
+  const void* k;          /* [n_slots][n_kv_groups][n_cap][head_dim]  main keys       */
+  const void* v;          /* [n_slots][n_kv_groups][n_cap][head_dim]  main values     */
+  int32_t n_slots;
+  int64_t n_cap;          /* multiple of r                                          */
+} qsa_cache_t;
+
+typedef enum {
+  QSA_OP_COMPRESS = 0,
+  QSA_OP_INDEX = 1,
+  QSA_OP_SELECT = 2,
+  QSA_OP_ATTN = 3,
+  QSA_OP_FORWARD = 4
+} qsa_op_t;
+
+/*
+ * Key pooling + block position encoding (design report, QSA item: keys are
+ * averaged per micro-block, then position-encoded).  For each i < n_ranges,
+ * writes k^ of blocks [blk_begin[i], blk_end[i]) of cache slot slots[i]:
+ *   cache->khat[slot][b][:] = RoPE_{r*b}(mean of cache->k_idx[slot][r*b .. r*b+r-1][:]).
+ * slots, blk_begin, blk_end: host arrays [n_ranges].  Requires
+ * 0 <= blk_begin <= blk_end <= n_cap/r.  Reads k_idx, writes khat only.
+ */
+qsa_status_t qsa_compress_keys(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                               const int32_t* slots, const int64_t* blk_begin,
+                               const int64_t* blk_end, int32_t n_ranges, void* stream);
+
+/*
+ * Indexer scores (design report, QSA item: 4-head MQA indexer scoring
+ * micro-blocks; Miles docs section 1: each layer scores its own compressed
+ * keys).  For every query token i at position t (segments, host array):
+ *   scores[i][b] = sum_h w[i][h] * max(0, RoPE_t(q_idx[i][h]) . khat[slot][b]),
+ *   b in [0, floor(t/r)).
+ * q_idx: device [T][idx_heads][idx_dim] (I/O dtype); w: device [T][idx_heads]
+ * fp32; cache->khat must hold blocks [0, floor(t/r)) for every query.
+ * scores: device fp32 [T][ld_scores]; entries b >= floor(t/r) of a row are not
+ * written.  ld_scores >= max floor(t/r) over all queries, and >= 1.
+ * n_tokens: T, the row count of the token-major arrays.
+ */
+qsa_status_t qsa_index_scores(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                              const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                              const void* q_idx, const float* w, float* scores,
+                              int64_t ld_scores, void* stream);
+
+/*
+ * Top-k block selection (pages: budget 2048 tokens per query; the own block
+ * rule and the tie order are this library's readings, see top of file).
+ * For every query token i at position t: sel[i][0..nsel[i]) = the kept blocks
+ * in ascending order (the own block floor(t/r) last), sel[i][nsel[i]..S) = -1,
+ * nsel[i] = min(S, floor(t/r)+1), S = budget_tokens/r.
+ * scores: device fp32 [T][ld_scores] as written by qsa_index_scores.
+ * sel: device int32 [T][S]; nsel: device int32 [T].
+ * workspace: device, >= qsa_workspace_size(..., QSA_OP_SELECT) bytes (may be
+ * NULL when that size is 0).  Contents on entry are ignored.
+ */
+qsa_status_t qsa_select_topk(const qsa_config_t* cfg, const qsa_segment_t* segs,
+                             int32_t n_segs, int32_t n_tokens, const float* scores,
+                             int64_t ld_scores, int32_t* sel, int32_t* nsel, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * Sparse GQA softmax attention over the kept tokens (Miles docs section 1:
+ * attention reads only the kept key tokens; 24 heads, 2 query groups, head
+ * dim 256).  For every query token i at position t and head h (group
+ * g = h / (n_q_heads/n_kv_groups)):
+ *   J = { j : floor(j/r) in sel[i][0..nsel[i]), j <= t },
+ *   o[i][h][:]  = sum_{j in J} softmax_j(scale * q[i][h] . K[slot][g][j]) V[slot][g][j][:],
+ *   lse[i][h]   = log sum_{j in J} exp(scale * q[i][h] . K[slot][g][j])   (natural log).
+ * q, o: device [T][n_q_heads][head_dim] (I/O dtype).  lse: device fp32
+ * [T][n_q_heads] or NULL.  sel/nsel as produced by qsa_select_topk (entries
+ * must lie in [0, n_cap/r)).  workspace >= qsa_workspace_size(..., QSA_OP_ATTN).
+ */
+qsa_status_t qsa_sparse_attn_fwd(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                 const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                                 const void* q, const int32_t* sel, const int32_t* nsel, void* o,
+                                 float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The whole QSA forward pass for a token batch (prefill, chunked prefill over
+ * a cached prefix, decode, or a mix), enqueued on one stream with no host
+ * synchronisation:
+ *   1. qsa_compress_keys for the blocks each segment completes:
+ *      [floor(pos0/r), floor((pos0+q_len)/r));
+ *   2. qsa_index_scores; 3. qsa_select_topk; 4. qsa_sparse_attn_fwd.
+ * Blocks before floor(pos0/r) must already be pooled in cache->khat.
+ * sel/nsel: device outputs as in qsa_select_topk, or both NULL to keep them in
+ * the workspace.  workspace >= qsa_workspace_size(..., QSA_OP_FORWARD).
+ */
+qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                         const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                         const void* q, const void* q_idx, const float* w, void* o, float* lse,
+                         int32_t* sel, int32_t* nsel, void* workspace, size_t ws_bytes,
+                         void* stream);
+
+/* Workspace bytes an operation needs for this batch (0 if none; SIZE_MAX on an
+ * invalid argument).  Host-only; no CUDA call. */
+size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* segs, int32_t n_segs,
+                          int32_t n_tokens, qsa_op_t op);
+
+/* Reads and clears the current device's error word written by bounded
+ * device-side waits; synchronises `stream`.  QSA_OK if no wait gave up. */
+qsa_status_t qsa_device_status(void* stream);
+
+/* Static description of a status code. */
+const char* qsa_status_string(qsa_status_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t qsa_version(void);
+
+/* Number of CUDA kernels this library has enqueued since it was loaded, in
+ * this process (all devices, all streams).  Host counter; no CUDA call. */
+int64_t qsa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QSA_H */

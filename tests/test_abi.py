@@ -1,0 +1,119 @@
+"""The C ABI library: loads without a GPU, exports every entry point that
+include/qsa.h declares, and rejects bad arguments on the host before any
+CUDA call (CPU only; no compute is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_22_b200 as qsa
+from block_sparse_attention_22_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(qsa_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert {"qsa_compress_keys", "qsa_index_scores", "qsa_select_topk", "qsa_sparse_attn_fwd",
+            "qsa_forward", "qsa_workspace_size"} <= set(names)
+    lib = ctypes.CDLL(qsa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_exports_nothing_else():
+    out = os.popen(f"nm -D --defined-only {qsa.LIB_PATH}").read()
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    ours = {n for n in exported if n.startswith("qsa_")}
+    assert ours == set(declared_functions())
+
+
+def _setup(shape=None):
+    sh = shape or synth.Shape()
+    cfg = qsa.make_config(sh)
+    segs = qsa.make_segments([(0, 16, 100, 0)])
+    cache = qsa.qsa_cache_t(16, 16, 16, 16, 1, 1024)    # fake aligned addresses: never dereferenced
+    return sh, cfg, segs, cache
+
+
+def _call_forward(cfg, cache, segs, T=16, ws_bytes=1 << 40, **kw):
+    L = qsa.get_lib()
+    args = dict(q=16, q_idx=16, w=16, o=16, lse=None, sel=None, nsel=None, ws=16)
+    args.update(kw)
+    return L.qsa_forward(ctypes.byref(cfg), ctypes.byref(cache), segs[0], segs[1], T, args["q"], args["q_idx"],
+                         args["w"], args["o"], args["lse"], args["sel"], args["nsel"], args["ws"], ws_bytes, None)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("r", 8, qsa.QSA_ERR_UNSUPPORTED),
+    ("r", 0, qsa.QSA_ERR_INVALID_ARG),
+    ("budget_tokens", 2047, qsa.QSA_ERR_INVALID_ARG),
+    ("budget_tokens", 8192, qsa.QSA_ERR_UNSUPPORTED),
+    ("head_dim", 128, qsa.QSA_ERR_UNSUPPORTED),
+    ("n_kv_groups", 5, qsa.QSA_ERR_INVALID_ARG),
+    ("n_kv_groups", 1, qsa.QSA_ERR_UNSUPPORTED),
+    ("idx_heads", 8, qsa.QSA_ERR_UNSUPPORTED),
+    ("idx_dim", 96, qsa.QSA_ERR_UNSUPPORTED),
+    ("rope_fraction", 1.5, qsa.QSA_ERR_INVALID_ARG),
+    ("rope_base", -1.0, qsa.QSA_ERR_INVALID_ARG),
+    ("dtype", 7, qsa.QSA_ERR_INVALID_ARG),
+])
+def test_bad_config_is_rejected_on_host(field, value, status):
+    sh, cfg, segs, cache = _setup()
+    setattr(cfg, field, value)
+    assert _call_forward(cfg, cache, segs) == status
+
+
+def test_bad_segments_pointers_and_workspace_are_rejected_on_host():
+    sh, cfg, segs, cache = _setup()
+    for bad in [(0, 16, 1020, 0), (8, 16, 0, 0), (0, -1, 0, 0), (0, 4, 0, 3), (-1, 4, 0, 0)]:
+        assert _call_forward(cfg, cache, qsa.make_segments([bad])) == qsa.QSA_ERR_INVALID_ARG, bad
+    assert _call_forward(cfg, cache, segs, q=None) == qsa.QSA_ERR_INVALID_ARG
+    assert _call_forward(cfg, cache, segs, q=18) == qsa.QSA_ERR_INVALID_ARG      # misaligned
+    assert _call_forward(cfg, cache, segs, sel=16) == qsa.QSA_ERR_INVALID_ARG   # sel without nsel
+    assert _call_forward(cfg, cache, segs, ws_bytes=10) == qsa.QSA_ERR_WORKSPACE
+    assert _call_forward(cfg, cache, segs, ws=None) == qsa.QSA_ERR_WORKSPACE
+    bad_cache = qsa.qsa_cache_t(16, 16, 16, 16, 1, 1023)
+    assert _call_forward(cfg, bad_cache, segs) == qsa.QSA_ERR_INVALID_ARG
+
+
+def test_empty_batches_are_noops_without_touching_the_device():
+    sh, cfg, segs, cache = _setup()
+    empty = qsa.make_segments([(0, 0, 100, 0)])
+    assert _call_forward(cfg, cache, empty, T=0, ws=None, ws_bytes=0) == qsa.QSA_OK
+    none = qsa.make_segments([])
+    assert _call_forward(cfg, cache, none, T=0, ws=None, ws_bytes=0) == qsa.QSA_OK
+
+
+def test_workspace_sizes_are_host_only_and_grow_with_the_batch():
+    sh = synth.Shape()
+    cfg = qsa.make_config(sh)
+    small = qsa.make_segments([(0, 1024, 0, 0)])
+    big = qsa.make_segments([(0, 131072, 0, 0)])
+    a = qsa.workspace_size(cfg, small, 1024, qsa.QSA_OP_FORWARD)
+    b = qsa.workspace_size(cfg, big, 131072, qsa.QSA_OP_FORWARD)
+    assert 0 < a < b
+    assert b >= 131072 * 32767 * 4           # the score rows
+    assert qsa.workspace_size(cfg, small, 1024, qsa.QSA_OP_COMPRESS) == 0
+    dec = qsa.make_segments([(i, 1, (1 << 20) - 1, i) for i in range(8)])
+    assert qsa.workspace_size(cfg, dec, 8, qsa.QSA_OP_SELECT) > 0     # long rows are split
+    assert qsa.workspace_size(cfg, dec, 8, qsa.QSA_OP_ATTN) > 0       # few units: split-K
+    bad = qsa.make_segments([(0, 10, 0, 0)])
+    assert qsa.workspace_size(cfg, bad, 5, qsa.QSA_OP_FORWARD) == 2 ** 64 - 1
+
+
+def test_status_strings_and_version():
+    assert qsa.status_string(qsa.QSA_OK) == "ok"
+    assert "workspace" in qsa.status_string(qsa.QSA_ERR_WORKSPACE)
+    assert qsa.version() >= 100
