@@ -61,6 +61,7 @@ def _load():
         "qsa_sparse_attn_fwd": [C, K, S, I32, I32, P, P, P, P, P, P, SZ, P],
         "qsa_forward": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, SZ, P],
         "qsa_device_status": [P],
+        "qsa_select_topk_noalloc": [C, S, I32, I32, P, I64, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -152,6 +153,14 @@ def qsa_select_topk(cfg, segs, n_tokens, scores, ld_scores, sel, nsel, workspace
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(get_lib().qsa_select_topk(ctypes.byref(cfg), arr, n, n_tokens, _ptr(scores), ld_scores, _ptr(sel),
                                _ptr(nsel), _ptr(workspace), ws_bytes, _stream(stream)), "qsa_select_topk")
+
+
+def qsa_select_topk_noalloc(cfg, segs, n_tokens, scores, ld_scores, sel, nsel, stream=None):
+    """qsa_select_topk with its scratch in the library's static device array
+    (no workspace argument; for callers that cannot allocate device memory)."""
+    arr, n = segs
+    _check(get_lib().qsa_select_topk_noalloc(ctypes.byref(cfg), arr, n, n_tokens, _ptr(scores), ld_scores,
+                                             _ptr(sel), _ptr(nsel), _stream(stream)), "qsa_select_topk_noalloc")
 
 
 def qsa_sparse_attn_fwd(cfg, cache, segs, n_tokens, q, sel, nsel, o, lse=None, workspace=None,

@@ -12,6 +12,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "qsa_internal.cuh"
@@ -523,3 +524,58 @@ QSA_API const char* qsa_status_string(qsa_status_t status) {
 QSA_API int32_t qsa_version(void) { return 100; }
 
 QSA_API int64_t qsa_launch_count(void) { return (int64_t)launch_counter().load(); }
+
+// ------------------------------------------------------------------ allocation-free selection
+// Top-k selection for callers that cannot allocate device memory: the
+// split-row candidate buffers live in this file-scope device array instead
+// of a caller workspace.  Every device that loads the library holds the
+// array until the process exits.  All calls on a device share it, so calls
+// whose work overlaps on the GPU (different streams, no ordering) race on
+// it; calls on one stream are ordered and safe.  Nothing in it needs to start
+// at zero: every candidate count the merge pass reads is written first by
+// the chunk pass of the same call.
+static __device__ __align__(256) unsigned char g_select_scratch[QSA_NOALLOC_SCRATCH_BYTES];
+
+namespace qsa {
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices];
+
+// Device address of g_select_scratch on the current device.  In host code
+// the array's name only stands for a host-side shadow, so the address is
+// looked up once per device, with that device current, and cached.
+qsa_status_t select_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || !p) return QSA_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return QSA_OK;
+}
+}  // namespace
+}  // namespace qsa
+
+QSA_API qsa_status_t qsa_select_topk_noalloc(const qsa_config_t* cfg, const qsa_segment_t* segs,
+                                             int32_t n_segs, int32_t n_tokens, const float* scores,
+                                             int64_t ld_scores, int32_t* sel, int32_t* nsel,
+                                             void* stream) {
+  qsa_status_t s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if ((s = check_segments(segs, n_segs, n_tokens, nullptr, 0)) != QSA_OK) return s;
+  if (seg_rows(segs, n_segs) == 0) return QSA_OK;
+  if (!scores || !sel || !nsel || !aligned16(sel)) return QSA_ERR_INVALID_ARG;
+  const int64_t nblk = seg_max_blocks(segs, n_segs, cfg->r);
+  if (ld_scores < std::max<int64_t>(1, nblk)) return QSA_ERR_INVALID_ARG;
+  if (nblk > (int64_t)topk::kChunkLarge * 32) return QSA_ERR_UNSUPPORTED;
+  const Geo g = make_geo(cfg, nullptr);
+  if (topk_plan(g, segs, n_segs).ws > (size_t)QSA_NOALLOC_SCRATCH_BYTES) return QSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((s = select_scratch(&scratch)) != QSA_OK) return s;
+  return run_select(g, segs, n_segs, scores, ld_scores, sel, nsel, scratch,
+                    (size_t)QSA_NOALLOC_SCRATCH_BYTES, (cudaStream_t)stream);
+}

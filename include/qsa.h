@@ -200,6 +200,35 @@ qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cache,
                          int32_t* sel, int32_t* nsel, void* workspace, size_t ws_bytes,
                          void* stream);
 
+/*
+ * qsa_select_topk without a caller workspace, for callers that cannot call
+ * cudaMalloc: code running where the allocator is off limits (a custom
+ * allocator or memory pool owns all device memory, an embedding that forbids
+ * allocation after start-up, or a section whose memory use must be fixed in
+ * advance).  The pages have no counterpart to this call; it is an interface
+ * convenience, not part of the method.
+ *
+ * Same arguments, results and errors as qsa_select_topk, minus the
+ * workspace.  Rows long enough to be split keep their per-chunk candidates
+ * in a device array built into the library, QSA_NOALLOC_SCRATCH_BYTES (16 MiB)
+ * per device, held by every GPU that loads the library until the process
+ * exits.  A batch whose selection needs more than that (see
+ * qsa_workspace_size(..., QSA_OP_SELECT)) returns QSA_ERR_WORKSPACE and
+ * enqueues nothing.  Nothing is allocated or freed.
+ *
+ * The first call on a device looks up the array's device address (a CUDA
+ * runtime query, once per device, with that device current); make that first
+ * call before any stream capture on the device.  All calls on a device share
+ * the one array and it keeps the last call's contents: calls that can
+ * overlap on the GPU (other streams without ordering between them) race on
+ * it; calls ordered on one stream do not.
+ */
+#define QSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+qsa_status_t qsa_select_topk_noalloc(const qsa_config_t* cfg, const qsa_segment_t* segs,
+                                     int32_t n_segs, int32_t n_tokens, const float* scores,
+                                     int64_t ld_scores, int32_t* sel, int32_t* nsel,
+                                     void* stream);
+
 /* Workspace bytes an operation needs for this batch (0 if none; SIZE_MAX on an
  * invalid argument).  Host-only; no CUDA call. */
 size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* segs, int32_t n_segs,
