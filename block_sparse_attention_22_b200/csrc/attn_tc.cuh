@@ -1,0 +1,499 @@
+// attn_tc.cuh -- sparse GQA attention on tcgen05 tensor cores (bf16 I/O).
+//
+// Miles docs "Qwen3.8-Flash-Next", section 1: attention reads only the kept
+// key tokens; 24 heads in 2 query groups, head dim 256.  The heads of a group
+// share one selection, so a work unit is (query token, KV group): its hpg<=16
+// heads against the group's kept blocks (up to 512 blocks = 2048 keys).
+//
+// The MMAs are swapped so that the gathered keys fill the 128-row M side:
+//   S^T[key, head]  = K_chunk[key, :] . Q[head, :]       (M=128 keys, N=16, K=256)
+//   O_c^T[d, head]  = V_chunk^T[d, key] . P^T[key, head]  (M=128 dims x2, N=16, K=128)
+// A chunk is 32 kept blocks (128 keys).  Kept blocks are contiguous 4-row
+// runs of the group's K/V cache; each is copied into the 128-byte-swizzled
+// K-major layout the MMA reads (8-row atoms are filled by two blocks).
+// Loads and MMAs walk one item sequence per unit, K(0), K(1), V(0), K(2),
+// V(1), ..., V(n-1); an item is two 32 KiB half-slots (128 keys x 128 dims)
+// of a 6-slot ring, reused in the order the MMAs consume them.
+//
+// The gather is HBM/L2-bound and scattered (2 KiB per kept block and tensor),
+// so it is issued as 16-byte cp.async copies by eight producer warps: on
+// B200 a 4-row block only forms 512-byte TMA boxes, and the TMA request rate
+// held such gathers near 1 TB/s, while wide cp.async issue reaches the
+// memory system's rate.
+//
+// Roles (17 warps, persistent over work units, one CTA per SM):
+//   warps 0..7   producers: every half-slot is shared, warp w copying kept
+//                blocks 4w..4w+3 (one 512-byte row quad per instruction);
+//                a warp publishes a half-slot once its own copies of it have
+//                landed, keeping kArmDepth newer half-slots in flight.  Warp 0
+//                also loads each unit's Q tile with TMA.
+//   warp 8       TMEM owner and single-thread MMA issuer;
+//   warps 9..16  softmax and epilogue: a thread owns TMEM lane i (key i of the
+//                chunk for S; dims i and 128+i for O) and 8 of the 16 heads.
+//                Online softmax in the exp2 domain; each chunk's P.V lands in
+//                TMEM and is added into fp32 registers with the running rescale.
+// Every mbarrier wait is bounded (sm100::mbar_wait); a timeout records an
+// error and the CTA's roles drain and return.
+#pragma once
+#include "qsa_internal.cuh"
+#include "sm100.cuh"
+#include "attn_simt.cuh"
+
+namespace qsa {
+namespace tc_attn {
+constexpr int kProducers = 8;
+constexpr int kMmaWarp = kProducers;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 32 * (kProducers + 1 + kSoftmaxWarps);   // 544
+constexpr int kArmDepth = 4;               // half-slots a producer keeps in flight beyond the one it publishes
+constexpr int kKeys = 128;                 // keys per chunk
+constexpr int kBlk = 32;                   // blocks per chunk
+constexpr int kSlots = 6;                  // 32 KiB K/V half-chunk slots
+constexpr int kSlotBytes = 32768;
+constexpr int kQBytes = 8192;              // 16 heads x 256 dims, 4 slabs x 2 KiB
+constexpr int kPBytes = 4096;              // 16 heads x 128 keys, 2 slabs x 2 KiB
+constexpr int kN = 16;                     // heads per MMA tile
+constexpr int kHH = 8;                     // heads per softmax thread
+constexpr int kOffQ = kSlots * kSlotBytes;                 // 196608
+constexpr int kOffP = kOffQ + 2 * kQBytes;                 // 212992
+constexpr int kOffBar = kOffP + 2 * kPBytes;               // 221184
+constexpr int kSmemBytes = kOffBar + 1024 + 1024;          // + control block + alignment slack
+constexpr uint32_t kTmemCols = 128;        // S: 2 x 16 cols at 0; O: 2 x 32 cols at 32
+constexpr uint32_t kIdescS = sm100::idesc_bf16(128, kN, false, false);
+constexpr uint32_t kIdescPV = sm100::idesc_bf16(128, kN, true, false);
+static_assert(kArmDepth < kSlots, "a producer must publish a slot before it needs that slot again");
+}
+
+struct AttnTcArgs {
+  const void* k;           // bf16 [n_slots][G][n_cap][D]
+  const void* v;
+  const int32_t* sel;
+  const int32_t* nsel;
+  void* o;                 // bf16 [T][H][D]
+  float* lse;              // [T][H] or null
+  float* part_o;           // split partials (n_split > 1)
+  float* part_ml;
+  int n_split;
+  int blocks_per_split;    // multiple of 32
+  int64_t units_per_group; // = st.item0[st.n]
+};
+
+struct AttnTcCtl {
+  uint64_t slot_full[tc_attn::kSlots];
+  uint64_t slot_empty[tc_attn::kSlots];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full[2], p_free[2];
+  uint64_t o_full[2], o_free[2];
+  uint64_t mma_done;
+  float red[2][4][16];
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct TcUnit {
+  int64_t tok;
+  int64_t t;
+  int64_t slot;
+  int grp;
+  int split;
+  int blk_begin;   // first position in the sel row
+  int blk_end;     // one past the last
+  int nchunks;
+};
+
+// Warp-uniform wait: lane 0 waits, every lane gets its verdict.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = sm100::mbar_wait(bar, parity, abort_flag) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ bool warp_aborted(volatile int* abort_flag) {
+  return __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
+}
+
+__device__ __forceinline__ TcUnit tc_unit(const Geo& g, const SegTable& st, const AttnTcArgs& a, int64_t w) {
+  TcUnit u;
+  u.grp = (int)(w / a.units_per_group);
+  const int rem = (int)(w - (int64_t)u.grp * a.units_per_group);
+  const int si = find_segment(st, rem);
+  const int local = rem - st.item0[si];
+  const int j = local / a.n_split;
+  u.split = local - j * a.n_split;
+  u.tok = st.q_offset[si] + j;
+  u.t = (int64_t)st.pos0[si] + j;
+  u.slot = st.slot[si];
+  const int nsel = min(max(a.nsel[u.tok], 0), g.S);
+  u.blk_begin = u.split * a.blocks_per_split;
+  u.blk_end = min(nsel, u.blk_begin + a.blocks_per_split);
+  u.nchunks = u.blk_end > u.blk_begin ? (int)cdiv(u.blk_end - u.blk_begin, tc_attn::kBlk) : 0;
+  return u;
+}
+
+__global__ void __launch_bounds__(tc_attn::kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Geo g, SegTable st, AttnTcArgs a) {
+  using namespace tc_attn;
+  using namespace sm100;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  AttnTcCtl& ctl = *reinterpret_cast<AttnTcCtl*>(smem + kOffBar);
+  volatile int* abort_flag = &ctl.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_units = (int64_t)g.G * a.units_per_group;
+
+  // ---------------------------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&ctl.slot_full[i], kProducers);
+      mbar_init(&ctl.slot_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ctl.q_full[i], 1);
+      mbar_init(&ctl.q_empty[i], 1);
+      mbar_init(&ctl.s_full[i], 1);
+      mbar_init(&ctl.s_free[i], kSoftmaxWarps);
+      mbar_init(&ctl.p_full[i], kSoftmaxWarps);
+      mbar_init(&ctl.p_free[i], 1);
+      mbar_init(&ctl.o_full[i], 1);
+      mbar_init(&ctl.o_free[i], kSoftmaxWarps);
+    }
+    mbar_init(&ctl.mma_done, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_q);
+  }
+  // zero both Q tiles: rows hpg..15 are never loaded and must read as zero
+  for (int i = threadIdx.x; i < 2 * kQBytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem + kOffQ)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (warp == kMmaWarp) {
+    tmem_alloc(&ctl.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp < kProducers) {
+    // ============================================================ producers
+    int64_t hs_next = 0, uc = 0;                 // half-slots issued so far (shared numbering)
+    bool ok = true;
+    auto publish = [&](int64_t hs) {             // this warp's copies of hs have landed
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.slot_full[hs % kSlots]);
+    };
+    const int r = (lane >> 3) & 3, jc = lane & 7;   // row of a block and 16-byte chunk of a line
+    for (int64_t w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
+      if (warp_aborted(abort_flag)) break;
+      const TcUnit u = tc_unit(g, st, a, w);
+      if (u.nchunks == 0) continue;
+      if (warp == 0) {
+        const int qb = (int)(uc & 1);
+        if (!(ok = warp_wait(&ctl.q_empty[qb], (uint32_t)(((uc >> 1) & 1) ^ 1), abort_flag))) break;
+        if (lane == 0) {
+          mbar_expect_tx(&ctl.q_full[qb], (uint32_t)(g.hpg * 128 * 4));
+          const int32_t qrow = (int32_t)(u.tok * g.H + (int64_t)u.grp * g.hpg);
+          for (int s = 0; s < 4; ++s)
+            tma_load_2d(smem + kOffQ + qb * kQBytes + s * 2048, &tm_q, 64 * s, qrow, &ctl.q_full[qb]);
+        }
+        __syncwarp();
+      }
+      ++uc;
+      const __nv_bfloat16* kg = (const __nv_bfloat16*)a.k + (u.slot * g.G + u.grp) * g.n_cap * kHeadDim;
+      const __nv_bfloat16* vg = (const __nv_bfloat16*)a.v + (u.slot * g.G + u.grp) * g.n_cap * kHeadDim;
+      const int32_t* selrow = a.sel + u.tok * g.S;
+      for (int c = 0; c <= u.nchunks && ok; ++c) {
+        for (int kind = 0; kind < 2 && ok; ++kind) {   // K(c), then V(c-1)
+          if ((kind == 0 && c == u.nchunks) || (kind == 1 && c == 0)) continue;
+          const int cc = kind == 0 ? c : c - 1;
+          // kept blocks 4w..4w+3 of the chunk: lanes 0..3 look up their cache rows
+          int64_t myrow = -1;
+          if (lane < 4) {
+            const int pos = u.blk_begin + cc * kBlk + 4 * warp + lane;
+            if (pos < u.blk_end) myrow = block_row(selrow[pos], 0, g);
+          }
+          const __nv_bfloat16* base = kind == 0 ? kg : vg;
+          for (int h = 0; h < 2 && ok; ++h) {
+            const int64_t hs = hs_next++;
+            const int slot = (int)(hs % kSlots);
+            if (!(ok = warp_wait(&ctl.slot_empty[slot], (uint32_t)(((hs / kSlots) & 1) ^ 1), abort_flag))) break;
+            const uint32_t dst0 = smem_u32(smem + slot * kSlotBytes);
+#pragma unroll
+            for (int bq = 0; bq < 4; ++bq) {
+              const int b = 4 * warp + bq;
+              const int64_t row = __shfl_sync(0xffffffffu, myrow, bq);
+              const int line = 4 * b + r;
+              const uint32_t dst = dst0 + line * 128 + ((jc ^ (line & 7)) << 4);
+              const __nv_bfloat16* src = base + 128 * h + 8 * jc + (row >= 0 ? (row + r) * kHeadDim : 0);
+              const uint32_t nb = row >= 0 ? 16u : 0u;
+              cp_async16(dst, src, nb);                       // dims 128h + 8jc .. +8
+              cp_async16(dst + 16384, src + 64, nb);          // dims 128h + 64 + 8jc .. +8
+            }
+            cp_async_commit();
+            if (hs >= kArmDepth) {
+              cp_async_wait<kArmDepth>();
+              publish(hs - kArmDepth);
+            }
+          }
+        }
+      }
+    }
+    cp_async_wait<0>();                          // no copy of this warp outlives the CTA
+    if (ok)
+      for (int64_t hs = hs_next > kArmDepth ? hs_next - kArmDepth : 0; hs < hs_next; ++hs) publish(hs);
+  } else if (warp == kMmaWarp) {
+    // ============================================================ MMA issuer
+    // Whole warp in the loop; lane 0 issues the MMAs and commits.
+    int64_t gc = 0, uc = 0, it = 0;
+    const uint32_t smem_base = smem_u32(smem);
+    bool ok = true;
+    for (int64_t w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
+      if (warp_aborted(abort_flag)) break;
+      const TcUnit u = tc_unit(g, st, a, w);
+      if (u.nchunks == 0) continue;
+      const int qb = (int)(uc & 1);
+      if (!(ok = warp_wait(&ctl.q_full[qb], (uint32_t)((uc >> 1) & 1), abort_flag))) break;
+      ++uc;
+      const uint32_t q_addr = smem_base + kOffQ + qb * kQBytes;
+      for (int c = 0; c <= u.nchunks && ok; ++c) {
+        if (c < u.nchunks) {
+          const int64_t gs = gc + c;
+          const int sb = (int)(gs & 1);
+          if (!(ok = warp_wait(&ctl.s_free[sb], (uint32_t)(((gs >> 1) & 1) ^ 1), abort_flag))) break;
+          for (int half = 0; half < 2 && ok; ++half) {
+            const int64_t i = 2 * it + half;
+            const int slot = (int)(i % kSlots);
+            if (!(ok = warp_wait(&ctl.slot_full[slot], (uint32_t)((i / kSlots) & 1), abort_flag))) break;
+            tc_fence_after();
+            if (lane == 0) {
+              const uint32_t k_addr = smem_base + slot * kSlotBytes;
+              for (int kk = 0; kk < 8; ++kk) {          // 8 k-steps of 16 dims per half
+                const int slab = kk >> 2, sub = kk & 3;
+                const uint64_t da = desc_sw128(k_addr + slab * 16384 + sub * 32, 16, 1024);
+                const uint64_t db = desc_sw128(q_addr + (half * 2 + slab) * 2048 + sub * 32, 16, 1024);
+                umma_bf16(tmem + sb * kN, da, db, kIdescS, (half | kk) != 0);
+              }
+              umma_commit(&ctl.slot_empty[slot]);
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
+          ++it;
+          if (lane == 0) {
+            umma_commit(&ctl.s_full[sb]);
+            if (c == u.nchunks - 1) umma_commit(&ctl.q_empty[qb]);
+          }
+          __syncwarp();
+        }
+        if (c >= 1) {
+          const int64_t gp = gc + c - 1;
+          const int pb = (int)(gp & 1);
+          if (!(ok = warp_wait(&ctl.p_full[pb], (uint32_t)((gp >> 1) & 1), abort_flag))) break;
+          if (!(ok = warp_wait(&ctl.o_free[pb], (uint32_t)(((gp >> 1) & 1) ^ 1), abort_flag))) break;
+          const uint32_t p_addr = smem_base + kOffP + pb * kPBytes;
+          for (int half = 0; half < 2 && ok; ++half) {
+            const int64_t i = 2 * it + half;
+            const int slot = (int)(i % kSlots);
+            if (!(ok = warp_wait(&ctl.slot_full[slot], (uint32_t)((i / kSlots) & 1), abort_flag))) break;
+            tc_fence_after();
+            if (lane == 0) {
+              const uint32_t v_addr = smem_base + slot * kSlotBytes;
+              for (int kk = 0; kk < 8; ++kk) {          // 8 k-steps of 16 keys
+                const uint64_t da = desc_sw128(v_addr + kk * 2048, 16384, 1024);
+                const uint64_t db = desc_sw128(p_addr + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+                umma_bf16(tmem + 32 + pb * 32 + half * kN, da, db, kIdescPV, kk != 0);
+              }
+              umma_commit(&ctl.slot_empty[slot]);
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
+          ++it;
+          if (lane == 0) {
+            umma_commit(&ctl.o_full[pb]);
+            umma_commit(&ctl.p_free[pb]);
+          }
+          __syncwarp();
+        }
+      }
+      gc += u.nchunks;
+    }
+    // every MMA issued above has finished before TMEM is freed
+    if (lane == 0) {
+      umma_commit(&ctl.mma_done);
+      volatile int never = 0;
+      mbar_wait(&ctl.mma_done, 0, &never);
+    }
+    __syncwarp();
+  } else {
+    // ============================================================ softmax + epilogue
+    const int sw = warp - kMmaWarp - 1;                 // 0..7
+    const int quad = warp & 3;                          // TMEM lane quadrant this warp may access
+    const int h0 = (sw >> 2) * kHH;                     // first of this thread's 8 heads
+    const int li = quad * 32 + lane;                    // TMEM lane: key of the chunk / dim
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t smem_base = smem_u32(smem);
+    const float scale_log2 = g.scale * 1.4426950408889634f;
+    const int nthr = 32 * kSoftmaxWarps;
+    int64_t gc = 0;
+    // No early exit in this role: its warps meet at named barriers, so they
+    // must run the same iterations.  After an abort every wait returns at
+    // once and the loop runs through without blocking.
+    for (int64_t w = blockIdx.x; w < n_units; w += gridDim.x) {
+      const TcUnit u = tc_unit(g, st, a, w);
+      float m[kHH], lp[kHH], al[kHH], oacc[2 * kHH];
+#pragma unroll
+      for (int h = 0; h < kHH; ++h) {
+        m[h] = -INFINITY;
+        lp[h] = 0.f;
+        al[h] = 1.f;
+        oacc[h] = 0.f;
+        oacc[kHH + h] = 0.f;
+      }
+      const int32_t* selrow = a.sel + u.tok * g.S;
+      for (int c = 0; c <= u.nchunks; ++c) {
+        float alpha[kHH];
+        if (c < u.nchunks) {
+          const int64_t gs = gc + c;
+          const int sb = (int)(gs & 1);
+          // key validity (kept block, causal within the own block): fetched before the wait
+          const int pos = u.blk_begin + c * kBlk + (li >> 2);
+          bool valid = false;
+          if (pos < u.blk_end) {
+            const int64_t row = block_row(selrow[pos], li & 3, g);
+            valid = row >= 0 && row <= u.t;
+          }
+          mbar_wait(&ctl.s_full[sb], (uint32_t)((gs >> 1) & 1), abort_flag);
+          tc_fence_after();
+          float s[kHH];
+          tmem_ld8(lane_addr + sb * kN + h0, s);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.s_free[sb]);
+          float mx[kHH];
+#pragma unroll
+          for (int h = 0; h < kHH; ++h) {
+            s[h] = valid ? s[h] * scale_log2 : -INFINITY;
+            mx[h] = s[h];
+          }
+#pragma unroll
+          for (int off = 16; off; off >>= 1)
+#pragma unroll
+            for (int h = 0; h < kHH; ++h) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], off));
+          if (lane == 0)
+#pragma unroll
+            for (int h = 0; h < kHH; ++h) ctl.red[gs & 1][quad][h0 + h] = mx[h];
+          named_bar_sync(1, nthr);
+          const int pb = sb;
+          mbar_wait(&ctl.p_free[pb], (uint32_t)(((gs >> 1) & 1) ^ 1), abort_flag);
+          const uint32_t p_addr = smem_base + kOffP + pb * kPBytes;
+          const int slab = li >> 6, kin = li & 63;
+          const uint32_t p_lane = p_addr + slab * 2048 + (kin & 7) * 2;
+#pragma unroll
+          for (int h = 0; h < kHH; ++h) {
+            const int hh = h0 + h;
+            const float cm = fmaxf(fmaxf(ctl.red[gs & 1][0][hh], ctl.red[gs & 1][1][hh]),
+                                   fmaxf(ctl.red[gs & 1][2][hh], ctl.red[gs & 1][3][hh]));
+            const float mn = fmaxf(m[h], cm);
+            alpha[h] = (mn == -INFINITY) ? 1.f : exp2f(m[h] - mn);
+            const float p = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - mn);
+            m[h] = mn;
+            lp[h] = lp[h] * alpha[h] + p;          // fp32 denominator (exact log-sum-exp)
+            const uint32_t addr = p_lane + (hh >> 3) * 1024 + (hh & 7) * 128 + (((kin >> 3) ^ (hh & 7)) << 4);
+            st_shared_u16(addr, __bfloat16_as_ushort(__float2bfloat16_rn(p)));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.p_full[pb]);
+        }
+        if (c >= 1) {
+          const int64_t gp = gc + c - 1;
+          const int ob = (int)(gp & 1);
+          mbar_wait(&ctl.o_full[ob], (uint32_t)((gp >> 1) & 1), abort_flag);
+          tc_fence_after();
+          float o0[kHH], o1[kHH];
+          tmem_ld8(lane_addr + 32 + ob * 32 + h0, o0);
+          tmem_ld8(lane_addr + 32 + ob * 32 + kN + h0, o1);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.o_free[ob]);
+#pragma unroll
+          for (int h = 0; h < kHH; ++h) {
+            oacc[h] = oacc[h] * al[h] + o0[h];
+            oacc[kHH + h] = oacc[kHH + h] * al[h] + o1[h];
+          }
+        }
+        if (c < u.nchunks) {
+#pragma unroll
+          for (int h = 0; h < kHH; ++h) al[h] = alpha[h];
+        }
+      }
+      gc += u.nchunks;
+      // ---- epilogue: denominators, normalisation, stores
+      float l[kHH];
+#pragma unroll
+      for (int h = 0; h < kHH; ++h) l[h] = lp[h];
+#pragma unroll
+      for (int off = 16; off; off >>= 1)
+#pragma unroll
+        for (int h = 0; h < kHH; ++h) l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
+      named_bar_sync(1, nthr);                // red[] of the last chunk fully read
+      if (lane == 0)
+#pragma unroll
+        for (int h = 0; h < kHH; ++h) ctl.red[0][quad][h0 + h] = l[h];
+      named_bar_sync(1, nthr);
+#pragma unroll
+      for (int h = 0; h < kHH; ++h)
+        l[h] = ctl.red[0][0][h0 + h] + ctl.red[0][1][h0 + h] + ctl.red[0][2][h0 + h] + ctl.red[0][3][h0 + h];
+      named_bar_sync(1, nthr);                // before red[] is reused
+      const int64_t unit = u.tok * g.G + u.grp;
+      if (a.n_split == 1) {
+        __nv_bfloat16* og = (__nv_bfloat16*)a.o + (u.tok * g.H + (int64_t)u.grp * g.hpg) * kHeadDim;
+#pragma unroll
+        for (int h = 0; h < kHH; ++h) {
+          if (h0 + h < g.hpg) {
+            const float inv = 1.f / l[h];
+            og[(h0 + h) * kHeadDim + li] = __float2bfloat16_rn(oacc[h] * inv);
+            og[(h0 + h) * kHeadDim + 128 + li] = __float2bfloat16_rn(oacc[kHH + h] * inv);
+          }
+        }
+        if (a.lse && li == 0) {
+#pragma unroll
+          for (int h = 0; h < kHH; ++h)
+            if (h0 + h < g.hpg)
+              a.lse[u.tok * g.H + u.grp * g.hpg + h0 + h] = (m[h] + log2f(l[h])) * 0.6931471805599453f;
+        }
+      } else {
+        const int64_t base = (unit * a.n_split + u.split) * g.hpg;
+#pragma unroll
+        for (int h = 0; h < kHH; ++h) {
+          if (h0 + h < g.hpg) {
+            a.part_o[(base + h0 + h) * kHeadDim + li] = oacc[h];
+            a.part_o[(base + h0 + h) * kHeadDim + 128 + li] = oacc[kHH + h];
+          }
+        }
+        if (li == 0) {
+#pragma unroll
+          for (int h = 0; h < kHH; ++h)
+            if (h0 + h < g.hpg) {
+              a.part_ml[(base + h0 + h) * 2] = u.nchunks ? m[h] * 0.6931471805599453f : -INFINITY;
+              a.part_ml[(base + h0 + h) * 2 + 1] = l[h];
+            }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace qsa

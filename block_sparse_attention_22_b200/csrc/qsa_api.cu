@@ -20,6 +20,9 @@
 #include "index_simt.cuh"
 #include "topk.cuh"
 #include "attn_simt.cuh"
+#include "attn_tc.cuh"
+
+#include <cudaTypedefs.h>
 
 #define QSA_API extern "C" __attribute__((visibility("default")))
 
@@ -176,12 +179,14 @@ struct AttnPlan {
   size_t ws;
 };
 
-AttnPlan attn_plan(const Geo& g, const qsa_segment_t* segs, int n) {
+// bf16 runs on the tensor-core kernel (splits in whole 32-block chunks),
+// fp32 on the CUDA-core kernel (8-block chunks).
+AttnPlan attn_plan(const Geo& g, const qsa_segment_t* segs, int n, bool tc) {
   int64_t T = 0;
   for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
   const int64_t units = seg_rows(segs, n) * g.G;
   AttnPlan p{1, g.S, 0};
-  const int gran = simt_attn::KC / 4;
+  const int gran = tc ? tc_attn::kBlk : simt_attn::KC / 4;
   if (units > 0 && units < 2 * kNumSms) {
     int ns = (int)std::min<int64_t>(cdiv(2 * kNumSms, units), cdiv(g.S, gran));
     p.blocks_per_split = (int)(cdiv(cdiv(g.S, ns), gran) * gran);
@@ -289,12 +294,49 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
       });
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][inner] (row stride inner*2 bytes), box box_inner x
+// box_rows, 128-byte swizzle, out-of-range rows read as zero.
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                   uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return kNumSms;
+  return n > 0 ? n : kNumSms;
+}
+
 qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
-                      const qsa_segment_t* segs, int n, const void* q, const int32_t* sel,
+                      const qsa_segment_t* segs, int n, int32_t n_tokens, const void* q, const int32_t* sel,
                       const int32_t* nsel, void* o, float* lse, void* ws, size_t ws_bytes,
                       cudaStream_t st) {
   const bool bf = c->dtype == QSA_DTYPE_BF16;
-  const AttnPlan p = attn_plan(g, segs, n);
+  const AttnPlan p = attn_plan(g, segs, n, bf);
   if (p.ws > 0 && (!ws || ws_bytes < p.ws)) return QSA_ERR_WORKSPACE;
   AttnArgs a;
   memset(&a, 0, sizeof a);
@@ -313,16 +355,46 @@ qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* ca
     a.part_o = (float*)ws;
     a.part_ml = (float*)((char*)ws + align_up((size_t)T * g.G * p.n_split * g.hpg * kHeadDim * 4, 256));
   }
-  const size_t smem = attn_simt_smem();
-  cudaFuncSetAttribute(attn_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  qsa_status_t r = for_each_table(
-      segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len * g.G * p.n_split; },
-      [&](const SegTable& t) {
-        if (bf) { count_launch(); attn_simt_kernel<__nv_bfloat16><<<t.item0[t.n], simt_attn::THREADS, smem, st>>>(g, t, a); }
-        else { count_launch(); attn_simt_kernel<float><<<t.item0[t.n], simt_attn::THREADS, smem, st>>>(g, t, a); }
-        return cudaGetLastError();
-      });
+  qsa_status_t r;
+  if (bf) {
+    CUtensorMap tq;
+    if (!make_map_bf16(&tq, q, kHeadDim, (uint64_t)n_tokens * g.H, 64, (uint32_t)g.hpg)) return QSA_ERR_CUDA;
+    AttnTcArgs ta;
+    memset(&ta, 0, sizeof ta);
+    ta.k = cache->k;
+    ta.v = cache->v;
+    ta.sel = sel;
+    ta.nsel = nsel;
+    ta.o = o;
+    ta.lse = lse;
+    ta.part_o = a.part_o;
+    ta.part_ml = a.part_ml;
+    ta.n_split = p.n_split;
+    ta.blocks_per_split = p.blocks_per_split;
+    const int smem = tc_attn::kSmemBytes;
+    cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int sms = sm_count();
+    r = for_each_table(
+        segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len * p.n_split; },
+        [&](const SegTable& t) {
+          ta.units_per_group = t.item0[t.n];
+          const int64_t units = ta.units_per_group * g.G;
+          const int grid = (int)std::min<int64_t>(units, sms);
+          count_launch();
+          attn_tc_kernel<<<grid, tc_attn::kThreads, smem, st>>>(tq, g, t, ta);
+          return cudaGetLastError();
+        });
+  } else {
+    const size_t smem = attn_simt_smem();
+    cudaFuncSetAttribute(attn_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    r = for_each_table(
+        segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len * g.G * p.n_split; },
+        [&](const SegTable& t) {
+          count_launch();
+          attn_simt_kernel<float><<<t.item0[t.n], simt_attn::THREADS, smem, st>>>(g, t, a);
+          return cudaGetLastError();
+        });
+  }
   if (r != QSA_OK || p.n_split == 1) return r;
   return for_each_table(
       segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
@@ -341,7 +413,7 @@ struct FwdLayout {
   size_t scores, sel, nsel, topk, attn, total;
 };
 
-FwdLayout fwd_layout(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens) {
+FwdLayout fwd_layout(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens, bool tc) {
   FwdLayout L;
   L.ld = std::max<int64_t>(4, cdiv(seg_max_blocks(segs, n, g.r), 4) * 4);
   size_t off = 0;
@@ -354,7 +426,7 @@ FwdLayout fwd_layout(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_t
   L.topk = off;
   off += align_up(topk_plan(g, segs, n).ws, 256);
   L.attn = off;
-  off += align_up(attn_plan(g, segs, n).ws, 256);
+  off += align_up(attn_plan(g, segs, n, tc).ws, 256);
   L.total = off;
   return L;
 }
@@ -431,7 +503,7 @@ QSA_API qsa_status_t qsa_sparse_attn_fwd(const qsa_config_t* cfg, const qsa_cach
       !aligned16(cache->k) || !aligned16(cache->v) || !aligned16(sel))
     return QSA_ERR_INVALID_ARG;
   const Geo g = make_geo(cfg, cache);
-  return run_attn(g, cfg, cache, segs, n_segs, q, sel, nsel, o, lse, workspace, ws_bytes,
+  return run_attn(g, cfg, cache, segs, n_segs, n_tokens, q, sel, nsel, o, lse, workspace, ws_bytes,
                   (cudaStream_t)stream);
 }
 
@@ -444,8 +516,8 @@ QSA_API size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* 
     case QSA_OP_COMPRESS:
     case QSA_OP_INDEX: return 0;
     case QSA_OP_SELECT: return topk_plan(g, segs, n_segs).ws;
-    case QSA_OP_ATTN: return attn_plan(g, segs, n_segs).ws;
-    case QSA_OP_FORWARD: return fwd_layout(g, segs, n_segs, n_tokens).total;
+    case QSA_OP_ATTN: return attn_plan(g, segs, n_segs, cfg->dtype == QSA_DTYPE_BF16).ws;
+    case QSA_OP_FORWARD: return fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16).total;
   }
   return SIZE_MAX;
 }
@@ -469,7 +541,7 @@ QSA_API qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cac
   const int64_t nblk = seg_max_blocks(segs, n_segs, cfg->r);
   if (nblk > (int64_t)topk::kChunkLarge * 32) return QSA_ERR_UNSUPPORTED;
   const Geo g = make_geo(cfg, cache);
-  const FwdLayout L = fwd_layout(g, segs, n_segs, n_tokens);
+  const FwdLayout L = fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16);
   if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return QSA_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
   char* ws = (char*)workspace;
@@ -493,7 +565,7 @@ QSA_API qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cac
   if ((s = run_index(g, cfg, cache, segs, n_segs, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
   if ((s = run_select(g, segs, n_segs, scores, L.ld, sel, nsel, ws + L.topk, L.attn - L.topk, st)) != QSA_OK)
     return s;
-  return run_attn(g, cfg, cache, segs, n_segs, q, sel, nsel, o, lse, ws + L.attn, L.total - L.attn, st);
+  return run_attn(g, cfg, cache, segs, n_segs, n_tokens, q, sel, nsel, o, lse, ws + L.attn, L.total - L.attn, st);
 }
 
 QSA_API qsa_status_t qsa_device_status(void* stream) {

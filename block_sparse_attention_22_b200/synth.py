@@ -16,6 +16,9 @@ kv-channels 256, rotary 0.25 at base 1e7; design report, QSA item: r=4, a
   decode_256k   32 sequences x 1 decode query against a 262144-token cache
   mixed_1m      8 decode queries at 1048576-token context plus one 4096-query
                 prefill chunk at [942080, 946176) of a 90%-cached sequence
+  chunk_128k    one 4096-query prefill chunk at [126976, 131072) of a
+                131072-token sequence whose prefix is cached (a ~1 GB case
+                whose K/V still exceeds L2; used for kernel profiles)
 
 Distributions: q, k, v, indexer q and indexer k ~ N(0, 1) drawn in fp32 and
 rounded once to the I/O dtype; head weights w ~ U(0, 1) in fp32.
@@ -189,6 +192,14 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
         cached = [(ctx - 1) // sh.r] * n_dec + [pos0 // sh.r]
         return Workload(name, sh, segs, n_dec + 1, _round_cap(max(ctx, pos0 + chunk), sh.r), fill, cached, needles,
                         seed if seed is not None else 4)
+    if name == "chunk_128k":
+        sh = Shape()
+        n = over.get("n", 131072)
+        chunk = over.get("chunk", 4096)
+        pos0 = n - chunk
+        needles = _needles_per_window(rng, 0, pos0, n, 4, sh.r)
+        return Workload(name, sh, [Segment(0, pos0, chunk)], 1, _round_cap(n, sh.r), [n], [pos0 // sh.r],
+                        needles, seed if seed is not None else 5)
     raise KeyError(name)
 
 
