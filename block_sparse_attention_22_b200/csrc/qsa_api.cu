@@ -21,6 +21,7 @@
 #include "topk.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "index_tc.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -53,6 +54,7 @@ qsa_status_t check_cfg(const qsa_config_t* c) {
   if (c->n_q_heads / c->n_kv_groups > kMaxHpg) return QSA_ERR_UNSUPPORTED;
   if (c->budget_tokens / c->r > kMaxBudgetBlocks) return QSA_ERR_UNSUPPORTED;
   if (rope_dims_of(c) / 2 > kMaxRopeHalf) return QSA_ERR_UNSUPPORTED;
+  if (c->dtype == QSA_DTYPE_BF16 && rope_dims_of(c) / 2 > tc_index::kMaxRopeHalf) return QSA_ERR_UNSUPPORTED;
   return QSA_OK;
 }
 
@@ -226,21 +228,48 @@ qsa_status_t run_compress(const Geo& g, const qsa_config_t* c, const qsa_cache_t
   return flush();
 }
 
+// Tensor map of the k^ cache: [n_slots * n_cap/r rows][idx_dim] bf16, boxes of
+// 64 dims x 128 rows.
+bool make_khat_map(CUtensorMap* m, const qsa_config_t* c, const qsa_cache_t* cache);
+
+template <int NQ>
+cudaError_t launch_index_tc(const Geo& g, const SegTable& t, const CUtensorMap& tm, const IndexTcArgs& a,
+                            cudaStream_t st) {
+  const int items = t.item0[t.n];
+  if (items == 0) return cudaSuccess;
+  const int smem = IndexTcCfg<NQ>::kSmemBytes;
+  cudaFuncSetAttribute(index_tc_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  count_launch();
+  index_tc_kernel<NQ><<<items, tc_index::kThreads, smem, st>>>(tm, g, t, a);
+  return cudaGetLastError();
+}
+
 qsa_status_t run_index(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
                        const qsa_segment_t* segs, int n, const void* q_idx, const float* w,
                        float* scores, int64_t ld, cudaStream_t st) {
-  const bool bf = c->dtype == QSA_DTYPE_BF16;
-  size_t smem = sizeof(float) * (simt_index::QT * g.HI * g.DI + simt_index::QT * g.HI);
-  if (smem > 48 * 1024) {
-    cudaFuncSetAttribute(index_scores_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(index_scores_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (c->dtype == QSA_DTYPE_BF16) {
+    CUtensorMap tm;
+    if (!make_khat_map(&tm, c, cache)) return QSA_ERR_CUDA;
+    IndexTcArgs a{(const __nv_bfloat16*)q_idx, w, scores, ld};
+    // prefill-like segments on 64-query tiles, decode-like ones on 4-query tiles
+    std::vector<qsa_segment_t> wide, narrow;
+    for (int i = 0; i < n; ++i) (segs[i].q_len >= 16 ? wide : narrow).push_back(segs[i]);
+    qsa_status_t r = for_each_table(
+        wide.data(), (int)wide.size(),
+        [&](const qsa_segment_t& s) { return index_tc_items<64>(s.q_len, s.pos0, g.r); },
+        [&](const SegTable& t) { return launch_index_tc<64>(g, t, tm, a, st); });
+    if (r != QSA_OK) return r;
+    return for_each_table(
+        narrow.data(), (int)narrow.size(),
+        [&](const qsa_segment_t& s) { return index_tc_items<4>(s.q_len, s.pos0, g.r); },
+        [&](const SegTable& t) { return launch_index_tc<4>(g, t, tm, a, st); });
   }
+  size_t smem = sizeof(float) * (simt_index::QT * g.HI * g.DI + simt_index::QT * g.HI);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(index_scores_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   return for_each_table(
       segs, n, [&](const qsa_segment_t& s) { return (int64_t)simt_index_items(s.q_len, s.pos0, g.r); },
-      [&](const SegTable& t) {
-        return bf ? launch_index_simt<__nv_bfloat16>(g, t, q_idx, w, cache->khat, scores, ld, st)
-                  : launch_index_simt<float>(g, t, q_idx, w, cache->khat, scores, ld, st);
-      });
+      [&](const SegTable& t) { return launch_index_simt<float>(g, t, q_idx, w, cache->khat, scores, ld, st); });
 }
 
 qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const float* scores,
@@ -322,6 +351,11 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ro
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_khat_map(CUtensorMap* m, const qsa_config_t* c, const qsa_cache_t* cache) {
+  const uint64_t rows = (uint64_t)cache->n_slots * (uint64_t)(cache->n_cap / c->r);
+  return make_map_bf16(m, cache->khat, (uint64_t)c->idx_dim, rows, 64, tc_index::kTileRows);
 }
 
 int sm_count() {
