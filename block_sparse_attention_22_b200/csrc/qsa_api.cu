@@ -157,19 +157,22 @@ struct TopkPlan {
   size_t ws;
 };
 
+// Rows are split into chunks (local top S-1, then a merge) only when there
+// are too few rows to fill the GPU.
 TopkPlan topk_plan(const Geo& g, const qsa_segment_t* segs, int n) {
   TopkPlan p{topk::kChunkLarge, 1, 0};
   const int64_t nblk = seg_max_blocks(segs, n, g.r);
   const int64_t rows = seg_rows(segs, n);
-  if (nblk + 1 <= g.S) return p;
-  if (rows * cdiv(nblk, topk::kChunkLarge) < 2 * kNumSms) p.chunk = topk::kChunkSmall;
-  if (cdiv(nblk, p.chunk) > 32) p.chunk = (int)std::min<int64_t>(topk::kChunkLarge, cdiv(nblk, 32));
+  if (nblk + 1 <= g.S || rows >= 4 * kNumSms) return p;
+  p.chunk = (int)std::max<int64_t>(topk::kChunkSmall, cdiv(nblk, 32));
   p.max_ch = (int)cdiv(nblk, p.chunk);
   if (p.max_ch > 1) {
     int64_t T = 0;
     for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
     const size_t K = (size_t)(g.S - 1);
     p.ws = align_up((size_t)T * p.max_ch * K * 4, 256) * 2 + align_up((size_t)T * p.max_ch * 4, 256);
+  } else {
+    p.chunk = topk::kChunkLarge;
   }
   return p;
 }
@@ -296,8 +299,7 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
     base += align_up((size_t)T * p.max_ch * K * 4, 256);
     a.cand_cnt = (int32_t*)base;
   }
-  const size_t smem_c = topk_chunk_smem(p.chunk);
-  cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
+  const size_t smem_c = 0;
   const int64_t nblk = seg_max_blocks(segs, n, g.r);
   (void)nblk;
   qsa_status_t r = for_each_table(
@@ -312,8 +314,7 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
         return cudaGetLastError();
       });
   if (r != QSA_OK || p.max_ch <= 1) return r;
-  const size_t smem_m = topk_merge_smem(p.max_ch, g.S - 1);
-  cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_m);
+  const size_t smem_m = 0;
   return for_each_table(
       segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
       [&](const SegTable& t) {

@@ -6,154 +6,221 @@
 // always kept; the other S-1 are the best candidates b < floor(t/r) under
 // the total order (score descending, block index ascending), -0 == +0.
 //
-// Algorithm: scores are mapped to order-preserving uint32 keys and held in
-// shared memory; a 3-pass MSB radix select (11/11/10-bit digits, warp-
-// aggregated shared-memory histograms) finds the threshold key and how many
-// keys equal to it are taken; an index-ordered ballot compaction then emits
-// the kept blocks already sorted ascending, taking tied keys lowest index
-// first.  Rows longer than one chunk are split: every chunk keeps its own
-// top S-1 (exact under the same total order, so the union contains the
-// answer), and a merge pass selects from the union.
+// Algorithm (one CTA per row, or per row chunk for long rows; the row is
+// streamed from global memory, so several CTAs fit on an SM):
+//   1. radix narrowing: a histogram of the next 11/11/10 key bits over the
+//      elements still in the threshold bucket (warp-aggregated shared
+//      atomics) locates the bucket holding the K-th largest key; repeated
+//      until that bucket fits the shared candidate buffer;
+//   2. gather: elements above the bucket are kept outright, elements in it
+//      become candidates, ordered by the 64-bit composite (key, ~index) so
+//      that ties go to the lower index;
+//   3. the best candidates complete the K, found by a bitonic sort of the
+//      composite keys; the kept block indices are finally sorted ascending.
+// If the bucket is still larger than the buffer after all 32 bits (many
+// exactly equal keys), the tied elements are taken in index order by an
+// ordered ballot compaction instead.  Long rows are split into chunks whose
+// local top K (exact under the same order) are merged by a second pass of
+// the same routine over the chunk candidates.
 #pragma once
 #include "qsa_internal.cuh"
 
 namespace qsa {
 namespace topk {
-constexpr int THREADS = 512;
+constexpr int THREADS = 256;
 constexpr int WARPS = THREADS / 32;
 constexpr int NBINS = 2048;
-constexpr int kChunkLarge = 32768;
+constexpr int CAP = 4096;                  // candidate buffer (composite keys)
+constexpr int KMAX = kMaxBudgetBlocks;     // kept entries per row (S-1 <= 511)
+constexpr int kChunkLarge = 1 << 30;       // no split
 constexpr int kChunkSmall = 8192;
 }
 
-struct RadixState {
-  uint32_t prefix;
-  uint32_t mask;
-  int k_rem;
-};
-
 struct TopkShared {
   uint32_t hist[topk::NBINS];
+  unsigned long long cand[topk::CAP];      // (key << 32) | ~index
+  uint32_t kept[topk::KMAX];               // indices kept outright / final list
   int warp_a[topk::WARPS];
   int warp_b[topk::WARPS];
+  int n_kept, n_cand;
   uint32_t sel_digit;
-  int sel_above;
-  int sel_count;
+  int sel_above, sel_count;
 };
 
-// Finds the K-th largest key among keys[0..n) (K <= n): on return, a key x
-// is kept iff (x & mask) > prefix, or (x & mask) == prefix and it is among
-// the first k_rem such keys in index order.
-__device__ RadixState radix_select(const uint32_t* keys, int n, int K, TopkShared& sh) {
+// Source of one selection: element i has key(i) and index idx(i).
+struct RowSrc {
+  const float* scores;          // score row (keys from scores), or null
+  const uint32_t* keys;         // candidate keys (merge), or null
+  const int32_t* idx;           // candidate indices (merge)
+  int64_t base;                 // index of element 0 (score rows)
+  __device__ __forceinline__ uint32_t key(int i) const {
+    return scores ? score_key(scores[i]) : keys[i];
+  }
+  __device__ __forceinline__ uint32_t index(int i) const {
+    return scores ? (uint32_t)(base + i) : (uint32_t)idx[i];
+  }
+};
+
+// Histogram of digit (key >> shift) & dmask over elements with (key & mask) == prefix.
+__device__ void topk_hist(const RowSrc& src, int n, uint32_t prefix, uint32_t mask, int shift, uint32_t dmask,
+                          TopkShared& sh) {
   using namespace topk;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  RadixState rs{0u, 0u, K};
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < NBINS; i += THREADS) sh.hist[i] = 0;
+  __syncthreads();
+  for (int b = warp * 32; b < n; b += THREADS) {
+    const int i = b + lane;
+    const uint32_t key = i < n ? src.key(i) : 0u;
+    const bool valid = i < n && (key & mask) == prefix;
+    const uint32_t digit = (key >> shift) & dmask;
+    const uint32_t peers = __match_any_sync(0xffffffffu, valid ? digit : 0xffffffffu);
+    if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[digit], (uint32_t)__popc(peers));
+  }
+  __syncthreads();
+}
+
+// Finds the digit whose bucket holds the k_rem-th largest element: sets
+// sh.sel_digit, sh.sel_above (count in higher buckets), sh.sel_count.
+__device__ void topk_locate(int k_rem, TopkShared& sh) {
+  using namespace topk;
+  constexpr int PER = NBINS / THREADS;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int local = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) local += sh.hist[threadIdx.x * PER + j];
+  int suf = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_down_sync(0xffffffffu, suf, off);
+    if (lane + off < 32) suf += v;
+  }
+  if (lane == 0) sh.warp_a[warp] = suf;
+  __syncthreads();
+  int above_warps = 0;
+  for (int w = warp + 1; w < WARPS; ++w) above_warps += sh.warp_a[w];
+  const int incl = suf + above_warps, excl = incl - local;
+  if (excl < k_rem && k_rem <= incl) {
+    int above = excl;
+    for (int j = PER - 1; j >= 0; --j) {
+      const int b = threadIdx.x * PER + j;
+      const int c = (int)sh.hist[b];
+      if (above + c >= k_rem) {
+        sh.sel_digit = (uint32_t)b;
+        sh.sel_above = above;
+        sh.sel_count = c;
+        break;
+      }
+      above += c;
+    }
+  }
+  __syncthreads();
+}
+
+// Bitonic sort of a[0..n) (n a power of two), descending or ascending.
+template <typename T>
+__device__ void bitonic(T* a, int n, bool descending) {
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int p = i ^ j;
+        if (p > i) {
+          const bool up = ((i & k) == 0) != descending;
+          const T x = a[i], y = a[p];
+          if ((x > y) == up) {
+            a[i] = y;
+            a[p] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Selects the K best elements of src[0..n) (K <= n) under (key desc, index
+// asc).  On return sh.kept[0..K) holds their indices, in no particular order.
+__device__ void topk_select(const RowSrc& src, int n, int K, TopkShared& sh) {
+  using namespace topk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t prefix = 0, mask = 0;
+  int k_rem = K;
+  int bucket = n;
   const int shifts[3] = {21, 10, 0};
   const int widths[3] = {11, 11, 10};
-  for (int p = 0; p < 3; ++p) {
-    const int shift = shifts[p];
+  for (int p = 0; p < 3 && bucket > CAP; ++p) {
     const uint32_t dmask = (1u << widths[p]) - 1u;
-    for (int i = tid; i < NBINS; i += THREADS) sh.hist[i] = 0;
+    topk_hist(src, n, prefix, mask, shifts[p], dmask, sh);
+    topk_locate(k_rem, sh);
+    k_rem -= sh.sel_above;
+    prefix |= sh.sel_digit << shifts[p];
+    mask |= dmask << shifts[p];
+    bucket = sh.sel_count;
     __syncthreads();
-    for (int base = warp * 32; base < n; base += THREADS) {
-      const int i = base + lane;
-      uint32_t key = i < n ? keys[i] : 0u;
-      const bool valid = i < n && (key & rs.mask) == rs.prefix;
-      const uint32_t digit = (key >> shift) & dmask;
-      const uint32_t tag = valid ? digit : 0xffffffffu;
-      const uint32_t peers = __match_any_sync(0xffffffffu, tag);
-      if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[digit], (uint32_t)__popc(peers));
-    }
-    __syncthreads();
-    // locate the digit where the count of larger-or-equal keys reaches k_rem
-    constexpr int PER = NBINS / THREADS;
-    int local = 0;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) local += sh.hist[tid * PER + j];
-    int suf = local;   // inclusive suffix sum within the warp (lanes >= this lane)
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      int v = __shfl_down_sync(0xffffffffu, suf, off);
-      if (lane + off < 32) suf += v;
-    }
-    if (lane == 0) sh.warp_a[warp] = suf;
-    __syncthreads();
-    int above_warps = 0;
-    for (int w = warp + 1; w < WARPS; ++w) above_warps += sh.warp_a[w];
-    const int incl = suf + above_warps;          // keys with digit >= tid*PER
-    const int excl = incl - local;               // keys with digit >= (tid+1)*PER
-    if (excl < rs.k_rem && rs.k_rem <= incl) {
-      int above = excl;
-      for (int j = PER - 1; j >= 0; --j) {
-        const int b = tid * PER + j;
-        const int c = (int)sh.hist[b];
-        if (above + c >= rs.k_rem) {
-          sh.sel_digit = (uint32_t)b;
-          sh.sel_above = above;
-          sh.sel_count = c;
-          break;
-        }
-        above += c;
+  }
+  if (threadIdx.x == 0) {
+    sh.n_kept = 0;
+    sh.n_cand = 0;
+  }
+  __syncthreads();
+  if (bucket <= CAP) {
+    // gather: above the bucket -> kept; in the bucket -> candidates
+    for (int i = threadIdx.x; i < n; i += THREADS) {
+      const uint32_t key = src.key(i);
+      const uint32_t mk = key & mask;
+      if (mk > prefix) {
+        sh.kept[atomicAdd(&sh.n_kept, 1)] = src.index(i);
+      } else if (mk == prefix) {
+        sh.cand[atomicAdd(&sh.n_cand, 1)] = ((unsigned long long)key << 32) | (0xffffffffu - src.index(i));
       }
     }
     __syncthreads();
-    rs.k_rem -= sh.sel_above;
-    rs.prefix |= sh.sel_digit << shift;
-    rs.mask |= dmask << shift;
-    const int cnt = sh.sel_count;
+    const int nc = sh.n_cand;
+    int P = 1;
+    while (P < nc) P <<= 1;
+    for (int i = nc + threadIdx.x; i < P; i += THREADS) sh.cand[i] = 0ull;
     __syncthreads();
-    if (cnt == rs.k_rem) break;                  // the whole bucket is kept
+    bitonic(sh.cand, P, true);
+    const int nk = sh.n_kept;                 // = K - k_rem
+    for (int i = threadIdx.x; i < k_rem; i += THREADS)
+      sh.kept[nk + i] = 0xffffffffu - (uint32_t)(sh.cand[i] & 0xffffffffull);
+    __syncthreads();
+  } else {
+    // every element of the bucket has the same key: keep the k_rem lowest
+    // indices among them, in index order, plus everything above the bucket.
+    // Element order is index order for both sources.
+    const int per = (int)cdiv(cdiv(n, WARPS), 32) * 32;
+    const int beg = warp * per, end = min(n, beg + per);
+    int n_gt = 0, n_tie = 0;
+    for (int b = beg; b < end; b += 32) {
+      const int i = b + lane;
+      const uint32_t mk = i < end ? (src.key(i) & mask) : 0u;
+      n_gt += __popc(__ballot_sync(0xffffffffu, i < end && mk > prefix));
+      n_tie += __popc(__ballot_sync(0xffffffffu, i < end && mk == prefix));
+    }
+    if (lane == 0) {
+      sh.warp_a[warp] = n_gt;
+      sh.warp_b[warp] = n_tie;
+    }
+    __syncthreads();
+    int gt_run = 0, tie_run = 0;
+    for (int w = 0; w < warp; ++w) {
+      gt_run += sh.warp_a[w];
+      tie_run += sh.warp_b[w];
+    }
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int b = beg; b < end; b += 32) {
+      const int i = b + lane;
+      const uint32_t mk = i < end ? (src.key(i) & mask) : 0u;
+      const bool gt = i < end && mk > prefix, tie = i < end && mk == prefix;
+      const uint32_t bg = __ballot_sync(0xffffffffu, gt), bt = __ballot_sync(0xffffffffu, tie);
+      const int gb = gt_run + __popc(bg & lt), tb = tie_run + __popc(bt & lt);
+      if (gt) sh.kept[gb + min(tb, k_rem)] = src.index(i);
+      else if (tie && tb < k_rem) sh.kept[gb + tb] = src.index(i);
+      gt_run += __popc(bg);
+      tie_run += __popc(bt);
+    }
+    __syncthreads();
   }
-  return rs;
-}
-
-// Emits the kept elements of keys[0..n) in index order.  emit(pos, i) is
-// called once per kept element with its output position.  keep_all keeps
-// every element.
-template <typename Emit>
-__device__ void compact_in_order(const uint32_t* keys, int n, const RadixState& rs, bool keep_all,
-                                 TopkShared& sh, Emit emit) {
-  using namespace topk;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (int)cdiv(cdiv(n, WARPS), 32) * 32;
-  const int beg = warp * per, end = min(n, beg + per);
-  int n_gt = 0, n_tie = 0;
-  for (int base = beg; base < end; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < end ? keys[i] : 0u;
-    const uint32_t mk = key & rs.mask;
-    const bool gt = i < end && (keep_all || mk > rs.prefix);
-    const bool tie = i < end && !keep_all && mk == rs.prefix;
-    n_gt += __popc(__ballot_sync(0xffffffffu, gt));
-    n_tie += __popc(__ballot_sync(0xffffffffu, tie));
-  }
-  if (lane == 0) {
-    sh.warp_a[warp] = n_gt;
-    sh.warp_b[warp] = n_tie;
-  }
-  __syncthreads();
-  int gt_run = 0, tie_run = 0;
-  for (int w = 0; w < warp; ++w) {
-    gt_run += sh.warp_a[w];
-    tie_run += sh.warp_b[w];
-  }
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int base = beg; base < end; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < end ? keys[i] : 0u;
-    const uint32_t mk = key & rs.mask;
-    const bool gt = i < end && (keep_all || mk > rs.prefix);
-    const bool tie = i < end && !keep_all && mk == rs.prefix;
-    const uint32_t bg = __ballot_sync(0xffffffffu, gt);
-    const uint32_t bt = __ballot_sync(0xffffffffu, tie);
-    const int gt_before = gt_run + __popc(bg & lt_mask);
-    const int tie_before = tie_run + __popc(bt & lt_mask);
-    if (gt) emit(gt_before + min(tie_before, rs.k_rem), i);
-    else if (tie && tie_before < rs.k_rem) emit(gt_before + tie_before, i);
-    gt_run += __popc(bg);
-    tie_run += __popc(bt);
-  }
-  __syncthreads();
 }
 
 struct TopkArgs {
@@ -168,17 +235,20 @@ struct TopkArgs {
   int max_ch;           // chunks per row in the workspace layout
 };
 
-// Writes the final selection of a row: kept[0..K) ascending, then the own block.
-__device__ __forceinline__ void write_tail(int32_t* sel_row, int K, int S, int64_t bt) {
-  for (int i = K + threadIdx.x; i < S; i += blockDim.x) sel_row[i] = (i == K) ? (int32_t)bt : -1;
+// Sorts sh.kept[0..K) ascending and writes the final row: kept blocks, the
+// own block, -1 padding.
+__device__ void topk_write_final(TopkShared& sh, int K, int S, int64_t bt, int32_t* sel_row) {
+  constexpr int P = topk::KMAX;
+  for (int i = K + threadIdx.x; i < P; i += blockDim.x) sh.kept[i] = 0xffffffffu;
+  __syncthreads();
+  bitonic(sh.kept, P, false);
+  for (int i = threadIdx.x; i < S; i += blockDim.x)
+    sel_row[i] = i < K ? (int32_t)sh.kept[i] : (i == K ? (int32_t)bt : -1);
 }
 
 __global__ void __launch_bounds__(topk::THREADS) topk_chunk_kernel(Geo g, SegTable st, TopkArgs a) {
   using namespace topk;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkShared));
-
+  __shared__ TopkShared sh;
   const int item = blockIdx.x;
   const int si = find_segment(st, item);
   const int local = item - st.item0[si];
@@ -203,34 +273,35 @@ __global__ void __launch_bounds__(topk::THREADS) topk_chunk_kernel(Geo g, SegTab
   if (c >= n_ch_row) return;
   const int64_t c0 = (int64_t)c * a.chunk;
   const int n = (int)((bt - c0) < a.chunk ? (bt - c0) : a.chunk);
-  const float* row = a.scores + tok * a.ld + c0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = score_key(row[i]);
-  __syncthreads();
-  const bool keep_all = n <= K;
-  RadixState rs{0u, 0u, 0};
-  if (!keep_all) rs = radix_select(keys, n, K, sh);
+  const RowSrc src{a.scores + tok * a.ld + c0, nullptr, nullptr, c0};
+  const int kk = min(n, K);
+  if (n <= K) {
+    for (int i = threadIdx.x; i < n; i += THREADS) sh.kept[i] = (uint32_t)(c0 + i);
+    __syncthreads();
+  } else {
+    topk_select(src, n, K, sh);
+  }
   if (n_ch_row == 1) {
-    compact_in_order(keys, n, rs, keep_all, sh, [&](int p, int i) { sel_row[p] = (int32_t)(c0 + i); });
-    write_tail(sel_row, K, S, bt);
+    topk_write_final(sh, K, S, bt, sel_row);
     if (threadIdx.x == 0) a.nsel[tok] = S;
   } else {
     const int64_t base = (tok * a.max_ch + c) * (int64_t)K;
-    compact_in_order(keys, n, rs, keep_all, sh, [&](int p, int i) {
-      a.cand_key[base + p] = keys[i];
-      a.cand_idx[base + p] = (int32_t)(c0 + i);
-    });
-    if (threadIdx.x == 0) a.cand_cnt[tok * a.max_ch + c] = min(n, K);
+    for (int i = threadIdx.x; i < kk; i += THREADS) {
+      const uint32_t idx = sh.kept[i];
+      a.cand_idx[base + i] = (int32_t)idx;
+      a.cand_key[base + i] = score_key(a.scores[tok * a.ld + idx]);
+    }
+    if (threadIdx.x == 0) a.cand_cnt[tok * a.max_ch + c] = kk;
   }
 }
 
+// Merge of split rows.  Every chunk but a row's last holds at least
+// kChunkSmall > S-1 elements and so stores exactly S-1 candidates; the
+// chunk lists therefore lie back to back, in chunk (= index) order.
 __global__ void __launch_bounds__(topk::THREADS) topk_merge_kernel(Geo g, SegTable st, TopkArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
+  using namespace topk;
+  __shared__ TopkShared sh;
   const int S = g.S, K = S - 1;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkShared));
-  int32_t* idx = reinterpret_cast<int32_t*>(keys + (size_t)a.max_ch * K);
-  __shared__ int offs[64 + 1];
-
   const int item = blockIdx.x;
   const int si = find_segment(st, item);
   const int j = item - st.item0[si];
@@ -240,35 +311,15 @@ __global__ void __launch_bounds__(topk::THREADS) topk_merge_kernel(Geo g, SegTab
   if (bt + 1 <= S) return;
   const int n_ch_row = (int)cdiv(bt, a.chunk);
   if (n_ch_row <= 1) return;
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int c = 0; c < n_ch_row; ++c) {
-      offs[c] = acc;
-      acc += a.cand_cnt[tok * a.max_ch + c];
-    }
-    offs[n_ch_row] = acc;
-  }
-  __syncthreads();
-  const int n = offs[n_ch_row];
-  for (int c = 0; c < n_ch_row; ++c) {
-    const int64_t base = (tok * a.max_ch + c) * (int64_t)K;
-    const int cnt = offs[c + 1] - offs[c];
-    for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
-      keys[offs[c] + i] = a.cand_key[base + i];
-      idx[offs[c] + i] = a.cand_idx[base + i];
-    }
-  }
-  __syncthreads();
-  int32_t* sel_row = a.sel + tok * S;
-  const RadixState rs = radix_select(keys, n, K, sh);
-  compact_in_order(keys, n, rs, false, sh, [&](int p, int i) { sel_row[p] = idx[i]; });
-  write_tail(sel_row, K, S, bt);
+  const int n = (n_ch_row - 1) * K + a.cand_cnt[tok * a.max_ch + n_ch_row - 1];
+  const int64_t row_base = tok * a.max_ch * (int64_t)K;
+  const RowSrc src{nullptr, a.cand_key + row_base, a.cand_idx + row_base, 0};
+  topk_select(src, n, K, sh);
+  topk_write_final(sh, K, S, bt, a.sel + tok * S);
   if (threadIdx.x == 0) a.nsel[tok] = S;
 }
 
-inline size_t topk_chunk_smem(int chunk) { return sizeof(TopkShared) + sizeof(uint32_t) * (size_t)chunk; }
-inline size_t topk_merge_smem(int max_ch, int K) {
-  return sizeof(TopkShared) + (sizeof(uint32_t) + sizeof(int32_t)) * (size_t)max_ch * K;
-}
+inline size_t topk_chunk_smem(int) { return 0; }
+inline size_t topk_merge_smem(int, int) { return 0; }
 
 }  // namespace qsa

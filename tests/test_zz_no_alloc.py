@@ -64,8 +64,8 @@ def test_noalloc_selection_matches_workspace_entry_point_on_consecutive_calls():
 def test_noalloc_rejects_a_batch_larger_than_its_scratch():
     sh = synth.Shape()
     cfg = qsa.make_config(sh)
-    T = 4096        # 4096 rows x 8 chunks x 511 candidates x 8 bytes > 16 MiB
-    segs = qsa.make_segments([(0, T, (1 << 20) - T, 0)])
+    T = 500         # 500 decode rows at 1M context, split into 32 chunks each: ~65 MB of candidates
+    segs = qsa.make_segments([(i, 1, (1 << 20) - 1, 0) for i in range(T)])
     assert qsa.workspace_size(cfg, segs, T, qsa.QSA_OP_SELECT) > (16 << 20)
     scores = torch.zeros((1, 1), device="cuda")   # never read: rejected before any launch
     sel = torch.zeros((1, 512), dtype=torch.int32, device="cuda")
