@@ -324,13 +324,19 @@ def dist_setup():
     return ws, rank
 
 
-def max_over_ranks(v: float, ws: int) -> float:
+def max_over_ranks(v: float, ws: int, device: str = "cuda") -> float:
+    """Max of a per-rank value over all ranks (device timing: the slowest replica)."""
     if ws == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], device="cuda", dtype=torch.float64)
+    t = torch.tensor([v], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, slowest_ms: float, ws: int) -> float:
+    """Whole-job tokens/s: every rank runs its own replica, timed by the slowest."""
+    return ws * tokens_per_rank / (slowest_ms * 1e-3)
 
 
 def barrier(ws):
@@ -371,16 +377,36 @@ def measure(prep: Prepared, steps, warmup, ws, flush, peaks, clocks=None):
                 clocks=clk)
 
 
-def traffic_record(kernel: str, workload: str):
-    """dram bytes per launch recorded from an ncu capture of the current kernel build, if any."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = {
+    "attn": ["attn_tc.cuh", "sm100.cuh", "qsa_internal.cuh"],
+    "index": ["index_tc.cuh", "sm100.cuh", "qsa_internal.cuh"],
+    "select": ["topk.cuh", "qsa_internal.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(ROOT, "block_sparse_attention_22_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel: str, alg_bytes: float):
+    """DRAM bytes per launch from the committed ncu record of this kernel build
+    (profiles/traffic.txt: kernel, source hash, captured workload, dram bytes
+    read+write per launch, algorithmic bytes of that launch), scaled to this
+    launch by its algorithmic bytes.  None if no record matches the current
+    kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    try:
-        rec = json.load(open(p)).get(f"{kernel}:{workload}")
-        return rec.get("dram_bytes_per_launch") if rec else None
-    except Exception:
-        return None
+    want = kernel_source_hash(kernel)
+    for line in open(p):
+        f = line.split()
+        if len(f) == 5 and not line.startswith("#") and f[0] == kernel and f[1] == want:
+            return float(f[3]) * alg_bytes / float(f[4])
+    return None
 
 
 def run_reference(args):
@@ -434,21 +460,21 @@ def main():
     clocks = ClockSampler(torch.cuda.current_device())
     m = measure(prep, args.steps, args.warmup, ws, flush, peaks, clocks)
     tokens = wl.n_tokens
-    value = ws * tokens / (m["fused_ms"] * 1e-3)
+    value = job_throughput(tokens, m["fused_ms"], ws)
 
     work = m["work"]
     attn_ms = m["stage_ms"][3]
     achieved = work["attn"]["bytes"] / (attn_ms * 1e-3) / 1e9
     roofline = {"kernel": "sparse attention (attn stage)", "bound": "hbm", "achieved": achieved,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                "traffic": traffic_record("attn", args.workload), "peak_source": peaks["source"],
+                "traffic": traffic_record("attn", work["attn"]["bytes"]), "peak_source": peaks["source"],
                 "bytes_per_launch": work["attn"]["bytes"]}
 
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = e2e_prefill(prep, args.steps, args.warmup)
         e2e_ms = max_over_ranks(e2e_ms, ws)
-        e2e = {"value": ws * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_throughput(tokens, e2e_ms, ws), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     cpu = None

@@ -205,16 +205,19 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       const __nv_bfloat16* kg = (const __nv_bfloat16*)a.k + (u.slot * g.G + u.grp) * g.n_cap * kHeadDim;
       const __nv_bfloat16* vg = (const __nv_bfloat16*)a.v + (u.slot * g.G + u.grp) * g.n_cap * kHeadDim;
       const int32_t* selrow = a.sel + u.tok * g.S;
+      // cache rows of this warp's kept blocks 4w..4w+3 of a chunk (lanes 0..3)
+      auto rows_of = [&](int cc) -> int64_t {
+        int64_t row = -1;
+        if (lane < 4 && cc < u.nchunks) {
+          const int pos = u.blk_begin + cc * kBlk + 4 * warp + lane;
+          if (pos < u.blk_end) row = block_row(selrow[pos], 0, g);
+        }
+        return row;
+      };
       for (int c = 0; c <= u.nchunks && ok; ++c) {
         for (int kind = 0; kind < 2 && ok; ++kind) {   // K(c), then V(c-1)
           if ((kind == 0 && c == u.nchunks) || (kind == 1 && c == 0)) continue;
-          const int cc = kind == 0 ? c : c - 1;
-          // kept blocks 4w..4w+3 of the chunk: lanes 0..3 look up their cache rows
-          int64_t myrow = -1;
-          if (lane < 4) {
-            const int pos = u.blk_begin + cc * kBlk + 4 * warp + lane;
-            if (pos < u.blk_end) myrow = block_row(selrow[pos], 0, g);
-          }
+          const int64_t myrow = rows_of(kind == 0 ? c : c - 1);
           const __nv_bfloat16* base = kind == 0 ? kg : vg;
           for (int h = 0; h < 2 && ok; ++h) {
             const int64_t hs = hs_next++;
