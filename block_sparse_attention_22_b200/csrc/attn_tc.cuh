@@ -7,13 +7,19 @@
 //
 // The MMAs are swapped so that the gathered keys fill the 128-row M side:
 //   S^T[key, head]  = K_chunk[key, :] . Q[head, :]       (M=128 keys, N=16, K=256)
-//   O_c^T[d, head]  = V_chunk^T[d, key] . P^T[key, head]  (M=128 dims x2, N=16, K=128)
+//   O^T[d, head]   += V_chunk^T[d, key] . P^T[key, head]  (M=128 dims x2, N=16, K=128)
 // A chunk is 32 kept blocks (128 keys).  Kept blocks are contiguous 4-row
 // runs of the group's K/V cache; each is copied into the 128-byte-swizzled
 // K-major layout the MMA reads (8-row atoms are filled by two blocks).
-// Loads and MMAs walk one item sequence per unit, K(0), K(1), V(0), K(2),
-// V(1), ..., V(n-1); an item is two 32 KiB half-slots (128 keys x 128 dims)
-// of a 6-slot ring, reused in the order the MMAs consume them.
+//
+// Two-phase softmax per unit: every chunk's S^T goes to its own TMEM buffer
+// (16 x 16 columns), the exact per-head maximum is taken once over all of
+// them, then P = exp2(S - max) is written chunk by chunk and P.V accumulates
+// straight into a TMEM output buffer.  K slots are therefore freed as soon
+// as their MMA has run, V slots as soon as their P is written, and the load
+// stream waits on the softmax only between units.  Loads and MMAs walk one
+// item sequence, K(0..n-1) then V(0..n-1) per unit; an item is two 32 KiB
+// half-slots (128 keys x 128 dims) of a 6-slot ring.
 //
 // The gather is HBM/L2-bound and scattered (2 KiB per kept block and tensor),
 // so it is issued as 16-byte cp.async copies by eight producer warps: on
@@ -24,14 +30,12 @@
 // Roles (17 warps, persistent over work units, one CTA per SM):
 //   warps 0..7   producers: every half-slot is shared, warp w copying kept
 //                blocks 4w..4w+3 (one 512-byte row quad per instruction);
-//                a warp publishes a half-slot once its own copies of it have
-//                landed, keeping kArmDepth newer half-slots in flight.  Warp 0
-//                also loads each unit's Q tile with TMA.
+//                each lane's cp.async completion arrives on the slot's
+//                barrier, so producers run ahead as far as the ring allows.
+//                Warp 0 also loads each unit's Q tile with TMA.
 //   warp 8       TMEM owner and single-thread MMA issuer;
-//   warps 9..16  softmax and epilogue: a thread owns TMEM lane i (key i of the
+//   warps 9..16  softmax and epilogue: a thread owns TMEM lane i (key i of a
 //                chunk for S; dims i and 128+i for O) and 8 of the 16 heads.
-//                Online softmax in the exp2 domain; each chunk's P.V lands in
-//                TMEM and is added into fp32 registers with the running rescale.
 // Every mbarrier wait is bounded (sm100::mbar_wait); a timeout records an
 // error and the CTA's roles drain and return.
 #pragma once
@@ -45,7 +49,6 @@ constexpr int kProducers = 8;
 constexpr int kMmaWarp = kProducers;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = 32 * (kProducers + 1 + kSoftmaxWarps);   // 544
-constexpr int kArmDepth = 4;               // half-slots a producer keeps in flight beyond the one it publishes
 constexpr int kKeys = 128;                 // keys per chunk
 constexpr int kBlk = 32;                   // blocks per chunk
 constexpr int kSlots = 6;                  // 32 KiB K/V half-chunk slots
@@ -58,10 +61,11 @@ constexpr int kOffQ = kSlots * kSlotBytes;                 // 196608
 constexpr int kOffP = kOffQ + 2 * kQBytes;                 // 212992
 constexpr int kOffBar = kOffP + 2 * kPBytes;               // 221184
 constexpr int kSmemBytes = kOffBar + 1024 + 1024;          // + control block + alignment slack
-constexpr uint32_t kTmemCols = 128;        // S: 2 x 16 cols at 0; O: 2 x 32 cols at 32
+constexpr int kMaxChunks = kMaxBudgetBlocks / 32;   // 16 S buffers
+constexpr uint32_t kTmemCols = 512;        // S: 16 x 16 cols at 0; O: 2 x 32 cols at 256
+constexpr uint32_t kTmemO = 256;
 constexpr uint32_t kIdescS = sm100::idesc_bf16(128, kN, false, false);
 constexpr uint32_t kIdescPV = sm100::idesc_bf16(128, kN, true, false);
-static_assert(kArmDepth < kSlots, "a producer must publish a slot before it needs that slot again");
 }
 
 struct AttnTcArgs {
@@ -82,7 +86,7 @@ struct AttnTcCtl {
   uint64_t slot_full[tc_attn::kSlots];
   uint64_t slot_empty[tc_attn::kSlots];
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[2], s_free[2];
+  uint64_t s_full[tc_attn::kMaxChunks], s_free[tc_attn::kMaxChunks];
   uint64_t p_full[2], p_free[2];
   uint64_t o_full[2], o_free[2];
   uint64_t mma_done;
@@ -145,14 +149,16 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlots; ++i) {
-      mbar_init(&ctl.slot_full[i], kProducers);
+      mbar_init(&ctl.slot_full[i], kProducers * 32);   // one cp.async completion arrival per producer lane
       mbar_init(&ctl.slot_empty[i], 1);
+    }
+    for (int i = 0; i < kMaxChunks; ++i) {
+      mbar_init(&ctl.s_full[i], 1);
+      mbar_init(&ctl.s_free[i], kSoftmaxWarps);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl.q_full[i], 1);
       mbar_init(&ctl.q_empty[i], 1);
-      mbar_init(&ctl.s_full[i], 1);
-      mbar_init(&ctl.s_free[i], kSoftmaxWarps);
       mbar_init(&ctl.p_full[i], kSoftmaxWarps);
       mbar_init(&ctl.p_free[i], 1);
       mbar_init(&ctl.o_full[i], 1);
@@ -180,11 +186,6 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
     // ============================================================ producers
     int64_t hs_next = 0, uc = 0;                 // half-slots issued so far (shared numbering)
     bool ok = true;
-    auto publish = [&](int64_t hs) {             // this warp's copies of hs have landed
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.slot_full[hs % kSlots]);
-    };
     const int r = (lane >> 3) & 3, jc = lane & 7;   // row of a block and 16-byte chunk of a line
     for (int64_t w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
       if (warp_aborted(abort_flag)) break;
@@ -214,10 +215,9 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
         }
         return row;
       };
-      for (int c = 0; c <= u.nchunks && ok; ++c) {
-        for (int kind = 0; kind < 2 && ok; ++kind) {   // K(c), then V(c-1)
-          if ((kind == 0 && c == u.nchunks) || (kind == 1 && c == 0)) continue;
-          const int64_t myrow = rows_of(kind == 0 ? c : c - 1);
+      for (int kind = 0; kind < 2 && ok; ++kind) {     // all K chunks, then all V chunks
+        for (int c = 0; c < u.nchunks && ok; ++c) {
+          const int64_t myrow = rows_of(c);
           const __nv_bfloat16* base = kind == 0 ? kg : vg;
           for (int h = 0; h < 2 && ok; ++h) {
             const int64_t hs = hs_next++;
@@ -235,94 +235,87 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
               cp_async16(dst, src, nb);                       // dims 128h + 8jc .. +8
               cp_async16(dst + 16384, src + 64, nb);          // dims 128h + 64 + 8jc .. +8
             }
-            cp_async_commit();
-            if (hs >= kArmDepth) {
-              cp_async_wait<kArmDepth>();
-              publish(hs - kArmDepth);
-            }
+            cp_async_mbar_arrive(&ctl.slot_full[slot]);    // completes once these copies land
           }
         }
       }
     }
-    cp_async_wait<0>();                          // no copy of this warp outlives the CTA
-    if (ok)
-      for (int64_t hs = hs_next > kArmDepth ? hs_next - kArmDepth : 0; hs < hs_next; ++hs) publish(hs);
+    cp_async_wait_all();                         // no copy of this warp outlives the CTA
   } else if (warp == kMmaWarp) {
     // ============================================================ MMA issuer
     // Whole warp in the loop; lane 0 issues the MMAs and commits.
-    int64_t gc = 0, uc = 0, it = 0;
+    int64_t gp = 0, uc = 0, it = 0;
+    uint32_t sbits = 0;                          // parity of each S buffer's next use
     const uint32_t smem_base = smem_u32(smem);
     bool ok = true;
     for (int64_t w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
       if (warp_aborted(abort_flag)) break;
       const TcUnit u = tc_unit(g, st, a, w);
       if (u.nchunks == 0) continue;
-      const int qb = (int)(uc & 1);
+      const int qb = (int)(uc & 1), ob = (int)(uc & 1);
       if (!(ok = warp_wait(&ctl.q_full[qb], (uint32_t)((uc >> 1) & 1), abort_flag))) break;
-      ++uc;
       const uint32_t q_addr = smem_base + kOffQ + qb * kQBytes;
-      for (int c = 0; c <= u.nchunks && ok; ++c) {
-        if (c < u.nchunks) {
-          const int64_t gs = gc + c;
-          const int sb = (int)(gs & 1);
-          if (!(ok = warp_wait(&ctl.s_free[sb], (uint32_t)(((gs >> 1) & 1) ^ 1), abort_flag))) break;
-          for (int half = 0; half < 2 && ok; ++half) {
-            const int64_t i = 2 * it + half;
-            const int slot = (int)(i % kSlots);
-            if (!(ok = warp_wait(&ctl.slot_full[slot], (uint32_t)((i / kSlots) & 1), abort_flag))) break;
-            tc_fence_after();
-            if (lane == 0) {
-              const uint32_t k_addr = smem_base + slot * kSlotBytes;
-              for (int kk = 0; kk < 8; ++kk) {          // 8 k-steps of 16 dims per half
-                const int slab = kk >> 2, sub = kk & 3;
-                const uint64_t da = desc_sw128(k_addr + slab * 16384 + sub * 32, 16, 1024);
-                const uint64_t db = desc_sw128(q_addr + (half * 2 + slab) * 2048 + sub * 32, 16, 1024);
-                umma_bf16(tmem + sb * kN, da, db, kIdescS, (half | kk) != 0);
-              }
-              umma_commit(&ctl.slot_empty[slot]);
-            }
-            __syncwarp();
-          }
-          if (!ok) break;
-          ++it;
+      // phase 1: S^T of every chunk into its own buffer
+      for (int c = 0; c < u.nchunks && ok; ++c) {
+        if (!(ok = warp_wait(&ctl.s_free[c], ((sbits >> c) & 1u) ^ 1u, abort_flag))) break;
+        for (int half = 0; half < 2 && ok; ++half) {
+          const int64_t i = 2 * it + half;
+          const int slot = (int)(i % kSlots);
+          if (!(ok = warp_wait(&ctl.slot_full[slot], (uint32_t)((i / kSlots) & 1), abort_flag))) break;
+          tc_fence_after();
           if (lane == 0) {
-            umma_commit(&ctl.s_full[sb]);
-            if (c == u.nchunks - 1) umma_commit(&ctl.q_empty[qb]);
+            fence_proxy_async_smem();
+            const uint32_t k_addr = smem_base + slot * kSlotBytes;
+            for (int kk = 0; kk < 8; ++kk) {            // 8 k-steps of 16 dims per half
+              const int slab = kk >> 2, sub = kk & 3;
+              const uint64_t da = desc_sw128(k_addr + slab * 16384 + sub * 32, 16, 1024);
+              const uint64_t db = desc_sw128(q_addr + (half * 2 + slab) * 2048 + sub * 32, 16, 1024);
+              umma_bf16(tmem + c * kN, da, db, kIdescS, (half | kk) != 0);
+            }
+            umma_commit(&ctl.slot_empty[slot]);
           }
           __syncwarp();
         }
-        if (c >= 1) {
-          const int64_t gp = gc + c - 1;
-          const int pb = (int)(gp & 1);
-          if (!(ok = warp_wait(&ctl.p_full[pb], (uint32_t)((gp >> 1) & 1), abort_flag))) break;
-          if (!(ok = warp_wait(&ctl.o_free[pb], (uint32_t)(((gp >> 1) & 1) ^ 1), abort_flag))) break;
-          const uint32_t p_addr = smem_base + kOffP + pb * kPBytes;
-          for (int half = 0; half < 2 && ok; ++half) {
-            const int64_t i = 2 * it + half;
-            const int slot = (int)(i % kSlots);
-            if (!(ok = warp_wait(&ctl.slot_full[slot], (uint32_t)((i / kSlots) & 1), abort_flag))) break;
-            tc_fence_after();
-            if (lane == 0) {
-              const uint32_t v_addr = smem_base + slot * kSlotBytes;
-              for (int kk = 0; kk < 8; ++kk) {          // 8 k-steps of 16 keys
-                const uint64_t da = desc_sw128(v_addr + kk * 2048, 16384, 1024);
-                const uint64_t db = desc_sw128(p_addr + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
-                umma_bf16(tmem + 32 + pb * 32 + half * kN, da, db, kIdescPV, kk != 0);
-              }
-              umma_commit(&ctl.slot_empty[slot]);
-            }
-            __syncwarp();
-          }
-          if (!ok) break;
-          ++it;
-          if (lane == 0) {
-            umma_commit(&ctl.o_full[pb]);
-            umma_commit(&ctl.p_free[pb]);
-          }
-          __syncwarp();
-        }
+        if (!ok) break;
+        ++it;
+        sbits ^= 1u << c;
+        if (lane == 0) umma_commit(&ctl.s_full[c]);
+        __syncwarp();
       }
-      gc += u.nchunks;
+      if (!ok) break;
+      if (lane == 0) umma_commit(&ctl.q_empty[qb]);
+      // phase 2: O^T += V^T P^T over the chunks, straight into the unit's O buffer
+      if (!(ok = warp_wait(&ctl.o_free[ob], (uint32_t)(((uc >> 1) & 1) ^ 1), abort_flag))) break;
+      for (int c = 0; c < u.nchunks && ok; ++c, ++gp) {
+        const int pb = (int)(gp & 1);
+        if (!(ok = warp_wait(&ctl.p_full[pb], (uint32_t)((gp >> 1) & 1), abort_flag))) break;
+        const uint32_t p_addr = smem_base + kOffP + pb * kPBytes;
+        for (int half = 0; half < 2 && ok; ++half) {
+          const int64_t i = 2 * it + half;
+          const int slot = (int)(i % kSlots);
+          if (!(ok = warp_wait(&ctl.slot_full[slot], (uint32_t)((i / kSlots) & 1), abort_flag))) break;
+          tc_fence_after();
+          if (lane == 0) {
+            fence_proxy_async_smem();
+            const uint32_t v_addr = smem_base + slot * kSlotBytes;
+            for (int kk = 0; kk < 8; ++kk) {            // 8 k-steps of 16 keys
+              const uint64_t da = desc_sw128(v_addr + kk * 2048, 16384, 1024);
+              const uint64_t db = desc_sw128(p_addr + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+              umma_bf16(tmem + kTmemO + ob * 32 + half * kN, da, db, kIdescPV, (c | kk) != 0);
+            }
+            umma_commit(&ctl.slot_empty[slot]);
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        ++it;
+        if (lane == 0) umma_commit(&ctl.p_free[pb]);
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(&ctl.o_full[ob]);
+      __syncwarp();
+      ++uc;
     }
     // every MMA issued above has finished before TMEM is freed
     if (lane == 0) {
@@ -336,116 +329,90 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
     const int sw = warp - kMmaWarp - 1;                 // 0..7
     const int quad = warp & 3;                          // TMEM lane quadrant this warp may access
     const int h0 = (sw >> 2) * kHH;                     // first of this thread's 8 heads
-    const int li = quad * 32 + lane;                    // TMEM lane: key of the chunk / dim
+    const int li = quad * 32 + lane;                    // TMEM lane: key of a chunk / dim
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t smem_base = smem_u32(smem);
     const float scale_log2 = g.scale * 1.4426950408889634f;
     const int nthr = 32 * kSoftmaxWarps;
-    int64_t gc = 0;
+    int64_t gp = 0, uc = 0;
+    uint32_t sbits = 0;
     // No early exit in this role: its warps meet at named barriers, so they
     // must run the same iterations.  After an abort every wait returns at
     // once and the loop runs through without blocking.
     for (int64_t w = blockIdx.x; w < n_units; w += gridDim.x) {
       const TcUnit u = tc_unit(g, st, a, w);
-      float m[kHH], lp[kHH], al[kHH], oacc[2 * kHH];
+      const int32_t* selrow = a.sel + u.tok * g.S;
+      float m[kHH], l[kHH];
 #pragma unroll
       for (int h = 0; h < kHH; ++h) {
         m[h] = -INFINITY;
-        lp[h] = 0.f;
-        al[h] = 1.f;
-        oacc[h] = 0.f;
-        oacc[kHH + h] = 0.f;
+        l[h] = 0.f;
       }
-      const int32_t* selrow = a.sel + u.tok * g.S;
-      for (int c = 0; c <= u.nchunks; ++c) {
-        float alpha[kHH];
-        if (c < u.nchunks) {
-          const int64_t gs = gc + c;
-          const int sb = (int)(gs & 1);
-          // key validity (kept block, causal within the own block): fetched before the wait
-          const int pos = u.blk_begin + c * kBlk + (li >> 2);
-          bool valid = false;
-          if (pos < u.blk_end) {
-            const int64_t row = block_row(selrow[pos], li & 3, g);
-            valid = row >= 0 && row <= u.t;
-          }
-          mbar_wait(&ctl.s_full[sb], (uint32_t)((gs >> 1) & 1), abort_flag);
-          tc_fence_after();
-          float s[kHH];
-          tmem_ld8(lane_addr + sb * kN + h0, s);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl.s_free[sb]);
-          float mx[kHH];
-#pragma unroll
-          for (int h = 0; h < kHH; ++h) {
-            s[h] = valid ? s[h] * scale_log2 : -INFINITY;
-            mx[h] = s[h];
-          }
-#pragma unroll
-          for (int off = 16; off; off >>= 1)
-#pragma unroll
-            for (int h = 0; h < kHH; ++h) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], off));
-          if (lane == 0)
-#pragma unroll
-            for (int h = 0; h < kHH; ++h) ctl.red[gs & 1][quad][h0 + h] = mx[h];
-          named_bar_sync(1, nthr);
-          const int pb = sb;
-          mbar_wait(&ctl.p_free[pb], (uint32_t)(((gs >> 1) & 1) ^ 1), abort_flag);
-          const uint32_t p_addr = smem_base + kOffP + pb * kPBytes;
-          const int slab = li >> 6, kin = li & 63;
-          const uint32_t p_lane = p_addr + slab * 2048 + (kin & 7) * 2;
-#pragma unroll
-          for (int h = 0; h < kHH; ++h) {
-            const int hh = h0 + h;
-            const float cm = fmaxf(fmaxf(ctl.red[gs & 1][0][hh], ctl.red[gs & 1][1][hh]),
-                                   fmaxf(ctl.red[gs & 1][2][hh], ctl.red[gs & 1][3][hh]));
-            const float mn = fmaxf(m[h], cm);
-            alpha[h] = (mn == -INFINITY) ? 1.f : exp2f(m[h] - mn);
-            const float p = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - mn);
-            m[h] = mn;
-            lp[h] = lp[h] * alpha[h] + p;          // fp32 denominator (exact log-sum-exp)
-            const uint32_t addr = p_lane + (hh >> 3) * 1024 + (hh & 7) * 128 + (((kin >> 3) ^ (hh & 7)) << 4);
-            st_shared_u16(addr, __bfloat16_as_ushort(__float2bfloat16_rn(p)));
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl.p_full[pb]);
-        }
-        if (c >= 1) {
-          const int64_t gp = gc + c - 1;
-          const int ob = (int)(gp & 1);
-          mbar_wait(&ctl.o_full[ob], (uint32_t)((gp >> 1) & 1), abort_flag);
-          tc_fence_after();
-          float o0[kHH], o1[kHH];
-          tmem_ld8(lane_addr + 32 + ob * 32 + h0, o0);
-          tmem_ld8(lane_addr + 32 + ob * 32 + kN + h0, o1);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl.o_free[ob]);
-#pragma unroll
-          for (int h = 0; h < kHH; ++h) {
-            oacc[h] = oacc[h] * al[h] + o0[h];
-            oacc[kHH + h] = oacc[kHH + h] * al[h] + o1[h];
-          }
-        }
-        if (c < u.nchunks) {
-#pragma unroll
-          for (int h = 0; h < kHH; ++h) al[h] = alpha[h];
+      // key validity of this thread's key in each chunk (kept block, causal within the own block)
+      uint32_t vbits = 0;
+      for (int c = 0; c < u.nchunks; ++c) {
+        const int pos = u.blk_begin + c * kBlk + (li >> 2);
+        if (pos < u.blk_end) {
+          const int64_t row = block_row(selrow[pos], li & 3, g);
+          if (row >= 0 && row <= u.t) vbits |= 1u << c;
         }
       }
-      gc += u.nchunks;
-      // ---- epilogue: denominators, normalisation, stores
-      float l[kHH];
+      // phase 1: exact per-head maximum over every chunk
+      for (int c = 0; c < u.nchunks; ++c) {
+        mbar_wait(&ctl.s_full[c], (sbits >> c) & 1u, abort_flag);
+        tc_fence_after();
+        float s[kHH];
+        tmem_ld8(lane_addr + c * kN + h0, s);
+        tmem_wait_ld();
+        if ((vbits >> c) & 1u) {
 #pragma unroll
-      for (int h = 0; h < kHH; ++h) l[h] = lp[h];
+          for (int h = 0; h < kHH; ++h) m[h] = fmaxf(m[h], s[h] * scale_log2);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off; off >>= 1)
+#pragma unroll
+        for (int h = 0; h < kHH; ++h) m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], off));
+      if (lane == 0)
+#pragma unroll
+        for (int h = 0; h < kHH; ++h) ctl.red[0][quad][h0 + h] = m[h];
+      named_bar_sync(1, nthr);
+#pragma unroll
+      for (int h = 0; h < kHH; ++h)
+        m[h] = fmaxf(fmaxf(ctl.red[0][0][h0 + h], ctl.red[0][1][h0 + h]),
+                     fmaxf(ctl.red[0][2][h0 + h], ctl.red[0][3][h0 + h]));
+      // phase 2: P = exp2(S - max) per chunk, written as the B operand of P.V
+      const int slab = li >> 6, kin = li & 63;
+      for (int c = 0; c < u.nchunks; ++c, ++gp) {
+        float s[kHH];
+        tmem_ld8(lane_addr + c * kN + h0, s);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.s_free[c]);
+        const bool valid = (vbits >> c) & 1u;
+        const int pb = (int)(gp & 1);
+        mbar_wait(&ctl.p_free[pb], (uint32_t)(((gp >> 1) & 1) ^ 1), abort_flag);
+        const uint32_t p_lane = smem_base + kOffP + pb * kPBytes + slab * 2048 + (kin & 7) * 2;
+#pragma unroll
+        for (int h = 0; h < kHH; ++h) {
+          const int hh = h0 + h;
+          const float p = (valid && m[h] != -INFINITY) ? exp2f(s[h] * scale_log2 - m[h]) : 0.f;
+          l[h] += p;
+          const uint32_t addr = p_lane + (hh >> 3) * 1024 + (hh & 7) * 128 + (((kin >> 3) ^ (hh & 7)) << 4);
+          st_shared_u16(addr, __bfloat16_as_ushort(__float2bfloat16_rn(p)));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.p_full[pb]);
+      }
+      sbits ^= (u.nchunks >= 32 ? 0xffffffffu : ((1u << u.nchunks) - 1u));
+      // denominators over all keys
 #pragma unroll
       for (int off = 16; off; off >>= 1)
 #pragma unroll
         for (int h = 0; h < kHH; ++h) l[h] += __shfl_xor_sync(0xffffffffu, l[h], off);
-      named_bar_sync(1, nthr);                // red[] of the last chunk fully read
+      named_bar_sync(1, nthr);                // every thread has read red[0] (the maxima)
       if (lane == 0)
 #pragma unroll
         for (int h = 0; h < kHH; ++h) ctl.red[0][quad][h0 + h] = l[h];
@@ -454,6 +421,25 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       for (int h = 0; h < kHH; ++h)
         l[h] = ctl.red[0][0][h0 + h] + ctl.red[0][1][h0 + h] + ctl.red[0][2][h0 + h] + ctl.red[0][3][h0 + h];
       named_bar_sync(1, nthr);                // before red[] is reused
+      // output: O^T from TMEM, normalised
+      float o0[kHH], o1[kHH];
+#pragma unroll
+      for (int h = 0; h < kHH; ++h) {
+        o0[h] = 0.f;
+        o1[h] = 0.f;
+      }
+      if (u.nchunks > 0) {
+        const int ob = (int)(uc & 1);
+        mbar_wait(&ctl.o_full[ob], (uint32_t)((uc >> 1) & 1), abort_flag);
+        tc_fence_after();
+        tmem_ld8(lane_addr + kTmemO + ob * 32 + h0, o0);
+        tmem_ld8(lane_addr + kTmemO + ob * 32 + kN + h0, o1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.o_free[ob]);
+        ++uc;
+      }
       const int64_t unit = u.tok * g.G + u.grp;
       if (a.n_split == 1) {
         __nv_bfloat16* og = (__nv_bfloat16*)a.o + (u.tok * g.H + (int64_t)u.grp * g.hpg) * kHeadDim;
@@ -461,8 +447,8 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
         for (int h = 0; h < kHH; ++h) {
           if (h0 + h < g.hpg) {
             const float inv = 1.f / l[h];
-            og[(h0 + h) * kHeadDim + li] = __float2bfloat16_rn(oacc[h] * inv);
-            og[(h0 + h) * kHeadDim + 128 + li] = __float2bfloat16_rn(oacc[kHH + h] * inv);
+            og[(h0 + h) * kHeadDim + li] = __float2bfloat16_rn(o0[h] * inv);
+            og[(h0 + h) * kHeadDim + 128 + li] = __float2bfloat16_rn(o1[h] * inv);
           }
         }
         if (a.lse && li == 0) {
@@ -476,8 +462,8 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
 #pragma unroll
         for (int h = 0; h < kHH; ++h) {
           if (h0 + h < g.hpg) {
-            a.part_o[(base + h0 + h) * kHeadDim + li] = oacc[h];
-            a.part_o[(base + h0 + h) * kHeadDim + 128 + li] = oacc[kHH + h];
+            a.part_o[(base + h0 + h) * kHeadDim + li] = o0[h];
+            a.part_o[(base + h0 + h) * kHeadDim + 128 + li] = o1[h];
           }
         }
         if (li == 0) {
