@@ -42,7 +42,8 @@ struct IndexTcCfg {
   static constexpr int kBBytes = N * 128 * 2;              // rotated queries, 2 slabs
   static constexpr int kOffB = tc_index::kStages * kABytes;
   static constexpr int kOffW = kOffB + kBBytes;            // w[NQ][4] fp32
-  static constexpr int kOffCS = kOffW + ((NQ * 16 + 1023) / 1024) * 1024;   // cos/sin[NQ][half][2]
+  static constexpr int kOffLim = kOffW + NQ * 16;          // floor(t/r) per query (int64)
+  static constexpr int kOffCS = kOffW + ((NQ * 24 + 1023) / 1024) * 1024;   // cos/sin[NQ][half][2]
   static constexpr int kOffBar = kOffCS + ((NQ * tc_index::kMaxRopeHalf * 8 + 1023) / 1024) * 1024;
   static constexpr int kSmemBytes = kOffBar + 1024 + 1024;
   static constexpr uint32_t kTmemCols = 2 * N < 32 ? 32 : 2 * N;
@@ -231,6 +232,8 @@ __global__ void __launch_bounds__(tc_index::kThreads, 1)
     }
     for (int i = et; i < NQ * 4; i += 32 * kEpiWarps)
       ws[i] = (i >> 2) < it.nq ? a.w[it.tok0 * 4 + i] : 0.f;
+    int64_t* lim = reinterpret_cast<int64_t*>(smem + C::kOffLim);   // blocks each query scores
+    for (int q = et; q < NQ; q += 32 * kEpiWarps) lim[q] = q < it.nq ? (it.t_first + q) / g.r : 0;
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&ctl.b_ready);
@@ -246,29 +249,26 @@ __global__ void __launch_bounds__(tc_index::kThreads, 1)
       mbar_wait(&ctl.acc_full[ab], (uint32_t)((i >> 1) & 1), abort_flag);
       tc_fence_after();
       const int64_t b = (int64_t)(it.tile0 + i) * kTileRows + quad * 32 + lane;
-      constexpr int kChunk = kCols >= 16 ? 16 : 8;  // TMEM columns per load (4 or 2 queries)
+      constexpr int kChunk = kCols >= 32 ? 32 : (kCols >= 16 ? 16 : 8);   // TMEM columns per load
       for (int c0 = 0; c0 < kCols; c0 += kChunk) {
-        float v[16];
-        if constexpr (kChunk == 16) {
-          tmem_ld16(lane_addr + ab * C::N + colhalf * kCols + c0, v);
+        float v[32];
+        if constexpr (kChunk == 32) {
+          tmem_ld16(lane_addr + ab * C::N + colhalf * kCols + c0, *reinterpret_cast<float(*)[16]>(v));
+          tmem_ld16(lane_addr + ab * C::N + colhalf * kCols + c0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+        } else if constexpr (kChunk == 16) {
+          tmem_ld16(lane_addr + ab * C::N + colhalf * kCols + c0, *reinterpret_cast<float(*)[16]>(v));
         } else {
-          float v8[8];
-          tmem_ld8(lane_addr + ab * C::N + colhalf * kCols + c0, v8);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) v[k] = v8[k];
+          tmem_ld8(lane_addr + ab * C::N + colhalf * kCols + c0, *reinterpret_cast<float(*)[8]>(v));
         }
         tmem_wait_ld();
 #pragma unroll
         for (int qq = 0; qq < kChunk / 4; ++qq) {
           const int q = (colhalf * kCols + c0) / 4 + qq;
-          if (q < it.nq) {
-            const int64_t t = it.t_first + q;
-            if (b < t / g.r) {
-              float sc = 0.f;
+          if (q < it.nq && b < lim[q]) {
+            float sc = 0.f;
 #pragma unroll
-              for (int h = 0; h < 4; ++h) sc += ws[q * 4 + h] * fmaxf(v[qq * 4 + h], 0.f);
-              a.scores[(it.tok0 + q) * a.ld + b] = sc;
-            }
+            for (int h = 0; h < 4; ++h) sc = fmaf(ws[q * 4 + h], fmaxf(v[qq * 4 + h], 0.f), sc);
+            a.scores[(it.tok0 + q) * a.ld + b] = sc;
           }
         }
       }

@@ -7,17 +7,20 @@
 // the total order (score descending, block index ascending), -0 == +0.
 //
 // Algorithm (one CTA per row, or per row chunk for long rows; the row is
-// streamed from global memory, so several CTAs fit on an SM):
-//   1. radix narrowing: a histogram of the next 11/11/10 key bits over the
-//      elements still in the threshold bucket (warp-aggregated shared
-//      atomics) locates the bucket holding the K-th largest key; repeated
-//      until that bucket fits the shared candidate buffer;
-//   2. gather: elements above the bucket are kept outright, elements in it
-//      become candidates, ordered by the 64-bit composite (key, ~index) so
-//      that ties go to the lower index;
-//   3. the best candidates complete the K, found by a bitonic sort of the
-//      composite keys; the kept block indices are finally sorted ascending.
-// If the bucket is still larger than the buffer after all 32 bits (many
+// streamed from global memory, so several CTAs fit on an SM).  Elements are
+// ranked by the 64-bit composite (key << 32) | ~index, which orders them by
+// score and then by lower block index, so every composite is distinct:
+//   1. radix narrowing over the row: histograms of the next 11/11/10 key bits
+//      over the elements still in the threshold bucket (warp-aggregated
+//      shared atomics) locate the bucket holding the K-th largest element,
+//      until that bucket fits a 4096-entry shared buffer;
+//   2. gather: elements above the bucket are kept outright, the bucket's
+//      elements are copied to the buffer as composites;
+//   3. narrowing continues on the composites in shared memory (remaining key
+//      bits, then index bits) until the bucket holds exactly the elements
+//      still needed; every buffered composite at or above it is kept;
+//   4. the kept block indices are sorted ascending (bitonic, 512 entries).
+// If a bucket is still larger than the buffer after all 32 key bits (many
 // exactly equal keys), the tied elements are taken in index order by an
 // ordered ballot compaction instead.  Long rows are split into chunks whose
 // local top K (exact under the same order) are merged by a second pass of
@@ -38,7 +41,7 @@ constexpr int kChunkSmall = 8192;
 
 struct TopkShared {
   uint32_t hist[topk::NBINS];
-  unsigned long long cand[topk::CAP];      // (key << 32) | ~index
+  unsigned long long cand[topk::CAP];      // composites (key << 32) | ~index
   uint32_t kept[topk::KMAX];               // indices kept outright / final list
   int warp_a[topk::WARPS];
   int warp_b[topk::WARPS];
@@ -137,11 +140,108 @@ __device__ void bitonic(T* a, int n, bool descending) {
   }
 }
 
+// Finishes a selection whose candidates sh.cand[0..nc) are the composites of
+// every element in the current bucket (key & mask == prefix) and k_rem of
+// them are still needed: narrows on the remaining key bits, then on the
+// index bits, until the bucket holds exactly the elements still needed, and
+// appends every candidate at or above it to sh.kept.
+__device__ void refine_and_keep(int nc, int k_rem, uint32_t prefix, uint32_t mask, TopkShared& sh) {
+  using namespace topk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long cprefix = (unsigned long long)prefix << 32, cmask = (unsigned long long)mask << 32;
+  const int cshifts[6] = {53, 42, 32, 21, 10, 0};
+  const int cwidths[6] = {11, 11, 10, 11, 11, 10};
+  int q0 = 0;                               // first composite digit not yet resolved
+  while (q0 < 3 && ((cmask >> cshifts[q0]) & 1ull)) ++q0;
+  int count = nc;
+  for (int q = q0; q < 6 && count != k_rem; ++q) {
+    const unsigned long long dm = (1ull << cwidths[q]) - 1ull;
+    for (int i = threadIdx.x; i < NBINS; i += THREADS) sh.hist[i] = 0;
+    __syncthreads();
+    for (int b = warp * 32; b < nc; b += THREADS) {
+      const int i = b + lane;
+      const unsigned long long c = i < nc ? sh.cand[i] : 0ull;
+      const bool valid = i < nc && (c & cmask) == cprefix;
+      const uint32_t digit = (uint32_t)((c >> cshifts[q]) & dm);
+      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? digit : 0xffffffffu);
+      if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[digit], (uint32_t)__popc(peers));
+    }
+    __syncthreads();
+    topk_locate(k_rem, sh);
+    k_rem -= sh.sel_above;
+    cprefix |= (unsigned long long)sh.sel_digit << cshifts[q];
+    cmask |= dm << cshifts[q];
+    count = sh.sel_count;
+    __syncthreads();
+  }
+  for (int i = threadIdx.x; i < nc; i += THREADS) {
+    const unsigned long long c = sh.cand[i];
+    if ((c & cmask) >= cprefix) sh.kept[atomicAdd(&sh.n_kept, 1)] = 0xffffffffu - (uint32_t)(c & 0xffffffffull);
+  }
+  __syncthreads();
+}
+
+// Fast path for rows longer than the candidate buffer: a strided sample of
+// the keys gives a threshold expected to admit about kSampleTarget elements;
+// one pass collects every element at or above it.  If between K and CAP
+// elements qualify, the K best are among them (at least K elements are at or
+// above the threshold, so the K-th largest is too) and are found exactly on
+// the buffered composites; otherwise returns false and nothing is kept.
+constexpr int kSamples = 2048;
+constexpr int kSampleTarget = 2048;
+
+__device__ bool select_by_sample(const RowSrc& src, int n, int K, TopkShared& sh) {
+  using namespace topk;
+  uint32_t* samp = reinterpret_cast<uint32_t*>(sh.cand);      // reused before the candidates land
+  const int m = min(kSamples, n / 4);
+  for (int s = threadIdx.x; s < m; s += THREADS) samp[s] = src.key((int)((int64_t)s * n / m));
+  __syncthreads();
+  const int target = max(4 * K, kSampleTarget);
+  const int rank = max(1, (int)((int64_t)m * target / n));
+  // exact rank-th largest sample key
+  const RowSrc ssrc{nullptr, samp, nullptr, 0};
+  uint32_t prefix = 0, mask = 0;
+  int k_rem = rank;
+  const int shifts[3] = {21, 10, 0};
+  const int widths[3] = {11, 11, 10};
+  for (int p = 0; p < 3; ++p) {
+    const uint32_t dmask = (1u << widths[p]) - 1u;
+    topk_hist(ssrc, m, prefix, mask, shifts[p], dmask, sh);
+    topk_locate(k_rem, sh);
+    k_rem -= sh.sel_above;
+    prefix |= sh.sel_digit << shifts[p];
+    mask |= dmask << shifts[p];
+    __syncthreads();
+  }
+  const uint32_t tau = prefix;
+  if (threadIdx.x == 0) {
+    sh.n_kept = 0;
+    sh.n_cand = 0;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += THREADS) {
+    const uint32_t key = src.key(i);
+    if (key >= tau) {
+      const int slot = atomicAdd(&sh.n_cand, 1);
+      if (slot < CAP) sh.cand[slot] = ((unsigned long long)key << 32) | (0xffffffffu - src.index(i));
+    }
+  }
+  __syncthreads();
+  const int nc = sh.n_cand;
+  if (nc < K || nc > CAP) {
+    __syncthreads();
+    return false;
+  }
+  refine_and_keep(nc, K, 0u, 0u, sh);
+  return true;
+}
+
 // Selects the K best elements of src[0..n) (K <= n) under (key desc, index
 // asc).  On return sh.kept[0..K) holds their indices, in no particular order.
 __device__ void topk_select(const RowSrc& src, int n, int K, TopkShared& sh) {
   using namespace topk;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (n > CAP && select_by_sample(src, n, K, sh)) return;
   uint32_t prefix = 0, mask = 0;
   int k_rem = K;
   int bucket = n;
@@ -163,7 +263,7 @@ __device__ void topk_select(const RowSrc& src, int n, int K, TopkShared& sh) {
   }
   __syncthreads();
   if (bucket <= CAP) {
-    // gather: above the bucket -> kept; in the bucket -> candidates
+    // gather: above the bucket -> kept; in the bucket -> composite candidates
     for (int i = threadIdx.x; i < n; i += THREADS) {
       const uint32_t key = src.key(i);
       const uint32_t mk = key & mask;
@@ -174,16 +274,7 @@ __device__ void topk_select(const RowSrc& src, int n, int K, TopkShared& sh) {
       }
     }
     __syncthreads();
-    const int nc = sh.n_cand;
-    int P = 1;
-    while (P < nc) P <<= 1;
-    for (int i = nc + threadIdx.x; i < P; i += THREADS) sh.cand[i] = 0ull;
-    __syncthreads();
-    bitonic(sh.cand, P, true);
-    const int nk = sh.n_kept;                 // = K - k_rem
-    for (int i = threadIdx.x; i < k_rem; i += THREADS)
-      sh.kept[nk + i] = 0xffffffffu - (uint32_t)(sh.cand[i] & 0xffffffffull);
-    __syncthreads();
+    refine_and_keep(sh.n_cand, k_rem, prefix, mask, sh);
   } else {
     // every element of the bucket has the same key: keep the k_rem lowest
     // indices among them, in index order, plus everything above the bucket.
