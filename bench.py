@@ -216,41 +216,73 @@ def timed(prep: Prepared, steps: int, warmup: int, flush: torch.Tensor, staged: 
 
 
 def e2e_prefill(prep: Prepared, steps: int, warmup: int):
-    """qsa_forward with the step's inputs copied from pinned host memory and the
-    output read back, all inside the timed region."""
+    """qsa_forward with every step's inputs copied from pinned host memory and its
+    output read back, all inside the timed region.  Steps are pipelined over
+    three streams (copy-in, compute, copy-out) with two device buffer sets, so
+    step i's compute overlaps step i+1's upload and step i-1's download."""
     x = prep.x
     slot = prep.wl.segments[0].slot
     fill = prep.wl.fill[slot]
-    host = {"q": x["q"], "q_idx": x["q_idx"], "w": x["w"], "k_idx": x["k_idx"][slot, :fill],
-            "k": x["k"][slot, :, :fill], "v": x["v"][slot, :, :fill]}
-    host = {k: v.cpu().pin_memory() for k, v in host.items()}
+    names = ["q", "q_idx", "w", "k_idx", "k", "v"]
+    views = [lambda d: d["q"], lambda d: d["q_idx"], lambda d: d["w"], lambda d: d["k_idx"][slot, :fill],
+             lambda d: d["k"][slot, :, :fill], lambda d: d["v"][slot, :, :fill]]
+    host = {n: f(x).cpu().pin_memory() for n, f in zip(names, views)}
     o_host = torch.empty(prep.o.shape, dtype=prep.o.dtype).pin_memory()
     lse_host = torch.empty(prep.lse.shape, dtype=prep.lse.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * lse_host.element_size()
-    st = torch.cuda.current_stream()
+    # two device buffer sets (inputs, caches, outputs); the score workspace is shared
+    sets = []
+    for b in range(2):
+        d = x if b == 0 else {k: torch.empty_like(v) for k, v in x.items()}
+        khat = prep.khat if b == 0 else torch.empty_like(prep.khat)
+        o = prep.o if b == 0 else torch.empty_like(prep.o)
+        lse = prep.lse if b == 0 else torch.empty_like(prep.lse)
+        sets.append(dict(d=d, khat=khat, o=o, lse=lse, cache=qsa.make_cache(d["k_idx"], khat, d["k"], d["v"])))
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_done, cmp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    used = [False, False]
 
-    def one():
-        x["q"].copy_(host["q"], non_blocking=True)
-        x["q_idx"].copy_(host["q_idx"], non_blocking=True)
-        x["w"].copy_(host["w"], non_blocking=True)
-        x["k_idx"][slot, :fill].copy_(host["k_idx"], non_blocking=True)
-        x["k"][slot, :, :fill].copy_(host["k"], non_blocking=True)
-        x["v"][slot, :, :fill].copy_(host["v"], non_blocking=True)
-        prep.forward()
-        o_host.copy_(prep.o, non_blocking=True)
-        lse_host.copy_(prep.lse, non_blocking=True)
+    def step(i):
+        b = i & 1
+        st_ = sets[b]
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(cmp_done[b])          # compute of step i-2 is done with this set
+            for n, f in zip(names, views):
+                f(st_["d"]).copy_(host[n], non_blocking=True)
+            in_done[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(in_done[b])
+            if used[b]:
+                s_cmp.wait_event(out_done[b])         # download of step i-2 has read this set's output
+            d = st_["d"]
+            qsa.qsa_forward(prep.cfg, st_["cache"], prep.segs, prep.T, d["q"], d["q_idx"], d["w"], st_["o"],
+                            st_["lse"], prep.sel, prep.nsel, prep.ws, stream=s_cmp)
+            cmp_done[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(cmp_done[b])
+            o_host.copy_(st_["o"], non_blocking=True)
+            lse_host.copy_(st_["lse"], non_blocking=True)
+            out_done[b].record(s_out)
+        used[b] = True
 
-    for _ in range(warmup):
-        one()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(steps):
-        one()
-    e1.record(st)
+    e0.record(s_in)
+    s_cmp.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(warmup, warmup + steps):
+        step(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_cmp)
+    e1.record(s_out)
     torch.cuda.synchronize()
+    del sets
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
