@@ -7,19 +7,29 @@
 //   ACC[b, (q,h)] = k^[b, :] . q~[q, h, :]      M = 128 blocks, N = 4*NQ, K = idx_dim
 // followed by a per-block epilogue s = sum_h w[q,h] * max(ACC, 0).
 //
-// A work item is (segment, tile of NQ consecutive query tokens, range of up to
-// KT 128-block tiles).  NQ = 64 for prefill (N = 256; TMEM holds two 128x256
-// fp32 accumulators), NQ = 4 for decode (N = 16; the kernel then streams the
-// sequence's k^ at HBM rate).  Roles (10 warps, one CTA per SM):
-//   warp 0      TMA producer: k^ tiles (128 rows x idx_dim, two 16 KiB boxes
-//               for idx_dim 128) into a 4-stage ring;
+// Work is the flat sequence of (segment, tile of NQ consecutive queries,
+// 128-block k^ tile) triples, ordered by segment, query tile, k^ tile.  The
+// kernel is persistent: CTA c takes the c-th of grid equal contiguous slices
+// of that sequence (measured in k^ tiles plus a fixed weight per query tile
+// for building its rotated queries), so every SM gets the same work and
+// walks few query tiles (the rotated query tile is built once per query
+// tile, not once per k^ tile).  The number of k^ tiles before query tile J of
+// a segment has a closed form (a floor sum), which lets a CTA seek to its
+// slice.
+//
+// NQ = 64 for prefill (N = 256; TMEM holds two 128x256 fp32 accumulators),
+// NQ = 4 for decode (N = 16; the kernel then streams each sequence's k^ at
+// HBM rate through a deeper ring).  Roles (one CTA per SM):
+//   warp 0      TMA producer: k^ tiles (128 rows x idx_dim as 64-dim boxes)
+//               into a ring of shared-memory stages;
 //   warp 1      TMEM owner and single-thread MMA issuer;
-//   warps 2..9  q~ = RoPE_t(q_idx) rounded to bf16, written once per item into
-//               the swizzled B tile (fp32 arithmetic in the same fixed order
-//               as the key pooling), then the epilogue: warp pair per TMEM lane
-//               quadrant, each thread owns one block row and half of the
-//               columns, and writes scores[t][b] for b < floor(t/r) as
-//               coalesced 128-byte rows.
+//   warps 2..   at each new query tile: q~ = RoPE_t(q_idx) rounded to bf16
+//               into the swizzled B tile (fp32 arithmetic in the same fixed
+//               order as the key pooling; the partner of a rotated pair comes
+//               from the neighbouring lane), then per k^ tile the epilogue:
+//               4 warps per TMEM lane quadrant, each reading its share of the
+//               columns into registers, releasing the accumulator, and
+//               writing scores[t][b] for b < floor(t/r) as 128-byte rows.
 // Every mbarrier wait is bounded.
 #pragma once
 #include "qsa_internal.cuh"
@@ -27,9 +37,6 @@
 
 namespace qsa {
 namespace tc_index {
-constexpr int kThreads = 320;
-constexpr int kEpiWarps = 8;
-constexpr int kStages = 4;
 constexpr int kTileRows = 128;             // k^ blocks per tile (MMA M)
 constexpr int kMaxRopeHalf = 32;           // rotated pairs per vector (rope_dims <= 64)
 }
@@ -37,17 +44,21 @@ constexpr int kMaxRopeHalf = 32;           // rotated pairs per vector (rope_dim
 template <int NQ>
 struct IndexTcCfg {
   static constexpr int N = 4 * NQ;                         // MMA N = queries x 4 heads
-  static constexpr int kKT = NQ >= 64 ? 16 : 64;           // tiles per work item
+  static constexpr int kEpiWarps = NQ >= 64 ? 8 : 4;       // 2 per TMEM lane quadrant for prefill
+  static constexpr int kEpiThreads = 32 * kEpiWarps;
+  static constexpr int kThreads = 64 + kEpiThreads;
+  static constexpr int kColsPerWarp = N / (kEpiWarps / 4);  // 64 (16 queries) or 16 (4 queries)
+  static constexpr int kStages = NQ >= 64 ? 4 : 6;
   static constexpr int kABytes = 128 * 128 * 2;            // one k^ tile, idx_dim 128
   static constexpr int kBBytes = N * 128 * 2;              // rotated queries, 2 slabs
-  static constexpr int kOffB = tc_index::kStages * kABytes;
+  static constexpr int kOffB = kStages * kABytes;
   static constexpr int kOffW = kOffB + kBBytes;            // w[NQ][4] fp32
-  static constexpr int kOffLim = kOffW + NQ * 16;          // floor(t/r) per query (int64)
-  static constexpr int kOffCS = kOffW + ((NQ * 24 + 1023) / 1024) * 1024;   // cos/sin[NQ][half][2]
+  static constexpr int kOffCS = kOffW + ((NQ * 16 + 1023) / 1024) * 1024;   // cos/sin[NQ][half]
   static constexpr int kOffBar = kOffCS + ((NQ * tc_index::kMaxRopeHalf * 8 + 1023) / 1024) * 1024;
   static constexpr int kSmemBytes = kOffBar + 1024 + 1024;
   static constexpr uint32_t kTmemCols = 2 * N < 32 ? 32 : 2 * N;
   static constexpr uint32_t kIdesc = sm100::idesc_bf16(128, N, false, false);
+  static constexpr int kRotTasks = (N * 16 + kEpiThreads - 1) / kEpiThreads;   // 16-byte chunks per thread
 };
 
 struct IndexTcArgs {
@@ -58,8 +69,8 @@ struct IndexTcArgs {
 };
 
 struct IndexTcCtl {
-  uint64_t a_full[tc_index::kStages];
-  uint64_t a_empty[tc_index::kStages];
+  uint64_t a_full[8];
+  uint64_t a_empty[8];
   uint64_t b_ready;
   uint64_t acc_full[2];
   uint64_t acc_free[2];
@@ -68,41 +79,127 @@ struct IndexTcCtl {
   int abort;
 };
 
-// Item geometry shared by every role.
-struct IndexItem {
-  int si;
-  int q0, nq;          // query tile within the segment
-  int64_t pos0;        // position of the segment's first query
-  int64_t tok0;        // token row of the tile's first query
-  int64_t t_first, t_last;
-  int tile0, ntiles;   // 128-block tiles [tile0, tile0+ntiles)
+// sum_{i=0}^{n-1} floor((a*i + b) / m) for n >= 0, m >= 1, a >= 0, b >= 0.
+// Each round strips the integer parts of a/m and b/m, then counts the
+// lattice points under the line the other way round:
+//   S(n, m, a, b) = K*n - S(K, a, m, m - b + a - 1),  K = floor((a(n-1) + b)/m),
+// whose (m, a) pair shrinks like Euclid's algorithm.
+__host__ __device__ inline int64_t floor_sum(int64_t n, int64_t m, int64_t a, int64_t b) {
+  int64_t total = 0, sign = 1;
+  while (n > 0) {
+    if (a >= m) {
+      total += sign * (a / m) * (n * (n - 1) / 2);
+      a %= m;
+    }
+    if (b >= m) {
+      total += sign * (b / m) * n;
+      b %= m;
+    }
+    const int64_t K = (a * (n - 1) + b) / m;
+    if (K == 0) break;
+    total += sign * K * n;
+    sign = -sign;
+    const int64_t nb = m - b + a - 1;
+    n = K;
+    const int64_t nm = a;
+    a = m;
+    m = nm;
+    b = nb;
+  }
+  return total;
+}
+
+// k^ tiles scored by query tile qt of a segment (the blocks its last query
+// scores, floor(t_last / r), in tiles of 128).
+template <int NQ>
+__host__ __device__ inline int index_qtile_tiles(int64_t pos0, int q_len, int qt, int r) {
+  const int64_t t_last = pos0 + (int64_t)min(NQ * (qt + 1), q_len) - 1;
+  return (int)cdiv(t_last / r, tc_index::kTileRows);
+}
+
+// Balancing weight of a query tile's prologue (building its rotated B tile),
+// in k^ tiles: the slices are equal in k^ tiles + kPrologueUnits per query
+// tile, so CTAs whose slice crosses many short early query tiles of a
+// prefill get fewer k^ tiles.
+template <int NQ>
+constexpr int index_prologue_units() { return NQ >= 64 ? 6 : 2; }
+
+// Work units (k^ tiles plus prologue weights) of the full query tiles
+// 0..J-1 of a segment, where the k^ tiles of full query tile j are
+//   ceil(floor((pos0 + NQ j + NQ - 1) / r) / 128) = floor((pos0 + NQ - 1 + 127 r + NQ j) / (128 r)).
+template <int NQ>
+__host__ __device__ inline int64_t index_units_before(int64_t pos0, int J, int r) {
+  return floor_sum(J, (int64_t)tc_index::kTileRows * r, NQ, pos0 + NQ - 1 + (int64_t)(tc_index::kTileRows - 1) * r) +
+         (int64_t)index_prologue_units<NQ>() * J;
+}
+
+// All work units of a segment.
+template <int NQ>
+inline int64_t index_tc_units(int q_len, int64_t pos0, int r) {
+  if (q_len <= 0) return 0;
+  const int nqt = (int)cdiv(q_len, NQ);
+  return index_units_before<NQ>(pos0, nqt - 1, r) + index_prologue_units<NQ>() +
+         index_qtile_tiles<NQ>(pos0, q_len, nqt - 1, r);
+}
+
+// Position in the flat sequence of work units: per segment, per query tile,
+// kPrologueUnits weights then one unit per k^ tile.  A CTA processes the k^
+// tiles whose units fall in its slice.
+struct IndexCursor {
+  int si, qt, tile, nt;
+  int64_t left;        // units left in this CTA's slice, the current tile included
 };
 
+// Moves to the next query tile that has k^ tiles (consuming its prologue
+// weight) while the current one is exhausted.
 template <int NQ>
-__device__ __forceinline__ bool index_item(const Geo& g, const SegTable& st, int item, IndexItem& it) {
-  using C = IndexTcCfg<NQ>;
-  it.si = find_segment(st, item);
-  const int local = item - st.item0[it.si];
-  const int q_len = st.q_len[it.si];
-  it.pos0 = st.pos0[it.si];
-  const int64_t nb_max = (it.pos0 + q_len - 1) / g.r;
-  const int max_chunks = (int)cdiv(cdiv(nb_max, tc_index::kTileRows), C::kKT);
-  if (max_chunks == 0) return false;
-  const int qt = local / max_chunks, ch = local - qt * max_chunks;
-  it.q0 = qt * NQ;
-  it.nq = min(NQ, q_len - it.q0);
-  it.tok0 = st.q_offset[it.si] + it.q0;
-  it.t_first = it.pos0 + it.q0;
-  it.t_last = it.t_first + it.nq - 1;
-  const int64_t nb = it.t_last / g.r;                       // blocks the tile's last query scores
-  const int nt = (int)cdiv(nb, tc_index::kTileRows);
-  it.tile0 = ch * C::kKT;
-  it.ntiles = min(C::kKT, nt - it.tile0);
-  return it.ntiles > 0;
+__device__ __forceinline__ void index_skip(const Geo& g, const SegTable& st, IndexCursor& c) {
+  while (c.left > 0 && c.tile >= c.nt) {
+    c.tile = 0;
+    if (++c.qt >= (int)cdiv(st.q_len[c.si], NQ)) {
+      c.qt = 0;
+      ++c.si;
+    }
+    c.nt = index_qtile_tiles<NQ>(st.pos0[c.si], st.q_len[c.si], c.qt, g.r);
+    c.left -= index_prologue_units<NQ>();
+  }
 }
 
 template <int NQ>
-__global__ void __launch_bounds__(tc_index::kThreads, 1)
+__device__ __forceinline__ void index_seek(const Geo& g, const SegTable& st, int64_t L, int64_t R, IndexCursor& c) {
+  constexpr int W = index_prologue_units<NQ>();
+  c.left = R - L;
+  if (c.left <= 0) return;
+  c.si = find_segment(st, (int)L);
+  const int64_t local = L - st.item0[c.si];
+  const int64_t pos0 = st.pos0[c.si];
+  const int nqt = (int)cdiv(st.q_len[c.si], NQ);
+  int lo = 0, hi = nqt - 1;                       // largest J with units_before(J) <= local
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (index_units_before<NQ>(pos0, mid, g.r) <= local) lo = mid; else hi = mid - 1;
+  }
+  c.qt = lo;
+  const int64_t o = local - index_units_before<NQ>(pos0, lo, g.r);
+  c.nt = index_qtile_tiles<NQ>(pos0, st.q_len[c.si], lo, g.r);
+  if (o < W) {                                    // the slice starts inside the prologue weight
+    c.left -= W - o;
+    c.tile = 0;
+  } else {
+    c.tile = (int)(o - W);
+  }
+  index_skip<NQ>(g, st, c);
+}
+
+template <int NQ>
+__device__ __forceinline__ void index_advance(const Geo& g, const SegTable& st, IndexCursor& c) {
+  --c.left;
+  ++c.tile;
+  index_skip<NQ>(g, st, c);
+}
+
+template <int NQ>
+__global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
     index_tc_kernel(const __grid_constant__ CUtensorMap tm_khat, Geo g, SegTable st, IndexTcArgs a) {
   using namespace tc_index;
   using namespace sm100;
@@ -111,22 +208,21 @@ __global__ void __launch_bounds__(tc_index::kThreads, 1)
   unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   IndexTcCtl& ctl = *reinterpret_cast<IndexTcCtl*>(smem + C::kOffBar);
   volatile int* abort_flag = &ctl.abort;
-  float* ws = reinterpret_cast<float*>(smem + C::kOffW);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  IndexItem it;
-  if (!index_item<NQ>(g, st, blockIdx.x, it)) return;          // uniform across the CTA
-  const int64_t kh_row0 = (int64_t)st.slot[it.si] * (g.n_cap / g.r);
+  const int64_t total = st.item0[st.n];
+  const int64_t L = total * blockIdx.x / gridDim.x, R = total * (blockIdx.x + 1) / gridDim.x;
+  if (L >= R) return;                                          // uniform across the CTA
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&ctl.a_full[i], 1);
       mbar_init(&ctl.a_empty[i], 1);
     }
-    mbar_init(&ctl.b_ready, kEpiWarps);
+    mbar_init(&ctl.b_ready, C::kEpiWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ctl.acc_full[i], 1);
-      mbar_init(&ctl.acc_free[i], kEpiWarps);
+      mbar_init(&ctl.acc_free[i], C::kEpiWarps);
     }
     mbar_init(&ctl.mma_done, 1);
     ctl.abort = 0;
@@ -143,14 +239,17 @@ __global__ void __launch_bounds__(tc_index::kThreads, 1)
   const uint32_t tmem = ctl.tmem_base;
   const uint32_t smem_base = smem_u32(smem);
 
+  IndexCursor cur;
+  index_seek<NQ>(g, st, L, R, cur);
+
   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0) {
-      for (int i = 0; i < it.ntiles; ++i) {
-        const int s = i % kStages;
-        if (!mbar_wait(&ctl.a_empty[s], (uint32_t)(((i / kStages) & 1) ^ 1), abort_flag)) break;
+      for (int i = 0; cur.left > 0; ++i, index_advance<NQ>(g, st, cur)) {
+        const int s = i % C::kStages;
+        if (!mbar_wait(&ctl.a_empty[s], (uint32_t)(((i / C::kStages) & 1) ^ 1), abort_flag)) break;
         mbar_expect_tx(&ctl.a_full[s], (uint32_t)(kTileRows * g.DI * 2));
-        const int32_t y = (int32_t)(kh_row0 + (int64_t)(it.tile0 + i) * kTileRows);
+        const int32_t y = (int32_t)((int64_t)st.slot[cur.si] * (g.n_cap / g.r) + (int64_t)cur.tile * kTileRows);
         for (int slab = 0; slab < g.DI / 64; ++slab)
           tma_load_2d(smem + s * C::kABytes + slab * 16384, &tm_khat, 64 * slab, y, &ctl.a_full[s]);
       }
@@ -159,12 +258,16 @@ __global__ void __launch_bounds__(tc_index::kThreads, 1)
   } else if (warp == 1) {
     // ============================================================ MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait(&ctl.b_ready, 0, abort_flag);
-      tc_fence_after();
-      for (int i = 0; i < it.ntiles && ok; ++i) {
-        const int s = i % kStages, ab = i & 1;
+      bool ok = true;
+      int nqt_seen = 0;
+      for (int i = 0; ok && cur.left > 0; ++i, index_advance<NQ>(g, st, cur)) {
+        if (i == 0 || cur.tile == 0) {                 // a new rotated query tile in B
+          if (!(ok = mbar_wait(&ctl.b_ready, (uint32_t)(nqt_seen & 1), abort_flag))) break;
+          ++nqt_seen;
+        }
+        const int s = i % C::kStages, ab = i & 1;
         if (!(ok = mbar_wait(&ctl.acc_free[ab], (uint32_t)(((i >> 1) & 1) ^ 1), abort_flag))) break;
-        if (!(ok = mbar_wait(&ctl.a_full[s], (uint32_t)((i / kStages) & 1), abort_flag))) break;
+        if (!(ok = mbar_wait(&ctl.a_full[s], (uint32_t)((i / C::kStages) & 1), abort_flag))) break;
         tc_fence_after();
         const uint32_t a_addr = smem_base + s * C::kABytes;
         const uint32_t b_addr = smem_base + C::kOffB;
@@ -184,97 +287,154 @@ __global__ void __launch_bounds__(tc_index::kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ============================================================ q~ tile, then epilogue
-    const int e = warp - 2;                         // 0..7
-    const int et = threadIdx.x - 64;                // 0..255
+    // ============================================================ q~ tiles and epilogue
+    const int et = threadIdx.x - 64;                // 0 .. kEpiThreads-1
     const int DI = g.DI, half = g.rope_half;
-    // cos/sin of every (query position, rotated pair) of the tile, once
+    const int chunks = DI / 8;                      // 16-byte chunks per q~ row
+    float* ws = reinterpret_cast<float*>(smem + C::kOffW);
     float2* cs = reinterpret_cast<float2*>(smem + C::kOffCS);
-    for (int k = et; k < it.nq * half; k += 32 * kEpiWarps) {
-      const int q = k / half, i = k - q * half;
-      float c, sn;
-      rope_cs(g, it.t_first + q, i, c, sn);
-      cs[k] = make_float2(c, sn);
-    }
-    named_bar_sync(1, 32 * kEpiWarps);
-    // rotated queries: row n = q*4 + h of the B tile (K-major, 128-byte swizzle)
-    for (int n = et; n < C::N; n += 32 * kEpiWarps) {
-      const int q = n >> 2, h = n & 3;
-      const bool live = q < it.nq;
-      const __nv_bfloat16* src = a.q_idx + ((it.tok0 + q) * 4 + h) * (int64_t)DI;
-      for (int j = 0; j < DI / 8; ++j) {            // 16-byte chunk j: dims 8j .. 8j+7
-        __align__(16) __nv_bfloat16 out[8];
-        if (live) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(src + 8 * j);
-          const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int d = 8 * j + k;
-            float v = __bfloat162float(x[k]);
-            if (d < 2 * half) {
-              const int i = d < half ? d : d - half;
-              const float xa = __bfloat162float(src[i]), xb = __bfloat162float(src[i + half]);
-              const float2 t = cs[q * half + i];
-              float o0, o1;
-              rope_pair(xa, xb, t.x, t.y, o0, o1);
-              v = d < half ? o0 : o1;
-            }
-            out[k] = __float2bfloat16_rn(v);
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) out[k] = __float2bfloat16_rn(0.f);
-        }
-        const int slab = j >> 3, jc = j & 7;
-        const uint32_t addr = C::kOffB + slab * (C::N * 128) + (n >> 3) * 1024 + (n & 7) * 128 + ((jc ^ (n & 7)) << 4);
-        *reinterpret_cast<uint4*>(smem + addr) = *reinterpret_cast<const uint4*>(out);
-      }
-    }
-    for (int i = et; i < NQ * 4; i += 32 * kEpiWarps)
-      ws[i] = (i >> 2) < it.nq ? a.w[it.tok0 * 4 + i] : 0.f;
-    int64_t* lim = reinterpret_cast<int64_t*>(smem + C::kOffLim);   // blocks each query scores
-    for (int q = et; q < NQ; q += 32 * kEpiWarps) lim[q] = q < it.nq ? (it.t_first + q) / g.r : 0;
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl.b_ready);
-    named_bar_sync(1, 32 * kEpiWarps);              // w[] visible to every epilogue thread
-
-    // epilogue: warp pair per lane quadrant; each warp takes half of the columns
     const int quad = warp & 3;
-    const int colhalf = e >> 2;                      // 0 or 1
-    constexpr int kCols = C::N / 2;                  // columns per warp
-    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    for (int i = 0; i < it.ntiles; ++i) {
-      const int ab = i & 1;
-      mbar_wait(&ctl.acc_full[ab], (uint32_t)((i >> 1) & 1), abort_flag);
-      tc_fence_after();
-      const int64_t b = (int64_t)(it.tile0 + i) * kTileRows + quad * 32 + lane;
-      constexpr int kChunk = kCols >= 32 ? 32 : (kCols >= 16 ? 16 : 8);   // TMEM columns per load
-      for (int c0 = 0; c0 < kCols; c0 += kChunk) {
-        float v[32];
-        if constexpr (kChunk == 32) {
-          tmem_ld16(lane_addr + ab * C::N + colhalf * kCols + c0, *reinterpret_cast<float(*)[16]>(v));
-          tmem_ld16(lane_addr + ab * C::N + colhalf * kCols + c0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
-        } else if constexpr (kChunk == 16) {
-          tmem_ld16(lane_addr + ab * C::N + colhalf * kCols + c0, *reinterpret_cast<float(*)[16]>(v));
-        } else {
-          tmem_ld8(lane_addr + ab * C::N + colhalf * kCols + c0, *reinterpret_cast<float(*)[8]>(v));
+    const int cq = (warp - 2) >> 2;                 // column share within the quadrant
+    constexpr int kCols = C::kColsPerWarp;
+    constexpr int kQ = kCols / 4;                   // queries per warp share
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(cq * kCols);
+    // pairs are whole 16-byte chunks when half is a multiple of 8: the partner
+    // chunk then sits hc lanes away in the same warp
+    const int hc = (half % 8 == 0) ? half / 8 : -1;
+
+    int64_t tok0 = 0, t_first = 0;
+    int nq = 0;
+    for (int i = 0; cur.left > 0; ++i, index_advance<NQ>(g, st, cur)) {
+      if (i == 0 || cur.tile == 0) {
+        // ---------------------------------------------- new query tile
+        const int q0 = cur.qt * NQ;
+        tok0 = st.q_offset[cur.si] + q0;
+        t_first = (int64_t)st.pos0[cur.si] + q0;
+        nq = min(NQ, st.q_len[cur.si] - q0);
+        named_bar_sync(1, C::kEpiThreads);          // every share is done with the previous w, cos/sin
+        for (int k = et; k < nq * half; k += C::kEpiThreads) {
+          const int q = k / half, p = k - q * half;
+          float c, sn;
+          rope_cs(g, t_first + q, p, c, sn);
+          cs[k] = make_float2(c, sn);
         }
-        tmem_wait_ld();
+        for (int k = et; k < NQ * 4; k += C::kEpiThreads) ws[k] = (k >> 2) < nq ? a.w[tok0 * 4 + k] : 0.f;
+        named_bar_sync(1, C::kEpiThreads);
+        // rotated queries: row n = q*4 + h of the B tile (K-major, 128-byte swizzle).
+        // The accumulators of the previous query tile were all observed full,
+        // so no MMA still reads B.
+        uint4 raw[C::kRotTasks];
 #pragma unroll
-        for (int qq = 0; qq < kChunk / 4; ++qq) {
-          const int q = (colhalf * kCols + c0) / 4 + qq;
-          if (q < it.nq && b < lim[q]) {
-            float sc = 0.f;
+        for (int k = 0; k < C::kRotTasks; ++k) {
+          const int task = et + k * C::kEpiThreads;
+          const int n = task / chunks, j = task - n * chunks;
+          raw[k] = make_uint4(0, 0, 0, 0);
+          if (n < C::N && (n >> 2) < nq)
+            raw[k] = *reinterpret_cast<const uint4*>(a.q_idx + ((tok0 + (n >> 2)) * 4 + (n & 3)) * (int64_t)DI + 8 * j);
+        }
 #pragma unroll
-            for (int h = 0; h < 4; ++h) sc = fmaf(ws[q * 4 + h], fmaxf(v[qq * 4 + h], 0.f), sc);
-            a.scores[(it.tok0 + q) * a.ld + b] = sc;
+        for (int k = 0; k < C::kRotTasks; ++k) {
+          const int task = et + k * C::kEpiThreads;
+          const int n = task / chunks, j = task - n * chunks;
+          const int q = n >> 2;
+          uint4 out = raw[k];
+          if (hc > 0) {
+            // partner chunk of a rotated pair: j + hc for first halves, j - hc for second halves
+            const int src = j < hc ? lane + hc : (j < 2 * hc ? lane - hc : lane);
+            uint4 pr;
+            pr.x = __shfl_sync(0xffffffffu, raw[k].x, src);
+            pr.y = __shfl_sync(0xffffffffu, raw[k].y, src);
+            pr.z = __shfl_sync(0xffffffffu, raw[k].z, src);
+            pr.w = __shfl_sync(0xffffffffu, raw[k].w, src);
+            if (j < 2 * hc && n < C::N && q < nq) {
+              const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(&raw[k]);
+              const __nv_bfloat16* y = reinterpret_cast<const __nv_bfloat16*>(&pr);
+              __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(&out);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int p = 8 * (j < hc ? j : j - hc) + e;          // pair index
+                const float2 t = cs[q * half + p];
+                float o0, o1;
+                if (j < hc) {
+                  rope_pair(__bfloat162float(x[e]), __bfloat162float(y[e]), t.x, t.y, o0, o1);
+                  o[e] = __float2bfloat16_rn(o0);
+                } else {
+                  rope_pair(__bfloat162float(y[e]), __bfloat162float(x[e]), t.x, t.y, o0, o1);
+                  o[e] = __float2bfloat16_rn(o1);
+                }
+              }
+            }
+          } else if (n < C::N && q < nq && 8 * j < 2 * half) {
+            // general pairing: fetch each partner element from the row in global memory
+            const __nv_bfloat16* row = a.q_idx + ((tok0 + q) * 4 + (n & 3)) * (int64_t)DI;
+            const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(&raw[k]);
+            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(&out);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int d = 8 * j + e;
+              if (d < 2 * half) {
+                const int p = d < half ? d : d - half;
+                const float2 t = cs[q * half + p];
+                float o0, o1;
+                rope_pair(__bfloat162float(row[p]), __bfloat162float(row[p + half]), t.x, t.y, o0, o1);
+                o[e] = __float2bfloat16_rn(d < half ? o0 : o1);
+              } else {
+                o[e] = x[e];
+              }
+            }
+          }
+          if (n < C::N) {
+            const int slab = j >> 3, jc = j & 7;
+            const uint32_t addr = C::kOffB + slab * (C::N * 128) + (n >> 3) * 1024 + (n & 7) * 128 + ((jc ^ (n & 7)) << 4);
+            *reinterpret_cast<uint4*>(smem + addr) = out;
           }
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.b_ready);
       }
+      // -------------------------------------------------- epilogue of k^ tile cur.tile
+      const int ab = i & 1;
+      if (!mbar_wait_sleep(&ctl.acc_full[ab], (uint32_t)((i >> 1) & 1), abort_flag)) continue;
+      tc_fence_after();
+      float v[kCols];
+#pragma unroll
+      for (int c0 = 0; c0 < kCols; c0 += 16)
+        tmem_ld16(lane_addr + ab * C::N + c0, *reinterpret_cast<float(*)[16]>(v + c0));
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.acc_free[ab]);
+      if (lane == 0) mbar_arrive(&ctl.acc_free[ab]);  // values are in registers: the MMA may reuse it
+
+      const int64_t b0 = (int64_t)cur.tile * kTileRows;
+      const int bl = quad * 32 + lane;                // block within the tile
+      const int qb = cq * kQ;                         // first query of this share
+      const int64_t t0 = t_first + qb;
+      const int64_t ld = a.ld;
+      float* p = a.scores + (tok0 + qb) * ld + b0 + bl;
+      const float4* w4 = reinterpret_cast<const float4*>(ws) + qb;
+      float sc[kQ];
+#pragma unroll
+      for (int qq = 0; qq < kQ; ++qq) {
+        const float4 wq = w4[qq];
+        float s = 0.f;
+        s = fmaf(wq.x, fmaxf(v[4 * qq + 0], 0.f), s);
+        s = fmaf(wq.y, fmaxf(v[4 * qq + 1], 0.f), s);
+        s = fmaf(wq.z, fmaxf(v[4 * qq + 2], 0.f), s);
+        s = fmaf(wq.w, fmaxf(v[4 * qq + 3], 0.f), s);
+        sc[qq] = s;
+      }
+      if (qb + kQ <= nq && (b0 + kTileRows) * g.r <= t0) {
+        // every block of the tile is a candidate of every query of the share
+#pragma unroll
+        for (int qq = 0; qq < kQ; ++qq, p += ld) *p = sc[qq];
+      } else {
+        // block b is a candidate of the query at t iff (b + 1) r <= t
+        const int64_t lim = t0 - (b0 + bl + 1) * g.r;
+#pragma unroll
+        for (int qq = 0; qq < kQ; ++qq, p += ld)
+          if (qb + qq < nq && lim + qq >= 0) *p = sc[qq];
+      }
     }
   }
   tc_fence_before();
@@ -283,14 +443,6 @@ __global__ void __launch_bounds__(tc_index::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
-}
-
-template <int NQ>
-inline int64_t index_tc_items(int q_len, int pos0, int r) {
-  using C = IndexTcCfg<NQ>;
-  if (q_len <= 0) return 0;
-  const int64_t nb_max = ((int64_t)pos0 + q_len - 1) / r;
-  return cdiv(q_len, NQ) * cdiv(cdiv(nb_max, tc_index::kTileRows), C::kKT);
 }
 
 }  // namespace qsa

@@ -234,16 +234,19 @@ qsa_status_t run_compress(const Geo& g, const qsa_config_t* c, const qsa_cache_t
 // Tensor map of the k^ cache: [n_slots * n_cap/r rows][idx_dim] bf16, boxes of
 // 64 dims x 128 rows.
 bool make_khat_map(CUtensorMap* m, const qsa_config_t* c, const qsa_cache_t* cache);
+int sm_count();
 
 template <int NQ>
 cudaError_t launch_index_tc(const Geo& g, const SegTable& t, const CUtensorMap& tm, const IndexTcArgs& a,
                             cudaStream_t st) {
-  const int items = t.item0[t.n];
-  if (items == 0) return cudaSuccess;
+  const int units = t.item0[t.n];
+  if (units == 0) return cudaSuccess;
   const int smem = IndexTcCfg<NQ>::kSmemBytes;
   cudaFuncSetAttribute(index_tc_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   count_launch();
-  index_tc_kernel<NQ><<<items, tc_index::kThreads, smem, st>>>(tm, g, t, a);
+  // persistent: one CTA per SM, each an equal slice of the work units
+  const int grid = std::min(units, sm_count());
+  index_tc_kernel<NQ><<<grid, IndexTcCfg<NQ>::kThreads, smem, st>>>(tm, g, t, a);
   return cudaGetLastError();
 }
 
@@ -259,12 +262,12 @@ qsa_status_t run_index(const Geo& g, const qsa_config_t* c, const qsa_cache_t* c
     for (int i = 0; i < n; ++i) (segs[i].q_len >= 16 ? wide : narrow).push_back(segs[i]);
     qsa_status_t r = for_each_table(
         wide.data(), (int)wide.size(),
-        [&](const qsa_segment_t& s) { return index_tc_items<64>(s.q_len, s.pos0, g.r); },
+        [&](const qsa_segment_t& s) { return index_tc_units<64>(s.q_len, s.pos0, g.r); },
         [&](const SegTable& t) { return launch_index_tc<64>(g, t, tm, a, st); });
     if (r != QSA_OK) return r;
     return for_each_table(
         narrow.data(), (int)narrow.size(),
-        [&](const qsa_segment_t& s) { return index_tc_items<4>(s.q_len, s.pos0, g.r); },
+        [&](const qsa_segment_t& s) { return index_tc_units<4>(s.q_len, s.pos0, g.r); },
         [&](const SegTable& t) { return launch_index_tc<4>(g, t, tm, a, st); });
   }
   size_t smem = sizeof(float) * (simt_index::QT * g.HI * g.DI + simt_index::QT * g.HI);

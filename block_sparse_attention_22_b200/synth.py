@@ -16,6 +16,8 @@ kv-channels 256, rotary 0.25 at base 1e7; design report, QSA item: r=4, a
   decode_256k   32 sequences x 1 decode query against a 262144-token cache
   mixed_1m      8 decode queries at 1048576-token context plus one 4096-query
                 prefill chunk at [942080, 946176) of a 90%-cached sequence
+  decode_1m     the decode part of mixed_1m alone: 8 sequences x 1 decode
+                query against a 1048576-token cache
   chunk_128k    one 4096-query prefill chunk at [126976, 131072) of a
                 131072-token sequence whose prefix is cached (a ~1 GB case
                 whose K/V still exceeds L2; used for kernel profiles)
@@ -161,10 +163,11 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
             needles.append((0, t, b))
         return Workload(name, sh, [Segment(0, 0, n)], 1, _round_cap(n, sh.r), [n], [0], needles,
                         seed if seed is not None else 2)
-    if name == "decode_256k":
+    if name in ("decode_256k", "decode_1m"):
         sh = Shape()
-        ctx = over.get("ctx", 262144)
-        n_seqs = over.get("n_seqs", 32)
+        big = name == "decode_1m"
+        ctx = over.get("ctx", (1 << 20) if big else 262144)
+        n_seqs = over.get("n_seqs", 8 if big else 32)
         segs = [Segment(s, ctx - 1, 1) for s in range(n_seqs)]
         needles = []
         for s in range(n_seqs):
@@ -174,7 +177,7 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
         # the decode token completes block (ctx-1)//r; earlier blocks are cached
         cached = [(ctx - 1) // sh.r] * n_seqs
         return Workload(name, sh, segs, n_seqs, _round_cap(ctx, sh.r), [ctx] * n_seqs, cached, needles,
-                        seed if seed is not None else 3)
+                        seed if seed is not None else (6 if big else 3))
     if name == "mixed_1m":
         sh = Shape()
         ctx = over.get("ctx", 1 << 20)
