@@ -313,7 +313,9 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
       },
       [&](const SegTable& t) {
         count_launch();
-        topk_chunk_kernel<<<t.item0[t.n], topk::THREADS, smem_c, st>>>(g, t, a);
+        // persistent: as many CTAs as fit (six per SM by shared memory)
+        const int grid = std::min(t.item0[t.n], 6 * sm_count());
+        topk_chunk_kernel<<<grid, topk::THREADS, smem_c, st>>>(g, t, a);
         return cudaGetLastError();
       });
   if (r != QSA_OK || p.max_ch <= 1) return r;

@@ -6,51 +6,74 @@
 // always kept; the other S-1 are the best candidates b < floor(t/r) under
 // the total order (score descending, block index ascending), -0 == +0.
 //
-// Algorithm (one CTA per row, or per row chunk for long rows; the row is
-// streamed from global memory, so several CTAs fit on an SM).  Elements are
-// ranked by the 64-bit composite (key << 32) | ~index, which orders them by
-// score and then by lower block index, so every composite is distinct:
-//   1. radix narrowing over the row: histograms of the next 11/11/10 key bits
-//      over the elements still in the threshold bucket (warp-aggregated
-//      shared atomics) locate the bucket holding the K-th largest element,
-//      until that bucket fits a 4096-entry shared buffer;
-//   2. gather: elements above the bucket are kept outright, the bucket's
-//      elements are copied to the buffer as composites;
-//   3. narrowing continues on the composites in shared memory (remaining key
-//      bits, then index bits) until the bucket holds exactly the elements
-//      still needed; every buffered composite at or above it is kept;
-//   4. the kept block indices are sorted ascending (bitonic, 512 entries).
-// If a bucket is still larger than the buffer after all 32 key bits (many
-// exactly equal keys), the tied elements are taken in index order by an
-// ordered ballot compaction instead.  Long rows are split into chunks whose
-// local top K (exact under the same order) are merged by a second pass of
-// the same routine over the chunk candidates.
+// One CTA of 4 warps per row (or per row chunk for long rows when rows are
+// few), persistent over rows, ~35 KB of shared memory so that six CTAs share
+// an SM.  Scores are compared as 32-bit keys whose unsigned order is the
+// float order.  For a row of n candidates and K = S-1:
+//   1. threshold: m = n/16 keys (1024 .. 8192, in runs of 8 neighbours spread
+//      evenly over the row) are reduced by a radix select to the 16-bit
+//      bucket of their rank-th largest, rank chosen so that about
+//      kSampleTarget elements of the row are expected at or above the
+//      bucket's lower edge (rows of at most CAP elements take every element);
+//   2. filter: one pass over the row (16-byte streaming loads); each thread
+//      appends the elements at or above the threshold to its own 24 slots,
+//      spilling to shared overflow slots, with no coordination;
+//   3. if between K and CAP elements were collected, the K-th largest of the
+//      row is among them: a radix select over the candidates (8-bit digits,
+//      starting below the bits all candidates share) finds its key T and how
+//      many elements equal to T are needed; if fewer than all of the tied ones
+//      are needed, a second radix select over the tied elements' indices keeps
+//      the lowest ones;
+//   4. the kept block indices are put in ascending order through a bitmap of
+//      the row (set bits, then each thread emits the set bits of its words at
+//      its prefix-count offset).
+// If the sampled threshold admits fewer than K or more than CAP elements, an
+// exact fallback runs: a radix select streamed over the whole row (four
+// passes), then one ordered pass that keeps everything above T and the
+// lowest-indexed elements equal to T.  Long rows are split into chunks whose
+// local top K (exact under the same order, sorted by index) are merged by a
+// second pass of the same routine over the chunk candidates.  While a CTA
+// works on one row, the copy engine prefetches its next row into L2.
 #pragma once
 #include "qsa_internal.cuh"
 
 namespace qsa {
 namespace topk {
-constexpr int THREADS = 256;
+constexpr int THREADS = 128;
 constexpr int WARPS = THREADS / 32;
-constexpr int NBINS = 2048;
-constexpr int CAP = 4096;                  // candidate buffer (composite keys)
+constexpr int NBINS = 256;                 // one 8-bit digit per radix pass
+constexpr int CAPL = 24;                   // candidate slots per thread
+constexpr int OVF = 1024;                  // shared overflow slots
+constexpr int CAP = CAPL * THREADS + OVF;  // candidates a row may collect (4096)
 constexpr int KMAX = kMaxBudgetBlocks;     // kept entries per row (S-1 <= 511)
+constexpr int kBufWords = 2 * CAP;         // candidate buffer, reused for the sample and the bitmap
+constexpr int kMinSamples = 1024;
+constexpr int kMaxSamples = kBufWords;
+constexpr int kSampleGroup = 8;            // samples are runs of 8 neighbours (one 32-byte sector)
+constexpr int kSampleTarget = 1536;        // expected elements at or above the sampled threshold
 constexpr int kChunkLarge = 1 << 30;       // no split
 constexpr int kChunkSmall = 8192;
 }
 
 struct TopkShared {
   uint32_t hist[topk::NBINS];
-  unsigned long long cand[topk::CAP];      // composites (key << 32) | ~index
-  uint32_t kept[topk::KMAX];               // indices kept outright / final list
+  uint32_t cbuf[topk::kBufWords];          // candidates | sample | bitmap
+  uint32_t kept[topk::KMAX];               // kept indices / final sorted list
   int warp_a[topk::WARPS];
   int warp_b[topk::WARPS];
-  int n_kept, n_cand;
+  uint32_t warp_c[topk::WARPS];
+  int n_kept, n_ovf;
   uint32_t sel_digit;
   int sel_above, sel_count;
+  // candidate slot s of thread t: lkey[s * THREADS + t]; overflow slot o: okey[o]
+  __device__ __forceinline__ uint32_t* lkey() { return cbuf; }
+  __device__ __forceinline__ uint32_t* lidx() { return cbuf + topk::CAPL * topk::THREADS; }
+  __device__ __forceinline__ uint32_t* okey() { return cbuf + 2 * topk::CAPL * topk::THREADS; }
+  __device__ __forceinline__ uint32_t* oidx() { return cbuf + 2 * topk::CAPL * topk::THREADS + topk::OVF; }
 };
 
-// Source of one selection: element i has key(i) and index idx(i).
+// Source of one selection: element i has key(i) and index index(i); element
+// order is index order.
 struct RowSrc {
   const float* scores;          // score row (keys from scores), or null
   const uint32_t* keys;         // candidate keys (merge), or null
@@ -64,34 +87,74 @@ struct RowSrc {
   }
 };
 
-// Histogram of digit (key >> shift) & dmask over elements with (key & mask) == prefix.
-__device__ void topk_hist(const RowSrc& src, int n, uint32_t prefix, uint32_t mask, int shift, uint32_t dmask,
-                          TopkShared& sh) {
-  using namespace topk;
+// Float whose key is k (inverse of score_key on keys of finite floats); keys
+// below that of -inf map to -inf.
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  if (k & 0x80000000u) return __uint_as_float(k & 0x7fffffffu);
+  if (k < 0x007fffffu) return -__int_as_float(0x7f800000);
+  return __uint_as_float(~k);
+}
+
+// ---------------------------------------------------------------- block reductions
+__device__ __forceinline__ int block_sum(int v, TopkShared& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < NBINS; i += THREADS) sh.hist[i] = 0;
+  v = __reduce_add_sync(0xffffffffu, v);
+  if (lane == 0) sh.warp_b[warp] = v;
   __syncthreads();
-  for (int b = warp * 32; b < n; b += THREADS) {
-    const int i = b + lane;
-    const uint32_t key = i < n ? src.key(i) : 0u;
-    const bool valid = i < n && (key & mask) == prefix;
-    const uint32_t digit = (key >> shift) & dmask;
-    const uint32_t peers = __match_any_sync(0xffffffffu, valid ? digit : 0xffffffffu);
-    if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[digit], (uint32_t)__popc(peers));
+  int t = 0;
+#pragma unroll
+  for (int w = 0; w < topk::WARPS; ++w) t += sh.warp_b[w];
+  __syncthreads();
+  return t;
+}
+
+__device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, TopkShared& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0) {
+    sh.warp_c[warp] = lo;
+    sh.warp_a[warp] = (int)hi;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < topk::WARPS; ++w) {
+    lo = min(lo, sh.warp_c[w]);
+    hi = max(hi, (uint32_t)sh.warp_a[w]);
   }
   __syncthreads();
 }
 
+// ---------------------------------------------------------------- radix helpers
+__device__ __forceinline__ void hist_clear(TopkShared& sh) {
+  for (int i = threadIdx.x; i < topk::NBINS; i += topk::THREADS) sh.hist[i] = 0;
+}
+
+// Adds element (key, valid) to the histogram of digit (key >> shift) & 255.
+// The top digit of keys of similar magnitude is shared by most of a warp, so
+// that pass aggregates equal digits into one shared atomic.
+__device__ __forceinline__ void hist_add(uint32_t key, bool valid, int shift, bool aggregate, TopkShared& sh) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t digit = (key >> shift) & 255u;
+  if (aggregate) {
+    const uint32_t peers = __match_any_sync(0xffffffffu, valid ? digit : 0xffffffffu);
+    if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[digit], (uint32_t)__popc(peers));
+  } else if (valid) {
+    atomicAdd(&sh.hist[digit], 1u);
+  }
+}
+
 // Finds the digit whose bucket holds the k_rem-th largest element: sets
 // sh.sel_digit, sh.sel_above (count in higher buckets), sh.sel_count.
-__device__ void topk_locate(int k_rem, TopkShared& sh) {
+// Ends with a barrier.
+__device__ void hist_locate(int k_rem, TopkShared& sh) {
   using namespace topk;
   constexpr int PER = NBINS / THREADS;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int local = 0;
 #pragma unroll
   for (int j = 0; j < PER; ++j) local += sh.hist[threadIdx.x * PER + j];
-  int suf = local;
+  int suf = local;                       // sum over this and higher threads of the warp
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int v = __shfl_down_sync(0xffffffffu, suf, off);
@@ -119,16 +182,317 @@ __device__ void topk_locate(int k_rem, TopkShared& sh) {
   __syncthreads();
 }
 
-// Bitonic sort of a[0..n) (n a power of two), descending or ascending.
-template <typename T>
-__device__ void bitonic(T* a, int n, bool descending) {
+// Radix select of the k-th largest value among the n values produced by
+// val(i) that satisfy ok(i): 8-bit passes from the top down to bit
+// last_shift.  Returns the value with the bits below last_shift cleared;
+// *above = how many values are larger in the resolved bits, *equal = how
+// many share them (with last_shift = 0: strictly larger, and equal).
+template <class Val, class Ok>
+__device__ uint32_t radix_select(int n, int k, Val val, Ok ok, int* above, int* equal, TopkShared& sh,
+                                 int last_shift = 0) {
+  using namespace topk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t prefix = 0, mask = 0;
+  int k_rem = k, n_above = 0, count = 0;
+  for (int shift = 24; shift >= last_shift; shift -= 8) {
+    hist_clear(sh);
+    __syncthreads();
+    for (int b = warp * 32; b < n; b += THREADS) {
+      const int i = b + lane;
+      const bool in = i < n && ok(i);
+      const uint32_t v = in ? val(i) : 0u;
+      hist_add(v, in && (v & mask) == prefix, shift, shift == 24, sh);
+    }
+    __syncthreads();
+    hist_locate(k_rem, sh);
+    k_rem -= sh.sel_above;
+    n_above += sh.sel_above;
+    prefix |= sh.sel_digit << shift;
+    mask |= 255u << shift;
+    count = sh.sel_count;
+    __syncthreads();
+  }
+  *above = n_above;
+  *equal = count;
+  return prefix;
+}
+
+// Appends idx to sh.kept when `take` (warp-aggregated; every lane calls it).
+__device__ __forceinline__ void keep_if(bool take, uint32_t idx, TopkShared& sh) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t m = __ballot_sync(0xffffffffu, take);
+  if (m == 0) return;
+  int base = 0;
+  if (lane == 0) base = atomicAdd(&sh.n_kept, __popc(m));
+  base = __shfl_sync(0xffffffffu, base, 0);
+  const int pos = base + __popc(m & ((1u << lane) - 1u));
+  if (take && pos < topk::KMAX) sh.kept[pos] = idx;
+}
+
+// ---------------------------------------------------------------- candidates
+// Each thread appends the candidates it finds to its own slots (no
+// coordination); past CAPL they go to the shared overflow slots.  `cnt`
+// counts every candidate of the thread.
+__device__ __forceinline__ void cand_append(uint32_t key, uint32_t idx, int& cnt, TopkShared& sh) {
+  using namespace topk;
+  if (cnt < CAPL) {
+    sh.lkey()[cnt * THREADS + threadIdx.x] = key;
+    sh.lidx()[cnt * THREADS + threadIdx.x] = idx;
+  } else {
+    const int o = atomicAdd(&sh.n_ovf, 1);
+    if (o < OVF) {
+      sh.okey()[o] = key;
+      sh.oidx()[o] = idx;
+    }
+  }
+  ++cnt;
+}
+
+// Calls f(key, idx, valid) for this thread's candidates in a loop whose trip
+// count is uniform across the warp (own slots, then a strided share of the
+// overflow slots).
+template <class F>
+__device__ __forceinline__ void cand_for_each(int cnt, TopkShared& sh, F f) {
+  using namespace topk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int mine = min(cnt, CAPL);
+  const int wmax = __reduce_max_sync(0xffffffffu, mine);
+  for (int s = 0; s < wmax; ++s) {
+    const bool v = s < mine;
+    f(v ? sh.lkey()[s * THREADS + threadIdx.x] : 0u, v ? sh.lidx()[s * THREADS + threadIdx.x] : 0u, v);
+  }
+  const int no = min(sh.n_ovf, OVF);
+  for (int b = warp * 32; b < no; b += THREADS) {
+    const int o = b + lane;
+    const bool v = o < no;
+    f(v ? sh.okey()[o] : 0u, v ? sh.oidx()[o] : 0u, v);
+  }
+}
+
+// Radix select of the k-th largest of val(key, idx) over the candidates
+// with ok(key, idx).  The passes start below the common high bits of the
+// smallest and largest participating value.  Returns the value; *above =
+// how many are larger, *equal = how many equal it.
+template <class Val, class Ok>
+__device__ uint32_t cand_radix(int cnt, int k, Val val, Ok ok, int* above, int* equal, TopkShared& sh) {
+  uint32_t vmin = 0xffffffffu, vmax = 0u;
+  int n_ok = 0;
+  cand_for_each(cnt, sh, [&](uint32_t key, uint32_t idx, bool v) {
+    if (v && ok(key, idx)) {
+      const uint32_t x = val(key, idx);
+      vmin = min(vmin, x);
+      vmax = max(vmax, x);
+      ++n_ok;
+    }
+  });
+  block_minmax(vmin, vmax, sh);
+  n_ok = block_sum(n_ok, sh);
+  if (vmin == vmax) {
+    *above = 0;
+    *equal = n_ok;
+    return vmin;
+  }
+  const int h = 31 - __clz(vmin ^ vmax);              // highest bit that differs
+  uint32_t mask = h == 31 ? 0u : ~((2u << h) - 1u);   // bits above h: shared by all
+  uint32_t prefix = vmin & mask;
+  int k_rem = k, n_above = 0, count = n_ok;
+  for (int hi = h; hi >= 0; hi -= 8) {
+    const int lo = hi >= 7 ? hi - 7 : 0;
+    const uint32_t dm = (2u << (hi - lo)) - 1u;
+    hist_clear(sh);
+    __syncthreads();
+    cand_for_each(cnt, sh, [&](uint32_t key, uint32_t idx, bool v) {
+      if (v && ok(key, idx)) {
+        const uint32_t x = val(key, idx);
+        if ((x & mask) == prefix) atomicAdd(&sh.hist[(x >> lo) & dm], 1u);
+      }
+    });
+    __syncthreads();
+    hist_locate(k_rem, sh);
+    k_rem -= sh.sel_above;
+    n_above += sh.sel_above;
+    prefix |= sh.sel_digit << lo;
+    mask |= dm << lo;
+    count = sh.sel_count;
+    __syncthreads();
+  }
+  *above = n_above;
+  *equal = count;
+  return prefix;
+}
+
+// Exact selection over the collected candidates, which hold every element of
+// the row whose key is >= the K-th largest key: appends the indices of the K
+// best (key desc, index asc) to sh.kept.
+__device__ void select_candidates(int cnt, int K, TopkShared& sh) {
+  int above, equal;
+  const uint32_t T = cand_radix(
+      cnt, K, [](uint32_t k, uint32_t) { return k; }, [](uint32_t, uint32_t) { return true; }, &above, &equal,
+      sh);
+  const int need = K - above;                // elements equal to T to keep (>= 1)
+  uint32_t imax = 0xffffffffu;                // keep ties with index <= imax
+  if (need < equal) {
+    // the need lowest indices among the ties: the need-th largest of ~index
+    int a2, e2;
+    const uint32_t inv = cand_radix(
+        cnt, need, [](uint32_t, uint32_t i) { return ~i; }, [T](uint32_t k, uint32_t) { return k == T; }, &a2,
+        &e2, sh);
+    imax = ~inv;
+  }
+  cand_for_each(cnt, sh, [&](uint32_t k, uint32_t i, bool v) {
+    keep_if(v && (k > T || (k == T && i <= imax)), i, sh);
+  });
+  __syncthreads();
+}
+
+// Exact fallback streamed over the whole source (any n >= K): four radix
+// passes over global memory, then one pass in element (= index) order that
+// keeps every element above T and the lowest-indexed ones equal to T.
+__device__ void select_streamed(const RowSrc& src, int n, int K, TopkShared& sh) {
+  using namespace topk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int above, equal;
+  const uint32_t T = radix_select(
+      n, K, [&](int i) { return src.key(i); }, [](int) { return true; }, &above, &equal, sh);
+  const int need = K - above;
+  // ties in index order: warp w owns a contiguous range of elements
+  const int per = (int)cdiv(cdiv(n, WARPS), 32) * 32;
+  const int beg = warp * per, end = min(n, beg + per);
+  int n_tie = 0;
+  for (int b = beg; b < end; b += 32) {
+    const int i = b + lane;
+    n_tie += __popc(__ballot_sync(0xffffffffu, i < end && src.key(i) == T));
+  }
+  if (lane == 0) sh.warp_b[warp] = n_tie;
+  __syncthreads();
+  int tie_run = 0;
+  for (int w = 0; w < warp; ++w) tie_run += sh.warp_b[w];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int b = beg; b < end; b += 32) {
+    const int i = b + lane;
+    const uint32_t k = i < end ? src.key(i) : 0u;
+    const bool tie = i < end && k == T;
+    const uint32_t bt = __ballot_sync(0xffffffffu, tie);
+    const bool take = (i < end && k > T) || (tie && tie_run + __popc(bt & lt) < need);
+    keep_if(take, take ? src.index(i) : 0u, sh);
+    tie_run += __popc(bt);
+  }
+  __syncthreads();
+}
+
+// Filter pass of a score row: every element with score >= tau (as floats,
+// which matches key >= key(tau)) becomes a candidate of the thread that
+// reads it.  16-byte streaming loads over the aligned middle of the row.
+__device__ void filter_scores(const float* row, int64_t base, int n, float tau, int& cnt, TopkShared& sh) {
+  using namespace topk;
+  const int align_head = (int)(((16 - ((uintptr_t)row & 15)) & 15) / 4);
+  const int head = align_head < n ? align_head : n;
+  const int nvec = (n - head) / 4;
+  const int tail0 = head + nvec * 4;
+  if (threadIdx.x < head) {
+    const float s = row[threadIdx.x];
+    if (s >= tau) cand_append(score_key(s), (uint32_t)(base + threadIdx.x), cnt, sh);
+  } else if (threadIdx.x >= 32 && threadIdx.x < 32 + n - tail0) {
+    const int i = tail0 + (int)threadIdx.x - 32;
+    const float s = row[i];
+    if (s >= tau) cand_append(score_key(s), (uint32_t)(base + i), cnt, sh);
+  }
+  const float4* v4 = reinterpret_cast<const float4*>(row + head);
+  constexpr int U = 4;
+  for (int v0 = threadIdx.x; v0 < nvec; v0 += U * THREADS) {
+    float4 x[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + u * THREADS;
+      x[u] = v < nvec ? __ldg(v4 + v) : make_float4(NAN, NAN, NAN, NAN);   // NaN never passes
+    }
+    // hits of this thread's 4U elements as a bit mask; most threads have
+    // none or one, so the appends loop over set bits, re-reading the value
+    // from L1 instead of selecting it among registers
+    uint32_t hm = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      hm |= ((x[u].x >= tau) ? 1u : 0u) << (4 * u) | ((x[u].y >= tau) ? 2u : 0u) << (4 * u) |
+            ((x[u].z >= tau) ? 4u : 0u) << (4 * u) | ((x[u].w >= tau) ? 8u : 0u) << (4 * u);
+    while (hm) {
+      const int b = __ffs(hm) - 1;
+      hm &= hm - 1u;
+      const int i = head + 4 * (v0 + (b >> 2) * THREADS) + (b & 3);
+      cand_append(score_key(__ldg(row + i)), (uint32_t)(base + i), cnt, sh);
+    }
+  }
+}
+
+// Selects the K best elements of src[0..n) (K <= n) under (key desc, index
+// asc).  On return sh.kept[0..K) holds their indices, in no particular order.
+__device__ void topk_select(const RowSrc& src, int n, int K, TopkShared& sh) {
+  using namespace topk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    sh.n_kept = 0;
+    sh.n_ovf = 0;
+  }
+  uint32_t tkey = 0u;                            // every key is >= 0
+  if (n > CAP) {
+    // 1. sampled threshold: m keys in runs of kSampleGroup spread over the row
+    const int m0 = n / 16 < kMinSamples ? kMinSamples : (n / 16 > kMaxSamples ? kMaxSamples : n / 16);
+    const int groups = m0 / kSampleGroup;
+    const int m = groups * kSampleGroup;
+    // group gi starts at gi*(n-8)/(groups-1) <= n-8, so every position is < n
+#pragma unroll 8
+    for (int s = threadIdx.x; s < m; s += THREADS) {
+      const int gi = s / kSampleGroup, j = s - gi * kSampleGroup;
+      const int64_t pos = (int64_t)gi * (n - kSampleGroup) / (groups - 1) + j;
+      sh.cbuf[s] = src.key((int)pos);
+    }
+    __syncthreads();
+    const int rank = max(1, (int)((int64_t)m * kSampleTarget / n));
+    int a0, e0;
+    // the lower edge of the 16-bit bucket holding the rank-th largest sample
+    tkey = radix_select(
+        m, rank, [&](int i) { return sh.cbuf[i]; }, [](int) { return true; }, &a0, &e0, sh, 16);
+  }
+  __syncthreads();
+  // 2. filter
+  int cnt = 0;
+  if (src.scores) {
+    filter_scores(src.scores, src.base, n, key_to_float(tkey), cnt, sh);
+  } else {
+    // candidate lists of a merge: batches of loads in flight, then the appends
+    constexpr int B = 8;
+    for (int i0 = threadIdx.x; i0 < n; i0 += B * THREADS) {
+      uint32_t k[B], ix[B];
+#pragma unroll
+      for (int u = 0; u < B; ++u) {
+        const int i = i0 + u * THREADS;
+        k[u] = i < n ? __ldcs(src.keys + i) : 0u;
+        ix[u] = i < n ? (uint32_t)__ldcs(src.idx + i) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < B; ++u)
+        if (i0 + u * THREADS < n && k[u] >= tkey) cand_append(k[u], ix[u], cnt, sh);
+    }
+  }
+  __syncthreads();
+  const int nc = block_sum(cnt, sh);
+  if (nc >= K && sh.n_ovf <= OVF) {
+    select_candidates(cnt, K, sh);              // 3.
+  } else {
+    select_streamed(src, n, K, sh);             // exact fallback
+  }
+  (void)lane;
+  (void)warp;
+}
+
+// Bitonic sort of a[0..n) (n a power of two), ascending.
+__device__ void bitonic_asc(uint32_t* a, int n) {
   for (int k = 2; k <= n; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
       for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int p = i ^ j;
         if (p > i) {
-          const bool up = ((i & k) == 0) != descending;
-          const T x = a[i], y = a[p];
+          const bool up = (i & k) == 0;
+          const uint32_t x = a[i], y = a[p];
           if ((x > y) == up) {
             a[i] = y;
             a[p] = x;
@@ -137,180 +501,6 @@ __device__ void bitonic(T* a, int n, bool descending) {
       }
       __syncthreads();
     }
-  }
-}
-
-// Finishes a selection whose candidates sh.cand[0..nc) are the composites of
-// every element in the current bucket (key & mask == prefix) and k_rem of
-// them are still needed: narrows on the remaining key bits, then on the
-// index bits, until the bucket holds exactly the elements still needed, and
-// appends every candidate at or above it to sh.kept.
-__device__ void refine_and_keep(int nc, int k_rem, uint32_t prefix, uint32_t mask, TopkShared& sh) {
-  using namespace topk;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  unsigned long long cprefix = (unsigned long long)prefix << 32, cmask = (unsigned long long)mask << 32;
-  const int cshifts[6] = {53, 42, 32, 21, 10, 0};
-  const int cwidths[6] = {11, 11, 10, 11, 11, 10};
-  int q0 = 0;                               // first composite digit not yet resolved
-  while (q0 < 3 && ((cmask >> cshifts[q0]) & 1ull)) ++q0;
-  int count = nc;
-  for (int q = q0; q < 6 && count != k_rem; ++q) {
-    const unsigned long long dm = (1ull << cwidths[q]) - 1ull;
-    for (int i = threadIdx.x; i < NBINS; i += THREADS) sh.hist[i] = 0;
-    __syncthreads();
-    for (int b = warp * 32; b < nc; b += THREADS) {
-      const int i = b + lane;
-      const unsigned long long c = i < nc ? sh.cand[i] : 0ull;
-      const bool valid = i < nc && (c & cmask) == cprefix;
-      const uint32_t digit = (uint32_t)((c >> cshifts[q]) & dm);
-      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? digit : 0xffffffffu);
-      if (valid && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[digit], (uint32_t)__popc(peers));
-    }
-    __syncthreads();
-    topk_locate(k_rem, sh);
-    k_rem -= sh.sel_above;
-    cprefix |= (unsigned long long)sh.sel_digit << cshifts[q];
-    cmask |= dm << cshifts[q];
-    count = sh.sel_count;
-    __syncthreads();
-  }
-  for (int i = threadIdx.x; i < nc; i += THREADS) {
-    const unsigned long long c = sh.cand[i];
-    if ((c & cmask) >= cprefix) sh.kept[atomicAdd(&sh.n_kept, 1)] = 0xffffffffu - (uint32_t)(c & 0xffffffffull);
-  }
-  __syncthreads();
-}
-
-// Fast path for rows longer than the candidate buffer: a strided sample of
-// the keys gives a threshold expected to admit about kSampleTarget elements;
-// one pass collects every element at or above it.  If between K and CAP
-// elements qualify, the K best are among them (at least K elements are at or
-// above the threshold, so the K-th largest is too) and are found exactly on
-// the buffered composites; otherwise returns false and nothing is kept.
-constexpr int kSamples = 2048;
-constexpr int kSampleTarget = 2048;
-
-__device__ bool select_by_sample(const RowSrc& src, int n, int K, TopkShared& sh) {
-  using namespace topk;
-  uint32_t* samp = reinterpret_cast<uint32_t*>(sh.cand);      // reused before the candidates land
-  const int m = min(kSamples, n / 4);
-  for (int s = threadIdx.x; s < m; s += THREADS) samp[s] = src.key((int)((int64_t)s * n / m));
-  __syncthreads();
-  const int target = max(4 * K, kSampleTarget);
-  const int rank = max(1, (int)((int64_t)m * target / n));
-  // exact rank-th largest sample key
-  const RowSrc ssrc{nullptr, samp, nullptr, 0};
-  uint32_t prefix = 0, mask = 0;
-  int k_rem = rank;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-  for (int p = 0; p < 3; ++p) {
-    const uint32_t dmask = (1u << widths[p]) - 1u;
-    topk_hist(ssrc, m, prefix, mask, shifts[p], dmask, sh);
-    topk_locate(k_rem, sh);
-    k_rem -= sh.sel_above;
-    prefix |= sh.sel_digit << shifts[p];
-    mask |= dmask << shifts[p];
-    __syncthreads();
-  }
-  const uint32_t tau = prefix;
-  if (threadIdx.x == 0) {
-    sh.n_kept = 0;
-    sh.n_cand = 0;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < n; i += THREADS) {
-    const uint32_t key = src.key(i);
-    if (key >= tau) {
-      const int slot = atomicAdd(&sh.n_cand, 1);
-      if (slot < CAP) sh.cand[slot] = ((unsigned long long)key << 32) | (0xffffffffu - src.index(i));
-    }
-  }
-  __syncthreads();
-  const int nc = sh.n_cand;
-  if (nc < K || nc > CAP) {
-    __syncthreads();
-    return false;
-  }
-  refine_and_keep(nc, K, 0u, 0u, sh);
-  return true;
-}
-
-// Selects the K best elements of src[0..n) (K <= n) under (key desc, index
-// asc).  On return sh.kept[0..K) holds their indices, in no particular order.
-__device__ void topk_select(const RowSrc& src, int n, int K, TopkShared& sh) {
-  using namespace topk;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (n > CAP && select_by_sample(src, n, K, sh)) return;
-  uint32_t prefix = 0, mask = 0;
-  int k_rem = K;
-  int bucket = n;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-  for (int p = 0; p < 3 && bucket > CAP; ++p) {
-    const uint32_t dmask = (1u << widths[p]) - 1u;
-    topk_hist(src, n, prefix, mask, shifts[p], dmask, sh);
-    topk_locate(k_rem, sh);
-    k_rem -= sh.sel_above;
-    prefix |= sh.sel_digit << shifts[p];
-    mask |= dmask << shifts[p];
-    bucket = sh.sel_count;
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
-    sh.n_kept = 0;
-    sh.n_cand = 0;
-  }
-  __syncthreads();
-  if (bucket <= CAP) {
-    // gather: above the bucket -> kept; in the bucket -> composite candidates
-    for (int i = threadIdx.x; i < n; i += THREADS) {
-      const uint32_t key = src.key(i);
-      const uint32_t mk = key & mask;
-      if (mk > prefix) {
-        sh.kept[atomicAdd(&sh.n_kept, 1)] = src.index(i);
-      } else if (mk == prefix) {
-        sh.cand[atomicAdd(&sh.n_cand, 1)] = ((unsigned long long)key << 32) | (0xffffffffu - src.index(i));
-      }
-    }
-    __syncthreads();
-    refine_and_keep(sh.n_cand, k_rem, prefix, mask, sh);
-  } else {
-    // every element of the bucket has the same key: keep the k_rem lowest
-    // indices among them, in index order, plus everything above the bucket.
-    // Element order is index order for both sources.
-    const int per = (int)cdiv(cdiv(n, WARPS), 32) * 32;
-    const int beg = warp * per, end = min(n, beg + per);
-    int n_gt = 0, n_tie = 0;
-    for (int b = beg; b < end; b += 32) {
-      const int i = b + lane;
-      const uint32_t mk = i < end ? (src.key(i) & mask) : 0u;
-      n_gt += __popc(__ballot_sync(0xffffffffu, i < end && mk > prefix));
-      n_tie += __popc(__ballot_sync(0xffffffffu, i < end && mk == prefix));
-    }
-    if (lane == 0) {
-      sh.warp_a[warp] = n_gt;
-      sh.warp_b[warp] = n_tie;
-    }
-    __syncthreads();
-    int gt_run = 0, tie_run = 0;
-    for (int w = 0; w < warp; ++w) {
-      gt_run += sh.warp_a[w];
-      tie_run += sh.warp_b[w];
-    }
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int b = beg; b < end; b += 32) {
-      const int i = b + lane;
-      const uint32_t mk = i < end ? (src.key(i) & mask) : 0u;
-      const bool gt = i < end && mk > prefix, tie = i < end && mk == prefix;
-      const uint32_t bg = __ballot_sync(0xffffffffu, gt), bt = __ballot_sync(0xffffffffu, tie);
-      const int gb = gt_run + __popc(bg & lt), tb = tie_run + __popc(bt & lt);
-      if (gt) sh.kept[gb + min(tb, k_rem)] = src.index(i);
-      else if (tie && tb < k_rem) sh.kept[gb + tb] = src.index(i);
-      gt_run += __popc(bg);
-      tie_run += __popc(bt);
-    }
-    __syncthreads();
   }
 }
 
@@ -326,63 +516,154 @@ struct TopkArgs {
   int max_ch;           // chunks per row in the workspace layout
 };
 
-// Sorts sh.kept[0..K) ascending and writes the final row: kept blocks, the
-// own block, -1 padding.
-__device__ void topk_write_final(TopkShared& sh, int K, int S, int64_t bt, int32_t* sel_row) {
-  constexpr int P = topk::KMAX;
-  for (int i = K + threadIdx.x; i < P; i += blockDim.x) sh.kept[i] = 0xffffffffu;
+// Puts sh.kept[0..K) (distinct indices in [lo, hi)) in ascending order.  A
+// bitmap of the range in the candidate buffer orders them when it fits
+// (rows up to 2^18 blocks); otherwise a bitonic sort does.
+__device__ void topk_sort_kept(TopkShared& sh, int K, int64_t lo, int64_t hi) {
+  using namespace topk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t span = hi - lo;
+  if (span > (int64_t)kBufWords * 32) {
+    constexpr int P = KMAX;
+    for (int i = K + threadIdx.x; i < P; i += blockDim.x) sh.kept[i] = 0xffffffffu;
+    __syncthreads();
+    bitonic_asc(sh.kept, P);
+    return;
+  }
+  uint32_t* bm = sh.cbuf;
+  const int nw = (int)((span + 31) >> 5);
+  for (int w = threadIdx.x; w < nw; w += THREADS) bm[w] = 0u;
   __syncthreads();
-  bitonic(sh.kept, P, false);
+  for (int i = threadIdx.x; i < K; i += THREADS) {
+    const uint32_t off = (uint32_t)(sh.kept[i] - lo);
+    atomicOr(&bm[off >> 5], 1u << (off & 31));
+  }
+  __syncthreads();
+  const int wpt = (nw + THREADS - 1) / THREADS;         // words per thread, contiguous
+  const int w0 = min(nw, (int)threadIdx.x * wpt), w1 = min(nw, w0 + wpt);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+  int incl = cnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) sh.warp_a[warp] = incl;
+  __syncthreads();
+  int pos = incl - cnt;
+  for (int w = 0; w < warp; ++w) pos += sh.warp_a[w];
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = bm[w];
+    while (bits) {
+      const int b = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (pos < KMAX) sh.kept[pos] = (uint32_t)(lo + ((int64_t)w << 5) + b);
+      ++pos;
+    }
+  }
+  __syncthreads();
+}
+
+// Writes the final row: kept blocks ascending, the own block, -1 padding.
+__device__ void topk_write_final(TopkShared& sh, int K, int S, int64_t bt, int32_t* sel_row) {
+  topk_sort_kept(sh, K, 0, bt);
   for (int i = threadIdx.x; i < S; i += blockDim.x)
     sel_row[i] = i < K ? (int32_t)sh.kept[i] : (i == K ? (int32_t)bt : -1);
 }
 
-__global__ void __launch_bounds__(topk::THREADS) topk_chunk_kernel(Geo g, SegTable st, TopkArgs a) {
-  using namespace topk;
-  __shared__ TopkShared sh;
-  const int item = blockIdx.x;
+// One row, or one chunk of a split row.
+struct TopkItem {
+  int64_t tok, bt, c0;
+  int n, c, n_ch_row;
+  bool all;            // every block in reach is kept (short context)
+  bool skip;           // nothing to do for this item
+};
+
+__device__ __forceinline__ TopkItem topk_item(const Geo& g, const SegTable& st, const TopkArgs& a, int item) {
+  TopkItem it;
   const int si = find_segment(st, item);
   const int local = item - st.item0[si];
   const int64_t pos0 = st.pos0[si];
   const int q_len = st.q_len[si];
   const int64_t nb_seg = cdiv((pos0 + q_len - 1) / g.r, a.chunk);
   const int n_ch_seg = (int)(nb_seg > 1 ? nb_seg : 1);
-  const int j = local / n_ch_seg, c = local - j * n_ch_seg;
-  const int64_t tok = st.q_offset[si] + j;
-  const int64_t t = pos0 + j;
-  const int64_t bt = t / g.r;
-  const int S = g.S, K = S - 1;
-  int32_t* sel_row = a.sel + tok * S;
+  const int j = local / n_ch_seg;
+  it.c = local - j * n_ch_seg;
+  it.tok = st.q_offset[si] + j;
+  it.bt = (pos0 + j) / g.r;
+  it.all = it.bt + 1 <= g.S;
+  it.n_ch_row = it.all ? 1 : (int)cdiv(it.bt, a.chunk);
+  it.c0 = (int64_t)it.c * a.chunk;
+  it.n = it.all ? 0 : (int)((it.bt - it.c0) < a.chunk ? (it.bt - it.c0) : a.chunk);
+  it.skip = it.all ? it.c != 0 : it.c >= it.n_ch_row;
+  return it;
+}
 
-  if (bt + 1 <= S) {                           // every block in reach is kept
-    if (c != 0) return;
-    for (int i = threadIdx.x; i < S; i += blockDim.x) sel_row[i] = (i <= bt) ? i : -1;
-    if (threadIdx.x == 0) a.nsel[tok] = (int32_t)(bt + 1);
-    return;
+// Asks the copy engine to bring a score range into L2 (16-byte granules
+// inside the range, pieces of at most 32 KiB, one per lane of the calling warp).
+__device__ __forceinline__ void prefetch_row_l2(const float* row, int n) {
+  const uintptr_t p0 = ((uintptr_t)row + 15) & ~(uintptr_t)15;
+  const uintptr_t p1 = ((uintptr_t)(row + n)) & ~(uintptr_t)15;
+  if (p1 <= p0) return;
+  constexpr uintptr_t kPiece = 32768;
+  const int lane = threadIdx.x & 31;
+  for (uintptr_t q = p0 + lane * kPiece; q < p1; q += 32 * kPiece) {
+    const uint32_t bytes = (uint32_t)((p1 - q) < kPiece ? (p1 - q) : kPiece);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(q), "r"(bytes) : "memory");
   }
-  const int n_ch_row = (int)cdiv(bt, a.chunk);
-  if (c >= n_ch_row) return;
-  const int64_t c0 = (int64_t)c * a.chunk;
-  const int n = (int)((bt - c0) < a.chunk ? (bt - c0) : a.chunk);
-  const RowSrc src{a.scores + tok * a.ld + c0, nullptr, nullptr, c0};
-  const int kk = min(n, K);
-  if (n <= K) {
-    for (int i = threadIdx.x; i < n; i += THREADS) sh.kept[i] = (uint32_t)(c0 + i);
-    __syncthreads();
-  } else {
-    topk_select(src, n, K, sh);
+}
+
+// Persistent over rows (or row chunks): while a CTA selects on one item, the
+// copy engine prefetches its next item's scores into L2.
+__global__ void __launch_bounds__(topk::THREADS, 6) topk_chunk_kernel(Geo g, SegTable st, TopkArgs a) {
+  using namespace topk;
+  __shared__ TopkShared sh;
+  const int n_items = st.item0[st.n];
+  const int S = g.S, K = S - 1;
+  if ((int)blockIdx.x < n_items && threadIdx.x < 32) {
+    const TopkItem f = topk_item(g, st, a, blockIdx.x);
+    if (!f.all && !f.skip) prefetch_row_l2(a.scores + f.tok * a.ld + f.c0, f.n);
   }
-  if (n_ch_row == 1) {
-    topk_write_final(sh, K, S, bt, sel_row);
-    if (threadIdx.x == 0) a.nsel[tok] = S;
-  } else {
-    const int64_t base = (tok * a.max_ch + c) * (int64_t)K;
-    for (int i = threadIdx.x; i < kk; i += THREADS) {
-      const uint32_t idx = sh.kept[i];
-      a.cand_idx[base + i] = (int32_t)idx;
-      a.cand_key[base + i] = score_key(a.scores[tok * a.ld + idx]);
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const TopkItem it = topk_item(g, st, a, item);
+    if (threadIdx.x < 32 && item + (int)gridDim.x < n_items) {
+      const TopkItem nx = topk_item(g, st, a, item + gridDim.x);
+      if (!nx.all && !nx.skip) prefetch_row_l2(a.scores + nx.tok * a.ld + nx.c0, nx.n);
     }
-    if (threadIdx.x == 0) a.cand_cnt[tok * a.max_ch + c] = kk;
+    if (it.skip) continue;
+    int32_t* sel_row = a.sel + it.tok * S;
+    if (it.all) {
+      for (int i = threadIdx.x; i < S; i += blockDim.x) sel_row[i] = (i <= it.bt) ? i : -1;
+      if (threadIdx.x == 0) a.nsel[it.tok] = (int32_t)(it.bt + 1);
+      continue;
+    }
+    const int64_t c0 = it.c0;
+    const int n = it.n;
+    const RowSrc src{a.scores + it.tok * a.ld + c0, nullptr, nullptr, c0};
+    const int kk = min(n, K);
+    if (n <= K) {
+      for (int i = threadIdx.x; i < n; i += THREADS) sh.kept[i] = (uint32_t)(c0 + i);
+      __syncthreads();
+    } else {
+      topk_select(src, n, K, sh);
+    }
+    if (it.n_ch_row == 1) {
+      topk_write_final(sh, K, S, it.bt, sel_row);
+      if (threadIdx.x == 0) a.nsel[it.tok] = S;
+    } else {
+      // chunk candidates in index order, so the chunk lists of a row lie in
+      // index order back to back
+      topk_sort_kept(sh, kk, c0, c0 + n);
+      const int64_t base = (it.tok * a.max_ch + it.c) * (int64_t)K;
+      for (int i = threadIdx.x; i < kk; i += THREADS) {
+        const uint32_t idx = sh.kept[i];
+        a.cand_idx[base + i] = (int32_t)idx;
+        a.cand_key[base + i] = score_key(a.scores[it.tok * a.ld + idx]);
+      }
+      if (threadIdx.x == 0) a.cand_cnt[it.tok * a.max_ch + it.c] = kk;
+    }
+    __syncthreads();                           // shared state is reused by the next item
   }
 }
 
@@ -409,8 +690,5 @@ __global__ void __launch_bounds__(topk::THREADS) topk_merge_kernel(Geo g, SegTab
   topk_write_final(sh, K, S, bt, a.sel + tok * S);
   if (threadIdx.x == 0) a.nsel[tok] = S;
 }
-
-inline size_t topk_chunk_smem(int) { return 0; }
-inline size_t topk_merge_smem(int, int) { return 0; }
 
 }  // namespace qsa
