@@ -163,35 +163,46 @@ __global__ void __launch_bounds__(simt_attn::THREADS) attn_simt_kernel(Geo g, Se
   }
 }
 
-// Log-sum-exp combine of split partials: one thread per (token, head, dim);
-// the table's item0 counts tokens per segment.
+// Log-sum-exp combine of split partials: one thread per (token, head, 4
+// dims); the table's item0 counts tokens per segment.  The loops over splits
+// are unrolled so their loads are in flight together.
 template <typename T>
 __global__ void __launch_bounds__(256) attn_combine_kernel(Geo g, SegTable st, AttnArgs a) {
-  constexpr int D = kHeadDim;
-  const int64_t total = (int64_t)st.item0[st.n] * g.H * D;
+  constexpr int D = kHeadDim, V = 4;
+  const int64_t total = (int64_t)st.item0[st.n] * g.H * (D / V);
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
-    const int d = (int)(e % D);
-    const int64_t lh = e / D;                   // local token * H + head
+    const int d = (int)(e % (D / V)) * V;
+    const int64_t lh = e / (D / V);             // local token * H + head
     const int lt = (int)(lh / g.H);
     const int hh = (int)(lh % g.H);
     const int si = find_segment(st, lt);
     const int64_t tok = st.q_offset[si] + (lt - st.item0[si]);
     const int grp = hh / g.hpg, h = hh % g.hpg;
-    const int64_t unit = tok * g.G + grp;
+    const int64_t p0 = (tok * g.G + grp) * a.n_split * g.hpg + h;   // partial of split s: p0 + s*hpg
     float m = -INFINITY;
-    for (int s = 0; s < a.n_split; ++s) m = fmaxf(m, a.part_ml[((unit * a.n_split + s) * g.hpg + h) * 2]);
-    float l = 0.f, o = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < a.n_split; ++s) m = fmaxf(m, a.part_ml[(p0 + (int64_t)s * g.hpg) * 2]);
+    float l = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
     for (int s = 0; s < a.n_split; ++s) {
-      const int64_t p = (unit * a.n_split + s) * g.hpg + h;
-      const float ms = a.part_ml[p * 2];
-      if (ms == -INFINITY) continue;
-      const float f = expf(ms - m);
-      l += a.part_ml[p * 2 + 1] * f;
-      o += a.part_o[p * D + d] * f;
+      const int64_t p = p0 + (int64_t)s * g.hpg;
+      const float2 ml = *reinterpret_cast<const float2*>(a.part_ml + p * 2);
+      const float4 po = *reinterpret_cast<const float4*>(a.part_o + p * D + d);
+      const float f = ml.x == -INFINITY ? 0.f : expf(ml.x - m);
+      l += ml.y * f;
+      o.x += po.x * f;
+      o.y += po.y * f;
+      o.z += po.z * f;
+      o.w += po.w * f;
     }
     const int64_t th = tok * g.H + hh;
-    ((T*)a.o)[th * D + d] = IO<T>::from_f(o / l);
+    T* out = (T*)a.o + th * D + d;
+    out[0] = IO<T>::from_f(o.x / l);
+    out[1] = IO<T>::from_f(o.y / l);
+    out[2] = IO<T>::from_f(o.z / l);
+    out[3] = IO<T>::from_f(o.w / l);
     if (a.lse && d == 0) a.lse[th] = m + logf(l);
   }
 }

@@ -150,30 +150,35 @@ qsa_status_t for_each_table(const qsa_segment_t* segs, int n_segs, Items items, 
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+int sm_count();
+
 // ------------------------------------------------------------------ selection plan
 struct TopkPlan {
   int chunk;
   int max_ch;      // chunks per row in the workspace (1: no split rows)
+  bool wide;       // few rows: one wide CTA per row
   size_t ws;
 };
 
-// Rows are split into chunks (local top S-1, then a merge) only when there
-// are too few rows to fill the GPU.
+// Many rows: one 4-warp CTA per row.  Few rows (too few to fill the GPU with
+// 4-warp CTAs): one 32-warp CTA per row, or, for rows beyond 2^18 blocks, a
+// split into chunks that share a sampled row threshold, then a merge.
 TopkPlan topk_plan(const Geo& g, const qsa_segment_t* segs, int n) {
-  TopkPlan p{topk::kChunkLarge, 1, 0};
+  TopkPlan p{topk::kChunkLarge, 1, false, 0};
   const int64_t nblk = seg_max_blocks(segs, n, g.r);
   const int64_t rows = seg_rows(segs, n);
   if (nblk + 1 <= g.S || rows >= 4 * kNumSms) return p;
+  if (nblk <= topk::kWideMaxBlocks) {
+    p.wide = true;
+    return p;
+  }
   p.chunk = (int)std::max<int64_t>(topk::kChunkSmall, cdiv(nblk, 32));
   p.max_ch = (int)cdiv(nblk, p.chunk);
-  if (p.max_ch > 1) {
-    int64_t T = 0;
-    for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
-    const size_t K = (size_t)(g.S - 1);
-    p.ws = align_up((size_t)T * p.max_ch * K * 4, 256) * 2 + align_up((size_t)T * p.max_ch * 4, 256);
-  } else {
-    p.chunk = topk::kChunkLarge;
-  }
+  int64_t T = 0;
+  for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
+  const size_t K = (size_t)(g.S - 1);
+  p.ws = align_up((size_t)T * p.max_ch * K * 4, 256) * 2 + align_up((size_t)T * p.max_ch * 4, 256) +
+         align_up((size_t)T * 4, 256);
   return p;
 }
 
@@ -184,16 +189,19 @@ struct AttnPlan {
   size_t ws;
 };
 
-// bf16 runs on the tensor-core kernel (splits in whole 32-block chunks),
-// fp32 on the CUDA-core kernel (8-block chunks).
+// bf16 runs on the tensor-core kernel (splits in whole 32-block chunks,
+// one CTA per SM: as many splits as keep every (query, group) split in one
+// round of CTAs), fp32 on the CUDA-core kernel (8-block chunks, several
+// CTAs per SM).
 AttnPlan attn_plan(const Geo& g, const qsa_segment_t* segs, int n, bool tc) {
   int64_t T = 0;
   for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
   const int64_t units = seg_rows(segs, n) * g.G;
   AttnPlan p{1, g.S, 0};
   const int gran = tc ? tc_attn::kBlk : simt_attn::KC / 4;
-  if (units > 0 && units < 2 * kNumSms) {
-    int ns = (int)std::min<int64_t>(cdiv(2 * kNumSms, units), cdiv(g.S, gran));
+  const int64_t slots = tc ? kNumSms : 2 * kNumSms;      // fixed: workspace sizes make no CUDA call
+  if (units > 0 && units * 2 <= slots) {
+    int ns = (int)std::min<int64_t>(tc ? slots / units : cdiv(slots, units), cdiv(g.S, gran));
     p.blocks_per_split = (int)(cdiv(cdiv(g.S, ns), gran) * gran);
     p.n_split = (int)cdiv(g.S, p.blocks_per_split);
   }
@@ -301,10 +309,30 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
     a.cand_idx = (int32_t*)base;
     base += align_up((size_t)T * p.max_ch * K * 4, 256);
     a.cand_cnt = (int32_t*)base;
+    base += align_up((size_t)T * p.max_ch * 4, 256);
+    a.row_tau = (uint32_t*)base;
   }
   const size_t smem_c = 0;
-  const int64_t nblk = seg_max_blocks(segs, n, g.r);
-  (void)nblk;
+  if (p.wide) {
+    return for_each_table(
+        segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
+        [&](const SegTable& t) {
+          count_launch();
+          topk_wide_kernel<<<t.item0[t.n], topk::kWideThreads, 0, st>>>(g, t, a);
+          return cudaGetLastError();
+        });
+  }
+  if (p.max_ch > 1) {
+    // one sampled threshold per long row, shared by its chunks
+    qsa_status_t r0 = for_each_table(
+        segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
+        [&](const SegTable& t) {
+          count_launch();
+          topk_row_threshold_kernel<<<t.item0[t.n], topk::THREADS, 0, st>>>(g, t, a);
+          return cudaGetLastError();
+        });
+    if (r0 != QSA_OK) return r0;
+  }
   qsa_status_t r = for_each_table(
       segs, n,
       [&](const qsa_segment_t& s) {
@@ -439,7 +467,7 @@ qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* ca
   return for_each_table(
       segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
       [&](const SegTable& t) {
-        const int64_t total = (int64_t)t.item0[t.n] * g.H * kHeadDim;
+        const int64_t total = (int64_t)t.item0[t.n] * g.H * (kHeadDim / 4);
         const unsigned blocks = (unsigned)std::min<int64_t>(cdiv(total, 256), kNumSms * 32);
         if (bf) { count_launch(); attn_combine_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(g, t, a); }
         else { count_launch(); attn_combine_kernel<float><<<blocks, 256, 0, st>>>(g, t, a); }

@@ -6,18 +6,19 @@
 // always kept; the other S-1 are the best candidates b < floor(t/r) under
 // the total order (score descending, block index ascending), -0 == +0.
 //
-// One CTA of 4 warps per row (or per row chunk for long rows when rows are
-// few), persistent over rows, ~35 KB of shared memory so that six CTAs share
-// an SM.  Scores are compared as 32-bit keys whose unsigned order is the
-// float order.  For a row of n candidates and K = S-1:
+// One CTA per row: 4 warps, persistent over rows, ~35 KB of shared memory
+// so that six CTAs share an SM, when rows are many; 32 warps per row when
+// rows are few (rows up to 2^18 blocks).  Scores are compared as 32-bit keys
+// whose unsigned order is the float order.  For a row of n candidates and
+// K = S-1:
 //   1. threshold: m = n/16 keys (1024 .. 8192, in runs of 8 neighbours spread
 //      evenly over the row) are reduced by a radix select to the 16-bit
 //      bucket of their rank-th largest, rank chosen so that about
 //      kSampleTarget elements of the row are expected at or above the
 //      bucket's lower edge (rows of at most CAP elements take every element);
-//   2. filter: one pass over the row (16-byte streaming loads); each thread
-//      appends the elements at or above the threshold to its own 24 slots,
-//      spilling to shared overflow slots, with no coordination;
+//   2. filter: one pass over the row (16-byte loads, several per thread in
+//      flight); each thread appends the elements at or above the threshold to
+//      its own slots, spilling to shared overflow slots, with no coordination;
 //   3. if between K and CAP elements were collected, the K-th largest of the
 //      row is among them: a radix select over the candidates (8-bit digits,
 //      starting below the bits all candidates share) finds its key T and how
@@ -30,21 +31,20 @@
 // If the sampled threshold admits fewer than K or more than CAP elements, an
 // exact fallback runs: a radix select streamed over the whole row (four
 // passes), then one ordered pass that keeps everything above T and the
-// lowest-indexed elements equal to T.  Long rows are split into chunks whose
-// local top K (exact under the same order, sorted by index) are merged by a
-// second pass of the same routine over the chunk candidates.  While a CTA
-// works on one row, the copy engine prefetches its next row into L2.
+// lowest-indexed elements equal to T.  Rows longer than 2^18 blocks, when
+// few, are split into chunks: one CTA per row computes the row's sampled
+// threshold, one CTA per chunk writes the chunk's elements at or above it,
+// and a merge runs steps 3-4 on the union (or the exact fallback).
 #pragma once
 #include "qsa_internal.cuh"
 
 namespace qsa {
 namespace topk {
-constexpr int THREADS = 128;
-constexpr int WARPS = THREADS / 32;
+constexpr int THREADS = 128;               // CTA of the per-row kernel (six CTAs per SM)
+constexpr int kWideThreads = 1024;         // CTA of the kernel for few long rows (one row per SM)
 constexpr int NBINS = 256;                 // one 8-bit digit per radix pass
-constexpr int CAPL = 24;                   // candidate slots per thread
 constexpr int OVF = 1024;                  // shared overflow slots
-constexpr int CAP = CAPL * THREADS + OVF;  // candidates a row may collect (4096)
+constexpr int CAP = 4096;                  // candidates a row may collect (thread slots + overflow)
 constexpr int KMAX = kMaxBudgetBlocks;     // kept entries per row (S-1 <= 511)
 constexpr int kBufWords = 2 * CAP;         // candidate buffer, reused for the sample and the bitmap
 constexpr int kMinSamples = 1024;
@@ -53,23 +53,36 @@ constexpr int kSampleGroup = 8;            // samples are runs of 8 neighbours (
 constexpr int kSampleTarget = 1536;        // expected elements at or above the sampled threshold
 constexpr int kChunkLarge = 1 << 30;       // no split
 constexpr int kChunkSmall = 8192;
+constexpr int kWideMaxBlocks = kBufWords * 32;   // longest row one CTA orders through its bitmap (2^18)
+constexpr int kMaxSplitChunks = 64;        // chunks per split row (the plan uses 32)
 }
 
+// Per-CTA-size constants: each thread owns CAPL candidate slots.
+template <int NT>
+struct TopkCfg {
+  static constexpr int THREADS = NT;
+  static constexpr int WARPS = NT / 32;
+  static constexpr int CAPL = (topk::CAP - topk::OVF) / NT;   // 24 at 128 threads, 3 at 1024
+  static constexpr int U = NT >= 512 ? 4 : 8;                 // 16-byte loads in flight per thread
+};
+
+template <int NT>
 struct TopkShared {
   uint32_t hist[topk::NBINS];
   uint32_t cbuf[topk::kBufWords];          // candidates | sample | bitmap
   uint32_t kept[topk::KMAX];               // kept indices / final sorted list
-  int warp_a[topk::WARPS];
-  int warp_b[topk::WARPS];
-  uint32_t warp_c[topk::WARPS];
+  int warp_a[NT / 32];
+  int warp_b[NT / 32];
+  uint32_t warp_c[NT / 32];
   int n_kept, n_ovf;
   uint32_t sel_digit;
   int sel_above, sel_count;
-  // candidate slot s of thread t: lkey[s * THREADS + t]; overflow slot o: okey[o]
+  // candidate slot s of thread t: lkey[s * NT + t]; overflow slot o: okey[o]
+  static constexpr int kSlots = TopkCfg<NT>::CAPL * NT;
   __device__ __forceinline__ uint32_t* lkey() { return cbuf; }
-  __device__ __forceinline__ uint32_t* lidx() { return cbuf + topk::CAPL * topk::THREADS; }
-  __device__ __forceinline__ uint32_t* okey() { return cbuf + 2 * topk::CAPL * topk::THREADS; }
-  __device__ __forceinline__ uint32_t* oidx() { return cbuf + 2 * topk::CAPL * topk::THREADS + topk::OVF; }
+  __device__ __forceinline__ uint32_t* lidx() { return cbuf + kSlots; }
+  __device__ __forceinline__ uint32_t* okey() { return cbuf + 2 * kSlots; }
+  __device__ __forceinline__ uint32_t* oidx() { return cbuf + 2 * kSlots + topk::OVF; }
 };
 
 // Source of one selection: element i has key(i) and index index(i); element
@@ -96,19 +109,44 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
 }
 
 // ---------------------------------------------------------------- block reductions
-__device__ __forceinline__ int block_sum(int v, TopkShared& sh) {
+template <int NT>
+__device__ __forceinline__ int block_sum(int v, TopkShared<NT>& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   v = __reduce_add_sync(0xffffffffu, v);
   if (lane == 0) sh.warp_b[warp] = v;
   __syncthreads();
   int t = 0;
 #pragma unroll
-  for (int w = 0; w < topk::WARPS; ++w) t += sh.warp_b[w];
+  for (int w = 0; w < TopkCfg<NT>::WARPS; ++w) t += sh.warp_b[w];
   __syncthreads();
   return t;
 }
 
-__device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, TopkShared& sh) {
+// Exclusive prefix sum of v over the block (thread order); *total = sum.
+template <int NT>
+__device__ __forceinline__ int block_exscan(int v, int* total, TopkShared<NT>& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  if (lane == 31) sh.warp_b[warp] = incl;
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < TopkCfg<NT>::WARPS; ++w) {
+    if (w < warp) before += sh.warp_b[w];
+    all += sh.warp_b[w];
+  }
+  __syncthreads();
+  *total = all;
+  return before + incl - v;
+}
+
+template <int NT>
+__device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, TopkShared<NT>& sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   lo = __reduce_min_sync(0xffffffffu, lo);
   hi = __reduce_max_sync(0xffffffffu, hi);
@@ -118,7 +156,7 @@ __device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, TopkSha
   }
   __syncthreads();
 #pragma unroll
-  for (int w = 0; w < topk::WARPS; ++w) {
+  for (int w = 0; w < TopkCfg<NT>::WARPS; ++w) {
     lo = min(lo, sh.warp_c[w]);
     hi = max(hi, (uint32_t)sh.warp_a[w]);
   }
@@ -126,14 +164,16 @@ __device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, TopkSha
 }
 
 // ---------------------------------------------------------------- radix helpers
-__device__ __forceinline__ void hist_clear(TopkShared& sh) {
-  for (int i = threadIdx.x; i < topk::NBINS; i += topk::THREADS) sh.hist[i] = 0;
+template <int NT>
+__device__ __forceinline__ void hist_clear(TopkShared<NT>& sh) {
+  for (int i = threadIdx.x; i < topk::NBINS; i += NT) sh.hist[i] = 0;
 }
 
 // Adds element (key, valid) to the histogram of digit (key >> shift) & 255.
 // The top digit of keys of similar magnitude is shared by most of a warp, so
 // that pass aggregates equal digits into one shared atomic.
-__device__ __forceinline__ void hist_add(uint32_t key, bool valid, int shift, bool aggregate, TopkShared& sh) {
+template <int NT>
+__device__ __forceinline__ void hist_add(uint32_t key, bool valid, int shift, bool aggregate, TopkShared<NT>& sh) {
   const int lane = threadIdx.x & 31;
   const uint32_t digit = (key >> shift) & 255u;
   if (aggregate) {
@@ -147,36 +187,44 @@ __device__ __forceinline__ void hist_add(uint32_t key, bool valid, int shift, bo
 // Finds the digit whose bucket holds the k_rem-th largest element: sets
 // sh.sel_digit, sh.sel_above (count in higher buckets), sh.sel_count.
 // Ends with a barrier.
-__device__ void hist_locate(int k_rem, TopkShared& sh) {
+template <int NT>
+__device__ void hist_locate(int k_rem, TopkShared<NT>& sh) {
   using namespace topk;
-  constexpr int PER = NBINS / THREADS;
+  constexpr int PER = NBINS >= NT ? NBINS / NT : 1;   // bins per thread
+  constexpr int ACT = NBINS / PER;                    // threads holding bins
+  constexpr int AW = (ACT + 31) / 32;                 // warps holding bins
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool act = (int)threadIdx.x < ACT;
   int local = 0;
+  if (act) {
 #pragma unroll
-  for (int j = 0; j < PER; ++j) local += sh.hist[threadIdx.x * PER + j];
+    for (int j = 0; j < PER; ++j) local += sh.hist[threadIdx.x * PER + j];
+  }
   int suf = local;                       // sum over this and higher threads of the warp
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int v = __shfl_down_sync(0xffffffffu, suf, off);
     if (lane + off < 32) suf += v;
   }
-  if (lane == 0) sh.warp_a[warp] = suf;
+  if (lane == 0 && warp < AW) sh.warp_a[warp] = suf;
   __syncthreads();
-  int above_warps = 0;
-  for (int w = warp + 1; w < WARPS; ++w) above_warps += sh.warp_a[w];
-  const int incl = suf + above_warps, excl = incl - local;
-  if (excl < k_rem && k_rem <= incl) {
-    int above = excl;
-    for (int j = PER - 1; j >= 0; --j) {
-      const int b = threadIdx.x * PER + j;
-      const int c = (int)sh.hist[b];
-      if (above + c >= k_rem) {
-        sh.sel_digit = (uint32_t)b;
-        sh.sel_above = above;
-        sh.sel_count = c;
-        break;
+  if (act) {
+    int above_warps = 0;
+    for (int w = warp + 1; w < AW; ++w) above_warps += sh.warp_a[w];
+    const int incl = suf + above_warps, excl = incl - local;
+    if (excl < k_rem && k_rem <= incl) {
+      int above = excl;
+      for (int j = PER - 1; j >= 0; --j) {
+        const int b = threadIdx.x * PER + j;
+        const int c = (int)sh.hist[b];
+        if (above + c >= k_rem) {
+          sh.sel_digit = (uint32_t)b;
+          sh.sel_above = above;
+          sh.sel_count = c;
+          break;
+        }
+        above += c;
       }
-      above += c;
     }
   }
   __syncthreads();
@@ -187,8 +235,8 @@ __device__ void hist_locate(int k_rem, TopkShared& sh) {
 // last_shift.  Returns the value with the bits below last_shift cleared;
 // *above = how many values are larger in the resolved bits, *equal = how
 // many share them (with last_shift = 0: strictly larger, and equal).
-template <class Val, class Ok>
-__device__ uint32_t radix_select(int n, int k, Val val, Ok ok, int* above, int* equal, TopkShared& sh,
+template <int NT, class Val, class Ok>
+__device__ uint32_t radix_select(int n, int k, Val val, Ok ok, int* above, int* equal, TopkShared<NT>& sh,
                                  int last_shift = 0) {
   using namespace topk;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -197,7 +245,7 @@ __device__ uint32_t radix_select(int n, int k, Val val, Ok ok, int* above, int* 
   for (int shift = 24; shift >= last_shift; shift -= 8) {
     hist_clear(sh);
     __syncthreads();
-    for (int b = warp * 32; b < n; b += THREADS) {
+    for (int b = warp * 32; b < n; b += NT) {
       const int i = b + lane;
       const bool in = i < n && ok(i);
       const uint32_t v = in ? val(i) : 0u;
@@ -218,7 +266,8 @@ __device__ uint32_t radix_select(int n, int k, Val val, Ok ok, int* above, int* 
 }
 
 // Appends idx to sh.kept when `take` (warp-aggregated; every lane calls it).
-__device__ __forceinline__ void keep_if(bool take, uint32_t idx, TopkShared& sh) {
+template <int NT>
+__device__ __forceinline__ void keep_if(bool take, uint32_t idx, TopkShared<NT>& sh) {
   const int lane = threadIdx.x & 31;
   const uint32_t m = __ballot_sync(0xffffffffu, take);
   if (m == 0) return;
@@ -233,11 +282,12 @@ __device__ __forceinline__ void keep_if(bool take, uint32_t idx, TopkShared& sh)
 // Each thread appends the candidates it finds to its own slots (no
 // coordination); past CAPL they go to the shared overflow slots.  `cnt`
 // counts every candidate of the thread.
-__device__ __forceinline__ void cand_append(uint32_t key, uint32_t idx, int& cnt, TopkShared& sh) {
+template <int NT>
+__device__ __forceinline__ void cand_append(uint32_t key, uint32_t idx, int& cnt, TopkShared<NT>& sh) {
   using namespace topk;
-  if (cnt < CAPL) {
-    sh.lkey()[cnt * THREADS + threadIdx.x] = key;
-    sh.lidx()[cnt * THREADS + threadIdx.x] = idx;
+  if (cnt < TopkCfg<NT>::CAPL) {
+    sh.lkey()[cnt * NT + threadIdx.x] = key;
+    sh.lidx()[cnt * NT + threadIdx.x] = idx;
   } else {
     const int o = atomicAdd(&sh.n_ovf, 1);
     if (o < OVF) {
@@ -251,18 +301,18 @@ __device__ __forceinline__ void cand_append(uint32_t key, uint32_t idx, int& cnt
 // Calls f(key, idx, valid) for this thread's candidates in a loop whose trip
 // count is uniform across the warp (own slots, then a strided share of the
 // overflow slots).
-template <class F>
-__device__ __forceinline__ void cand_for_each(int cnt, TopkShared& sh, F f) {
+template <int NT, class F>
+__device__ __forceinline__ void cand_for_each(int cnt, TopkShared<NT>& sh, F f) {
   using namespace topk;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int mine = min(cnt, CAPL);
+  const int mine = min(cnt, TopkCfg<NT>::CAPL);
   const int wmax = __reduce_max_sync(0xffffffffu, mine);
   for (int s = 0; s < wmax; ++s) {
     const bool v = s < mine;
-    f(v ? sh.lkey()[s * THREADS + threadIdx.x] : 0u, v ? sh.lidx()[s * THREADS + threadIdx.x] : 0u, v);
+    f(v ? sh.lkey()[s * NT + threadIdx.x] : 0u, v ? sh.lidx()[s * NT + threadIdx.x] : 0u, v);
   }
   const int no = min(sh.n_ovf, OVF);
-  for (int b = warp * 32; b < no; b += THREADS) {
+  for (int b = warp * 32; b < no; b += NT) {
     const int o = b + lane;
     const bool v = o < no;
     f(v ? sh.okey()[o] : 0u, v ? sh.oidx()[o] : 0u, v);
@@ -273,8 +323,8 @@ __device__ __forceinline__ void cand_for_each(int cnt, TopkShared& sh, F f) {
 // with ok(key, idx).  The passes start below the common high bits of the
 // smallest and largest participating value.  Returns the value; *above =
 // how many are larger, *equal = how many equal it.
-template <class Val, class Ok>
-__device__ uint32_t cand_radix(int cnt, int k, Val val, Ok ok, int* above, int* equal, TopkShared& sh) {
+template <int NT, class Val, class Ok>
+__device__ uint32_t cand_radix(int cnt, int k, Val val, Ok ok, int* above, int* equal, TopkShared<NT>& sh) {
   uint32_t vmin = 0xffffffffu, vmax = 0u;
   int n_ok = 0;
   cand_for_each(cnt, sh, [&](uint32_t key, uint32_t idx, bool v) {
@@ -324,7 +374,8 @@ __device__ uint32_t cand_radix(int cnt, int k, Val val, Ok ok, int* above, int* 
 // Exact selection over the collected candidates, which hold every element of
 // the row whose key is >= the K-th largest key: appends the indices of the K
 // best (key desc, index asc) to sh.kept.
-__device__ void select_candidates(int cnt, int K, TopkShared& sh) {
+template <int NT>
+__device__ void select_candidates(int cnt, int K, TopkShared<NT>& sh) {
   int above, equal;
   const uint32_t T = cand_radix(
       cnt, K, [](uint32_t k, uint32_t) { return k; }, [](uint32_t, uint32_t) { return true; }, &above, &equal,
@@ -348,7 +399,8 @@ __device__ void select_candidates(int cnt, int K, TopkShared& sh) {
 // Exact fallback streamed over the whole source (any n >= K): four radix
 // passes over global memory, then one pass in element (= index) order that
 // keeps every element above T and the lowest-indexed ones equal to T.
-__device__ void select_streamed(const RowSrc& src, int n, int K, TopkShared& sh) {
+template <int NT>
+__device__ void select_streamed(const RowSrc& src, int n, int K, TopkShared<NT>& sh) {
   using namespace topk;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int above, equal;
@@ -356,7 +408,7 @@ __device__ void select_streamed(const RowSrc& src, int n, int K, TopkShared& sh)
       n, K, [&](int i) { return src.key(i); }, [](int) { return true; }, &above, &equal, sh);
   const int need = K - above;
   // ties in index order: warp w owns a contiguous range of elements
-  const int per = (int)cdiv(cdiv(n, WARPS), 32) * 32;
+  const int per = (int)cdiv(cdiv(n, TopkCfg<NT>::WARPS), 32) * 32;
   const int beg = warp * per, end = min(n, beg + per);
   int n_tie = 0;
   for (int b = beg; b < end; b += 32) {
@@ -383,7 +435,8 @@ __device__ void select_streamed(const RowSrc& src, int n, int K, TopkShared& sh)
 // Filter pass of a score row: every element with score >= tau (as floats,
 // which matches key >= key(tau)) becomes a candidate of the thread that
 // reads it.  16-byte streaming loads over the aligned middle of the row.
-__device__ void filter_scores(const float* row, int64_t base, int n, float tau, int& cnt, TopkShared& sh) {
+template <int NT>
+__device__ void filter_scores(const float* row, int64_t base, int n, float tau, int& cnt, TopkShared<NT>& sh) {
   using namespace topk;
   const int align_head = (int)(((16 - ((uintptr_t)row & 15)) & 15) / 4);
   const int head = align_head < n ? align_head : n;
@@ -398,12 +451,12 @@ __device__ void filter_scores(const float* row, int64_t base, int n, float tau, 
     if (s >= tau) cand_append(score_key(s), (uint32_t)(base + i), cnt, sh);
   }
   const float4* v4 = reinterpret_cast<const float4*>(row + head);
-  constexpr int U = 4;
-  for (int v0 = threadIdx.x; v0 < nvec; v0 += U * THREADS) {
+  constexpr int U = TopkCfg<NT>::U;
+  for (int v0 = threadIdx.x; v0 < nvec; v0 += U * NT) {
     float4 x[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int v = v0 + u * THREADS;
+      const int v = v0 + u * NT;
       x[u] = v < nvec ? __ldg(v4 + v) : make_float4(NAN, NAN, NAN, NAN);   // NaN never passes
     }
     // hits of this thread's 4U elements as a bit mask; most threads have
@@ -417,41 +470,49 @@ __device__ void filter_scores(const float* row, int64_t base, int n, float tau, 
     while (hm) {
       const int b = __ffs(hm) - 1;
       hm &= hm - 1u;
-      const int i = head + 4 * (v0 + (b >> 2) * THREADS) + (b & 3);
+      const int i = head + 4 * (v0 + (b >> 2) * NT) + (b & 3);
       cand_append(score_key(__ldg(row + i)), (uint32_t)(base + i), cnt, sh);
     }
   }
 }
 
+// Sampled threshold of src[0..n) (n > CAP): m keys in runs of kSampleGroup
+// neighbours spread evenly over the source are reduced to the lower edge of
+// the 16-bit bucket of their rank-th largest, rank chosen so that about
+// kSampleTarget elements of the source are expected at or above it.  The
+// result depends only on the source, so CTAs sharing a row agree on it.
+// Ends with a barrier.
+template <int NT>
+__device__ uint32_t sampled_threshold(const RowSrc& src, int n, TopkShared<NT>& sh) {
+  using namespace topk;
+  const int m0 = n / 16 < kMinSamples ? kMinSamples : (n / 16 > kMaxSamples ? kMaxSamples : n / 16);
+  const int groups = m0 / kSampleGroup;
+  const int m = groups * kSampleGroup;
+  // group gi starts at gi*(n-8)/(groups-1) <= n-8, so every position is < n
+#pragma unroll 8
+  for (int s = threadIdx.x; s < m; s += NT) {
+    const int gi = s / kSampleGroup, j = s - gi * kSampleGroup;
+    const int64_t pos = (int64_t)gi * (n - kSampleGroup) / (groups - 1) + j;
+    sh.cbuf[s] = src.key((int)pos);
+  }
+  __syncthreads();
+  const int rank = max(1, (int)((int64_t)m * kSampleTarget / n));
+  int a0, e0;
+  return radix_select(
+      m, rank, [&](int i) { return sh.cbuf[i]; }, [](int) { return true; }, &a0, &e0, sh, 16);
+}
+
 // Selects the K best elements of src[0..n) (K <= n) under (key desc, index
 // asc).  On return sh.kept[0..K) holds their indices, in no particular order.
-__device__ void topk_select(const RowSrc& src, int n, int K, TopkShared& sh) {
+template <int NT>
+__device__ void topk_select(const RowSrc& src, int n, int K, TopkShared<NT>& sh) {
   using namespace topk;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     sh.n_kept = 0;
     sh.n_ovf = 0;
   }
-  uint32_t tkey = 0u;                            // every key is >= 0
-  if (n > CAP) {
-    // 1. sampled threshold: m keys in runs of kSampleGroup spread over the row
-    const int m0 = n / 16 < kMinSamples ? kMinSamples : (n / 16 > kMaxSamples ? kMaxSamples : n / 16);
-    const int groups = m0 / kSampleGroup;
-    const int m = groups * kSampleGroup;
-    // group gi starts at gi*(n-8)/(groups-1) <= n-8, so every position is < n
-#pragma unroll 8
-    for (int s = threadIdx.x; s < m; s += THREADS) {
-      const int gi = s / kSampleGroup, j = s - gi * kSampleGroup;
-      const int64_t pos = (int64_t)gi * (n - kSampleGroup) / (groups - 1) + j;
-      sh.cbuf[s] = src.key((int)pos);
-    }
-    __syncthreads();
-    const int rank = max(1, (int)((int64_t)m * kSampleTarget / n));
-    int a0, e0;
-    // the lower edge of the 16-bit bucket holding the rank-th largest sample
-    tkey = radix_select(
-        m, rank, [&](int i) { return sh.cbuf[i]; }, [](int) { return true; }, &a0, &e0, sh, 16);
-  }
+  const uint32_t tkey = n > CAP ? sampled_threshold(src, n, sh) : 0u;   // 1. (every key is >= 0)
   __syncthreads();
   // 2. filter
   int cnt = 0;
@@ -460,17 +521,17 @@ __device__ void topk_select(const RowSrc& src, int n, int K, TopkShared& sh) {
   } else {
     // candidate lists of a merge: batches of loads in flight, then the appends
     constexpr int B = 8;
-    for (int i0 = threadIdx.x; i0 < n; i0 += B * THREADS) {
+    for (int i0 = threadIdx.x; i0 < n; i0 += B * NT) {
       uint32_t k[B], ix[B];
 #pragma unroll
       for (int u = 0; u < B; ++u) {
-        const int i = i0 + u * THREADS;
+        const int i = i0 + u * NT;
         k[u] = i < n ? __ldcs(src.keys + i) : 0u;
         ix[u] = i < n ? (uint32_t)__ldcs(src.idx + i) : 0u;
       }
 #pragma unroll
       for (int u = 0; u < B; ++u)
-        if (i0 + u * THREADS < n && k[u] >= tkey) cand_append(k[u], ix[u], cnt, sh);
+        if (i0 + u * NT < n && k[u] >= tkey) cand_append(k[u], ix[u], cnt, sh);
     }
   }
   __syncthreads();
@@ -512,6 +573,7 @@ struct TopkArgs {
   uint32_t* cand_key;   // [T][max_ch][S-1]   (split rows only)
   int32_t* cand_idx;    // [T][max_ch][S-1]
   int32_t* cand_cnt;    // [T][max_ch]
+  uint32_t* row_tau;    // [T] sampled threshold key of rows split into many chunks
   int chunk;            // candidates per chunk
   int max_ch;           // chunks per row in the workspace layout
 };
@@ -519,7 +581,8 @@ struct TopkArgs {
 // Puts sh.kept[0..K) (distinct indices in [lo, hi)) in ascending order.  A
 // bitmap of the range in the candidate buffer orders them when it fits
 // (rows up to 2^18 blocks); otherwise a bitonic sort does.
-__device__ void topk_sort_kept(TopkShared& sh, int K, int64_t lo, int64_t hi) {
+template <int NT>
+__device__ void topk_sort_kept(TopkShared<NT>& sh, int K, int64_t lo, int64_t hi) {
   using namespace topk;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t span = hi - lo;
@@ -532,14 +595,14 @@ __device__ void topk_sort_kept(TopkShared& sh, int K, int64_t lo, int64_t hi) {
   }
   uint32_t* bm = sh.cbuf;
   const int nw = (int)((span + 31) >> 5);
-  for (int w = threadIdx.x; w < nw; w += THREADS) bm[w] = 0u;
+  for (int w = threadIdx.x; w < nw; w += NT) bm[w] = 0u;
   __syncthreads();
-  for (int i = threadIdx.x; i < K; i += THREADS) {
+  for (int i = threadIdx.x; i < K; i += NT) {
     const uint32_t off = (uint32_t)(sh.kept[i] - lo);
     atomicOr(&bm[off >> 5], 1u << (off & 31));
   }
   __syncthreads();
-  const int wpt = (nw + THREADS - 1) / THREADS;         // words per thread, contiguous
+  const int wpt = (nw + NT - 1) / NT;         // words per thread, contiguous
   const int w0 = min(nw, (int)threadIdx.x * wpt), w1 = min(nw, w0 + wpt);
   int cnt = 0;
   for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
@@ -566,7 +629,8 @@ __device__ void topk_sort_kept(TopkShared& sh, int K, int64_t lo, int64_t hi) {
 }
 
 // Writes the final row: kept blocks ascending, the own block, -1 padding.
-__device__ void topk_write_final(TopkShared& sh, int K, int S, int64_t bt, int32_t* sel_row) {
+template <int NT>
+__device__ void topk_write_final(TopkShared<NT>& sh, int K, int S, int64_t bt, int32_t* sel_row) {
   topk_sort_kept(sh, K, 0, bt);
   for (int i = threadIdx.x; i < S; i += blockDim.x)
     sel_row[i] = i < K ? (int32_t)sh.kept[i] : (i == K ? (int32_t)bt : -1);
@@ -600,37 +664,68 @@ __device__ __forceinline__ TopkItem topk_item(const Geo& g, const SegTable& st, 
   return it;
 }
 
-// Asks the copy engine to bring a score range into L2 (16-byte granules
-// inside the range, pieces of at most 32 KiB, one per lane of the calling warp).
-__device__ __forceinline__ void prefetch_row_l2(const float* row, int n) {
-  const uintptr_t p0 = ((uintptr_t)row + 15) & ~(uintptr_t)15;
-  const uintptr_t p1 = ((uintptr_t)(row + n)) & ~(uintptr_t)15;
-  if (p1 <= p0) return;
-  constexpr uintptr_t kPiece = 32768;
-  const int lane = threadIdx.x & 31;
-  for (uintptr_t q = p0 + lane * kPiece; q < p1; q += 32 * kPiece) {
-    const uint32_t bytes = (uint32_t)((p1 - q) < kPiece ? (p1 - q) : kPiece);
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(q), "r"(bytes) : "memory");
-  }
+// Row threshold of rows split into many chunks (one CTA per row): the
+// sampled threshold of the whole row, read by every chunk of the row.
+__global__ void __launch_bounds__(topk::THREADS) topk_row_threshold_kernel(Geo g, SegTable st, TopkArgs a) {
+  using namespace topk;
+  __shared__ TopkShared<topk::THREADS> sh;
+  const int item = blockIdx.x;
+  const int si = find_segment(st, item);
+  const int j = item - st.item0[si];
+  const int64_t tok = st.q_offset[si] + j;
+  const int64_t bt = (st.pos0[si] + j) / g.r;
+  if (bt + 1 <= g.S || cdiv(bt, a.chunk) <= 1) return;
+  const RowSrc row{a.scores + tok * a.ld, nullptr, nullptr, 0};
+  const uint32_t tkey = sampled_threshold(row, (int)bt, sh);
+  if (threadIdx.x == 0) a.row_tau[tok] = tkey;
 }
 
-// Persistent over rows (or row chunks): while a CTA selects on one item, the
-// copy engine prefetches its next item's scores into L2.
+// A chunk of a row split into many chunks: every chunk element at or above
+// the row's threshold is written out, up to K per chunk (more marks the
+// chunk as overflowed with a count of -1).
+template <int NT>
+__device__ void topk_chunk_row_threshold(const Geo& g, const TopkArgs& a, const TopkItem& it, TopkShared<NT>& sh) {
+  using namespace topk;
+  const int K = g.S - 1;
+  if (threadIdx.x == 0) {
+    sh.n_kept = 0;
+    sh.n_ovf = 0;
+  }
+  const uint32_t tkey = a.row_tau[it.tok];
+  __syncthreads();
+  int cnt = 0;
+  filter_scores(a.scores + it.tok * a.ld + it.c0, it.c0, it.n, key_to_float(tkey), cnt, sh);
+  __syncthreads();
+  const int own = min(cnt, TopkCfg<NT>::CAPL);
+  int own_total;
+  const int pos = block_exscan(own, &own_total, sh);
+  const int n_ovf = sh.n_ovf;
+  const int nc = own_total + n_ovf;
+  const int64_t base = (it.tok * a.max_ch + it.c) * (int64_t)K;
+  if (nc > K || n_ovf > OVF) {
+    if (threadIdx.x == 0) a.cand_cnt[it.tok * a.max_ch + it.c] = -1;
+    return;
+  }
+  for (int s = 0; s < own; ++s) {
+    a.cand_key[base + pos + s] = sh.lkey()[s * NT + threadIdx.x];
+    a.cand_idx[base + pos + s] = (int32_t)sh.lidx()[s * NT + threadIdx.x];
+  }
+  for (int o = threadIdx.x; o < n_ovf; o += NT) {
+    a.cand_key[base + own_total + o] = sh.okey()[o];
+    a.cand_idx[base + own_total + o] = (int32_t)sh.oidx()[o];
+  }
+  if (threadIdx.x == 0) a.cand_cnt[it.tok * a.max_ch + it.c] = nc;
+}
+
+// Persistent over rows (or row chunks of split rows, which write their
+// elements at or above the row's sampled threshold).
 __global__ void __launch_bounds__(topk::THREADS, 6) topk_chunk_kernel(Geo g, SegTable st, TopkArgs a) {
   using namespace topk;
-  __shared__ TopkShared sh;
+  __shared__ TopkShared<topk::THREADS> sh;
   const int n_items = st.item0[st.n];
   const int S = g.S, K = S - 1;
-  if ((int)blockIdx.x < n_items && threadIdx.x < 32) {
-    const TopkItem f = topk_item(g, st, a, blockIdx.x);
-    if (!f.all && !f.skip) prefetch_row_l2(a.scores + f.tok * a.ld + f.c0, f.n);
-  }
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const TopkItem it = topk_item(g, st, a, item);
-    if (threadIdx.x < 32 && item + (int)gridDim.x < n_items) {
-      const TopkItem nx = topk_item(g, st, a, item + gridDim.x);
-      if (!nx.all && !nx.skip) prefetch_row_l2(a.scores + nx.tok * a.ld + nx.c0, nx.n);
-    }
     if (it.skip) continue;
     int32_t* sel_row = a.sel + it.tok * S;
     if (it.all) {
@@ -638,41 +733,52 @@ __global__ void __launch_bounds__(topk::THREADS, 6) topk_chunk_kernel(Geo g, Seg
       if (threadIdx.x == 0) a.nsel[it.tok] = (int32_t)(it.bt + 1);
       continue;
     }
-    const int64_t c0 = it.c0;
-    const int n = it.n;
-    const RowSrc src{a.scores + it.tok * a.ld + c0, nullptr, nullptr, c0};
-    const int kk = min(n, K);
-    if (n <= K) {
-      for (int i = threadIdx.x; i < n; i += THREADS) sh.kept[i] = (uint32_t)(c0 + i);
-      __syncthreads();
+    if (it.n_ch_row > 1) {
+      topk_chunk_row_threshold(g, a, it, sh);
     } else {
-      topk_select(src, n, K, sh);
-    }
-    if (it.n_ch_row == 1) {
+      const RowSrc src{a.scores + it.tok * a.ld, nullptr, nullptr, 0};
+      topk_select(src, it.n, K, sh);
       topk_write_final(sh, K, S, it.bt, sel_row);
       if (threadIdx.x == 0) a.nsel[it.tok] = S;
-    } else {
-      // chunk candidates in index order, so the chunk lists of a row lie in
-      // index order back to back
-      topk_sort_kept(sh, kk, c0, c0 + n);
-      const int64_t base = (it.tok * a.max_ch + it.c) * (int64_t)K;
-      for (int i = threadIdx.x; i < kk; i += THREADS) {
-        const uint32_t idx = sh.kept[i];
-        a.cand_idx[base + i] = (int32_t)idx;
-        a.cand_key[base + i] = score_key(a.scores[it.tok * a.ld + idx]);
-      }
-      if (threadIdx.x == 0) a.cand_cnt[it.tok * a.max_ch + it.c] = kk;
     }
     __syncthreads();                           // shared state is reused by the next item
   }
 }
 
-// Merge of split rows.  Every chunk but a row's last holds at least
-// kChunkSmall > S-1 elements and so stores exactly S-1 candidates; the
-// chunk lists therefore lie back to back, in chunk (= index) order.
+// Few long rows: one CTA of kWideThreads per row, so a handful of rows still
+// keeps many loads in flight.  Rows up to kWideMaxBlocks blocks.
+__global__ void __launch_bounds__(topk::kWideThreads, 1) topk_wide_kernel(Geo g, SegTable st, TopkArgs a) {
+  using namespace topk;
+  __shared__ TopkShared<topk::kWideThreads> sh;
+  const int S = g.S, K = S - 1;
+  const int item = blockIdx.x;
+  const int si = find_segment(st, item);
+  const int j = item - st.item0[si];
+  const int64_t tok = st.q_offset[si] + j;
+  const int64_t bt = (st.pos0[si] + j) / g.r;
+  int32_t* sel_row = a.sel + tok * S;
+  if (bt + 1 <= S) {
+    for (int i = threadIdx.x; i < S; i += blockDim.x) sel_row[i] = (i <= bt) ? i : -1;
+    if (threadIdx.x == 0) a.nsel[tok] = (int32_t)(bt + 1);
+    return;
+  }
+  const RowSrc src{a.scores + tok * a.ld, nullptr, nullptr, 0};
+  topk_select(src, (int)bt, K, sh);
+  topk_write_final(sh, K, S, bt, sel_row);
+  if (threadIdx.x == 0) a.nsel[tok] = S;
+}
+
+// Merge of split rows: the union of the chunk lists (every chunk element at
+// or above the row's threshold) holds every element of the row at or above
+// the K-th largest once it has at least K elements, so the exact selection
+// runs on the union.  A chunk that overflowed, a union
+// smaller than K or larger than the candidate buffer sends the row to the
+// exact streamed fallback over its scores.
 __global__ void __launch_bounds__(topk::THREADS) topk_merge_kernel(Geo g, SegTable st, TopkArgs a) {
   using namespace topk;
-  __shared__ TopkShared sh;
+  __shared__ TopkShared<topk::THREADS> sh;
+  __shared__ int start[kMaxSplitChunks + 1];
+  __shared__ int bad;
   const int S = g.S, K = S - 1;
   const int item = blockIdx.x;
   const int si = find_segment(st, item);
@@ -683,10 +789,65 @@ __global__ void __launch_bounds__(topk::THREADS) topk_merge_kernel(Geo g, SegTab
   if (bt + 1 <= S) return;
   const int n_ch_row = (int)cdiv(bt, a.chunk);
   if (n_ch_row <= 1) return;
-  const int n = (n_ch_row - 1) * K + a.cand_cnt[tok * a.max_ch + n_ch_row - 1];
-  const int64_t row_base = tok * a.max_ch * (int64_t)K;
-  const RowSrc src{nullptr, a.cand_key + row_base, a.cand_idx + row_base, 0};
-  topk_select(src, n, K, sh);
+  if (threadIdx.x < 32) {
+    // chunk list offsets (n_ch_row <= kMaxSplitChunks)
+    const int lane = threadIdx.x;
+    int run = 0, neg = 0;
+    for (int c0 = 0; c0 < n_ch_row; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < n_ch_row ? a.cand_cnt[tok * a.max_ch + c] : 0;
+      neg |= v < 0;
+      int incl = v < 0 ? 0 : v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += u;
+      }
+      if (c < n_ch_row) start[c + 1] = run + incl;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    neg = __any_sync(0xffffffffu, neg);
+    if (lane == 0) {
+      start[0] = 0;
+      bad = neg;
+      sh.n_kept = 0;
+      sh.n_ovf = 0;
+    }
+  }
+  __syncthreads();
+  const int total = start[n_ch_row];
+  if (bad || total < K || total > CAP) {
+    const RowSrc row{a.scores + tok * a.ld, nullptr, nullptr, 0};
+    select_streamed(row, (int)bt, K, sh);
+  } else {
+    int cnt = 0;
+    const int64_t row_base = tok * a.max_ch * (int64_t)K;
+    constexpr int B = 8;                          // loads in flight per thread
+    for (int i0 = threadIdx.x; i0 < total; i0 += B * THREADS) {
+      uint32_t k[B], ix[B];
+#pragma unroll
+      for (int u = 0; u < B; ++u) {
+        const int i = i0 + u * THREADS;
+        k[u] = 0u;
+        ix[u] = 0u;
+        if (i < total) {
+          int lo = 0, hi = n_ch_row - 1;          // chunk c with start[c] <= i < start[c+1]
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (start[mid] <= i) lo = mid; else hi = mid - 1;
+          }
+          const int64_t e = row_base + (int64_t)lo * K + (i - start[lo]);
+          k[u] = a.cand_key[e];
+          ix[u] = (uint32_t)a.cand_idx[e];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < B; ++u)
+        if (i0 + u * THREADS < total) cand_append(k[u], ix[u], cnt, sh);
+    }
+    __syncthreads();
+    select_candidates(cnt, K, sh);
+  }
   topk_write_final(sh, K, S, bt, a.sel + tok * S);
   if (threadIdx.x == 0) a.nsel[tok] = S;
 }

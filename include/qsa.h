@@ -209,7 +209,8 @@ qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cache,
  * convenience, not part of the method.
  *
  * Same arguments, results and errors as qsa_select_topk, minus the
- * workspace.  Rows long enough to be split keep their per-chunk candidates
+ * workspace.  Rows long enough to be split (beyond 2^18 candidate blocks,
+ * in a batch of few rows) keep their per-chunk candidates and row thresholds
  * in a device array built into the library, QSA_NOALLOC_SCRATCH_BYTES (16 MiB)
  * per device, held by every GPU that loads the library until the process
  * exits.  A batch whose selection needs more than that (see

@@ -42,8 +42,9 @@ def test_noalloc_selection_matches_workspace_entry_point_on_consecutive_calls():
     sh = synth.Shape()
     cfg = qsa.make_config(sh)
     S = sh.budget_blocks
-    # long decode rows are split into chunks whose candidates use the scratch
-    lengths = [262143, 65535, 300, 40000, 131071]
+    # rows beyond 2^18 blocks (when rows are few) are split into chunks whose
+    # candidates use the scratch; the shorter rows take the one-CTA path
+    lengths = [300001, 65535, 300, 40000, 524287]
     segs = qsa.make_segments([(i, 1, 4 * n + 3, 0) for i, n in enumerate(lengths)])
     T = len(lengths)
     assert qsa.workspace_size(cfg, segs, T, qsa.QSA_OP_SELECT) > 0
@@ -64,11 +65,11 @@ def test_noalloc_selection_matches_workspace_entry_point_on_consecutive_calls():
 def test_noalloc_rejects_a_batch_larger_than_its_scratch():
     sh = synth.Shape()
     cfg = qsa.make_config(sh)
-    T = 500         # 500 decode rows at 1M context, split into 32 chunks each: ~65 MB of candidates
-    segs = qsa.make_segments([(i, 1, (1 << 20) - 1, 0) for i in range(T)])
+    T = 500         # 500 decode rows at 2M context, split into 32 chunks each: ~65 MB of candidates
+    segs = qsa.make_segments([(i, 1, (1 << 21) - 1, 0) for i in range(T)])
     assert qsa.workspace_size(cfg, segs, T, qsa.QSA_OP_SELECT) > (16 << 20)
     scores = torch.zeros((1, 1), device="cuda")   # never read: rejected before any launch
     sel = torch.zeros((1, 512), dtype=torch.int32, device="cuda")
     n0 = qsa.launch_count()
-    assert _noalloc(cfg, segs, T, scores.expand(T, 262144), sel, sel[0]) == qsa.QSA_ERR_WORKSPACE
+    assert _noalloc(cfg, segs, T, scores.expand(T, 524288), sel, sel[0]) == qsa.QSA_ERR_WORKSPACE
     assert qsa.launch_count() == n0
