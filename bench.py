@@ -412,7 +412,7 @@ def measure(prep: Prepared, steps, warmup, ws, flush, peaks, clocks=None):
 KERNEL_SOURCES = {
     "attn": ["attn_tc.cuh", "sm100.cuh", "qsa_internal.cuh"],
     "index": ["index_tc.cuh", "sm100.cuh", "qsa_internal.cuh"],
-    "select": ["topk.cuh", "qsa_internal.cuh"],
+    "select": ["topk.cuh", "sm100.cuh", "qsa_internal.cuh"],
 }
 
 

@@ -32,6 +32,8 @@ struct AttnArgs {
 
 template <typename T>
 __global__ void __launch_bounds__(simt_attn::THREADS) attn_simt_kernel(Geo g, SegTable st, AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   using namespace simt_attn;
   constexpr int D = kHeadDim;
   extern __shared__ float sm[];
@@ -168,6 +170,8 @@ __global__ void __launch_bounds__(simt_attn::THREADS) attn_simt_kernel(Geo g, Se
 // are unrolled so their loads are in flight together.
 template <typename T>
 __global__ void __launch_bounds__(256) attn_combine_kernel(Geo g, SegTable st, AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int D = kHeadDim, V = 4;
   const int64_t total = (int64_t)st.item0[st.n] * g.H * (D / V);
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;

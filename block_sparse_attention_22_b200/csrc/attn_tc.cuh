@@ -181,6 +181,8 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl.tmem_base;
+  pdl_wait();                                   // the previous kernel's results are visible from here
+  pdl_trigger();
 
   if (warp < kProducers) {
     // ============================================================ producers

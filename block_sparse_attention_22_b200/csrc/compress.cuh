@@ -24,6 +24,8 @@ struct RangeTable {
 template <typename T>
 __global__ void __launch_bounds__(256) compress_keys_kernel(Geo g, RangeTable rt, const T* __restrict__ k_idx,
                                                            T* __restrict__ khat) {
+  pdl_wait();
+  pdl_trigger();
   const int DI = g.DI, half = g.rope_half, r = g.r;
   const int64_t total = rt.item0[rt.n] * DI;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
@@ -67,7 +69,8 @@ cudaError_t launch_compress(const Geo& g, const RangeTable& rt, const void* k_id
   int64_t blocks = cdiv(total, 256);
   if (blocks > 148 * 64) blocks = 148 * 64;
   count_launch();
-  compress_keys_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(g, rt, (const T*)k_idx, (T*)khat);
+  const cudaError_t e = launch_chained(compress_keys_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, st, g, rt, (const T*)k_idx, (T*)khat);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

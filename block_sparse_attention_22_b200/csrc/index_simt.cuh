@@ -47,6 +47,8 @@ template <typename T>
 __global__ void __launch_bounds__(simt_index::BT) index_scores_simt_kernel(
     Geo g, SegTable st, const T* __restrict__ q_idx, const float* __restrict__ w,
     const T* __restrict__ khat, float* __restrict__ scores, int64_t ld) {
+  pdl_wait();
+  pdl_trigger();
   using namespace simt_index;
   extern __shared__ float smem[];
   const int HI = g.HI, DI = g.DI;
@@ -112,9 +114,9 @@ cudaError_t launch_index_simt(const Geo& g, const SegTable& st, const void* q_id
   if (items == 0) return cudaSuccess;
   size_t smem = sizeof(float) * (QT * g.HI * g.DI + QT * g.HI);
   count_launch();
-  index_scores_simt_kernel<T><<<items, BT, smem, s>>>(g, st, (const T*)q_idx, w, (const T*)khat,
-                                                      scores, ld);
-  return cudaGetLastError();
+  return launch_chained(index_scores_simt_kernel<T>, dim3(items), dim3(BT), smem, s, g, st, (const T*)q_idx, w,
+                        (const T*)khat,
+                        scores, ld);
 }
 
 }  // namespace qsa

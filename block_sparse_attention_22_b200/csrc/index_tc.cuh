@@ -238,6 +238,8 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctl.tmem_base;
   const uint32_t smem_base = smem_u32(smem);
+  pdl_wait();                                   // the previous kernel's results are visible from here
+  pdl_trigger();
 
   IndexCursor cur;
   index_seek<NQ>(g, st, L, R, cur);

@@ -161,8 +161,9 @@ struct TopkPlan {
 };
 
 // Many rows: one 4-warp CTA per row.  Few rows (too few to fill the GPU with
-// 4-warp CTAs): one 32-warp CTA per row, or, for rows beyond 2^18 blocks, a
-// split into chunks that share a sampled row threshold, then a merge.
+// 4-warp CTAs): one 32-warp CTA per row while rows are short, else a split
+// into chunks (one 16-warp CTA each) that share a sampled row threshold,
+// then a merge (one 32-warp CTA per row).
 TopkPlan topk_plan(const Geo& g, const qsa_segment_t* segs, int n) {
   TopkPlan p{topk::kChunkLarge, 1, false, 0};
   const int64_t nblk = seg_max_blocks(segs, n, g.r);
@@ -177,8 +178,7 @@ TopkPlan topk_plan(const Geo& g, const qsa_segment_t* segs, int n) {
   int64_t T = 0;
   for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
   const size_t K = (size_t)(g.S - 1);
-  p.ws = align_up((size_t)T * p.max_ch * K * 4, 256) * 2 + align_up((size_t)T * p.max_ch * 4, 256) +
-         align_up((size_t)T * 4, 256);
+  p.ws = align_up((size_t)T * p.max_ch * K * 4, 256) * 2 + align_up((size_t)T * p.max_ch * 4, 256);
   return p;
 }
 
@@ -254,8 +254,7 @@ cudaError_t launch_index_tc(const Geo& g, const SegTable& t, const CUtensorMap& 
   count_launch();
   // persistent: one CTA per SM, each an equal slice of the work units
   const int grid = std::min(units, sm_count());
-  index_tc_kernel<NQ><<<grid, IndexTcCfg<NQ>::kThreads, smem, st>>>(tm, g, t, a);
-  return cudaGetLastError();
+  return launch_chained(index_tc_kernel<NQ>, dim3(grid), dim3(IndexTcCfg<NQ>::kThreads), smem, st, tm, g, t, a);
 }
 
 qsa_status_t run_index(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
@@ -309,51 +308,43 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
     a.cand_idx = (int32_t*)base;
     base += align_up((size_t)T * p.max_ch * K * 4, 256);
     a.cand_cnt = (int32_t*)base;
-    base += align_up((size_t)T * p.max_ch * 4, 256);
-    a.row_tau = (uint32_t*)base;
   }
   const size_t smem_c = 0;
   if (p.wide) {
     return for_each_table(
         segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
         [&](const SegTable& t) {
+          cudaFuncSetAttribute(topk_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, topk::kWideRingBytes);
           count_launch();
-          topk_wide_kernel<<<t.item0[t.n], topk::kWideThreads, 0, st>>>(g, t, a);
-          return cudaGetLastError();
+          return launch_chained(topk_wide_kernel, dim3(t.item0[t.n]), dim3(topk::kWideThreads), topk::kWideRingBytes, st, g, t, a);
         });
   }
   if (p.max_ch > 1) {
-    // one sampled threshold per long row, shared by its chunks
-    qsa_status_t r0 = for_each_table(
+    qsa_status_t r = for_each_table(
+        segs, n,
+        [&](const qsa_segment_t& s) {
+          const int64_t nb = ((int64_t)s.pos0 + s.q_len - 1) / g.r;
+          return (int64_t)s.q_len * std::max<int64_t>(1, cdiv(nb, p.chunk));
+        },
+        [&](const SegTable& t) {
+          count_launch();
+          return launch_chained(topk_split_kernel, dim3(t.item0[t.n]), dim3(topk::kSplitThreads), 0, st, g, t, a);
+        });
+    if (r != QSA_OK) return r;
+    return for_each_table(
         segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
         [&](const SegTable& t) {
           count_launch();
-          topk_row_threshold_kernel<<<t.item0[t.n], topk::THREADS, 0, st>>>(g, t, a);
-          return cudaGetLastError();
+          return launch_chained(topk_merge_kernel, dim3(t.item0[t.n]), dim3(topk::kWideThreads), 0, st, g, t, a);
         });
-    if (r0 != QSA_OK) return r0;
   }
-  qsa_status_t r = for_each_table(
-      segs, n,
-      [&](const qsa_segment_t& s) {
-        const int64_t nb = ((int64_t)s.pos0 + s.q_len - 1) / g.r;
-        return (int64_t)s.q_len * std::max<int64_t>(1, cdiv(nb, p.chunk));
-      },
-      [&](const SegTable& t) {
-        count_launch();
-        // persistent: as many CTAs as fit (six per SM by shared memory)
-        const int grid = std::min(t.item0[t.n], 6 * sm_count());
-        topk_chunk_kernel<<<grid, topk::THREADS, smem_c, st>>>(g, t, a);
-        return cudaGetLastError();
-      });
-  if (r != QSA_OK || p.max_ch <= 1) return r;
-  const size_t smem_m = 0;
   return for_each_table(
       segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
       [&](const SegTable& t) {
         count_launch();
-        topk_merge_kernel<<<t.item0[t.n], topk::THREADS, smem_m, st>>>(g, t, a);
-        return cudaGetLastError();
+        // persistent: as many CTAs as fit (six per SM by shared memory)
+        const int grid = std::min(t.item0[t.n], 6 * sm_count());
+        return launch_chained(topk_chunk_kernel, dim3(grid), dim3(topk::THREADS), smem_c, st, g, t, a);
       });
 }
 
@@ -449,8 +440,7 @@ qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* ca
           const int64_t units = ta.units_per_group * g.G;
           const int grid = (int)std::min<int64_t>(units, sms);
           count_launch();
-          attn_tc_kernel<<<grid, tc_attn::kThreads, smem, st>>>(tq, g, t, ta);
-          return cudaGetLastError();
+          return launch_chained(attn_tc_kernel, dim3(grid), dim3(tc_attn::kThreads), smem, st, tq, g, t, ta);
         });
   } else {
     const size_t smem = attn_simt_smem();
@@ -459,7 +449,8 @@ qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* ca
         segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len * g.G * p.n_split; },
         [&](const SegTable& t) {
           count_launch();
-          attn_simt_kernel<float><<<t.item0[t.n], simt_attn::THREADS, smem, st>>>(g, t, a);
+          const cudaError_t e = launch_chained(attn_simt_kernel<float>, dim3(t.item0[t.n]), dim3(simt_attn::THREADS), smem, st, g, t, a);
+          if (e != cudaSuccess) return e;
           return cudaGetLastError();
         });
   }
@@ -469,9 +460,9 @@ qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* ca
       [&](const SegTable& t) {
         const int64_t total = (int64_t)t.item0[t.n] * g.H * (kHeadDim / 4);
         const unsigned blocks = (unsigned)std::min<int64_t>(cdiv(total, 256), kNumSms * 32);
-        if (bf) { count_launch(); attn_combine_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(g, t, a); }
-        else { count_launch(); attn_combine_kernel<float><<<blocks, 256, 0, st>>>(g, t, a); }
-        return cudaGetLastError();
+        count_launch();
+        return bf ? launch_chained(attn_combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, g, t, a)
+                  : launch_chained(attn_combine_kernel<float>, dim3(blocks), dim3(256), 0, st, g, t, a);
       });
 }
 

@@ -37,6 +37,7 @@
 // and a merge runs steps 3-4 on the union (or the exact fallback).
 #pragma once
 #include "qsa_internal.cuh"
+#include "sm100.cuh"
 
 namespace qsa {
 namespace topk {
@@ -52,9 +53,12 @@ constexpr int kMaxSamples = kBufWords;
 constexpr int kSampleGroup = 8;            // samples are runs of 8 neighbours (one 32-byte sector)
 constexpr int kSampleTarget = 1536;        // expected elements at or above the sampled threshold
 constexpr int kChunkLarge = 1 << 30;       // no split
-constexpr int kChunkSmall = 8192;
-constexpr int kWideMaxBlocks = kBufWords * 32;   // longest row one CTA orders through its bitmap (2^18)
+constexpr int kChunkSmall = 16384;         // chunk of a split row
+constexpr int kWideMaxBlocks = 32768;      // few rows up to this long: one wide CTA per row
+constexpr int kSplitThreads = 512;         // CTA of a split-row chunk
 constexpr int kMaxSplitChunks = 64;        // chunks per split row (the plan uses 32)
+constexpr int kWideStages = 8;             // cp.async slots per thread of the wide CTA
+constexpr int kWideRingBytes = kWideStages * kWideThreads * 16;
 }
 
 // Per-CTA-size constants: each thread owns CAPL candidate slots.
@@ -476,36 +480,103 @@ __device__ void filter_scores(const float* row, int64_t base, int n, float tau, 
   }
 }
 
+// filter_scores for the wide CTA: each thread streams its 16-byte pieces of
+// the row through R private shared-memory slots with cp.async, so R pieces
+// per thread are in flight without holding registers (a single CTA must keep
+// ~100 KB in flight to stream a long row at a useful rate).
+template <int NT, int R>
+__device__ void filter_scores_staged(const float* row, int64_t base, int n, float tau, int& cnt, TopkShared<NT>& sh,
+                                     float4* ring) {
+  const int align_head = (int)(((16 - ((uintptr_t)row & 15)) & 15) / 4);
+  const int head = align_head < n ? align_head : n;
+  const int nvec = (n - head) / 4;
+  const int tail0 = head + nvec * 4;
+  if ((int)threadIdx.x < head) {
+    const float s = row[threadIdx.x];
+    if (s >= tau) cand_append(score_key(s), (uint32_t)(base + threadIdx.x), cnt, sh);
+  } else if (threadIdx.x >= 32 && (int)threadIdx.x < 32 + n - tail0) {
+    const int i = tail0 + (int)threadIdx.x - 32;
+    const float s = row[i];
+    if (s >= tau) cand_append(score_key(s), (uint32_t)(base + i), cnt, sh);
+  }
+  const float4* v4 = reinterpret_cast<const float4*>(row + head);
+  const int mine = (int)threadIdx.x < nvec ? (nvec - (int)threadIdx.x + NT - 1) / NT : 0;
+#pragma unroll
+  for (int k = 0; k < R - 1; ++k) {
+    if (k < mine) sm100::cp_async16(sm100::smem_u32(ring + k * NT + threadIdx.x), v4 + threadIdx.x + k * NT, 16);
+    sm100::cp_async_commit();
+  }
+  for (int k = 0; k < mine; ++k) {
+    const int kn = k + R - 1;
+    if (kn < mine)
+      sm100::cp_async16(sm100::smem_u32(ring + (kn % R) * NT + threadIdx.x), v4 + threadIdx.x + (int64_t)kn * NT, 16);
+    sm100::cp_async_commit();
+    sm100::cp_async_wait<R - 1>();              // this thread's piece k has landed
+    const float4 x = ring[(k % R) * NT + threadIdx.x];
+    const uint32_t i0 = (uint32_t)(base + head + 4 * ((int)threadIdx.x + k * NT));
+    if (x.x >= tau) cand_append(score_key(x.x), i0 + 0, cnt, sh);
+    if (x.y >= tau) cand_append(score_key(x.y), i0 + 1, cnt, sh);
+    if (x.z >= tau) cand_append(score_key(x.z), i0 + 2, cnt, sh);
+    if (x.w >= tau) cand_append(score_key(x.w), i0 + 3, cnt, sh);
+  }
+  sm100::cp_async_wait_all();
+}
+
 // Sampled threshold of src[0..n) (n > CAP): m keys in runs of kSampleGroup
 // neighbours spread evenly over the source are reduced to the lower edge of
-// the 16-bit bucket of their rank-th largest, rank chosen so that about
-// kSampleTarget elements of the source are expected at or above it.  The
-// result depends only on the source, so CTAs sharing a row agree on it.
-// Ends with a barrier.
+// a 16-bit-wide bucket holding their rank-th largest, rank chosen so that
+// about kSampleTarget elements of the source are expected at or above it.
+// The two 8-bit radix passes start below the high bits all samples share (so
+// their digits spread over the histogram instead of piling onto a few
+// bins).  The result depends only on the source, so CTAs sharing a row agree
+// on it.  Ends with a barrier.
 template <int NT>
 __device__ uint32_t sampled_threshold(const RowSrc& src, int n, TopkShared<NT>& sh) {
   using namespace topk;
   const int m0 = n / 16 < kMinSamples ? kMinSamples : (n / 16 > kMaxSamples ? kMaxSamples : n / 16);
   const int groups = m0 / kSampleGroup;
   const int m = groups * kSampleGroup;
+  uint32_t vmin = 0xffffffffu, vmax = 0u;
   // group gi starts at gi*(n-8)/(groups-1) <= n-8, so every position is < n
 #pragma unroll 8
   for (int s = threadIdx.x; s < m; s += NT) {
     const int gi = s / kSampleGroup, j = s - gi * kSampleGroup;
     const int64_t pos = (int64_t)gi * (n - kSampleGroup) / (groups - 1) + j;
-    sh.cbuf[s] = src.key((int)pos);
+    const uint32_t k = src.key((int)pos);
+    sh.cbuf[s] = k;
+    vmin = min(vmin, k);
+    vmax = max(vmax, k);
   }
-  __syncthreads();
+  block_minmax(vmin, vmax, sh);
   const int rank = max(1, (int)((int64_t)m * kSampleTarget / n));
-  int a0, e0;
-  return radix_select(
-      m, rank, [&](int i) { return sh.cbuf[i]; }, [](int) { return true; }, &a0, &e0, sh, 16);
+  if (vmin == vmax) return vmin;
+  const int h = 31 - __clz(vmin ^ vmax);
+  uint32_t mask = h == 31 ? 0u : ~((2u << h) - 1u);
+  uint32_t prefix = vmin & mask;
+  int k_rem = rank;
+  for (int hi = h, pass = 0; hi >= 0 && pass < 2; hi -= 8, ++pass) {
+    const int lo = hi >= 7 ? hi - 7 : 0;
+    const uint32_t dm = (2u << (hi - lo)) - 1u;
+    hist_clear(sh);
+    __syncthreads();
+    for (int s = threadIdx.x; s < m; s += NT) {
+      const uint32_t x = sh.cbuf[s];
+      if ((x & mask) == prefix) atomicAdd(&sh.hist[(x >> lo) & dm], 1u);
+    }
+    __syncthreads();
+    hist_locate(k_rem, sh);
+    k_rem -= sh.sel_above;
+    prefix |= sh.sel_digit << lo;
+    mask |= dm << lo;
+    __syncthreads();
+  }
+  return prefix;
 }
 
 // Selects the K best elements of src[0..n) (K <= n) under (key desc, index
 // asc).  On return sh.kept[0..K) holds their indices, in no particular order.
 template <int NT>
-__device__ void topk_select(const RowSrc& src, int n, int K, TopkShared<NT>& sh) {
+__device__ void topk_select(const RowSrc& src, int n, int K, TopkShared<NT>& sh, float4* ring = nullptr) {
   using namespace topk;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
@@ -517,7 +588,10 @@ __device__ void topk_select(const RowSrc& src, int n, int K, TopkShared<NT>& sh)
   // 2. filter
   int cnt = 0;
   if (src.scores) {
-    filter_scores(src.scores, src.base, n, key_to_float(tkey), cnt, sh);
+    if (ring)
+      filter_scores_staged<NT, topk::kWideStages>(src.scores, src.base, n, key_to_float(tkey), cnt, sh, ring);
+    else
+      filter_scores(src.scores, src.base, n, key_to_float(tkey), cnt, sh);
   } else {
     // candidate lists of a merge: batches of loads in flight, then the appends
     constexpr int B = 8;
@@ -573,7 +647,6 @@ struct TopkArgs {
   uint32_t* cand_key;   // [T][max_ch][S-1]   (split rows only)
   int32_t* cand_idx;    // [T][max_ch][S-1]
   int32_t* cand_cnt;    // [T][max_ch]
-  uint32_t* row_tau;    // [T] sampled threshold key of rows split into many chunks
   int chunk;            // candidates per chunk
   int max_ch;           // chunks per row in the workspace layout
 };
@@ -664,25 +737,10 @@ __device__ __forceinline__ TopkItem topk_item(const Geo& g, const SegTable& st, 
   return it;
 }
 
-// Row threshold of rows split into many chunks (one CTA per row): the
-// sampled threshold of the whole row, read by every chunk of the row.
-__global__ void __launch_bounds__(topk::THREADS) topk_row_threshold_kernel(Geo g, SegTable st, TopkArgs a) {
-  using namespace topk;
-  __shared__ TopkShared<topk::THREADS> sh;
-  const int item = blockIdx.x;
-  const int si = find_segment(st, item);
-  const int j = item - st.item0[si];
-  const int64_t tok = st.q_offset[si] + j;
-  const int64_t bt = (st.pos0[si] + j) / g.r;
-  if (bt + 1 <= g.S || cdiv(bt, a.chunk) <= 1) return;
-  const RowSrc row{a.scores + tok * a.ld, nullptr, nullptr, 0};
-  const uint32_t tkey = sampled_threshold(row, (int)bt, sh);
-  if (threadIdx.x == 0) a.row_tau[tok] = tkey;
-}
-
-// A chunk of a row split into many chunks: every chunk element at or above
-// the row's threshold is written out, up to K per chunk (more marks the
-// chunk as overflowed with a count of -1).
+// A chunk of a split row: every chunk element at or above the row's sampled
+// threshold (computed by each chunk's CTA from the same sample, so all agree)
+// is written out, up to K per chunk (more marks the chunk as overflowed with
+// a count of -1).
 template <int NT>
 __device__ void topk_chunk_row_threshold(const Geo& g, const TopkArgs& a, const TopkItem& it, TopkShared<NT>& sh) {
   using namespace topk;
@@ -691,7 +749,8 @@ __device__ void topk_chunk_row_threshold(const Geo& g, const TopkArgs& a, const 
     sh.n_kept = 0;
     sh.n_ovf = 0;
   }
-  const uint32_t tkey = a.row_tau[it.tok];
+  const RowSrc row{a.scores + it.tok * a.ld, nullptr, nullptr, 0};
+  const uint32_t tkey = sampled_threshold(row, (int)it.bt, sh);
   __syncthreads();
   int cnt = 0;
   filter_scores(a.scores + it.tok * a.ld + it.c0, it.c0, it.n, key_to_float(tkey), cnt, sh);
@@ -717,10 +776,11 @@ __device__ void topk_chunk_row_threshold(const Geo& g, const TopkArgs& a, const 
   if (threadIdx.x == 0) a.cand_cnt[it.tok * a.max_ch + it.c] = nc;
 }
 
-// Persistent over rows (or row chunks of split rows, which write their
-// elements at or above the row's sampled threshold).
+// Many rows: persistent 4-warp CTAs, one row at a time.
 __global__ void __launch_bounds__(topk::THREADS, 6) topk_chunk_kernel(Geo g, SegTable st, TopkArgs a) {
   using namespace topk;
+  pdl_wait();
+  pdl_trigger();
   __shared__ TopkShared<topk::THREADS> sh;
   const int n_items = st.item0[st.n];
   const int S = g.S, K = S - 1;
@@ -733,23 +793,22 @@ __global__ void __launch_bounds__(topk::THREADS, 6) topk_chunk_kernel(Geo g, Seg
       if (threadIdx.x == 0) a.nsel[it.tok] = (int32_t)(it.bt + 1);
       continue;
     }
-    if (it.n_ch_row > 1) {
-      topk_chunk_row_threshold(g, a, it, sh);
-    } else {
-      const RowSrc src{a.scores + it.tok * a.ld, nullptr, nullptr, 0};
-      topk_select(src, it.n, K, sh);
-      topk_write_final(sh, K, S, it.bt, sel_row);
-      if (threadIdx.x == 0) a.nsel[it.tok] = S;
-    }
+    const RowSrc src{a.scores + it.tok * a.ld, nullptr, nullptr, 0};
+    topk_select(src, it.n, K, sh);
+    topk_write_final(sh, K, S, it.bt, sel_row);
+    if (threadIdx.x == 0) a.nsel[it.tok] = S;
     __syncthreads();                           // shared state is reused by the next item
   }
 }
 
-// Few long rows: one CTA of kWideThreads per row, so a handful of rows still
-// keeps many loads in flight.  Rows up to kWideMaxBlocks blocks.
+// Few rows, each up to kWideMaxBlocks blocks: one CTA of kWideThreads per
+// row, streaming the row through cp.async slots.
 __global__ void __launch_bounds__(topk::kWideThreads, 1) topk_wide_kernel(Geo g, SegTable st, TopkArgs a) {
   using namespace topk;
+  pdl_wait();
+  pdl_trigger();
   __shared__ TopkShared<topk::kWideThreads> sh;
+  extern __shared__ float4 ring[];              // kWideRingBytes
   const int S = g.S, K = S - 1;
   const int item = blockIdx.x;
   const int si = find_segment(st, item);
@@ -763,20 +822,50 @@ __global__ void __launch_bounds__(topk::kWideThreads, 1) topk_wide_kernel(Geo g,
     return;
   }
   const RowSrc src{a.scores + tok * a.ld, nullptr, nullptr, 0};
-  topk_select(src, (int)bt, K, sh);
+  topk_select(src, (int)bt, K, sh, ring);
   topk_write_final(sh, K, S, bt, sel_row);
   if (threadIdx.x == 0) a.nsel[tok] = S;
 }
 
-// Merge of split rows: the union of the chunk lists (every chunk element at
-// or above the row's threshold) holds every element of the row at or above
-// the K-th largest once it has at least K elements, so the exact selection
-// runs on the union.  A chunk that overflowed, a union
-// smaller than K or larger than the candidate buffer sends the row to the
-// exact streamed fallback over its scores.
-__global__ void __launch_bounds__(topk::THREADS) topk_merge_kernel(Geo g, SegTable st, TopkArgs a) {
+// Few long rows: one CTA of kSplitThreads per (row, chunk).  Rows of a
+// single chunk are selected in place; chunks of longer rows write their
+// elements at or above the row's sampled threshold for the merge.
+__global__ void __launch_bounds__(topk::kSplitThreads) topk_split_kernel(Geo g, SegTable st, TopkArgs a) {
   using namespace topk;
-  __shared__ TopkShared<topk::THREADS> sh;
+  pdl_wait();
+  pdl_trigger();
+  __shared__ TopkShared<topk::kSplitThreads> sh;
+  const int S = g.S, K = S - 1;
+  const TopkItem it = topk_item(g, st, a, blockIdx.x);
+  if (it.skip) return;
+  int32_t* sel_row = a.sel + it.tok * S;
+  if (it.all) {
+    for (int i = threadIdx.x; i < S; i += blockDim.x) sel_row[i] = (i <= it.bt) ? i : -1;
+    if (threadIdx.x == 0) a.nsel[it.tok] = (int32_t)(it.bt + 1);
+    return;
+  }
+  if (it.n_ch_row > 1) {
+    topk_chunk_row_threshold(g, a, it, sh);
+    return;
+  }
+  const RowSrc src{a.scores + it.tok * a.ld, nullptr, nullptr, 0};
+  topk_select(src, it.n, K, sh);
+  topk_write_final(sh, K, S, it.bt, sel_row);
+  if (threadIdx.x == 0) a.nsel[it.tok] = S;
+}
+
+// Merge of split rows (one CTA of kWideThreads per row): the union of the
+// chunk lists (every chunk element at or above the row's threshold) holds
+// every element of the row at or above the K-th largest once it has at
+// least K elements, so the exact selection runs on the union.  A chunk that
+// overflowed, a union smaller than K or larger than the candidate buffer
+// sends the row to the exact streamed fallback over its scores.
+__global__ void __launch_bounds__(topk::kWideThreads, 1) topk_merge_kernel(Geo g, SegTable st, TopkArgs a) {
+  using namespace topk;
+  pdl_wait();
+  pdl_trigger();
+  constexpr int NT = kWideThreads;
+  __shared__ TopkShared<NT> sh;
   __shared__ int start[kMaxSplitChunks + 1];
   __shared__ int bad;
   const int S = g.S, K = S - 1;
@@ -822,28 +911,14 @@ __global__ void __launch_bounds__(topk::THREADS) topk_merge_kernel(Geo g, SegTab
   } else {
     int cnt = 0;
     const int64_t row_base = tok * a.max_ch * (int64_t)K;
-    constexpr int B = 8;                          // loads in flight per thread
-    for (int i0 = threadIdx.x; i0 < total; i0 += B * THREADS) {
-      uint32_t k[B], ix[B];
-#pragma unroll
-      for (int u = 0; u < B; ++u) {
-        const int i = i0 + u * THREADS;
-        k[u] = 0u;
-        ix[u] = 0u;
-        if (i < total) {
-          int lo = 0, hi = n_ch_row - 1;          // chunk c with start[c] <= i < start[c+1]
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (start[mid] <= i) lo = mid; else hi = mid - 1;
-          }
-          const int64_t e = row_base + (int64_t)lo * K + (i - start[lo]);
-          k[u] = a.cand_key[e];
-          ix[u] = (uint32_t)a.cand_idx[e];
-        }
+    for (int i = threadIdx.x; i < total; i += NT) {
+      int lo = 0, hi = n_ch_row - 1;            // chunk c with start[c] <= i < start[c+1]
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (start[mid] <= i) lo = mid; else hi = mid - 1;
       }
-#pragma unroll
-      for (int u = 0; u < B; ++u)
-        if (i0 + u * THREADS < total) cand_append(k[u], ix[u], cnt, sh);
+      const int64_t e = row_base + (int64_t)lo * K + (i - start[lo]);
+      cand_append(a.cand_key[e], (uint32_t)a.cand_idx[e], cnt, sh);
     }
     __syncthreads();
     select_candidates(cnt, K, sh);

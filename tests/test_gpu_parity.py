@@ -95,9 +95,10 @@ def _score_rows(seed, lengths, tie_levels=None):
 @pytest.mark.parametrize("lengths,ties", [
     ([1, 3, 511, 512, 513, 600, 2047, 2048, 4096, 32767], None),
     ([600, 3000, 32767], 3),
-    ([32768, 40000, 65535], None),        # few rows: one wide CTA per row
+    ([20000, 32768, 3000], None),         # few rows: one wide CTA per row
+    ([32769, 40000, 65535], None),        # few long rows: chunks sharing a row threshold + merge
     ([65535, 262143], 5),
-    ([300001, 70000], 2),                 # rows beyond 2^18 blocks: chunks + row threshold + merge
+    ([300001, 70000], 2),                 # ties everywhere: chunk overflow, exact fallback
 ])
 def test_select_topk_matches_oracle_on_seeded_rows(lengths, ties):
     S = 512

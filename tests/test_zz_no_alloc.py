@@ -42,8 +42,8 @@ def test_noalloc_selection_matches_workspace_entry_point_on_consecutive_calls():
     sh = synth.Shape()
     cfg = qsa.make_config(sh)
     S = sh.budget_blocks
-    # rows beyond 2^18 blocks (when rows are few) are split into chunks whose
-    # candidates use the scratch; the shorter rows take the one-CTA path
+    # long rows (when rows are few) are split into chunks whose candidates use
+    # the scratch; the short row takes the in-place path
     lengths = [300001, 65535, 300, 40000, 524287]
     segs = qsa.make_segments([(i, 1, 4 * n + 3, 0) for i, n in enumerate(lengths)])
     T = len(lengths)
