@@ -172,10 +172,15 @@ class Prepared:
         comp_bytes = n_new_blocks * (sh.r + 1) * DI * el
         cand = bt.sum().item()
         idx_flops = 2.0 * HI * DI * cand
-        # scores: k^ rows read once per 64-query tile (L2-resident for prefill) + score writes
+        # scores: score writes + query rows; k^ of prefill-like segments (64-query tiles) is
+        # L2-resident, while decode-like segments (< 16 queries, 4-query tiles) stream their
+        # sequence's k^ from HBM once per tile of 4 consecutive queries
         idx_bytes = cand * 4 + self.T * HI * (DI * el + 4)
-        if self.T <= 64:   # decode: every query streams its whole k^ prefix from HBM
-            idx_bytes += cand * DI * el
+        for s in wl.segments:
+            if s.q_len < 16:
+                for q0 in range(0, s.q_len, 4):
+                    t_last = s.pos0 + min(q0 + 4, s.q_len) - 1
+                    idx_bytes += (t_last // sh.r) * DI * el
         sel_bytes = cand * 4 + self.T * (sh.budget_blocks + 1) * 4
         gathered = float((nsel * sh.r).sum().item()) * G * D * el * 2
         attn_bytes = gathered + self.T * H * D * el * 2 + self.T * H * 4 + self.T * (sh.budget_blocks + 1) * 4

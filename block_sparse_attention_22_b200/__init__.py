@@ -61,6 +61,7 @@ def _load():
         "qsa_sparse_attn_fwd": [C, K, S, I32, I32, P, P, P, P, P, P, SZ, P],
         "qsa_forward": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, SZ, P],
         "qsa_device_status": [P],
+        "qsa_selftest_wait_timeout": [P],
         "qsa_select_topk_noalloc": [C, S, I32, I32, P, I64, P, P, P],
     }
     for name, args in sig.items():
@@ -183,6 +184,16 @@ def qsa_forward(cfg, cache, segs, n_tokens, q, q_idx, w, o, lse=None, sel=None, 
 
 def qsa_device_status(stream=None):
     _check(get_lib().qsa_device_status(_stream(stream)), "qsa_device_status")
+
+
+def device_status(stream=None) -> int:
+    """Status code of qsa_device_status (reads and clears the device error word)."""
+    return int(get_lib().qsa_device_status(_stream(stream)))
+
+
+def qsa_selftest_wait_timeout(stream=None):
+    """Enqueue the bounded-wait diagnostic (a wait that runs out after ~0.1 s)."""
+    _check(get_lib().qsa_selftest_wait_timeout(_stream(stream)), "qsa_selftest_wait_timeout")
 
 
 def launch_count() -> int:

@@ -640,6 +640,27 @@ QSA_API qsa_status_t qsa_device_status(void* stream) {
   return QSA_OK;
 }
 
+// One thread waits, with the library's bounded wait and a short limit, for an
+// mbarrier phase that nothing completes: the wait gives up, records the
+// timeout in the error word and returns.
+__global__ void selftest_wait_kernel(long long limit_cycles) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) sm100::mbar_wait(&bar, 0, &abort_flag, limit_cycles);
+}
+
+QSA_API qsa_status_t qsa_selftest_wait_timeout(void* stream) {
+  count_launch();
+  selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(200000000LL);   // ~0.1 s
+  return cudaGetLastError() == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+}
+
 QSA_API const char* qsa_status_string(qsa_status_t status) {
   switch (status) {
     case QSA_OK: return "ok";

@@ -18,6 +18,9 @@ kv-channels 256, rotary 0.25 at base 1e7; design report, QSA item: r=4, a
                 prefill chunk at [942080, 946176) of a 90%-cached sequence
   decode_1m     the decode part of mixed_1m alone: 8 sequences x 1 decode
                 query against a 1048576-token cache
+  spec_decode_1m  8 sequences x 4 consecutive query tokens (a speculative
+                decode step) at the end of a 1048576-token cache; the 4
+                queries of a sequence share one stream of its k^
   chunk_128k    one 4096-query prefill chunk at [126976, 131072) of a
                 131072-token sequence whose prefix is cached (a ~1 GB case
                 whose K/V still exceeds L2; used for kernel profiles)
@@ -178,6 +181,19 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
         cached = [(ctx - 1) // sh.r] * n_seqs
         return Workload(name, sh, segs, n_seqs, _round_cap(ctx, sh.r), [ctx] * n_seqs, cached, needles,
                         seed if seed is not None else (6 if big else 3))
+    if name == "spec_decode_1m":
+        sh = Shape()
+        ctx = over.get("ctx", 1 << 20)
+        n_seqs = over.get("n_seqs", 8)
+        q_len = over.get("q_len", 4)
+        segs = [Segment(s, ctx - q_len, q_len) for s in range(n_seqs)]
+        needles = []
+        for s in range(n_seqs):
+            for b in _distinct_blocks(rng, (ctx - 1) // sh.r, 8):
+                needles.append((s, ctx - 1, b))
+        cached = [(ctx - q_len) // sh.r] * n_seqs
+        return Workload(name, sh, segs, n_seqs, _round_cap(ctx, sh.r), [ctx] * n_seqs, cached, needles,
+                        seed if seed is not None else 7)
     if name == "mixed_1m":
         sh = Shape()
         ctx = over.get("ctx", 1 << 20)

@@ -239,6 +239,14 @@ size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* segs, in
  * device-side waits; synchronises `stream`.  QSA_OK if no wait gave up. */
 qsa_status_t qsa_device_status(void* stream);
 
+/* Diagnostic for the failure path (the pages have no counterpart): enqueues
+ * one kernel whose thread waits, through the same bounded wait the
+ * tensor-core kernels use but with a ~0.1 s limit, on an mbarrier phase that
+ * nothing completes.  The wait gives up and records QSA_ERR_TIMEOUT in the
+ * device error word; no fault, no trap, the context stays usable.  A
+ * following qsa_device_status() returns QSA_ERR_TIMEOUT and clears it. */
+qsa_status_t qsa_selftest_wait_timeout(void* stream);
+
 /* Static description of a status code. */
 const char* qsa_status_string(qsa_status_t status);
 
