@@ -22,9 +22,13 @@ struct RangeTable {
 };
 
 template <typename T>
+// late_wait: the blocks pooled here are read by no kernel before the next
+// one in the stream (decode-like batches: every query's candidates predate
+// this step's blocks), so the pooling runs alongside the previous kernel and
+// only its exit waits for that kernel, which keeps completion order.
 __global__ void __launch_bounds__(256) compress_keys_kernel(Geo g, RangeTable rt, const T* __restrict__ k_idx,
-                                                           T* __restrict__ khat) {
-  pdl_wait();
+                                                           T* __restrict__ khat, int late_wait) {
+  if (!late_wait) pdl_wait();
   pdl_trigger();
   const int DI = g.DI, half = g.rope_half, r = g.r;
   const int64_t total = rt.item0[rt.n] * DI;
@@ -59,19 +63,19 @@ __global__ void __launch_bounds__(256) compress_keys_kernel(Geo g, RangeTable rt
       out[d] = IO<T>::from_f(m0);
     }
   }
+  if (late_wait) pdl_wait();
 }
 
 template <typename T>
 cudaError_t launch_compress(const Geo& g, const RangeTable& rt, const void* k_idx, void* khat,
-                            cudaStream_t st) {
+                            cudaStream_t st, bool late_wait = false) {
   int64_t total = rt.item0[rt.n] * g.DI;
   if (total == 0) return cudaSuccess;
   int64_t blocks = cdiv(total, 256);
   if (blocks > 148 * 64) blocks = 148 * 64;
   count_launch();
-  const cudaError_t e = launch_chained(compress_keys_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, st, g, rt, (const T*)k_idx, (T*)khat);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_chained(compress_keys_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, st, g, rt, (const T*)k_idx,
+                        (T*)khat, late_wait ? 1 : 0);
 }
 
 }  // namespace qsa

@@ -214,14 +214,14 @@ AttnPlan attn_plan(const Geo& g, const qsa_segment_t* segs, int n, bool tc) {
 // ------------------------------------------------------------------ stage launchers
 qsa_status_t run_compress(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
                           const int32_t* slots, const int64_t* b0, const int64_t* b1, int n,
-                          cudaStream_t st) {
+                          cudaStream_t st, bool late_wait = false) {
   RangeTable rt;
   memset(&rt, 0, sizeof rt);
   auto flush = [&]() -> qsa_status_t {
     if (rt.n == 0) return QSA_OK;
     cudaError_t e = c->dtype == QSA_DTYPE_BF16
-                        ? launch_compress<__nv_bfloat16>(g, rt, cache->k_idx, cache->khat, st)
-                        : launch_compress<float>(g, rt, cache->k_idx, cache->khat, st);
+                        ? launch_compress<__nv_bfloat16>(g, rt, cache->k_idx, cache->khat, st, late_wait)
+                        : launch_compress<float>(g, rt, cache->k_idx, cache->khat, st, late_wait);
     rt.n = 0;
     return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
   };
@@ -612,16 +612,27 @@ QSA_API qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cac
   // 1. pool the blocks each segment completes
   std::vector<int32_t> slots;
   std::vector<int64_t> b0, b1;
+  bool own_blocks_only = true;      // no query scores a block this step completes
   for (int i = 0; i < n_segs; ++i) {
     if (segs[i].q_len <= 0) continue;
     slots.push_back(segs[i].slot);
     b0.push_back(segs[i].pos0 / cfg->r);
     b1.push_back(((int64_t)segs[i].pos0 + segs[i].q_len) / cfg->r);
+    own_blocks_only &= ((int64_t)segs[i].pos0 + segs[i].q_len - 1) / cfg->r <= segs[i].pos0 / cfg->r;
   }
-  s = run_compress(g, cfg, cache, slots.data(), b0.data(), b1.data(), (int)slots.size(), st);
-  if (s != QSA_OK) return s;
-  // 2. indexer scores, 3. selection, 4. attention
-  if ((s = run_index(g, cfg, cache, segs, n_segs, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
+  if (own_blocks_only) {
+    // decode-like batch: the indexer reads no block pooled now, so the pooling
+    // runs alongside it (its exit still waits for the indexer)
+    if ((s = run_index(g, cfg, cache, segs, n_segs, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
+    s = run_compress(g, cfg, cache, slots.data(), b0.data(), b1.data(), (int)slots.size(), st, true);
+    if (s != QSA_OK) return s;
+  } else {
+    s = run_compress(g, cfg, cache, slots.data(), b0.data(), b1.data(), (int)slots.size(), st);
+    if (s != QSA_OK) return s;
+    // 2. indexer scores
+    if ((s = run_index(g, cfg, cache, segs, n_segs, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
+  }
+  // 3. selection, 4. attention
   if ((s = run_select(g, segs, n_segs, scores, L.ld, sel, nsel, ws + L.topk, L.attn - L.topk, st)) != QSA_OK)
     return s;
   return run_attn(g, cfg, cache, segs, n_segs, n_tokens, q, sel, nsel, o, lse, ws + L.attn, L.total - L.attn, st);
