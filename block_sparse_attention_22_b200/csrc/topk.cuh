@@ -8,7 +8,7 @@
 //
 // One CTA per row: 4 warps, persistent over rows, ~35 KB of shared memory
 // so that six CTAs share an SM, when rows are many; 32 warps per row when
-// rows are few (rows up to 2^18 blocks).  Scores are compared as 32-bit keys
+// rows are few and at most 32K blocks long.  Scores are compared as 32-bit keys
 // whose unsigned order is the float order.  For a row of n candidates and
 // K = S-1:
 //   1. threshold: m = n/16 keys (1024 .. 8192, in runs of 8 neighbours spread
@@ -31,10 +31,11 @@
 // If the sampled threshold admits fewer than K or more than CAP elements, an
 // exact fallback runs: a radix select streamed over the whole row (four
 // passes), then one ordered pass that keeps everything above T and the
-// lowest-indexed elements equal to T.  Rows longer than 2^18 blocks, when
-// few, are split into chunks: one CTA per row computes the row's sampled
-// threshold, one CTA per chunk writes the chunk's elements at or above it,
-// and a merge runs steps 3-4 on the union (or the exact fallback).
+// lowest-indexed elements equal to T.  Longer rows, when few, are split into
+// 16K-block chunks: the 16-warp CTA of each chunk derives the row's sampled
+// threshold (all chunks of a row agree on it) and writes the chunk's
+// elements at or above it, and a 32-warp merge runs steps 3-4 on the union
+// (or the exact fallback).
 #pragma once
 #include "qsa_internal.cuh"
 #include "sm100.cuh"

@@ -190,6 +190,8 @@ qsa_status_t qsa_sparse_attn_fwd(const qsa_config_t* cfg, const qsa_cache_t* cac
  *   1. qsa_compress_keys for the blocks each segment completes:
  *      [floor(pos0/r), floor((pos0+q_len)/r));
  *   2. qsa_index_scores; 3. qsa_select_topk; 4. qsa_sparse_attn_fwd.
+ * (When no query of the batch scores a block this call completes, as in
+ * decode, step 1 runs alongside step 2; the results are the same.)
  * Blocks before floor(pos0/r) must already be pooled in cache->khat.
  * sel/nsel: device outputs as in qsa_select_topk, or both NULL to keep them in
  * the workspace.  workspace >= qsa_workspace_size(..., QSA_OP_FORWARD).
@@ -209,9 +211,9 @@ qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cache,
  * convenience, not part of the method.
  *
  * Same arguments, results and errors as qsa_select_topk, minus the
- * workspace.  Rows long enough to be split (beyond 2^18 candidate blocks,
- * in a batch of few rows) keep their per-chunk candidates and row thresholds
- * in a device array built into the library, QSA_NOALLOC_SCRATCH_BYTES (16 MiB)
+ * workspace.  Rows long enough to be split (beyond 32K candidate blocks,
+ * in a batch of few rows) keep their per-chunk candidates in a device array
+ * built into the library, QSA_NOALLOC_SCRATCH_BYTES (16 MiB)
  * per device, held by every GPU that loads the library until the process
  * exits.  A batch whose selection needs more than that (see
  * qsa_workspace_size(..., QSA_OP_SELECT)) returns QSA_ERR_WORKSPACE and
