@@ -205,7 +205,9 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
   using namespace sm100;
   using C = IndexTcCfg<NQ>;
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  // 1 KiB-aligned base, offset from the shared array itself so that accesses
+  // through it stay shared-memory accesses (not generic ones)
+  unsigned char* smem = smem_raw + ((1024u - (sm100::smem_u32(smem_raw) & 1023u)) & 1023u);
   IndexTcCtl& ctl = *reinterpret_cast<IndexTcCtl*>(smem + C::kOffBar);
   volatile int* abort_flag = &ctl.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
