@@ -11,7 +11,8 @@ measured in the same run and reported beside the main line: "decode_1m"
 (the same decode queries plus a 4096-query chunk of a 90%-cached sequence).
 
 Inputs are synthetic (seeded, N(0,1) with planted needles) and resident in
-HBM before the timed region; L2 is flushed (a 256 MiB write, outside the
+HBM before the timed region; L2 is flushed (a 256 MiB write, then a 256 MiB
+read so that no dirty line is left for the step to write back; outside the
 timed events) before every timed step.  Times are CUDA events on the
 launching stream, max over ranks.  With torchrun and N > 1 every rank runs
 an independent replica of the workload on its own GPU (the method has no
@@ -190,7 +191,22 @@ class Prepared:
                                                             gathered_bytes=gathered))
 
 
-def timed(prep: Prepared, steps: int, warmup: int, flush: torch.Tensor, staged: bool):
+class L2Flush:
+    """Empties L2 between timed steps: a write of a buffer larger than L2, then
+    a read of another one, so the step starts with no useful line in L2 and
+    without a cache full of dirty lines whose write-back it would pay for."""
+
+    def __init__(self, nbytes: int = L2_FLUSH_BYTES):
+        self.w = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        self.r = torch.zeros(nbytes // 4, dtype=torch.float32, device="cuda")
+        self.sink = torch.empty((), dtype=torch.float32, device="cuda")
+
+    def zero_(self):
+        self.w.zero_()
+        torch.sum(self.r, dim=0, out=self.sink)
+
+
+def timed(prep: Prepared, steps: int, warmup: int, flush: L2Flush, staged: bool):
     """Device time of `steps` steps (ms each), L2 flushed before every step."""
     st = torch.cuda.current_stream()
     n_ev = 5 if staged else 2
@@ -492,7 +508,7 @@ def main():
 
     ws, rank = dist_setup()
     peaks = load_peaks()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     wl = synth.make_workload(args.workload)
     prep = Prepared(wl)
     clocks = ClockSampler(torch.cuda.current_device())
@@ -549,7 +565,8 @@ def main():
                            "budget_tokens": wl.shape.budget_tokens, "heads": wl.shape.n_heads,
                            "kv_groups": wl.shape.n_groups, "head_dim": wl.shape.head_dim,
                            "idx_heads": wl.shape.idx_heads, "idx_dim": wl.shape.idx_dim,
-                           "parallelism": f"replicas x{ws}", "l2": "flushed before every timed step"},
+                           "parallelism": f"replicas x{ws}",
+                           "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)"},
                 "roofline": roofline, "stages": m["stages"], "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": m["launches"], "clocks": m["clocks"]}
         line.update(extra)
