@@ -80,6 +80,8 @@ def _lib(acc="f64"):
         lib.qsa_ref_select.restype = ctypes.c_int
         lib.qsa_ref_attend.argtypes = [_C, _F, _F, _F, ctypes.c_int64, ctypes.c_int64, _I32,
                                        ctypes.c_int, _D, _D]
+        lib.qsa_ref_attend_bwd.argtypes = [_C, _F, _F, _F, ctypes.c_int64, ctypes.c_int64, _I32,
+                                           ctypes.c_int, _F, _D, _D, _D]
         lib.qsa_ref_forward.argtypes = [_C, _F, _F, _F, _I64, ctypes.c_int64, _F, _F, _F,
                                         ctypes.c_int64, _I32, _I32, _D, _D, ctypes.c_int]
         lib.qsa_ref_acc_bits.restype = ctypes.c_int
@@ -162,6 +164,27 @@ def attend(cfg: RefConfig, q, k, v, t: int, sel, nsel: int, acc="f64"):
     _lib(acc).qsa_ref_attend(ctypes.byref(cfg), pq, pk, pv, k.shape[1], t, _p(sel, _I32), nsel,
                              _p(o, _D), _p(lse, _D))
     return o, lse
+
+
+def attend_bwd(cfg: RefConfig, q, k, v, t: int, sel, nsel: int, dout, dk=None, dv=None, acc="f64"):
+    """Backward of one query's attention for the loss sum(dout * o): returns dq
+    [H, D]; adds this query's contributions to dk, dv ([G, ld, D] float64, created
+    zero if not given) and returns them too."""
+    q, pq = _f32(q)
+    k, pk = _f32(k)
+    v, pv = _f32(v)
+    dout, pdo = _f32(dout)
+    sel = np.ascontiguousarray(np.asarray(sel, dtype=np.int32))
+    dq = np.zeros((cfg.n_heads, cfg.head_dim), np.float64)
+    if dk is None:
+        dk = np.zeros(k.shape, np.float64)
+    if dv is None:
+        dv = np.zeros(v.shape, np.float64)
+    assert dk.dtype == np.float64 and dk.flags.c_contiguous and dk.shape == k.shape
+    assert dv.dtype == np.float64 and dv.flags.c_contiguous and dv.shape == v.shape
+    _lib(acc).qsa_ref_attend_bwd(ctypes.byref(cfg), pq, pk, pv, k.shape[1], t, _p(sel, _I32), nsel, pdo,
+                                 _p(dq, _D), _p(dk, _D), _p(dv, _D))
+    return dq, dk, dv
 
 
 def forward(cfg: RefConfig, q, q_idx, w, pos, k_idx, k, v, acc="f64",

@@ -282,6 +282,81 @@ void qsa_ref_attend(const qsa_ref_config* c, const float* q, const float* k,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Backward of one query's sparse attention (Miles docs "Qwen3.8-Flash-Next",  */
+/* section 1: the QSA kernel has a forward and a backward pass).  For the     */
+/* loss sum_h dout_h . o_h, with P_hj = softmax_j(scale q_h . k_j) over the     */
+/* same kept tokens as qsa_ref_attend, the derivative of softmax attention:   */
+/*   dv_j  += P_hj dout_h                                                      */
+/*   dp_hj  = dout_h . v_j,  delta_h = sum_j P_hj dp_hj                        */
+/*   ds_hj  = P_hj (dp_hj - delta_h)                                           */
+/*   dq_h   = scale sum_j ds_hj k_j,   dk_j += scale ds_hj q_h                 */
+/* q, dout: [n_heads][head_dim]; k, v: [n_groups][ld][head_dim];              */
+/* dq: out [n_heads][head_dim]; dk, dv: accumulated, [n_groups][ld][head_dim]. */
+/* ------------------------------------------------------------------------ */
+void qsa_ref_attend_bwd(const qsa_ref_config* c, const float* q, const float* k,
+                        const float* v, int64_t ld, int64_t t, const int32_t* sel,
+                        int nsel, const float* dout, double* dq, double* dk, double* dv) {
+  int H = c->n_heads, G = c->n_groups, D = c->head_dim, r = c->r;
+  int hpg = H / G;
+  int64_t maxtok = (int64_t)nsel * r;
+  acc_t* p = (acc_t*)malloc(sizeof(acc_t) * (size_t)(maxtok > 0 ? maxtok : 1));
+  acc_t* dp = (acc_t*)malloc(sizeof(acc_t) * (size_t)(maxtok > 0 ? maxtok : 1));
+  int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)(maxtok > 0 ? maxtok : 1));
+  for (int h = 0; h < H; ++h) {
+    int g = h / hpg;
+    const float* qh = q + (int64_t)h * D;
+    const float* doh = dout + (int64_t)h * D;
+    const float* kg = k + (int64_t)g * ld * D;
+    const float* vg = v + (int64_t)g * ld * D;
+    /* probabilities, as in the forward pass */
+    int64_t n = 0;
+    acc_t m = -INFINITY;
+    for (int i = 0; i < nsel; ++i) {
+      int64_t b = sel[i];
+      for (int64_t j = b * r; j < b * r + r; ++j) {
+        if (j > t) continue;
+        acc_t dot = 0;
+        for (int e = 0; e < D; ++e) dot += (acc_t)qh[e] * (acc_t)kg[j * D + e];
+        p[n] = (acc_t)c->softmax_scale * dot;
+        tok[n] = j;
+        if (p[n] > m) m = p[n];
+        ++n;
+      }
+    }
+    acc_t l = 0;
+    for (int64_t i = 0; i < n; ++i) {
+      p[i] = ACC_EXP(p[i] - m);
+      l += p[i];
+    }
+    for (int64_t i = 0; i < n; ++i) p[i] /= l;
+    /* dp and delta */
+    acc_t delta = 0;
+    for (int64_t i = 0; i < n; ++i) {
+      const float* vj = vg + tok[i] * D;
+      acc_t dot = 0;
+      for (int e = 0; e < D; ++e) dot += (acc_t)doh[e] * (acc_t)vj[e];
+      dp[i] = dot;
+      delta += p[i] * dot;
+    }
+    /* gradients */
+    for (int e = 0; e < D; ++e) dq[(int64_t)h * D + e] = 0;
+    for (int64_t i = 0; i < n; ++i) {
+      const int64_t j = tok[i];
+      const acc_t ds = p[i] * (dp[i] - delta);
+      const acc_t sds = (acc_t)c->softmax_scale * ds;
+      for (int e = 0; e < D; ++e) {
+        dq[(int64_t)h * D + e] += (double)(sds * (acc_t)kg[j * D + e]);
+        dk[((int64_t)g * ld + j) * D + e] += (double)(sds * (acc_t)qh[e]);
+        dv[((int64_t)g * ld + j) * D + e] += (double)(p[i] * (acc_t)doh[e]);
+      }
+    }
+  }
+  free(tok);
+  free(dp);
+  free(p);
+}
+
+/* ------------------------------------------------------------------------ */
 /* The whole path for nq query tokens of ONE sequence.                       */
 /* q: [nq][n_heads][head_dim]; q_idx: [nq][idx_heads][idx_dim]; w: [nq][idx_heads];
  * pos: [nq] absolute positions.  k_idx: [>= n][idx_dim]; k, v: [n_groups][ld][head_dim]

@@ -41,6 +41,9 @@ void qsa_ref_index_scores(const qsa_ref_config* c, const float* q_idx, const flo
 int qsa_ref_select(const qsa_ref_config* c, const double* s, int64_t t, int32_t* sel);
 void qsa_ref_attend(const qsa_ref_config* c, const float* q, const float* k, const float* v,
                     int64_t ld, int64_t t, const int32_t* sel, int nsel, double* o, double* lse);
+void qsa_ref_attend_bwd(const qsa_ref_config* c, const float* q, const float* k, const float* v,
+                        int64_t ld, int64_t t, const int32_t* sel, int nsel, const float* dout,
+                        double* dq, double* dk, double* dv);
 void qsa_ref_forward(const qsa_ref_config* c, const float* q, const float* q_idx, const float* w,
                      const int64_t* pos, int64_t nq, const float* k_idx, const float* k,
                      const float* v, int64_t ld, int32_t* sel, int32_t* nsel, double* o,

@@ -396,3 +396,93 @@ def test_fp32_accumulation_build_agrees_with_fp64_build():
     assert same.mean() > 0.99
     np.testing.assert_allclose(b["o"][same], a["o"][same], atol=1e-5)
     np.testing.assert_allclose(b["lse"][same], a["lse"][same], atol=1e-5)
+
+
+# --------------------------------------------------------------------------- attention backward
+def _loss(cfg, q, k, v, t, sel, nsel, dout):
+    o, _ = oracle.attend(cfg, q, k, v, t, sel, nsel)
+    return float((o * dout.astype(np.float64)).sum())
+
+
+def test_backward_matches_finite_differences_of_the_forward():
+    """Central differences of the forward oracle's loss sum(dout * o) against the
+    backward oracle, on coordinates of q, of kept keys and values, of a key outside
+    the causal range (zero gradient) and of a key not kept (zero gradient)."""
+    cfg = small_cfg(budget_tokens=12)
+    n, t = 40, 37                                  # own block 9 holds 36..39: 36, 37 attended
+    c = _rand_attn_case(21, n)
+    sel = np.array([2, 5, 9], np.int32)
+    rng = np.random.default_rng(5)
+    dout = rng.standard_normal((cfg.n_heads, cfg.head_dim)).astype(np.float32)
+    q, k, v = c["q"][t].copy(), c["k"].copy(), c["v"].copy()
+    dq, dk, dv = oracle.attend_bwd(cfg, q, k, v, t, sel, 3, dout)
+    eps = 2.0 ** -11
+
+    def fd(arr, idx):
+        x = arr[idx]
+        arr[idx] = x + eps
+        lp = _loss(cfg, q, k, v, t, sel, 3, dout)
+        arr[idx] = x - eps
+        lm = _loss(cfg, q, k, v, t, sel, 3, dout)
+        arr[idx] = x
+        return (lp - lm) / (2 * eps)
+
+    for h, d in [(0, 0), (1, 7), (3, 15), (2, 3)]:
+        np.testing.assert_allclose(fd(q, (h, d)), dq[h, d], rtol=2e-5, atol=1e-7)
+    for g, j, d in [(0, 8, 1), (1, 21, 4), (0, 36, 9), (1, 37, 15), (0, 11, 0)]:
+        np.testing.assert_allclose(fd(k, (g, j, d)), dk[g, j, d], rtol=2e-5, atol=1e-7)
+        np.testing.assert_allclose(fd(v, (g, j, d)), dv[g, j, d], rtol=2e-5, atol=1e-7)
+    # key 38 is in the own block but after t; key 12 is in a block not kept
+    for g, j in [(0, 38), (1, 38), (0, 12), (1, 12)]:
+        assert np.all(dk[g, j] == 0) and np.all(dv[g, j] == 0)
+        assert fd(k, (g, j, 3)) == 0.0 and fd(v, (g, j, 3)) == 0.0
+
+
+def test_backward_with_budget_covering_context_is_dense_attention_backward():
+    """Budget >= context: the sparse backward equals torch autograd of dense causal
+    GQA attention in fp64 (dq per query; dk, dv summed over the queries)."""
+    n = 48
+    cfg = small_cfg(budget_tokens=256)
+    c = _rand_attn_case(22, n)
+    rng = np.random.default_rng(6)
+    dout = rng.standard_normal((n, cfg.n_heads, cfg.head_dim)).astype(np.float32)
+    dk = np.zeros(c["k"].shape, np.float64)
+    dv = np.zeros(c["v"].shape, np.float64)
+    dqs = []
+    for t in range(n):
+        nb = t // 4 + 1
+        sel = np.arange(nb, dtype=np.int32)
+        dq, dk, dv = oracle.attend_bwd(cfg, c["q"][t], c["k"], c["v"], t, sel, nb, dout[t], dk, dv)
+        dqs.append(dq)
+    H, G = cfg.n_heads, cfg.n_groups
+    q = torch.from_numpy(c["q"]).double().permute(1, 0, 2).requires_grad_(True)     # [H, n, D]
+    k = torch.from_numpy(c["k"]).double().requires_grad_(True)                      # [G, n, D]
+    v = torch.from_numpy(c["v"]).double().requires_grad_(True)
+    kk = k.repeat_interleave(H // G, 0)
+    vv = v.repeat_interleave(H // G, 0)
+    s = (q @ kk.transpose(1, 2)) * cfg.softmax_scale
+    s = s.masked_fill(~torch.tril(torch.ones(n, n, dtype=torch.bool)), float("-inf"))
+    o = torch.softmax(s, -1) @ vv
+    (o * torch.from_numpy(dout).double().permute(1, 0, 2)).sum().backward()
+    np.testing.assert_allclose(np.stack(dqs), q.grad.permute(1, 0, 2).numpy(), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(dk, k.grad.numpy(), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(dv, v.grad.numpy(), rtol=1e-9, atol=1e-12)
+
+
+def test_backward_constant_values_give_zero_query_and_key_gradients():
+    """Constant V makes every dp equal to its mean: ds = 0, so dq = dk = 0, while dv
+    of each attended key is its probability times dout."""
+    cfg = small_cfg(budget_tokens=16)
+    n, t = 64, 50
+    c = _rand_attn_case(23, n)
+    c["v"][:] = 1.5
+    sel = np.array([3, 7, 11, 12], np.int32)
+    dout = np.random.default_rng(7).standard_normal((cfg.n_heads, cfg.head_dim)).astype(np.float32)
+    dq, dk, dv = oracle.attend_bwd(cfg, c["q"][t], c["k"], c["v"], t, sel, 4, dout)
+    np.testing.assert_allclose(dq, 0, atol=1e-12)
+    np.testing.assert_allclose(dk, 0, atol=1e-12)
+    # sum over attended keys of dv = (sum of probabilities) * dout per head = dout, per group
+    hpg = cfg.n_heads // cfg.n_groups
+    for g in range(cfg.n_groups):
+        np.testing.assert_allclose(dv[g].sum(0), dout[g * hpg:(g + 1) * hpg].astype(np.float64).sum(0),
+                                   rtol=1e-12, atol=1e-12)
