@@ -430,6 +430,60 @@ def measure(prep: Prepared, steps, warmup, ws, flush, peaks, clocks=None):
                 clocks=clk)
 
 
+def measure_backward(name, steps, warmup, ws, flush, peaks):
+    """qsa_sparse_attn_bwd on one workload: the forward runs once for o, lse and
+    the selection; each timed step zeroes dk/dv (outside the events) and runs the
+    backward.  Algorithmic work: five dot products of head_dim per (head, kept
+    key) -- scores, dp, and the dq, dk, dv contributions -- on CUDA cores, so the
+    roofline is the fp32 FMA peak from the unit count and clock (148 SMs x 128
+    lanes x 2 flop x 1.965 GHz)."""
+    wl = synth.make_workload(name)
+    prep = Prepared(wl)
+    prep.forward()
+    sh, x = prep.sh, prep.x
+    T = prep.T
+    g = torch.Generator(device="cuda").manual_seed(31)
+    dout = torch.randn((T, sh.n_heads, sh.head_dim), generator=g, device="cuda").to(sh.torch_dtype)
+    dq = torch.empty((T, sh.n_heads, sh.head_dim), dtype=torch.float32, device="cuda")
+    dk = torch.zeros(x["k"].shape, dtype=torch.float32, device="cuda")
+    dv = torch.zeros(x["v"].shape, dtype=torch.float32, device="cuda")
+    st = torch.cuda.current_stream()
+
+    def step():
+        qsa.qsa_sparse_attn_bwd(prep.cfg, prep.cache, prep.segs, T, x["q"], prep.o, prep.lse, dout, prep.sel,
+                                prep.nsel, dq, dk, dv)
+
+    for _ in range(warmup):
+        dk.zero_()
+        dv.zero_()
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        dk.zero_()
+        dv.zero_()
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        step()
+        e1.record(st)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = max_over_ranks(sum(times) / steps, ws)
+    pos = wl.token_positions().double()
+    keys = float((torch.clamp(torch.floor(pos / sh.r) + 1, max=sh.budget_blocks) * sh.r).sum().item())
+    flops = 10.0 * sh.head_dim * sh.n_heads * keys
+    peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    tflops = flops / (ms * 1e-3) / 1e12
+    del prep
+    torch.cuda.empty_cache()
+    return {"workload": name, "ms_per_step": ms, "tokens_per_s": job_throughput(T, ms, ws),
+            "roofline": {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak, "peak_source": "fp32 FMA lanes x clock (148 x 128 x 2 x 1.965 GHz)"}}
+
+
 KERNEL_SOURCES = {
     "attn": ["attn_tc.cuh", "sm100.cuh", "qsa_internal.cuh"],
     "index": ["index_tc.cuh", "sm100.cuh", "qsa_internal.cuh"],
@@ -497,6 +551,8 @@ def main():
     ap.add_argument("--workload", default="prefill_128k")
     ap.add_argument("--decode-workload", default="decode_1m,mixed_1m",
                     help="comma-separated extra workloads reported beside the main line; 'none' to skip")
+    ap.add_argument("--bwd-workload", default="prefill_8k",
+                    help="workload of the attention-backward measurement; 'none' to skip")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -556,6 +612,9 @@ def main():
         extra[name] = d
         del prep2
         torch.cuda.empty_cache()
+
+    if args.bwd_workload != "none":
+        extra["attn_backward"] = measure_backward(args.bwd_workload, args.steps, args.warmup, ws, flush, peaks)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,

@@ -59,6 +59,7 @@ def _load():
         "qsa_index_scores": [C, K, S, I32, I32, P, P, P, I64, P],
         "qsa_select_topk": [C, S, I32, I32, P, I64, P, P, P, SZ, P],
         "qsa_sparse_attn_fwd": [C, K, S, I32, I32, P, P, P, P, P, P, SZ, P],
+        "qsa_sparse_attn_bwd": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, P, P],
         "qsa_forward": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, SZ, P],
         "qsa_device_status": [P],
         "qsa_selftest_wait_timeout": [P],
@@ -171,6 +172,15 @@ def qsa_sparse_attn_fwd(cfg, cache, segs, n_tokens, q, sel, nsel, o, lse=None, w
     _check(get_lib().qsa_sparse_attn_fwd(ctypes.byref(cfg), ctypes.byref(cache), arr, n, n_tokens, _ptr(q),
                                    _ptr(sel), _ptr(nsel), _ptr(o), _ptr(lse), _ptr(workspace), ws_bytes,
                                    _stream(stream)), "qsa_sparse_attn_fwd")
+
+
+def qsa_sparse_attn_bwd(cfg, cache, segs, n_tokens, q, o, lse, dout, sel, nsel, dq, dk, dv, stream=None):
+    """Backward of qsa_sparse_attn_fwd: writes dq (fp32 [T,H,D]); adds into dk, dv
+    (fp32, laid out like the K/V caches)."""
+    arr, n = segs
+    _check(get_lib().qsa_sparse_attn_bwd(ctypes.byref(cfg), ctypes.byref(cache), arr, n, n_tokens, _ptr(q),
+                                         _ptr(o), _ptr(lse), _ptr(dout), _ptr(sel), _ptr(nsel), _ptr(dq),
+                                         _ptr(dk), _ptr(dv), _stream(stream)), "qsa_sparse_attn_bwd")
 
 
 def qsa_forward(cfg, cache, segs, n_tokens, q, q_idx, w, o, lse=None, sel=None, nsel=None,

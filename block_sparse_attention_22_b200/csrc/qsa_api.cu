@@ -19,6 +19,7 @@
 #include "compress.cuh"
 #include "index_simt.cuh"
 #include "topk.cuh"
+#include "attn_bwd.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "index_tc.cuh"
@@ -564,6 +565,41 @@ QSA_API qsa_status_t qsa_sparse_attn_fwd(const qsa_config_t* cfg, const qsa_cach
   const Geo g = make_geo(cfg, cache);
   return run_attn(g, cfg, cache, segs, n_segs, n_tokens, q, sel, nsel, o, lse, workspace, ws_bytes,
                   (cudaStream_t)stream);
+}
+
+QSA_API qsa_status_t qsa_sparse_attn_bwd(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                         const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                                         const void* q, const void* o, const float* lse, const void* dout,
+                                         const int32_t* sel, const int32_t* nsel, float* dq, float* dk,
+                                         float* dv, void* stream) {
+  qsa_status_t s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if ((s = check_cache(cfg, cache)) != QSA_OK) return s;
+  if ((s = check_segments(segs, n_segs, n_tokens, cache, 0)) != QSA_OK) return s;
+  if (seg_rows(segs, n_segs) == 0) return QSA_OK;
+  if (!q || !o || !lse || !dout || !sel || !nsel || !dq || !dk || !dv || !cache->k || !cache->v)
+    return QSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv) || !aligned16(cache->k) || !aligned16(cache->v))
+    return QSA_ERR_INVALID_ARG;
+  const Geo g = make_geo(cfg, cache);
+  AttnBwdArgs a{q, o, lse, dout, cache->k, cache->v, sel, nsel, dq, dk, dv};
+  const size_t smem = attn_bwd_smem();
+  const bool bf = cfg->dtype == QSA_DTYPE_BF16;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (bf)
+    cudaFuncSetAttribute(attn_bwd_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  else
+    cudaFuncSetAttribute(attn_bwd_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  return for_each_table(
+      segs, n_segs, [&](const qsa_segment_t& sg) { return (int64_t)sg.q_len * g.G; },
+      [&](const SegTable& t) {
+        count_launch();
+        return bf ? launch_chained(attn_bwd_kernel<__nv_bfloat16>, dim3(t.item0[t.n]), dim3(bwd_attn::THREADS),
+                                   smem, st, g, t, a)
+                  : launch_chained(attn_bwd_kernel<float>, dim3(t.item0[t.n]), dim3(bwd_attn::THREADS), smem,
+                                   st, g, t, a);
+      });
 }
 
 QSA_API size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* segs,

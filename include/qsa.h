@@ -184,6 +184,28 @@ qsa_status_t qsa_sparse_attn_fwd(const qsa_config_t* cfg, const qsa_cache_t* cac
                                  float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Backward of qsa_sparse_attn_fwd (Miles docs section 1: the QSA attention
+ * kernel has a forward and a backward pass over the same kept tokens).  For
+ * the loss sum over tokens and heads of dout . o, with the forward's
+ * probabilities P_hj = exp(scale q_h . k_j - lse_h) over the kept tokens:
+ *   dq_h  = scale sum_j P_hj (dout_h . v_j - dout_h . o_h) k_j
+ *   dk_j += scale sum_{t,h} P_hj (dout_h . v_j - dout_h . o_h) q_h
+ *   dv_j += sum_{t,h} P_hj dout_h
+ * q, o, dout: device [T][H][D] in the I/O dtype (o and lse as qsa_sparse_attn_fwd
+ * or qsa_forward wrote them); lse: device fp32 [T][H]; sel/nsel as the forward
+ * used them.  dq: device fp32 [T][H][D], written.  dk, dv: device fp32 arrays
+ * laid out like cache->k / cache->v ([n_slots][n_kv_groups][n_cap][head_dim]),
+ * ACCUMULATED into (fp32 atomic adds, so the order of additions and the last
+ * bits vary from run to run): zero them before the first call of a step.
+ * The indexer and the selection have no gradient here.
+ */
+qsa_status_t qsa_sparse_attn_bwd(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                 const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                                 const void* q, const void* o, const float* lse, const void* dout,
+                                 const int32_t* sel, const int32_t* nsel, float* dq, float* dk,
+                                 float* dv, void* stream);
+
+/*
  * The whole QSA forward pass for a token batch (prefill, chunked prefill over
  * a cached prefix, decode, or a mix), enqueued on one stream with no host
  * synchronisation:
