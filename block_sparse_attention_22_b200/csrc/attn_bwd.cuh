@@ -10,8 +10,9 @@
 //   dv_j += sum_h P_hj dout_h.
 // One CTA per (query token, KV group): the group's heads share the kept
 // keys, so each gathered K/V row serves all of them, and its dk/dv rows are
-// summed over the heads before one fp32 atomic add per element (keys are
-// shared by many queries, so the key gradients are accumulated in place).
+// summed over the heads before fp32 atomic adds, four elements per 16-byte
+// atomic (keys are shared by many queries, so the key gradients are
+// accumulated in place).
 // lse is the forward's natural-log normaliser, so probabilities are
 // recomputed without a second pass.
 #pragma once
@@ -154,19 +155,33 @@ __global__ void __launch_bounds__(bwd_attn::THREADS) attn_bwd_kernel(Geo g, SegT
         dq_acc[i] = fmaf(acc, g.scale, dq_acc[i]);
       }
     }
-    // dk_j += scale * sum_h ds_hj q_h ; dv_j += sum_h P_hj dout_h  (attended keys only)
-    for (int e = tid; e < KC * D; e += THREADS) {
-      const int kk = e / D, d = e % D;
+    // dk_j += scale * sum_h ds_hj q_h ; dv_j += sum_h P_hj dout_h  (attended keys only),
+    // four dims per thread and one 16-byte atomic add per tensor
+    for (int e = tid; e < KC * D / 4; e += THREADS) {
+      const int kk = e / (D / 4), d = 4 * (e % (D / 4));
       const int bi = kk >> 2;
       const int64_t row = bi < nb ? block_row(sel[c0 + bi], kk & 3, g) : -1;
       if (row < 0 || row > t) continue;
-      float sk = 0.f, sv = 0.f;
+      float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int h = 0; h < hpg; ++h) {
-        sk = fmaf(dss[h * KC + kk], qs[h * D + d], sk);
-        sv = fmaf(ps[h * KC + kk], dos[h * D + d], sv);
+        const float ds = dss[h * KC + kk], p = ps[h * KC + kk];
+        const float4 qv = *reinterpret_cast<const float4*>(qs + h * D + d);
+        const float4 ov = *reinterpret_cast<const float4*>(dos + h * D + d);
+        sk.x = fmaf(ds, qv.x, sk.x);
+        sk.y = fmaf(ds, qv.y, sk.y);
+        sk.z = fmaf(ds, qv.z, sk.z);
+        sk.w = fmaf(ds, qv.w, sk.w);
+        sv.x = fmaf(p, ov.x, sv.x);
+        sv.y = fmaf(p, ov.y, sv.y);
+        sv.z = fmaf(p, ov.z, sv.z);
+        sv.w = fmaf(p, ov.w, sv.w);
       }
-      atomicAdd(dkg + row * D + d, sk * g.scale);
-      atomicAdd(dvg + row * D + d, sv);
+      sk.x *= g.scale;
+      sk.y *= g.scale;
+      sk.z *= g.scale;
+      sk.w *= g.scale;
+      atomicAdd(reinterpret_cast<float4*>(dkg + row * D + d), sk);
+      atomicAdd(reinterpret_cast<float4*>(dvg + row * D + d), sv);
     }
     __syncthreads();
   }
