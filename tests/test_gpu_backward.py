@@ -104,5 +104,7 @@ def test_backward_accumulates_key_gradients():
     dk2, dv2 = dk1.clone(), dv1.clone()
     qsa.qsa_sparse_attn_bwd(cfg, cache, segs, T, x["q"], fwd.o, fwd.lse, dout, fwd.sel, fwd.nsel, dq, dk2, dv2)
     torch.cuda.synchronize()
-    torch.testing.assert_close(dk2, 2 * dk1, rtol=1e-5, atol=1e-6)
-    torch.testing.assert_close(dv2, 2 * dv1, rtol=1e-5, atol=1e-6)
+    # the second call adds the same contributions in another atomic order: equal up to
+    # fp32 rounding of sums of a few hundred terms, relative to each tensor's scale
+    torch.testing.assert_close(dk2, 2 * dk1, rtol=0, atol=1e-5 * float(dk1.abs().max()))
+    torch.testing.assert_close(dv2, 2 * dv1, rtol=0, atol=1e-5 * float(dv1.abs().max()))

@@ -287,3 +287,16 @@ def test_duplicate_blocks_tie_toward_lower_index():
     kept = run.sel[0, :511].tolist()
     dup = list(range(100, 1900, 3))
     assert sum(1 for b in kept if b in set(dup)) > 400
+
+
+# --------------------------------------------------------------------------- determinism
+def test_forward_is_deterministic_across_calls():
+    """No atomics order results on the forward path: two calls on the same inputs
+    give bit-identical outputs, log-sum-exps and selections."""
+    wl = synth.make_workload("mixed_1m", ctx=16384, n_decode=3, chunk=300, chunk_pos0=5001)
+    x = _cuda_inputs(wl)
+    a = gpu_forward(wl, x)
+    b = gpu_forward(wl, x)
+    assert torch.equal(a.sel, b.sel) and torch.equal(a.nsel, b.nsel)
+    assert torch.equal(a.o.view(torch.int16), b.o.view(torch.int16))
+    assert torch.equal(a.lse, b.lse)
