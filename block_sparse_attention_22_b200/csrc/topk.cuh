@@ -532,9 +532,10 @@ __device__ void filter_scores_staged(const float* row, int64_t base, int n, floa
 // bins).  The result depends only on the source, so CTAs sharing a row agree
 // on it.  Ends with a barrier.
 template <int NT>
-__device__ uint32_t sampled_threshold(const RowSrc& src, int n, TopkShared<NT>& sh) {
+__device__ uint32_t sampled_threshold(const RowSrc& src, int n, TopkShared<NT>& sh,
+                                      int max_samples = topk::kMaxSamples, int target = topk::kSampleTarget) {
   using namespace topk;
-  const int m0 = n / 16 < kMinSamples ? kMinSamples : (n / 16 > kMaxSamples ? kMaxSamples : n / 16);
+  const int m0 = n / 16 < kMinSamples ? kMinSamples : (n / 16 > max_samples ? max_samples : n / 16);
   const int groups = m0 / kSampleGroup;
   const int m = groups * kSampleGroup;
   uint32_t vmin = 0xffffffffu, vmax = 0u;
@@ -549,7 +550,7 @@ __device__ uint32_t sampled_threshold(const RowSrc& src, int n, TopkShared<NT>& 
     vmax = max(vmax, k);
   }
   block_minmax(vmin, vmax, sh);
-  const int rank = max(1, (int)((int64_t)m * kSampleTarget / n));
+  const int rank = max(1, (int)((int64_t)m * target / n));
   if (vmin == vmax) return vmin;
   const int h = 31 - __clz(vmin ^ vmax);
   uint32_t mask = h == 31 ? 0u : ~((2u << h) - 1u);
@@ -751,7 +752,10 @@ __device__ void topk_chunk_row_threshold(const Geo& g, const TopkArgs& a, const 
     sh.n_ovf = 0;
   }
   const RowSrc row{a.scores + it.tok * a.ld, nullptr, nullptr, 0};
-  const uint32_t tkey = sampled_threshold(row, (int)it.bt, sh);
+  // every chunk CTA of the row repeats this: a smaller sample with a larger
+  // target (about 2048 of the row, 32 sampled above it) keeps it short, and
+  // the chunk lists (K each) and the merge buffer (CAP) hold that many
+  const uint32_t tkey = sampled_threshold(row, (int)it.bt, sh, 4096, 2048);
   __syncthreads();
   int cnt = 0;
   filter_scores(a.scores + it.tok * a.ld + it.c0, it.c0, it.n, key_to_float(tkey), cnt, sh);
