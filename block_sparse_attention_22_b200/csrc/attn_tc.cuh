@@ -27,15 +27,20 @@
 // held such gathers near 1 TB/s, while wide cp.async issue reaches the
 // memory system's rate.
 //
-// Roles (17 warps, persistent over work units, one CTA per SM):
-//   warps 0..7   producers: every half-slot is shared, warp w copying kept
-//                blocks 4w..4w+3 (one 512-byte row quad per instruction);
-//                each lane's cp.async completion arrives on the slot's
-//                barrier, so producers run ahead as far as the ring allows.
-//                Warp 0 also loads each unit's Q tile with TMA.
-//   warp 8       TMEM owner and single-thread MMA issuer;
-//   warps 9..16  softmax and epilogue: a thread owns TMEM lane i (key i of a
-//                chunk for S; dims i and 128+i for O) and 8 of the 16 heads.
+// Roles (20 warps, persistent over work units, one CTA per SM; warp w runs
+// on sub-partition w % 4):
+//   9 producers  (three on each of sub-partitions 1..3): every half-slot is
+//                shared, producer p copying kept blocks p, p+9, p+18, p+27
+//                (one 512-byte row quad per instruction); each lane's
+//                cp.async completion arrives on the slot's barrier, so
+//                producers run ahead as far as the ring allows.  Producer 0
+//                also loads each unit's Q tile with TMA.
+//   warp 0       TMEM owner and single-thread MMA issuer, alone with two
+//                softmax warps on sub-partition 0;
+//   8 softmax    softmax and epilogue, two per TMEM lane quadrant: a thread
+//                owns TMEM lane i (key i of a chunk for S; dims i and 128+i
+//                for O) and 8 of the 16 heads;
+//   warps 12, 16 idle.
 // Every mbarrier wait is bounded (sm100::mbar_wait); a timeout records an
 // error and the CTA's roles drain and return.
 #pragma once
@@ -45,10 +50,11 @@
 
 namespace qsa {
 namespace tc_attn {
-constexpr int kProducers = 8;
-constexpr int kMmaWarp = kProducers;
-constexpr int kSoftmaxWarps = 8;
-constexpr int kThreads = 32 * (kProducers + 1 + kSoftmaxWarps);   // 544
+constexpr int kProducers = 9;              // three on each of sub-partitions 1..3
+constexpr int kSoftmaxWarps = 8;           // two per TMEM lane quadrant
+constexpr int kWarps = 20;                 // + the MMA warp and two idle warps
+constexpr int kThreads = 32 * kWarps;      // 640
+enum Role { kRoleProducer, kRoleMma, kRoleSoftmax, kRoleIdle };
 constexpr int kKeys = 128;                 // keys per chunk
 constexpr int kBlk = 32;                   // blocks per chunk
 constexpr int kSlots = 6;                  // 32 KiB K/V half-chunk slots
@@ -135,6 +141,32 @@ __device__ __forceinline__ TcUnit tc_unit(const Geo& g, const SegTable& st, cons
   return u;
 }
 
+// Role of warp w.  Warp w runs on sub-partition w % 4 and may access TMEM
+// lanes 32 (w % 4) .. +31.  Sub-partition 0 holds the MMA issuer and two
+// softmax warps, each other sub-partition three producers and two softmax
+// warps: an issuing tcgen05.mma holds its sub-partition for tens of cycles,
+// and producers beside it would fall behind the others and hold up every
+// shared half-slot.  `idx` is the producer number (0..8) or the softmax
+// warp's head half (0, 1).
+__device__ __forceinline__ tc_attn::Role tc_role(int w, int& idx) {
+  using namespace tc_attn;
+  const int q = w & 3, r = w >> 2;
+  if (q == 0) {
+    if (r == 0) {
+      idx = 0;
+      return kRoleMma;
+    }
+    idx = r - 1;
+    return r <= 2 ? kRoleSoftmax : kRoleIdle;
+  }
+  if (r <= 2) {
+    idx = (q - 1) * 3 + r;
+    return kRoleProducer;
+  }
+  idx = r - 3;
+  return kRoleSoftmax;
+}
+
 __global__ void __launch_bounds__(tc_attn::kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Geo g, SegTable st, AttnTcArgs a) {
   using namespace tc_attn;
@@ -145,6 +177,8 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
   volatile int* abort_flag = &ctl.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n_units = (int64_t)g.G * a.units_per_group;
+  int ridx = 0;
+  const Role role = tc_role(warp, ridx);
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
@@ -173,7 +207,7 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
   for (int i = threadIdx.x; i < 2 * kQBytes / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem + kOffQ)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
-  if (warp == kMmaWarp) {
+  if (role == kRoleMma) {
     tmem_alloc(&ctl.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -184,8 +218,9 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
   pdl_wait();                                   // the previous kernel's results are visible from here
   pdl_trigger();
 
-  if (warp < kProducers) {
+  if (role == kRoleProducer) {
     // ============================================================ producers
+    const int pw = ridx;                         // producer number: copies blocks pw, pw+9, pw+18, pw+27
     int64_t hs_next = 0, uc = 0;                 // half-slots issued so far (shared numbering)
     bool ok = true;
     const int r = (lane >> 3) & 3, jc = lane & 7;   // row of a block and 16-byte chunk of a line
@@ -193,7 +228,7 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       if (warp_aborted(abort_flag)) break;
       const TcUnit u = tc_unit(g, st, a, w);
       if (u.nchunks == 0) continue;
-      if (warp == 0) {
+      if (pw == 0) {
         const int qb = (int)(uc & 1);
         if (!(ok = warp_wait(&ctl.q_empty[qb], (uint32_t)(((uc >> 1) & 1) ^ 1), abort_flag))) break;
         if (lane == 0) {
@@ -208,11 +243,11 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       const __nv_bfloat16* kg = (const __nv_bfloat16*)a.k + (u.slot * g.G + u.grp) * g.n_cap * kHeadDim;
       const __nv_bfloat16* vg = (const __nv_bfloat16*)a.v + (u.slot * g.G + u.grp) * g.n_cap * kHeadDim;
       const int32_t* selrow = a.sel + u.tok * g.S;
-      // cache rows of this warp's kept blocks 4w..4w+3 of a chunk (lanes 0..3)
+      // cache rows of this warp's kept blocks pw + 9 i of a chunk (lane i < 4)
       auto rows_of = [&](int cc) -> int64_t {
         int64_t row = -1;
-        if (lane < 4 && cc < u.nchunks) {
-          const int pos = u.blk_begin + cc * kBlk + 4 * warp + lane;
+        if (lane < 4 && cc < u.nchunks && pw + kProducers * lane < kBlk) {
+          const int pos = u.blk_begin + cc * kBlk + pw + kProducers * lane;
           if (pos < u.blk_end) row = block_row(selrow[pos], 0, g);
         }
         return row;
@@ -228,7 +263,8 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
             const uint32_t dst0 = smem_u32(smem + slot * kSlotBytes);
 #pragma unroll
             for (int bq = 0; bq < 4; ++bq) {
-              const int b = 4 * warp + bq;
+              const int b = pw + kProducers * bq;
+              if (b >= kBlk) break;
               const int64_t row = __shfl_sync(0xffffffffu, myrow, bq);
               const int line = 4 * b + r;
               const uint32_t dst = dst0 + line * 128 + ((jc ^ (line & 7)) << 4);
@@ -243,7 +279,7 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       }
     }
     cp_async_wait_all();                         // no copy of this warp outlives the CTA
-  } else if (warp == kMmaWarp) {
+  } else if (role == kRoleMma) {
     // ============================================================ MMA issuer
     // Whole warp in the loop; lane 0 issues the MMAs and commits.
     int64_t gp = 0, uc = 0, it = 0;
@@ -326,11 +362,10 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       mbar_wait(&ctl.mma_done, 0, &never);
     }
     __syncwarp();
-  } else {
+  } else if (role == kRoleSoftmax) {
     // ============================================================ softmax + epilogue
-    const int sw = warp - kMmaWarp - 1;                 // 0..7
     const int quad = warp & 3;                          // TMEM lane quadrant this warp may access
-    const int h0 = (sw >> 2) * kHH;                     // first of this thread's 8 heads
+    const int h0 = ridx * kHH;                          // first of this thread's 8 heads
     const int li = quad * 32 + lane;                    // TMEM lane: key of a chunk / dim
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t smem_base = smem_u32(smem);
@@ -481,7 +516,7 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (role == kRoleMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
