@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(HERE, "libqsa.so")
 
 QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA, QSA_ERR_TIMEOUT = range(6)
 QSA_DTYPE_F32, QSA_DTYPE_BF16 = 0, 1
-QSA_OP_COMPRESS, QSA_OP_INDEX, QSA_OP_SELECT, QSA_OP_ATTN, QSA_OP_FORWARD = range(5)
+QSA_OP_COMPRESS, QSA_OP_INDEX, QSA_OP_SELECT, QSA_OP_ATTN, QSA_OP_FORWARD, QSA_OP_FORWARD_LOWMEM = range(6)
 
 
 class qsa_config_t(ctypes.Structure):
@@ -61,7 +61,9 @@ def _load():
         "qsa_sparse_attn_fwd": [C, K, S, I32, I32, P, P, P, P, P, P, SZ, P],
         "qsa_sparse_attn_bwd": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, P, P],
         "qsa_forward": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, SZ, P],
+        "qsa_forward_lowmem": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, SZ, P],
         "qsa_device_status": [P],
+        "qsa_select_fallbacks": [P, ctypes.POINTER(ctypes.c_int64)],
         "qsa_selftest_wait_timeout": [P],
         "qsa_select_topk_noalloc": [C, S, I32, I32, P, I64, P, P, P],
     }
@@ -192,6 +194,16 @@ def qsa_forward(cfg, cache, segs, n_tokens, q, q_idx, w, o, lse=None, sel=None, 
                            _stream(stream)), "qsa_forward")
 
 
+def qsa_forward_lowmem(cfg, cache, segs, n_tokens, q, q_idx, w, o, lse=None, sel=None, nsel=None,
+                       workspace=None, stream=None):
+    """qsa_forward without the score matrix (workspace: QSA_OP_FORWARD_LOWMEM)."""
+    arr, n = segs
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(get_lib().qsa_forward_lowmem(ctypes.byref(cfg), ctypes.byref(cache), arr, n, n_tokens, _ptr(q),
+                                        _ptr(q_idx), _ptr(w), _ptr(o), _ptr(lse), _ptr(sel), _ptr(nsel),
+                                        _ptr(workspace), ws_bytes, _stream(stream)), "qsa_forward_lowmem")
+
+
 def qsa_device_status(stream=None):
     _check(get_lib().qsa_device_status(_stream(stream)), "qsa_device_status")
 
@@ -199,6 +211,13 @@ def qsa_device_status(stream=None):
 def device_status(stream=None) -> int:
     """Status code of qsa_device_status (reads and clears the device error word)."""
     return int(get_lib().qsa_device_status(_stream(stream)))
+
+
+def select_fallbacks(stream=None) -> int:
+    """Rows whose selection took the exact fallback since the last call (reads and clears)."""
+    n = ctypes.c_int64(0)
+    _check(get_lib().qsa_select_fallbacks(_stream(stream), ctypes.byref(n)), "qsa_select_fallbacks")
+    return int(n.value)
 
 
 def qsa_selftest_wait_timeout(stream=None):

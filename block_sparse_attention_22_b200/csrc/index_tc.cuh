@@ -17,6 +17,13 @@
 // a segment has a closed form (a floor sum), which lets a CTA seek to its
 // slice.
 //
+// The k^ tensor map is [slot][row][dim] with row j = pooled block j*stride:
+// stride 1 scores every block; a larger stride scores an evenly spaced
+// sample of them (the row threshold of the fused selection comes from it).
+// In filter mode the epilogue writes no scores: it appends (key, block) for
+// the candidates at or above the token's threshold key to the token's
+// candidate list (warp-aggregated atomics on the list's count).
+//
 // NQ = 64 for prefill (N = 256; TMEM holds two 128x256 fp32 accumulators),
 // NQ = 4 for decode (N = 16; the kernel then streams each sequence's k^ at
 // HBM rate through a deeper ring).  Roles (one CTA per SM):
@@ -54,7 +61,8 @@ struct IndexTcCfg {
   static constexpr int kOffB = kStages * kABytes;
   static constexpr int kOffW = kOffB + kBBytes;            // w[NQ][4] fp32
   static constexpr int kOffCS = kOffW + ((NQ * 16 + 1023) / 1024) * 1024;   // cos/sin[NQ][half]
-  static constexpr int kOffBar = kOffCS + ((NQ * tc_index::kMaxRopeHalf * 8 + 1023) / 1024) * 1024;
+  static constexpr int kOffTau = kOffCS + ((NQ * tc_index::kMaxRopeHalf * 8 + 1023) / 1024) * 1024;   // float[NQ]
+  static constexpr int kOffBar = kOffTau + ((NQ * 4 + 1023) / 1024) * 1024;
   static constexpr int kSmemBytes = kOffBar + 1024 + 1024;
   static constexpr uint32_t kTmemCols = 2 * N < 32 ? 32 : 2 * N;
   static constexpr uint32_t kIdesc = sm100::idesc_bf16(128, N, false, false);
@@ -64,8 +72,18 @@ struct IndexTcCfg {
 struct IndexTcArgs {
   const __nv_bfloat16* q_idx;   // [T][4][DI]
   const float* w;               // [T][4]
-  float* scores;                // [T][ld]
+  float* scores;                // [T][ld] (score mode)
   int64_t ld;
+  int stride;                   // pooled blocks per scored row: 1, or the sample stride
+  // filter mode (tau != null): instead of writing scores, the (score, block)
+  // pairs of every candidate with score >= tau[token] are appended to the
+  // token's list; cand_cnt counts them all (entries past cand_cap are
+  // dropped, and the count tells the selection so)
+  const float* tau;             // [T]; -inf keeps every candidate, NaN none
+  float* cand_score;            // [T][cand_cap]
+  int32_t* cand_idx;            // [T][cand_cap]
+  int32_t* cand_cnt;            // [T], zero on entry
+  int cand_cap;
 };
 
 struct IndexTcCtl {
@@ -110,11 +128,12 @@ __host__ __device__ inline int64_t floor_sum(int64_t n, int64_t m, int64_t a, in
 }
 
 // k^ tiles scored by query tile qt of a segment (the blocks its last query
-// scores, floor(t_last / r), in tiles of 128).
+// scores, floor(t_last / r), in tiles of 128 scored rows; with stride s a row
+// is every s-th block, so a tile spans 128 s blocks).
 template <int NQ>
-__host__ __device__ inline int index_qtile_tiles(int64_t pos0, int q_len, int qt, int r) {
+__host__ __device__ inline int index_qtile_tiles(int64_t pos0, int q_len, int qt, int r, int stride) {
   const int64_t t_last = pos0 + (int64_t)min(NQ * (qt + 1), q_len) - 1;
-  return (int)cdiv(t_last / r, tc_index::kTileRows);
+  return (int)cdiv(t_last / r, (int64_t)tc_index::kTileRows * stride);
 }
 
 // Balancing weight of a query tile's prologue (building its rotated B tile),
@@ -125,21 +144,22 @@ template <int NQ>
 constexpr int index_prologue_units() { return NQ >= 64 ? 6 : 2; }
 
 // Work units (k^ tiles plus prologue weights) of the full query tiles
-// 0..J-1 of a segment, where the k^ tiles of full query tile j are
-//   ceil(floor((pos0 + NQ j + NQ - 1) / r) / 128) = floor((pos0 + NQ - 1 + 127 r + NQ j) / (128 r)).
+// 0..J-1 of a segment, where with P = 128 s blocks per tile the k^ tiles of
+// full query tile j are
+//   ceil(floor((pos0 + NQ j + NQ - 1) / r) / P) = floor((pos0 + NQ - 1 + (P-1) r + NQ j) / (P r)).
 template <int NQ>
-__host__ __device__ inline int64_t index_units_before(int64_t pos0, int J, int r) {
-  return floor_sum(J, (int64_t)tc_index::kTileRows * r, NQ, pos0 + NQ - 1 + (int64_t)(tc_index::kTileRows - 1) * r) +
-         (int64_t)index_prologue_units<NQ>() * J;
+__host__ __device__ inline int64_t index_units_before(int64_t pos0, int J, int r, int stride) {
+  const int64_t P = (int64_t)tc_index::kTileRows * stride;
+  return floor_sum(J, P * r, NQ, pos0 + NQ - 1 + (P - 1) * r) + (int64_t)index_prologue_units<NQ>() * J;
 }
 
 // All work units of a segment.
 template <int NQ>
-inline int64_t index_tc_units(int q_len, int64_t pos0, int r) {
+inline int64_t index_tc_units(int q_len, int64_t pos0, int r, int stride = 1) {
   if (q_len <= 0) return 0;
   const int nqt = (int)cdiv(q_len, NQ);
-  return index_units_before<NQ>(pos0, nqt - 1, r) + index_prologue_units<NQ>() +
-         index_qtile_tiles<NQ>(pos0, q_len, nqt - 1, r);
+  return index_units_before<NQ>(pos0, nqt - 1, r, stride) + index_prologue_units<NQ>() +
+         index_qtile_tiles<NQ>(pos0, q_len, nqt - 1, r, stride);
 }
 
 // Position in the flat sequence of work units: per segment, per query tile,
@@ -153,20 +173,21 @@ struct IndexCursor {
 // Moves to the next query tile that has k^ tiles (consuming its prologue
 // weight) while the current one is exhausted.
 template <int NQ>
-__device__ __forceinline__ void index_skip(const Geo& g, const SegTable& st, IndexCursor& c) {
+__device__ __forceinline__ void index_skip(const Geo& g, const SegTable& st, int stride, IndexCursor& c) {
   while (c.left > 0 && c.tile >= c.nt) {
     c.tile = 0;
     if (++c.qt >= (int)cdiv(st.q_len[c.si], NQ)) {
       c.qt = 0;
       ++c.si;
     }
-    c.nt = index_qtile_tiles<NQ>(st.pos0[c.si], st.q_len[c.si], c.qt, g.r);
+    c.nt = index_qtile_tiles<NQ>(st.pos0[c.si], st.q_len[c.si], c.qt, g.r, stride);
     c.left -= index_prologue_units<NQ>();
   }
 }
 
 template <int NQ>
-__device__ __forceinline__ void index_seek(const Geo& g, const SegTable& st, int64_t L, int64_t R, IndexCursor& c) {
+__device__ __forceinline__ void index_seek(const Geo& g, const SegTable& st, int stride, int64_t L, int64_t R,
+                                           IndexCursor& c) {
   constexpr int W = index_prologue_units<NQ>();
   c.left = R - L;
   if (c.left <= 0) return;
@@ -177,25 +198,25 @@ __device__ __forceinline__ void index_seek(const Geo& g, const SegTable& st, int
   int lo = 0, hi = nqt - 1;                       // largest J with units_before(J) <= local
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (index_units_before<NQ>(pos0, mid, g.r) <= local) lo = mid; else hi = mid - 1;
+    if (index_units_before<NQ>(pos0, mid, g.r, stride) <= local) lo = mid; else hi = mid - 1;
   }
   c.qt = lo;
-  const int64_t o = local - index_units_before<NQ>(pos0, lo, g.r);
-  c.nt = index_qtile_tiles<NQ>(pos0, st.q_len[c.si], lo, g.r);
+  const int64_t o = local - index_units_before<NQ>(pos0, lo, g.r, stride);
+  c.nt = index_qtile_tiles<NQ>(pos0, st.q_len[c.si], lo, g.r, stride);
   if (o < W) {                                    // the slice starts inside the prologue weight
     c.left -= W - o;
     c.tile = 0;
   } else {
     c.tile = (int)(o - W);
   }
-  index_skip<NQ>(g, st, c);
+  index_skip<NQ>(g, st, stride, c);
 }
 
 template <int NQ>
-__device__ __forceinline__ void index_advance(const Geo& g, const SegTable& st, IndexCursor& c) {
+__device__ __forceinline__ void index_advance(const Geo& g, const SegTable& st, int stride, IndexCursor& c) {
   --c.left;
   ++c.tile;
-  index_skip<NQ>(g, st, c);
+  index_skip<NQ>(g, st, stride, c);
 }
 
 template <int NQ>
@@ -244,18 +265,19 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
   pdl_trigger();
 
   IndexCursor cur;
-  index_seek<NQ>(g, st, L, R, cur);
+  index_seek<NQ>(g, st, a.stride, L, R, cur);
 
   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0) {
-      for (int i = 0; cur.left > 0; ++i, index_advance<NQ>(g, st, cur)) {
+      for (int i = 0; cur.left > 0; ++i, index_advance<NQ>(g, st, a.stride, cur)) {
         const int s = i % C::kStages;
         if (!mbar_wait(&ctl.a_empty[s], (uint32_t)(((i / C::kStages) & 1) ^ 1), abort_flag)) break;
         mbar_expect_tx(&ctl.a_full[s], (uint32_t)(kTileRows * g.DI * 2));
-        const int32_t y = (int32_t)((int64_t)st.slot[cur.si] * (g.n_cap / g.r) + (int64_t)cur.tile * kTileRows);
+        // tensor map [slot][scored row][dim]: rows past the slot's last read as zero
+        const int32_t y = (int32_t)((int64_t)cur.tile * kTileRows);
         for (int slab = 0; slab < g.DI / 64; ++slab)
-          tma_load_2d(smem + s * C::kABytes + slab * 16384, &tm_khat, 64 * slab, y, &ctl.a_full[s]);
+          tma_load_3d(smem + s * C::kABytes + slab * 16384, &tm_khat, 64 * slab, y, st.slot[cur.si], &ctl.a_full[s]);
       }
     }
     __syncwarp();
@@ -264,7 +286,7 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
     if (lane == 0) {
       bool ok = true;
       int nqt_seen = 0;
-      for (int i = 0; ok && cur.left > 0; ++i, index_advance<NQ>(g, st, cur)) {
+      for (int i = 0; ok && cur.left > 0; ++i, index_advance<NQ>(g, st, a.stride, cur)) {
         if (i == 0 || cur.tile == 0) {                 // a new rotated query tile in B
           if (!(ok = mbar_wait(&ctl.b_ready, (uint32_t)(nqt_seen & 1), abort_flag))) break;
           ++nqt_seen;
@@ -297,6 +319,7 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
     const int chunks = DI / 8;                      // 16-byte chunks per q~ row
     float* ws = reinterpret_cast<float*>(smem + C::kOffW);
     float2* cs = reinterpret_cast<float2*>(smem + C::kOffCS);
+    float* taus = reinterpret_cast<float*>(smem + C::kOffTau);
     const int quad = warp & 3;
     const int cq = (warp - 2) >> 2;                 // column share within the quadrant
     constexpr int kCols = C::kColsPerWarp;
@@ -308,7 +331,7 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
 
     int64_t tok0 = 0, t_first = 0;
     int nq = 0;
-    for (int i = 0; cur.left > 0; ++i, index_advance<NQ>(g, st, cur)) {
+    for (int i = 0; cur.left > 0; ++i, index_advance<NQ>(g, st, a.stride, cur)) {
       if (i == 0 || cur.tile == 0) {
         // ---------------------------------------------- new query tile
         const int q0 = cur.qt * NQ;
@@ -323,6 +346,8 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
           cs[k] = make_float2(c, sn);
         }
         for (int k = et; k < NQ * 4; k += C::kEpiThreads) ws[k] = (k >> 2) < nq ? a.w[tok0 * 4 + k] : 0.f;
+        if (a.tau)
+          for (int k = et; k < NQ; k += C::kEpiThreads) taus[k] = k < nq ? a.tau[tok0 + k] : __int_as_float(0x7fffffff);
         named_bar_sync(1, C::kEpiThreads);
         // rotated queries: row n = q*4 + h of the B tile (K-major, 128-byte swizzle).
         // The accumulators of the previous query tile were all observed full,
@@ -410,12 +435,13 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.acc_free[ab]);  // values are in registers: the MMA may reuse it
 
-      const int64_t b0 = (int64_t)cur.tile * kTileRows;
-      const int bl = quad * 32 + lane;                // block within the tile
+      const int64_t b0 = (int64_t)cur.tile * kTileRows;   // first scored row of the tile
+      const int bl = quad * 32 + lane;                // scored row within the tile
       const int qb = cq * kQ;                         // first query of this share
       const int64_t t0 = t_first + qb;
-      const int64_t ld = a.ld;
-      float* p = a.scores + (tok0 + qb) * ld + b0 + bl;
+      const int64_t blk = (b0 + bl) * a.stride;       // the pooled block of this row
+      // block blk is a candidate of the query at t iff (blk + 1) r <= t
+      const int64_t lim = t0 - (blk + 1) * g.r;
       const float4* w4 = reinterpret_cast<const float4*>(ws) + qb;
       float sc[kQ];
 #pragma unroll
@@ -428,16 +454,48 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
         s = fmaf(wq.w, fmaxf(v[4 * qq + 3], 0.f), s);
         sc[qq] = s;
       }
-      if (qb + kQ <= nq && (b0 + kTileRows) * g.r <= t0) {
-        // every block of the tile is a candidate of every query of the share
+      if (a.tau) {
+        // filter mode: the warp's hits of query qq form ballot m_qq; lane qq
+        // reserves them with one atomic on the query's count (the kQ round
+        // trips of a tile overlap), then the hits of each query are stored at
+        // consecutive positions
+        static_assert(kQ <= 32, "one lane per query of the share");
+        const bool full = qb + kQ <= nq && ((b0 + kTileRows - 1) * a.stride + 1) * g.r <= t0;
+        uint32_t hits = 0, my_m = 0;
 #pragma unroll
-        for (int qq = 0; qq < kQ; ++qq, p += ld) *p = sc[qq];
+        for (int qq = 0; qq < kQ; ++qq) {
+          const bool pass = sc[qq] >= taus[qb + qq] && (full || (qb + qq < nq && lim + qq >= 0));
+          const uint32_t m = __ballot_sync(0xffffffffu, pass);
+          hits |= (pass ? 1u : 0u) << qq;
+          if (lane == qq) my_m = m;
+        }
+        int my_base = 0;
+        if (my_m) my_base = atomicAdd(&a.cand_cnt[tok0 + qb + lane], __popc(my_m));
+        const uint32_t below = (1u << lane) - 1u;
+        const int cap = a.cand_cap;
+        float* ps = a.cand_score + (tok0 + qb) * (int64_t)cap;
+        int32_t* pi = a.cand_idx + (tok0 + qb) * (int64_t)cap;
+#pragma unroll
+        for (int qq = 0; qq < kQ; ++qq, ps += cap, pi += cap) {
+          const uint32_t m = __shfl_sync(0xffffffffu, my_m, qq);
+          const int pos = __shfl_sync(0xffffffffu, my_base, qq) + __popc(m & below);
+          if (((hits >> qq) & 1u) && pos < cap) {
+            ps[pos] = sc[qq];
+            pi[pos] = (int32_t)blk;
+          }
+        }
       } else {
-        // block b is a candidate of the query at t iff (b + 1) r <= t
-        const int64_t lim = t0 - (b0 + bl + 1) * g.r;
+        const int64_t ld = a.ld;
+        float* p = a.scores + (tok0 + qb) * ld + b0 + bl;
+        if (qb + kQ <= nq && ((b0 + kTileRows - 1) * a.stride + 1) * g.r <= t0) {
+          // every block of the tile is a candidate of every query of the share
 #pragma unroll
-        for (int qq = 0; qq < kQ; ++qq, p += ld)
-          if (qb + qq < nq && lim + qq >= 0) *p = sc[qq];
+          for (int qq = 0; qq < kQ; ++qq, p += ld) *p = sc[qq];
+        } else {
+#pragma unroll
+          for (int qq = 0; qq < kQ; ++qq, p += ld)
+            if (qb + qq < nq && lim + qq >= 0) *p = sc[qq];
+        }
       }
     }
   }

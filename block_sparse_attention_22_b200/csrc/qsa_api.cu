@@ -240,9 +240,8 @@ qsa_status_t run_compress(const Geo& g, const qsa_config_t* c, const qsa_cache_t
   return flush();
 }
 
-// Tensor map of the k^ cache: [n_slots * n_cap/r rows][idx_dim] bf16, boxes of
-// 64 dims x 128 rows.
-bool make_khat_map(CUtensorMap* m, const qsa_config_t* c, const qsa_cache_t* cache);
+// Tensor map of the k^ cache (every stride-th pooled block of each slot).
+bool make_khat_map(CUtensorMap* m, const qsa_config_t* c, const qsa_cache_t* cache, int stride);
 int sm_count();
 
 template <int NQ>
@@ -263,8 +262,13 @@ qsa_status_t run_index(const Geo& g, const qsa_config_t* c, const qsa_cache_t* c
                        float* scores, int64_t ld, cudaStream_t st) {
   if (c->dtype == QSA_DTYPE_BF16) {
     CUtensorMap tm;
-    if (!make_khat_map(&tm, c, cache)) return QSA_ERR_CUDA;
-    IndexTcArgs a{(const __nv_bfloat16*)q_idx, w, scores, ld};
+    if (!make_khat_map(&tm, c, cache, 1)) return QSA_ERR_CUDA;
+    IndexTcArgs a{};
+    a.q_idx = (const __nv_bfloat16*)q_idx;
+    a.w = w;
+    a.scores = scores;
+    a.ld = ld;
+    a.stride = 1;
     // prefill-like segments on 64-query tiles, decode-like ones on 4-query tiles
     std::vector<qsa_segment_t> wide, narrow;
     for (int i = 0; i < n; ++i) (segs[i].q_len >= 16 ? wide : narrow).push_back(segs[i]);
@@ -284,6 +288,72 @@ qsa_status_t run_index(const Geo& g, const qsa_config_t* c, const qsa_cache_t* c
   return for_each_table(
       segs, n, [&](const qsa_segment_t& s) { return (int64_t)simt_index_items(s.q_len, s.pos0, g.r); },
       [&](const SegTable& t) { return launch_index_simt<float>(g, t, q_idx, w, cache->khat, scores, ld, st); });
+}
+
+// Fused selection of prefill-like bf16 segments (no score matrix): sample
+// scores, row thresholds, filtered scoring into candidate lists, selection.
+struct FusedBufs {
+  float* samples;
+  int64_t ld_s;
+  float* tau;
+  float* cand_score;
+  int32_t* cand_idx;
+  int32_t* cand_cnt;
+};
+
+qsa_status_t run_fused_select(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
+                              const qsa_segment_t* segs, int n, const void* q_idx, const float* w,
+                              const FusedBufs& f, int32_t* sel, int32_t* nsel, cudaStream_t st) {
+  constexpr int kStride = topk::kFusedStride;
+  CUtensorMap tm_s, tm;
+  if (!make_khat_map(&tm_s, c, cache, kStride) || !make_khat_map(&tm, c, cache, 1)) return QSA_ERR_CUDA;
+  IndexTcArgs a{};
+  a.q_idx = (const __nv_bfloat16*)q_idx;
+  a.w = w;
+  a.scores = f.samples;
+  a.ld = f.ld_s;
+  a.stride = kStride;
+  qsa_status_t r = for_each_table(
+      segs, n, [&](const qsa_segment_t& s) { return index_tc_units<64>(s.q_len, s.pos0, g.r, kStride); },
+      [&](const SegTable& t) { return launch_index_tc<64>(g, t, tm_s, a, st); });
+  if (r != QSA_OK) return r;
+  FusedSelArgs fa;
+  memset(&fa, 0, sizeof fa);
+  fa.samples = f.samples;
+  fa.ld_s = f.ld_s;
+  fa.stride = kStride;
+  fa.tau = f.tau;
+  fa.cand_score = f.cand_score;
+  fa.cand_idx = f.cand_idx;
+  fa.cand_cnt = f.cand_cnt;
+  fa.sel = sel;
+  fa.nsel = nsel;
+  fa.q_idx = (const __nv_bfloat16*)q_idx;
+  fa.w = w;
+  fa.khat = (const __nv_bfloat16*)cache->khat;
+  const int ctas = 6 * sm_count();
+  auto rows = [](const qsa_segment_t& s) { return (int64_t)s.q_len; };
+  r = for_each_table(segs, n, rows, [&](const SegTable& t) {
+    count_launch();
+    return launch_chained(topk_tau_kernel, dim3(std::min(t.item0[t.n], ctas)), dim3(topk::THREADS), 0, st, g, t, fa);
+  });
+  if (r != QSA_OK) return r;
+  a.scores = nullptr;
+  a.ld = 0;
+  a.stride = 1;
+  a.tau = f.tau;
+  a.cand_score = f.cand_score;
+  a.cand_idx = f.cand_idx;
+  a.cand_cnt = f.cand_cnt;
+  a.cand_cap = topk::CAP;
+  r = for_each_table(
+      segs, n, [&](const qsa_segment_t& s) { return index_tc_units<64>(s.q_len, s.pos0, g.r, 1); },
+      [&](const SegTable& t) { return launch_index_tc<64>(g, t, tm, a, st); });
+  if (r != QSA_OK) return r;
+  return for_each_table(segs, n, rows, [&](const SegTable& t) {
+    count_launch();
+    return launch_chained(topk_cand_kernel, dim3(std::min(t.item0[t.n], ctas)), dim3(topk::THREADS), 0, st, g, t, fa);
+  });
 }
 
 qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const float* scores,
@@ -379,9 +449,20 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ro
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_khat_map(CUtensorMap* m, const qsa_config_t* c, const qsa_cache_t* cache) {
-  const uint64_t rows = (uint64_t)cache->n_slots * (uint64_t)(cache->n_cap / c->r);
-  return make_map_bf16(m, cache->khat, (uint64_t)c->idx_dim, rows, 64, tc_index::kTileRows);
+// Tensor map of the k^ cache as [n_slots][rows][idx_dim] bf16 with row j of
+// a slot = pooled block j*stride (stride 1: every block), boxes of 64 dims x
+// 128 rows x 1 slot, 128-byte swizzle; rows past a slot's end read as zero.
+bool make_khat_map(CUtensorMap* m, const qsa_config_t* c, const qsa_cache_t* cache, int stride) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const uint64_t blocks = (uint64_t)(cache->n_cap / c->r), di = (uint64_t)c->idx_dim;
+  cuuint64_t dims[3] = {di, (blocks + stride - 1) / stride, (uint64_t)cache->n_slots};
+  cuuint64_t strides[2] = {di * 2 * stride, di * 2 * blocks};
+  cuuint32_t box[3] = {64, (cuuint32_t)tc_index::kTileRows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, cache->khat, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int sm_count() {
@@ -468,25 +549,47 @@ qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* ca
 }
 
 // ------------------------------------------------------------------ forward workspace
+// In the low-memory forward, prefill-like segments (64-query index tiles) of
+// the bf16 path select through the fused path; the others (decode-like, or
+// fp32), and every segment of the default forward, through the score matrix.
+bool fused_segment(const qsa_segment_t& s, bool tc, bool lowmem) { return lowmem && tc && s.q_len >= 16; }
+
+void split_fused(const qsa_segment_t* segs, int n, bool tc, bool lowmem, std::vector<qsa_segment_t>& fused,
+                 std::vector<qsa_segment_t>& plain) {
+  for (int i = 0; i < n; ++i) (fused_segment(segs[i], tc, lowmem) ? fused : plain).push_back(segs[i]);
+}
+
 struct FwdLayout {
-  int64_t ld;
-  size_t scores, sel, nsel, topk, attn, total;
+  int64_t ld;      // score rows of the plain segments
+  int64_t ld_s;    // sample rows of the fused segments
+  size_t scores, sel, nsel, topk, attn, samples, tau, cnt, ckey, cidx, total;
 };
 
-FwdLayout fwd_layout(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens, bool tc) {
+FwdLayout fwd_layout(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens, bool tc, bool lowmem) {
+  std::vector<qsa_segment_t> fused, plain;
+  split_fused(segs, n, tc, lowmem, fused, plain);
   FwdLayout L;
-  L.ld = std::max<int64_t>(4, cdiv(seg_max_blocks(segs, n, g.r), 4) * 4);
+  L.ld = std::max<int64_t>(4, cdiv(seg_max_blocks(plain.data(), (int)plain.size(), g.r), 4) * 4);
+  const int64_t nb_f = seg_max_blocks(fused.data(), (int)fused.size(), g.r);
+  L.ld_s = std::max<int64_t>(4, cdiv(cdiv(nb_f, topk::kFusedStride), 4) * 4);
+  const size_t T = (size_t)n_tokens;
   size_t off = 0;
-  L.scores = off;
-  off += align_up((size_t)n_tokens * L.ld * 4, 256);
-  L.sel = off;
-  off += align_up((size_t)n_tokens * g.S * 4, 256);
-  L.nsel = off;
-  off += align_up((size_t)n_tokens * 4, 256);
-  L.topk = off;
-  off += align_up(topk_plan(g, segs, n).ws, 256);
-  L.attn = off;
-  off += align_up(attn_plan(g, segs, n, tc).ws, 256);
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align_up(bytes, 256);
+    return at;
+  };
+  L.scores = take(plain.empty() ? 0 : T * L.ld * 4);
+  L.sel = take(T * g.S * 4);
+  L.nsel = take(T * 4);
+  L.topk = take(topk_plan(g, plain.data(), (int)plain.size()).ws);
+  L.attn = take(attn_plan(g, segs, n, tc).ws);
+  const bool f = !fused.empty();
+  L.samples = take(f ? T * L.ld_s * 4 : 0);
+  L.tau = take(f ? T * 4 : 0);
+  L.cnt = take(f ? T * 4 : 0);
+  L.ckey = take(f ? T * topk::CAP * 4 : 0);
+  L.cidx = take(f ? T * topk::CAP * 4 : 0);
   L.total = off;
   return L;
 }
@@ -612,16 +715,19 @@ QSA_API size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* 
     case QSA_OP_INDEX: return 0;
     case QSA_OP_SELECT: return topk_plan(g, segs, n_segs).ws;
     case QSA_OP_ATTN: return attn_plan(g, segs, n_segs, cfg->dtype == QSA_DTYPE_BF16).ws;
-    case QSA_OP_FORWARD: return fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16).total;
+    case QSA_OP_FORWARD: return fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16, false).total;
+    case QSA_OP_FORWARD_LOWMEM:
+      return fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16, true).total;
   }
   return SIZE_MAX;
 }
 
-QSA_API qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cache,
-                                 const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
-                                 const void* q, const void* q_idx, const float* w, void* o,
-                                 float* lse, int32_t* sel, int32_t* nsel, void* workspace,
-                                 size_t ws_bytes, void* stream) {
+namespace qsa {
+namespace {
+qsa_status_t forward_impl(const qsa_config_t* cfg, const qsa_cache_t* cache, const qsa_segment_t* segs,
+                          int32_t n_segs, int32_t n_tokens, const void* q, const void* q_idx, const float* w,
+                          void* o, float* lse, int32_t* sel, int32_t* nsel, void* workspace, size_t ws_bytes,
+                          void* stream, bool lowmem) {
   qsa_status_t s = check_cfg(cfg);
   if (s != QSA_OK) return s;
   if ((s = check_cache(cfg, cache)) != QSA_OK) return s;
@@ -636,7 +742,7 @@ QSA_API qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cac
   const int64_t nblk = seg_max_blocks(segs, n_segs, cfg->r);
   if (nblk > (int64_t)topk::kChunkLarge * 32) return QSA_ERR_UNSUPPORTED;
   const Geo g = make_geo(cfg, cache);
-  const FwdLayout L = fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16);
+  const FwdLayout L = fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16, lowmem);
   if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return QSA_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
   char* ws = (char*)workspace;
@@ -645,6 +751,8 @@ QSA_API qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cac
     sel = (int32_t*)(ws + L.sel);
     nsel = (int32_t*)(ws + L.nsel);
   }
+  std::vector<qsa_segment_t> fused, plain;
+  split_fused(segs, n_segs, cfg->dtype == QSA_DTYPE_BF16, lowmem, fused, plain);
   // 1. pool the blocks each segment completes
   std::vector<int32_t> slots;
   std::vector<int64_t> b0, b1;
@@ -656,22 +764,65 @@ QSA_API qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cac
     b1.push_back(((int64_t)segs[i].pos0 + segs[i].q_len) / cfg->r);
     own_blocks_only &= ((int64_t)segs[i].pos0 + segs[i].q_len - 1) / cfg->r <= segs[i].pos0 / cfg->r;
   }
+  const int n_plain = (int)plain.size();
   if (own_blocks_only) {
-    // decode-like batch: the indexer reads no block pooled now, so the pooling
-    // runs alongside it (its exit still waits for the indexer)
-    if ((s = run_index(g, cfg, cache, segs, n_segs, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
+    // decode-like batch (no prefill-like segment completes no block): the
+    // indexer reads no block pooled now, so the pooling runs alongside it
+    // (its exit still waits for the indexer)
+    if ((s = run_index(g, cfg, cache, plain.data(), n_plain, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
     s = run_compress(g, cfg, cache, slots.data(), b0.data(), b1.data(), (int)slots.size(), st, true);
     if (s != QSA_OK) return s;
   } else {
     s = run_compress(g, cfg, cache, slots.data(), b0.data(), b1.data(), (int)slots.size(), st);
     if (s != QSA_OK) return s;
-    // 2. indexer scores
-    if ((s = run_index(g, cfg, cache, segs, n_segs, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
+    // 2. indexer scores of the plain segments
+    if ((s = run_index(g, cfg, cache, plain.data(), n_plain, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
   }
-  // 3. selection, 4. attention
-  if ((s = run_select(g, segs, n_segs, scores, L.ld, sel, nsel, ws + L.topk, L.attn - L.topk, st)) != QSA_OK)
+  // 2-3. fused scoring and selection of the prefill-like segments
+  if (!fused.empty()) {
+    const FusedBufs f{(float*)(ws + L.samples), L.ld_s, (float*)(ws + L.tau), (float*)(ws + L.ckey),
+                      (int32_t*)(ws + L.cidx), (int32_t*)(ws + L.cnt)};
+    if ((s = run_fused_select(g, cfg, cache, fused.data(), (int)fused.size(), q_idx, w, f, sel, nsel, st)) != QSA_OK)
+      return s;
+  }
+  // 3. selection of the plain segments, 4. attention
+  if (n_plain > 0 &&
+      (s = run_select(g, plain.data(), n_plain, scores, L.ld, sel, nsel, ws + L.topk, L.attn - L.topk, st)) != QSA_OK)
     return s;
-  return run_attn(g, cfg, cache, segs, n_segs, n_tokens, q, sel, nsel, o, lse, ws + L.attn, L.total - L.attn, st);
+  return run_attn(g, cfg, cache, segs, n_segs, n_tokens, q, sel, nsel, o, lse, ws + L.attn, L.samples - L.attn, st);
+}
+}  // namespace
+}  // namespace qsa
+
+QSA_API qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                 const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                                 const void* q, const void* q_idx, const float* w, void* o,
+                                 float* lse, int32_t* sel, int32_t* nsel, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  return forward_impl(cfg, cache, segs, n_segs, n_tokens, q, q_idx, w, o, lse, sel, nsel, workspace, ws_bytes,
+                      stream, false);
+}
+
+QSA_API qsa_status_t qsa_forward_lowmem(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                        const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                                        const void* q, const void* q_idx, const float* w, void* o,
+                                        float* lse, int32_t* sel, int32_t* nsel, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  return forward_impl(cfg, cache, segs, n_segs, n_tokens, q, q_idx, w, o, lse, sel, nsel, workspace, ws_bytes,
+                      stream, true);
+}
+
+QSA_API qsa_status_t qsa_select_fallbacks(void* stream, int64_t* count) {
+  if (!count) return QSA_ERR_INVALID_ARG;
+  unsigned long long h = 0, zero = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyFromSymbolAsync(&h, g_qsa_select_fallbacks, sizeof h, 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return QSA_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(g_qsa_select_fallbacks, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return QSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QSA_ERR_CUDA;
+  *count = (int64_t)h;
+  return QSA_OK;
 }
 
 QSA_API qsa_status_t qsa_device_status(void* stream) {

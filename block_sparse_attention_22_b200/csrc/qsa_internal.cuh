@@ -96,6 +96,14 @@ __device__ __forceinline__ void report_error(unsigned int code) {
   atomicCAS(&g_qsa_device_error, 0u, code);
 }
 
+// Rows whose selection took an exact fallback (the sampled threshold admitted
+// too few or too many candidates); read and reset by qsa_select_fallbacks().
+static __device__ unsigned long long g_qsa_select_fallbacks;
+
+__device__ __forceinline__ void count_fallback() {
+  if (threadIdx.x == 0) atomicAdd(&g_qsa_select_fallbacks, 1ull);
+}
+
 // Cache row of token `j_in_block` of kept block `b`, or -1 when b is not a
 // block of the cache (a caller-supplied selection out of range: reported and
 // skipped, never dereferenced).

@@ -60,6 +60,7 @@ constexpr int kSplitThreads = 512;         // CTA of a split-row chunk
 constexpr int kMaxSplitChunks = 64;        // chunks per split row (the plan uses 32)
 constexpr int kWideStages = 8;             // cp.async slots per thread of the wide CTA
 constexpr int kWideRingBytes = kWideStages * kWideThreads * 16;
+constexpr int kFusedStride = 16;          // fused prefill selection: one sampled block in 16
 }
 
 // Per-CTA-size constants: each thread owns CAPL candidate slots.
@@ -403,9 +404,10 @@ __device__ void select_candidates(int cnt, int K, TopkShared<NT>& sh) {
 
 // Exact fallback streamed over the whole source (any n >= K): four radix
 // passes over global memory, then one pass in element (= index) order that
-// keeps every element above T and the lowest-indexed ones equal to T.
-template <int NT>
-__device__ void select_streamed(const RowSrc& src, int n, int K, TopkShared<NT>& sh) {
+// keeps every element above T and the lowest-indexed ones equal to T.  Src
+// provides key(i) and index(i) (a score row, or scores computed on the fly).
+template <int NT, class Src>
+__device__ void select_streamed(const Src& src, int n, int K, TopkShared<NT>& sh) {
   using namespace topk;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int above, equal;
@@ -615,6 +617,7 @@ __device__ void topk_select(const RowSrc& src, int n, int K, TopkShared<NT>& sh,
   if (nc >= K && sh.n_ovf <= OVF) {
     select_candidates(cnt, K, sh);              // 3.
   } else {
+    count_fallback();
     select_streamed(src, n, K, sh);             // exact fallback
   }
   (void)lane;
@@ -912,6 +915,7 @@ __global__ void __launch_bounds__(topk::kWideThreads, 1) topk_merge_kernel(Geo g
   const int total = start[n_ch_row];
   if (bad || total < K || total > CAP) {
     const RowSrc row{a.scores + tok * a.ld, nullptr, nullptr, 0};
+    count_fallback();
     select_streamed(row, (int)bt, K, sh);
   } else {
     int cnt = 0;
@@ -930,6 +934,206 @@ __global__ void __launch_bounds__(topk::kWideThreads, 1) topk_merge_kernel(Geo g
   }
   topk_write_final(sh, K, S, bt, a.sel + tok * S);
   if (threadIdx.x == 0) a.nsel[tok] = S;
+}
+
+// ---------------------------------------------------------------- fused prefill selection
+// Many rows of prefill-like segments skip the score matrix:
+//   1. the indexer scores an evenly spaced sample, pooled block j*stride;
+//   2. topk_tau_kernel: per row, the threshold key below which about
+//      kSampleTarget elements of the row are expected (the lower edge of the
+//      16-bit bucket of the sample's matching rank), and a zeroed count;
+//   3. the indexer in filter mode appends every candidate with score >= tau
+//      (the float of that key) to the row's list (up to CAP entries; the
+//      count keeps counting);
+//   4. topk_cand_kernel: when the list holds between K and CAP elements it
+//      holds every element of the row at or above the K-th largest, so the
+//      exact candidate selection gives the row's answer; otherwise an exact
+//      streamed selection runs over scores recomputed on CUDA cores.
+// Rows with n <= CAP take tau = 0 (every key passes); rows that keep every
+// block take tau = ~0 and need no candidates.
+struct FusedSelArgs {
+  const float* samples;          // [T][ld_s] sample scores (row j = block j*stride)
+  int64_t ld_s;
+  int stride;
+  float* tau;                    // [T] threshold (-inf: keep all, NaN: none)
+  const float* cand_score;       // [T][CAP]
+  const int32_t* cand_idx;       // [T][CAP]
+  int32_t* cand_cnt;             // [T]
+  int32_t* sel;                  // [T][S]
+  int32_t* nsel;                 // [T]
+  // exact fallback: scores recomputed from the indexer inputs
+  const __nv_bfloat16* q_idx;    // [T][4][DI]
+  const float* w;                // [T][4]
+  const __nv_bfloat16* khat;     // [n_slots][n_cap/r][DI]
+};
+
+// Lower edge of the 16-bit bucket (below the bits all keys share) holding
+// the rank-th largest key of row[0..n); at least `rank` keys are >= it.
+// Keys are staged in shared memory when they fit.  Ends with a barrier.
+template <int NT>
+__device__ uint32_t rank_threshold(const float* row, int n, int rank, TopkShared<NT>& sh) {
+  using namespace topk;
+  const bool staged = n <= kBufWords;
+  uint32_t vmin = 0xffffffffu, vmax = 0u;
+  for (int i = threadIdx.x; i < n; i += NT) {
+    const uint32_t k = score_key(row[i]);
+    if (staged) sh.cbuf[i] = k;
+    vmin = min(vmin, k);
+    vmax = max(vmax, k);
+  }
+  block_minmax(vmin, vmax, sh);
+  if (vmin == vmax) return vmin;
+  const int h = 31 - __clz(vmin ^ vmax);
+  uint32_t mask = h == 31 ? 0u : ~((2u << h) - 1u);
+  uint32_t prefix = vmin & mask;
+  int k_rem = rank;
+  for (int hi = h, pass = 0; hi >= 0 && pass < 2; hi -= 8, ++pass) {
+    const int lo = hi >= 7 ? hi - 7 : 0;
+    const uint32_t dm = (2u << (hi - lo)) - 1u;
+    hist_clear(sh);
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += NT) {
+      const uint32_t x = staged ? sh.cbuf[i] : score_key(row[i]);
+      if ((x & mask) == prefix) atomicAdd(&sh.hist[(x >> lo) & dm], 1u);
+    }
+    __syncthreads();
+    hist_locate(k_rem, sh);
+    k_rem -= sh.sel_above;
+    prefix |= sh.sel_digit << lo;
+    mask |= dm << lo;
+    __syncthreads();
+  }
+  return prefix;
+}
+
+struct FusedRow {
+  int64_t tok, t, bt, slot;
+};
+
+__device__ __forceinline__ FusedRow fused_row(const Geo& g, const SegTable& st, int item) {
+  FusedRow r;
+  const int si = find_segment(st, item);
+  const int j = item - st.item0[si];
+  r.tok = st.q_offset[si] + j;
+  r.t = (int64_t)st.pos0[si] + j;
+  r.bt = r.t / g.r;
+  r.slot = st.slot[si];
+  return r;
+}
+
+__global__ void __launch_bounds__(topk::THREADS, 6) topk_tau_kernel(Geo g, SegTable st, FusedSelArgs a) {
+  using namespace topk;
+  pdl_wait();
+  pdl_trigger();
+  __shared__ TopkShared<topk::THREADS> sh;
+  const int n_items = st.item0[st.n];
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const FusedRow r = fused_row(g, st, item);
+    uint32_t tkey;
+    if (r.bt + 1 <= g.S) {
+      tkey = 0xffffffffu;                        // every block is kept: no candidates needed (NaN)
+    } else if (r.bt <= CAP) {
+      tkey = 0u;                                 // every element fits the list (-inf)
+    } else {
+      const int n = (int)r.bt;
+      const int n_s = (int)cdiv(n, a.stride);    // samples j*stride < n
+      const int rank = max(1, (int)((int64_t)n_s * kSampleTarget / n));
+      tkey = rank_threshold(a.samples + r.tok * a.ld_s, n_s, rank, sh);
+    }
+    if (threadIdx.x == 0) {
+      a.tau[r.tok] = key_to_float(tkey);         // score >= it  <=>  key >= tkey
+      a.cand_cnt[r.tok] = 0;
+    }
+    __syncthreads();                             // shared state is reused by the next item
+  }
+}
+
+// Scores of one row computed on CUDA cores for the exact fallback: element i
+// is block i, s = sum_h w_h ReLU(q~_h . k^_i) with q~ (rotated, rounded to
+// bf16 like the tensor-core path) staged in shared memory as fp32.
+struct ComputedRow {
+  const float* qt;               // [4][DI] shared
+  const __nv_bfloat16* kh;       // the slot's k^ rows
+  float4 w;
+  int DI;
+  __device__ __forceinline__ uint32_t key(int i) const {
+    const uint4* kr = reinterpret_cast<const uint4*>(kh + (int64_t)i * DI);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int c = 0; c < DI / 8; ++c) {
+      const uint4 raw = kr[c];
+      const __nv_bfloat16* kv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float x = __bfloat162float(kv[e]);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) acc[h] = fmaf(qt[h * DI + 8 * c + e], x, acc[h]);
+      }
+    }
+    float s = 0.f;
+    s = fmaf(w.x, fmaxf(acc[0], 0.f), s);
+    s = fmaf(w.y, fmaxf(acc[1], 0.f), s);
+    s = fmaf(w.z, fmaxf(acc[2], 0.f), s);
+    s = fmaf(w.w, fmaxf(acc[3], 0.f), s);
+    return score_key(s);
+  }
+  __device__ __forceinline__ uint32_t index(int i) const { return (uint32_t)i; }
+};
+
+__global__ void __launch_bounds__(topk::THREADS, 6) topk_cand_kernel(Geo g, SegTable st, FusedSelArgs a) {
+  using namespace topk;
+  pdl_wait();
+  pdl_trigger();
+  __shared__ TopkShared<topk::THREADS> sh;
+  const int n_items = st.item0[st.n];
+  const int S = g.S, K = S - 1;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const FusedRow r = fused_row(g, st, item);
+    int32_t* sel_row = a.sel + r.tok * S;
+    if (r.bt + 1 <= S) {
+      for (int i = threadIdx.x; i < S; i += blockDim.x) sel_row[i] = (i <= r.bt) ? i : -1;
+      if (threadIdx.x == 0) a.nsel[r.tok] = (int32_t)(r.bt + 1);
+      continue;
+    }
+    if (threadIdx.x == 0) {
+      sh.n_kept = 0;
+      sh.n_ovf = 0;
+    }
+    const int nc = a.cand_cnt[r.tok];
+    __syncthreads();
+    if (nc >= K && nc <= CAP) {
+      // at most CAP/THREADS per thread: CAPL own slots, the rest (<= OVF in all) in overflow
+      int cnt = 0;
+      const int64_t base = r.tok * (int64_t)CAP;
+      for (int i = threadIdx.x; i < nc; i += THREADS)
+        cand_append(score_key(a.cand_score[base + i]), (uint32_t)a.cand_idx[base + i], cnt, sh);
+      __syncthreads();
+      select_candidates(cnt, K, sh);
+    } else {
+      count_fallback();
+      float* qt = reinterpret_cast<float*>(sh.cbuf);        // unused by the streamed selection
+      const int DI = g.DI, half = g.rope_half;
+      const __nv_bfloat16* qr = a.q_idx + r.tok * 4 * (int64_t)DI;
+      for (int e = threadIdx.x; e < 4 * DI; e += THREADS) {
+        const int h = e / DI, d = e - h * DI;
+        float v = __bfloat162float(qr[e]);
+        if (d < 2 * half) {
+          const int p = d < half ? d : d - half;
+          float c, sn, o0, o1;
+          rope_cs(g, r.t, p, c, sn);
+          rope_pair(__bfloat162float(qr[h * DI + p]), __bfloat162float(qr[h * DI + p + half]), c, sn, o0, o1);
+          v = __bfloat162float(__float2bfloat16_rn(d < half ? o0 : o1));
+        }
+        qt[e] = v;
+      }
+      __syncthreads();
+      const float4 w4 = *reinterpret_cast<const float4*>(a.w + r.tok * 4);
+      const ComputedRow src{qt, a.khat + r.slot * (g.n_cap / g.r) * (int64_t)DI, w4, DI};
+      select_streamed(src, (int)r.bt, K, sh);
+    }
+    topk_write_final(sh, K, S, r.bt, sel_row);
+    if (threadIdx.x == 0) a.nsel[r.tok] = S;
+    __syncthreads();                             // shared state is reused by the next item
+  }
 }
 
 }  // namespace qsa

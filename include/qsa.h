@@ -118,7 +118,8 @@ typedef enum {
   QSA_OP_INDEX = 1,
   QSA_OP_SELECT = 2,
   QSA_OP_ATTN = 3,
-  QSA_OP_FORWARD = 4
+  QSA_OP_FORWARD = 4,
+  QSA_OP_FORWARD_LOWMEM = 5
 } qsa_op_t;
 
 /*
@@ -225,6 +226,33 @@ qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cache,
                          void* stream);
 
 /*
+ * qsa_forward without the score matrix, for callers short of device memory.
+ * The design report's QSA item defines the indexer scores and the top-k;
+ * fusing them is this library's choice, not the pages'.  Same
+ * arguments, results and errors; workspace >= qsa_workspace_size(...,
+ * QSA_OP_FORWARD_LOWMEM).  For bf16 segments of 16 or more queries steps 2-3
+ * run fused: the indexer scores every 16th pooled block; a threshold per
+ * query is taken from that sample (about 1536 of the query's blocks are
+ * expected at or above it); a second indexer pass keeps only the (score,
+ * block) pairs at or above it, at most 4096 per query; the selection runs
+ * exactly on those.  A query whose list holds fewer than S-1 or more than
+ * 4096 pairs is selected exactly over all of its blocks, scores recomputed
+ * on CUDA cores (qsa_select_fallbacks counts these).  Selections equal
+ * qsa_forward's up to the rounding order of the scores.  Other segments run
+ * as in qsa_forward.
+ *
+ * Memory: 4*ceil(n_blocks/16) + 32 KiB per query instead of 4*n_blocks bytes
+ * (128K-token prefill: 5.6 GB instead of 17.2 GB).  Time: slower than
+ * qsa_forward on B200 (the filtering costs the indexer's epilogue more
+ * instructions than the score writes it saves).
+ */
+qsa_status_t qsa_forward_lowmem(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                                const void* q, const void* q_idx, const float* w, void* o, float* lse,
+                                int32_t* sel, int32_t* nsel, void* workspace, size_t ws_bytes,
+                                void* stream);
+
+/*
  * qsa_select_topk without a caller workspace, for callers that cannot call
  * cudaMalloc: code running where the allocator is off limits (a custom
  * allocator or memory pool owns all device memory, an embedding that forbids
@@ -262,6 +290,13 @@ size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* segs, in
 /* Reads and clears the current device's error word written by bounded
  * device-side waits; synchronises `stream`.  QSA_OK if no wait gave up. */
 qsa_status_t qsa_device_status(void* stream);
+
+/* Reads into *count and clears the number of query rows whose selection took
+ * an exact fallback since the last call: the sampled threshold admitted too
+ * few or too many candidates (a diagnostic of the selection's speed, not an
+ * error; the result is exact either way).  Synchronises `stream`.
+ * QSA_ERR_INVALID_ARG if count is NULL. */
+qsa_status_t qsa_select_fallbacks(void* stream, int64_t* count);
 
 /* Diagnostic for the failure path (the pages have no counterpart): enqueues
  * one kernel whose thread waits, through the same bounded wait the

@@ -56,7 +56,7 @@ def gpu_prepare_cache(wl: synth.Workload, x: Dict[str, torch.Tensor]):
     return cfg, cache, khat
 
 
-def gpu_forward(wl: synth.Workload, x: Dict[str, torch.Tensor]) -> GpuRun:
+def gpu_forward(wl: synth.Workload, x: Dict[str, torch.Tensor], lowmem: bool = False) -> GpuRun:
     sh = wl.shape
     cfg, cache, khat = gpu_prepare_cache(wl, x)
     segs = segments_of(wl)
@@ -65,9 +65,10 @@ def gpu_forward(wl: synth.Workload, x: Dict[str, torch.Tensor]) -> GpuRun:
     lse = torch.full((T, sh.n_heads), float("nan"), dtype=torch.float32, device="cuda")
     sel = torch.full((T, sh.budget_blocks), -7, dtype=torch.int32, device="cuda")
     nsel = torch.full((T,), -7, dtype=torch.int32, device="cuda")
-    ws = torch.empty(max(1, qsa.workspace_size(cfg, segs, T, qsa.QSA_OP_FORWARD)), dtype=torch.uint8,
-                     device="cuda")
-    qsa.qsa_forward(cfg, cache, segs, T, x["q"], x["q_idx"], x["w"], o, lse, sel, nsel, ws)
+    op = qsa.QSA_OP_FORWARD_LOWMEM if lowmem else qsa.QSA_OP_FORWARD
+    ws = torch.empty(max(1, qsa.workspace_size(cfg, segs, T, op)), dtype=torch.uint8, device="cuda")
+    fwd = qsa.qsa_forward_lowmem if lowmem else qsa.qsa_forward
+    fwd(cfg, cache, segs, T, x["q"], x["q_idx"], x["w"], o, lse, sel, nsel, ws)
     torch.cuda.synchronize()
     qsa.qsa_device_status()
     return GpuRun(o, lse, sel, nsel, khat)

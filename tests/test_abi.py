@@ -105,6 +105,16 @@ def test_workspace_sizes_are_host_only_and_grow_with_the_batch():
     b = qsa.workspace_size(cfg, big, 131072, qsa.QSA_OP_FORWARD)
     assert 0 < a < b
     assert b >= 131072 * 32767 * 4           # the score rows
+    # the low-memory forward keeps sample scores (every 16th of 32767 blocks)
+    # and 4096-entry candidate lists per query instead of the score rows
+    lo = qsa.workspace_size(cfg, big, 131072, qsa.QSA_OP_FORWARD_LOWMEM)
+    assert 131072 * (2048 * 4 + 4096 * 8) <= lo < 131072 * 32767 * 4 // 3
+    # fp32 and decode-like segments keep the score rows in both
+    sh32 = synth.Shape(dtype="f32")
+    b32 = qsa.workspace_size(qsa.make_config(sh32), big, 131072, qsa.QSA_OP_FORWARD_LOWMEM)
+    assert b32 >= 131072 * 32767 * 4
+    dec_fwd = qsa.make_segments([(i, 1, (1 << 20) - 1, i) for i in range(8)])
+    assert qsa.workspace_size(cfg, dec_fwd, 8, qsa.QSA_OP_FORWARD_LOWMEM) >= 8 * 262143 * 4
     assert qsa.workspace_size(cfg, small, 1024, qsa.QSA_OP_COMPRESS) == 0
     dec = qsa.make_segments([(i, 1, (1 << 20) - 1, i) for i in range(8)])
     assert qsa.workspace_size(cfg, dec, 8, qsa.QSA_OP_SELECT) > 0     # few long rows are split
