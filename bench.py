@@ -140,11 +140,22 @@ class Prepared:
         self.ws_attn = torch.empty(max(1, qsa.workspace_size(self.cfg, self.segs, T, qsa.QSA_OP_ATTN)),
                                    dtype=torch.uint8, device="cuda")
         self.ranges = [(s.slot, s.pos0 // sh.r, (s.pos0 + s.q_len) // sh.r) for s in wl.segments]
+        self.ws_low = None
 
-    def forward(self):
+    def workspace_bytes(self, lowmem: bool) -> int:
+        op = qsa.QSA_OP_FORWARD_LOWMEM if lowmem else qsa.QSA_OP_FORWARD
+        return qsa.workspace_size(self.cfg, self.segs, self.T, op)
+
+    def forward(self, lowmem: bool = False):
         x = self.x
-        qsa.qsa_forward(self.cfg, self.cache, self.segs, self.T, x["q"], x["q_idx"], x["w"], self.o, self.lse,
-                        self.sel, self.nsel, self.ws)
+        if lowmem:
+            if self.ws_low is None:
+                self.ws_low = torch.empty(max(1, self.workspace_bytes(True)), dtype=torch.uint8, device="cuda")
+            qsa.qsa_forward_lowmem(self.cfg, self.cache, self.segs, self.T, x["q"], x["q_idx"], x["w"], self.o,
+                                   self.lse, self.sel, self.nsel, self.ws_low)
+        else:
+            qsa.qsa_forward(self.cfg, self.cache, self.segs, self.T, x["q"], x["q_idx"], x["w"], self.o, self.lse,
+                            self.sel, self.nsel, self.ws)
 
     # the same four calls qsa_forward makes, one public entry point each
     def stage(self, i):
@@ -206,7 +217,7 @@ class L2Flush:
         torch.sum(self.r, dim=0, out=self.sink)
 
 
-def timed(prep: Prepared, steps: int, warmup: int, flush: L2Flush, staged: bool):
+def timed(prep: Prepared, steps: int, warmup: int, flush: L2Flush, staged: bool, lowmem: bool = False):
     """Device time of `steps` steps (ms each), L2 flushed before every step."""
     st = torch.cuda.current_stream()
     n_ev = 5 if staged else 2
@@ -216,7 +227,7 @@ def timed(prep: Prepared, steps: int, warmup: int, flush: L2Flush, staged: bool)
             for i in range(4):
                 prep.stage(i)
         else:
-            prep.forward()
+            prep.forward(lowmem)
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(steps)]
     launches0 = qsa.launch_count()
@@ -228,7 +239,7 @@ def timed(prep: Prepared, steps: int, warmup: int, flush: L2Flush, staged: bool)
                 prep.stage(i)
                 evs[s][i + 1].record(st)
         else:
-            prep.forward()
+            prep.forward(lowmem)
             evs[s][1].record(st)
     torch.cuda.synchronize()
     launches = qsa.launch_count() - launches0
@@ -555,6 +566,7 @@ def main():
                     help="workload of the attention-backward measurement; 'none' to skip")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-lowmem", action="store_true", help="skip the low-memory forward line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -586,6 +598,18 @@ def main():
         e2e_ms = max_over_ranks(e2e_ms, ws)
         e2e = {"value": job_throughput(tokens, e2e_ms, ws), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    lowmem = None
+    if not args.no_lowmem:
+        # the same step through qsa_forward_lowmem (no score matrix)
+        qsa.select_fallbacks()
+        barrier(ws)
+        per_l, launches_l = timed(prep, args.steps, args.warmup, flush, staged=False, lowmem=True)
+        barrier(ws)
+        ms_l = max_over_ranks(sum(p[0] for p in per_l) / args.steps, ws)
+        lowmem = {"ms_per_step": ms_l, "tokens_per_s": job_throughput(tokens, ms_l, ws),
+                  "workspace_bytes": prep.workspace_bytes(True), "workspace_bytes_default": prep.workspace_bytes(False),
+                  "fallback_rows": qsa.select_fallbacks(), "gpu_launches": launches_l}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -627,7 +651,7 @@ def main():
                            "parallelism": f"replicas x{ws}",
                            "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)"},
                 "roofline": roofline, "stages": m["stages"], "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": m["launches"], "clocks": m["clocks"]}
+                "gpu_launches": m["launches"], "clocks": m["clocks"], "lowmem_forward": lowmem}
         line.update(extra)
         print(json.dumps(line), flush=True)
     if ws > 1:
