@@ -247,22 +247,40 @@ def timed(prep: Prepared, steps: int, warmup: int, flush: L2Flush, staged: bool,
     return per, launches
 
 
-def e2e_prefill(prep: Prepared, steps: int, warmup: int):
-    """qsa_forward with every step's inputs copied from pinned host memory and its
-    output read back, all inside the timed region.  Steps are pipelined over
-    three streams (copy-in, compute, copy-out) with two device buffer sets, so
-    step i's compute overlaps step i+1's upload and step i-1's download."""
-    x = prep.x
-    slot = prep.wl.segments[0].slot
-    fill = prep.wl.fill[slot]
-    names = ["q", "q_idx", "w", "k_idx", "k", "v"]
-    views = [lambda d: d["q"], lambda d: d["q_idx"], lambda d: d["w"], lambda d: d["k_idx"][slot, :fill],
-             lambda d: d["k"][slot, :, :fill], lambda d: d["v"][slot, :, :fill]]
-    host = {n: f(x).cpu().pin_memory() for n, f in zip(names, views)}
+def e2e_prefill(prep: Prepared, steps: int, warmup: int, n_chunks: int = 8):
+    """The prefill step end to end through the public API: every step's inputs
+    are copied from pinned host memory and its output read back, all inside the
+    timed region.  A step runs as n_chunks chunked-prefill calls of qsa_forward
+    (query rows [r0, r1) at positions [r0, r1), each call pooling its own blocks
+    over the prefix the earlier calls pooled: the same results as one call), so
+    the upload of chunk j+1 and the download of chunk j-1 overlap chunk j's
+    compute.  Three streams (copy-in, compute, copy-out) and two device buffer
+    sets let consecutive steps overlap the same way."""
+    x, wl = prep.x, prep.wl
+    assert len(wl.segments) == 1 and wl.segments[0].pos0 == 0, "a prefill from position 0"
+    o_single = prep.o.cpu()                           # the single-call output of the device-timed steps
+    slot = wl.segments[0].slot
+    T = prep.T
+    G = prep.sh.n_groups
+    host = {"q": x["q"].cpu().pin_memory(), "q_idx": x["q_idx"].cpu().pin_memory(), "w": x["w"].cpu().pin_memory(),
+            "k_idx": x["k_idx"][slot, :T].cpu().pin_memory(), "k": x["k"][slot, :, :T].cpu().pin_memory(),
+            "v": x["v"][slot, :, :T].cpu().pin_memory()}
     o_host = torch.empty(prep.o.shape, dtype=prep.o.dtype).pin_memory()
     lse_host = torch.empty(prep.lse.shape, dtype=prep.lse.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * lse_host.element_size()
+    C = -(-T // n_chunks)
+    C = -(-C // 64) * 64
+    chunks = [(r0, min(T, r0 + C)) for r0 in range(0, T, C)]
+    chunk_segs = [qsa.make_segments([(r0, r1 - r0, r0, slot)]) for r0, r1 in chunks]
+
+    def pieces(d, r0, r1):
+        out = [(d["q"][r0:r1], host["q"][r0:r1]), (d["q_idx"][r0:r1], host["q_idx"][r0:r1]),
+               (d["w"][r0:r1], host["w"][r0:r1]), (d["k_idx"][slot, r0:r1], host["k_idx"][r0:r1])]
+        for g in range(G):
+            out += [(d["k"][slot, g, r0:r1], host["k"][g, r0:r1]), (d["v"][slot, g, r0:r1], host["v"][g, r0:r1])]
+        return out
+
     # two device buffer sets (inputs, caches, outputs); the score workspace is shared
     sets = []
     for b in range(2):
@@ -272,32 +290,35 @@ def e2e_prefill(prep: Prepared, steps: int, warmup: int):
         lse = prep.lse if b == 0 else torch.empty_like(prep.lse)
         sets.append(dict(d=d, khat=khat, o=o, lse=lse, cache=qsa.make_cache(d["k_idx"], khat, d["k"], d["v"])))
     s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ev = lambda: torch.cuda.Event()
-    in_done, cmp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    nc = len(chunks)
+    in_done = [[torch.cuda.Event() for _ in range(nc)] for _ in range(2)]
+    cmp_done = [[torch.cuda.Event() for _ in range(nc)] for _ in range(2)]
+    out_done = [[torch.cuda.Event() for _ in range(nc)] for _ in range(2)]
     used = [False, False]
 
     def step(i):
         b = i & 1
         st_ = sets[b]
-        with torch.cuda.stream(s_in):
-            if used[b]:
-                s_in.wait_event(cmp_done[b])          # compute of step i-2 is done with this set
-            for n, f in zip(names, views):
-                f(st_["d"]).copy_(host[n], non_blocking=True)
-            in_done[b].record(s_in)
-        with torch.cuda.stream(s_cmp):
-            s_cmp.wait_event(in_done[b])
-            if used[b]:
-                s_cmp.wait_event(out_done[b])         # download of step i-2 has read this set's output
-            d = st_["d"]
-            qsa.qsa_forward(prep.cfg, st_["cache"], prep.segs, prep.T, d["q"], d["q_idx"], d["w"], st_["o"],
-                            st_["lse"], prep.sel, prep.nsel, prep.ws, stream=s_cmp)
-            cmp_done[b].record(s_cmp)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(cmp_done[b])
-            o_host.copy_(st_["o"], non_blocking=True)
-            lse_host.copy_(st_["lse"], non_blocking=True)
-            out_done[b].record(s_out)
+        d = st_["d"]
+        for j, (r0, r1) in enumerate(chunks):
+            with torch.cuda.stream(s_in):
+                if used[b]:
+                    s_in.wait_event(cmp_done[b][j])      # compute of step i-2 is done with these rows
+                for dst, src in pieces(d, r0, r1):
+                    dst.copy_(src, non_blocking=True)
+                in_done[b][j].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(in_done[b][j])
+                if used[b]:
+                    s_cmp.wait_event(out_done[b][j])     # download of step i-2 has read these output rows
+                qsa.qsa_forward(prep.cfg, st_["cache"], chunk_segs[j], T, d["q"], d["q_idx"], d["w"], st_["o"],
+                                st_["lse"], prep.sel, prep.nsel, prep.ws, stream=s_cmp)
+                cmp_done[b][j].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(cmp_done[b][j])
+                o_host[r0:r1].copy_(st_["o"][r0:r1], non_blocking=True)
+                lse_host[r0:r1].copy_(st_["lse"][r0:r1], non_blocking=True)
+                out_done[b][j].record(s_out)
         used[b] = True
 
     for i in range(warmup):
@@ -314,8 +335,9 @@ def e2e_prefill(prep: Prepared, steps: int, warmup: int):
     s_out.wait_stream(s_cmp)
     e1.record(s_out)
     torch.cuda.synchronize()
+    ok = bool(torch.equal(o_host, o_single))
     del sets
-    return e0.elapsed_time(e1) / steps, h2d, d2h
+    return e0.elapsed_time(e1) / steps, h2d, d2h, nc, ok
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -594,10 +616,12 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e2e_ms, h2d, d2h = e2e_prefill(prep, args.steps, args.warmup)
+        e2e_ms, h2d, d2h, n_calls, same = e2e_prefill(prep, args.steps, args.warmup)
         e2e_ms = max_over_ranks(e2e_ms, ws)
         e2e = {"value": job_throughput(tokens, e2e_ms, ws), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "api": f"qsa_forward, {n_calls} chunked-prefill calls per step",
+               "output_matches_single_call": same}
 
     lowmem = None
     if not args.no_lowmem:
