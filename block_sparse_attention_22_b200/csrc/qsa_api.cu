@@ -409,13 +409,21 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
           return launch_chained(topk_merge_kernel, dim3(t.item0[t.n]), dim3(topk::kWideThreads), 0, st, g, t, a);
         });
   }
+  (void)smem_c;
+  // many rows: one warp per row (five 4-warp CTAs per SM), then a CTA-level
+  // selection of the rows it left (long rows, sampled thresholds that
+  // missed).  Plain launches: chained, the pair ran 1.7x slower (the
+  // dependent's CTAs, resident early, held the SMs the other grid needed).
   return for_each_table(
       segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
       [&](const SegTable& t) {
+        const int rows = t.item0[t.n];
+        const int grid = std::min((int)cdiv(rows, topk_w::WARPS), 5 * sm_count());
         count_launch();
-        // persistent: as many CTAs as fit (six per SM by shared memory)
-        const int grid = std::min(t.item0[t.n], 6 * sm_count());
-        return launch_chained(topk_chunk_kernel, dim3(grid), dim3(topk::THREADS), smem_c, st, g, t, a);
+        topk_rows_kernel<<<dim3(grid), dim3(topk_w::THREADS), 0, st>>>(g, t, a);
+        count_launch();
+        topk_rows_fallback_kernel<<<dim3(std::min(rows, 6 * sm_count())), dim3(topk::THREADS), 0, st>>>(g, t, a);
+        return cudaGetLastError();
       });
 }
 

@@ -6,9 +6,11 @@
 // always kept; the other S-1 are the best candidates b < floor(t/r) under
 // the total order (score descending, block index ascending), -0 == +0.
 //
-// One CTA per row: 4 warps, persistent over rows, ~35 KB of shared memory
-// so that six CTAs share an SM, when rows are many; 32 warps per row when
-// rows are few and at most 32K blocks long.  Scores are compared as 32-bit keys
+// Many rows: one warp per row (topk_rows_kernel, below), with the rows it
+// leaves selected by a 4-warp CTA each (~35 KB of shared memory, six CTAs per
+// SM); 32 warps per row when rows are few and at most 32K blocks long; split
+// chunks and a merge for few longer rows.  The CTA-level selection of one
+// row (topk_select) runs as follows.  Scores are compared as 32-bit keys
 // whose unsigned order is the float order.  For a row of n candidates and
 // K = S-1:
 //   1. threshold: m = n/16 keys (1024 .. 8192, in runs of 8 neighbours spread
@@ -784,31 +786,6 @@ __device__ void topk_chunk_row_threshold(const Geo& g, const TopkArgs& a, const 
   if (threadIdx.x == 0) a.cand_cnt[it.tok * a.max_ch + it.c] = nc;
 }
 
-// Many rows: persistent 4-warp CTAs, one row at a time.
-__global__ void __launch_bounds__(topk::THREADS, 6) topk_chunk_kernel(Geo g, SegTable st, TopkArgs a) {
-  using namespace topk;
-  pdl_wait();
-  pdl_trigger();
-  __shared__ TopkShared<topk::THREADS> sh;
-  const int n_items = st.item0[st.n];
-  const int S = g.S, K = S - 1;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const TopkItem it = topk_item(g, st, a, item);
-    if (it.skip) continue;
-    int32_t* sel_row = a.sel + it.tok * S;
-    if (it.all) {
-      for (int i = threadIdx.x; i < S; i += blockDim.x) sel_row[i] = (i <= it.bt) ? i : -1;
-      if (threadIdx.x == 0) a.nsel[it.tok] = (int32_t)(it.bt + 1);
-      continue;
-    }
-    const RowSrc src{a.scores + it.tok * a.ld, nullptr, nullptr, 0};
-    topk_select(src, it.n, K, sh);
-    topk_write_final(sh, K, S, it.bt, sel_row);
-    if (threadIdx.x == 0) a.nsel[it.tok] = S;
-    __syncthreads();                           // shared state is reused by the next item
-  }
-}
-
 // Few rows, each up to kWideMaxBlocks blocks: one CTA of kWideThreads per
 // row, streaming the row through cp.async slots.
 __global__ void __launch_bounds__(topk::kWideThreads, 1) topk_wide_kernel(Geo g, SegTable st, TopkArgs a) {
@@ -934,6 +911,336 @@ __global__ void __launch_bounds__(topk::kWideThreads, 1) topk_merge_kernel(Geo g
   }
   topk_write_final(sh, K, S, bt, a.sel + tok * S);
   if (threadIdx.x == 0) a.nsel[tok] = S;
+}
+
+// ---------------------------------------------------------------- many rows: one warp per row
+// The 4-warp CTA per row above spends most of a row in barrier-separated
+// phases with no loads in flight.  Here each warp selects its own row with
+// warp-synchronous steps only, so an SM has 20 rows in flight (4 warps x 5
+// CTAs) whose load phases overlap each other's selection phases:
+//   1. rows of at most CAPW candidates take them all; longer rows take the
+//      lower edge of the 16-bit bucket of the rank-th largest of m = n/16
+//      sampled keys (runs of 8 neighbours), rank chosen so that about TARGET
+//      elements of the row are expected at or above it;
+//   2. filter: 16-byte loads, U in flight per lane; the lanes' hits are
+//      compacted into the warp's list by a warp prefix sum;
+//   3. if the list holds K..CAPW elements: exact radix select (8-bit digits
+//      below the common high bits, then lowest indices among the ties);
+//   4. ordering through a bitmap of the row.
+// A row whose list holds fewer than K or more than CAPW elements is marked
+// (nsel = -1) and selected exactly by topk_rows_fallback_kernel.  Rows of
+// more than 64K blocks are marked -2 and left to that kernel's 4-warp CTAs:
+// one warp keeps too few loads in flight to stream them.
+namespace topk_w {
+constexpr int WARPS = 4;
+constexpr int THREADS = 32 * WARPS;
+constexpr int CAPW = 1024;                 // candidates a row may collect
+constexpr int BUFW = 2 * CAPW;             // keys | indices; reused for the sample and the bitmap
+constexpr int TARGET = 768;                // expected elements at or above the sampled threshold
+constexpr int MIN_S = 512;
+constexpr int MAX_S = 16384;               // samples beyond BUFW are re-read from the row each pass
+constexpr int U = 4;                       // 16-byte loads in flight per lane
+constexpr int64_t kMaxRowBlocks = (int64_t)BUFW * 32;   // the bitmap of the row fits the buffer
+}
+
+struct WarpRowShared {
+  uint32_t hist[topk::NBINS];
+  uint32_t buf[topk_w::BUFW];
+  uint32_t kept[topk::KMAX];
+};
+
+// Bin holding the k-th largest counted value: each lane owns 8 consecutive
+// bins; suffix sums run from the top bin down.  Returns the digit; *above =
+// count in higher bins, *count = the bin's count.  Warp-uniform results.
+__device__ __forceinline__ uint32_t warp_hist_locate(const uint32_t* hist, int k, int* above, int* count) {
+  const int lane = threadIdx.x & 31;
+  uint32_t b[8];
+  int local = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    b[j] = hist[lane * 8 + j];
+    local += (int)b[j];
+  }
+  int suf = local;                              // this lane and the lanes above it
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_down_sync(0xffffffffu, suf, off);
+    if (lane + off < 32) suf += v;
+  }
+  const int excl = suf - local;                 // lanes above
+  uint32_t digit = 0;
+  int ab = 0, cnt = 0;
+  const bool mine = excl < k && k <= suf;
+  if (mine) {
+    int run = excl;
+    for (int j = 7; j >= 0; --j) {
+      if (run + (int)b[j] >= k) {
+        digit = (uint32_t)(lane * 8 + j);
+        ab = run;
+        cnt = (int)b[j];
+        break;
+      }
+      run += (int)b[j];
+    }
+  }
+  const int src = max(0, __ffs(__ballot_sync(0xffffffffu, mine)) - 1);
+  *above = __shfl_sync(0xffffffffu, ab, src);
+  *count = __shfl_sync(0xffffffffu, cnt, src);
+  return __shfl_sync(0xffffffffu, digit, src);
+}
+
+// Radix select over n values val(i) (those with ok(i)) held by the warp:
+// passes of 8-bit digits from the highest bit where min and max differ; at
+// most `max_passes` passes (2: a 16-bit bucket).  Returns the prefix; *above
+// and *equal as in cand_radix.
+template <class Val, class Ok>
+__device__ uint32_t warp_radix(int n, int k, Val val, Ok ok, int* above, int* equal, uint32_t* hist,
+                               int max_passes = 4) {
+  const int lane = threadIdx.x & 31;
+  uint32_t vmin = 0xffffffffu, vmax = 0u;
+  int n_ok = 0;
+  for (int i = lane; i < n; i += 32) {
+    if (ok(i)) {
+      const uint32_t x = val(i);
+      vmin = min(vmin, x);
+      vmax = max(vmax, x);
+      ++n_ok;
+    }
+  }
+  vmin = __reduce_min_sync(0xffffffffu, vmin);
+  vmax = __reduce_max_sync(0xffffffffu, vmax);
+  n_ok = __reduce_add_sync(0xffffffffu, n_ok);
+  if (vmin == vmax) {
+    *above = 0;
+    *equal = n_ok;
+    return vmin;
+  }
+  const int h = 31 - __clz(vmin ^ vmax);
+  uint32_t mask = h == 31 ? 0u : ~((2u << h) - 1u);
+  uint32_t prefix = vmin & mask;
+  int k_rem = k, n_above = 0, count = n_ok;
+  for (int hi = h, pass = 0; hi >= 0 && pass < max_passes; hi -= 8, ++pass) {
+    const int lo = hi >= 7 ? hi - 7 : 0;
+    const uint32_t dm = (2u << (hi - lo)) - 1u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0u;
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+      if (ok(i)) {
+        const uint32_t x = val(i);
+        if ((x & mask) == prefix) atomicAdd(&hist[(x >> lo) & dm], 1u);
+      }
+    }
+    __syncwarp();
+    int ab, cnt;
+    const uint32_t d = warp_hist_locate(hist, k_rem, &ab, &cnt);
+    k_rem -= ab;
+    n_above += ab;
+    prefix |= d << lo;
+    mask |= dm << lo;
+    count = cnt;
+    __syncwarp();
+  }
+  *above = n_above;
+  *equal = count;
+  return prefix;
+}
+
+__global__ void __launch_bounds__(topk_w::THREADS, 5) topk_rows_kernel(Geo g, SegTable st, TopkArgs a) {
+  using namespace topk;
+  using namespace topk_w;
+  pdl_wait();
+  pdl_trigger();
+  __shared__ WarpRowShared shw[WARPS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  WarpRowShared& sh = shw[warp];
+  uint32_t* ckey = sh.buf;
+  uint32_t* cidx = sh.buf + CAPW;
+  const int n_items = st.item0[st.n];
+  const int S = g.S, K = S - 1;
+  const uint32_t below = (1u << lane) - 1u;
+  for (int item = blockIdx.x * WARPS + warp; item < n_items; item += gridDim.x * WARPS) {
+    const int si = find_segment(st, item);
+    const int j = item - st.item0[si];
+    const int64_t tok = st.q_offset[si] + j;
+    const int64_t bt = ((int64_t)st.pos0[si] + j) / g.r;
+    int32_t* sel_row = a.sel + tok * S;
+    if (bt + 1 <= S) {
+      for (int i = lane; i < S; i += 32) sel_row[i] = (i <= bt) ? i : -1;
+      if (lane == 0) a.nsel[tok] = (int32_t)(bt + 1);
+      continue;
+    }
+    if (bt > kMaxRowBlocks) {
+      if (lane == 0) a.nsel[tok] = -2;            // a long row: selected by a 4-warp CTA
+      continue;
+    }
+    const int n = (int)bt;
+    const float* row = a.scores + tok * a.ld;
+    // 1. threshold
+    uint32_t tkey = 0u;
+    if (n > CAPW) {
+      const int m0 = n / 16 < MIN_S ? MIN_S : (n / 16 > MAX_S ? MAX_S : n / 16);
+      const int groups = m0 / kSampleGroup;
+      const int m = groups * kSampleGroup;
+      // sample s: element gi*(n-8)/(groups-1) + j of group gi = s/8 (< n)
+      auto sample = [&](int s_i) -> uint32_t {
+        const int gi = s_i / kSampleGroup, jj = s_i - gi * kSampleGroup;
+        return score_key(row[(int64_t)gi * (n - kSampleGroup) / (groups - 1) + jj]);
+      };
+      const int rank = max(1, (int)((int64_t)m * TARGET / n));
+      int ab, eq;
+      if (m <= BUFW) {
+        for (int s_i = lane; s_i < m; s_i += 32) sh.buf[s_i] = sample(s_i);
+        __syncwarp();
+        tkey = warp_radix(
+            m, rank, [&](int i) { return sh.buf[i]; }, [](int) { return true; }, &ab, &eq, sh.hist, 2);
+      } else {
+        tkey = warp_radix(m, rank, sample, [](int) { return true; }, &ab, &eq, sh.hist, 2);
+      }
+      __syncwarp();
+    }
+    const float tau = key_to_float(tkey);
+    // 2. filter into the warp's list
+    int nc = 0;                                   // warp-uniform count (may exceed CAPW)
+    const int head = min(n, (int)(((16 - ((uintptr_t)row & 15)) & 15) / 4));
+    const int nvec = (n - head) / 4;
+    const int tail0 = head + nvec * 4;
+    {
+      // ragged ends: at most 3 + 3 elements, one per lane
+      const int e = lane < head ? lane : (lane >= 4 && lane < 4 + n - tail0 ? tail0 + lane - 4 : -1);
+      const float v = e >= 0 ? row[e] : 0.f;
+      const bool hit = e >= 0 && v >= tau;
+      const uint32_t m = __ballot_sync(0xffffffffu, hit);
+      const int pos = nc + __popc(m & below);
+      if (hit && pos < CAPW) {
+        ckey[pos] = score_key(v);
+        cidx[pos] = (uint32_t)e;
+      }
+      nc += __popc(m);
+    }
+    const float4* v4 = reinterpret_cast<const float4*>(row + head);
+    for (int b = 0; b < nvec; b += 32 * U) {
+      float4 x[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int vi = b + u * 32 + lane;
+        x[u] = vi < nvec ? __ldcs(v4 + vi) : make_float4(NAN, NAN, NAN, NAN);   // NaN never passes
+      }
+      int cnt = 0;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        cnt += (x[u].x >= tau) + (x[u].y >= tau) + (x[u].z >= tau) + (x[u].w >= tau);
+      int incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+      }
+      int o = nc + incl - cnt;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t i0 = (uint32_t)(head + 4 * (b + u * 32 + lane));
+        const float c4[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c4[c] >= tau) {
+            if (o < CAPW) {
+              ckey[o] = score_key(c4[c]);
+              cidx[o] = i0 + c;
+            }
+            ++o;
+          }
+        }
+      }
+      nc += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    __syncwarp();
+    if (nc < K || nc > CAPW) {
+      if (lane == 0) {
+        a.nsel[tok] = -1;                         // exact selection by the fallback kernel
+        atomicAdd(&g_qsa_select_fallbacks, 1ull);
+      }
+      continue;
+    }
+    // 3. exact selection among the nc candidates
+    int above, equal;
+    const uint32_t T = warp_radix(
+        nc, K, [&](int i) { return ckey[i]; }, [](int) { return true; }, &above, &equal, sh.hist);
+    const int need = K - above;
+    uint32_t imax = 0xffffffffu;
+    if (need < equal) {
+      int a2, e2;
+      imax = ~warp_radix(
+          nc, need, [&](int i) { return ~cidx[i]; }, [&](int i) { return ckey[i] == T; }, &a2, &e2, sh.hist);
+    }
+    int nk = 0;
+    for (int b = 0; b < nc; b += 32) {
+      const int i = b + lane;
+      const bool take = i < nc && (ckey[i] > T || (ckey[i] == T && cidx[i] <= imax));
+      const uint32_t m = __ballot_sync(0xffffffffu, take);
+      const int pos = nk + __popc(m & below);
+      if (take && pos < KMAX) sh.kept[pos] = cidx[i];
+      nk += __popc(m);
+    }
+    __syncwarp();
+    // 4. ascending order, the own block, padding
+    {
+      uint32_t* bm = sh.buf;                      // the candidates are no longer needed
+      const int nw = (int)((bt + 31) >> 5);
+      for (int w = lane; w < nw; w += 32) bm[w] = 0u;
+      __syncwarp();
+      for (int i = lane; i < K; i += 32) atomicOr(&bm[sh.kept[i] >> 5], 1u << (sh.kept[i] & 31));
+      __syncwarp();
+      const int wpl = (nw + 31) / 32;
+      const int w0 = min(nw, lane * wpl), w1 = min(nw, w0 + wpl);
+      int cnt = 0;
+      for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+      int incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+      }
+      int pos = incl - cnt;
+      for (int w = w0; w < w1; ++w) {
+        uint32_t bits = bm[w];
+        while (bits) {
+          const int bb = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          if (pos < K) sel_row[pos] = (int32_t)(w * 32 + bb);
+          ++pos;
+        }
+      }
+    }
+    for (int i = K + lane; i < S; i += 32) sel_row[i] = i == K ? (int32_t)bt : -1;
+    if (lane == 0) a.nsel[tok] = S;
+    __syncwarp();                                 // shared state is reused by the next row
+  }
+}
+
+// Rows topk_rows_kernel marked (nsel = -1 or -2): selection by a 4-warp CTA
+// (sampled threshold, filter, candidate selection, or the streamed fallback).
+// Launched without programmatic chaining and with no early trigger: its CTAs
+// mostly skip rows, and a dependent kernel made resident early would take
+// the SMs its remaining CTAs need.
+__global__ void __launch_bounds__(topk::THREADS, 6) topk_rows_fallback_kernel(Geo g, SegTable st, TopkArgs a) {
+  using namespace topk;
+  __shared__ TopkShared<topk::THREADS> sh;
+  const int n_items = st.item0[st.n];
+  const int S = g.S, K = S - 1;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int si = find_segment(st, item);
+    const int j = item - st.item0[si];
+    const int64_t tok = st.q_offset[si] + j;
+    const int mark = a.nsel[tok];
+    if (mark != -1 && mark != -2) continue;      // uniform across the CTA
+    const int64_t bt = ((int64_t)st.pos0[si] + j) / g.r;
+    const RowSrc src{a.scores + tok * a.ld, nullptr, nullptr, 0};
+    topk_select(src, (int)bt, K, sh);
+    topk_write_final(sh, K, S, bt, a.sel + tok * S);
+    if (threadIdx.x == 0) a.nsel[tok] = S;
+    __syncthreads();
+  }
 }
 
 // ---------------------------------------------------------------- fused prefill selection

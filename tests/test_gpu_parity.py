@@ -123,6 +123,39 @@ def test_select_topk_matches_oracle_on_seeded_rows(lengths, ties):
         np.testing.assert_array_equal(sel[i].cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("tie_levels", [None, 2, 1000])
+def test_select_many_rows_matches_oracle(tie_levels):
+    """700 rows, enough for the many-rows kernel (one warp per row): lengths on
+    both sides of every threshold it has (S, the list capacity 1024, the
+    sampled threshold, 64K blocks for the bitmap ordering), random keys, two
+    tie levels (every list overflows: the exact fallback) or a thousand levels
+    (many ties at the K-th key)."""
+    S = 512
+    cfg_sh = synth.Shape()
+    cfg = qsa.make_config(cfg_sh)
+    base = [1, 3, 511, 512, 513, 600, 1023, 1024, 1025, 1536, 2047, 4096, 16384, 32767, 65535, 65536, 70001]
+    lengths = [base[i % len(base)] for i in range(700)]
+    rows = _score_rows(11 + (tie_levels or 0), lengths, tie_levels)
+    segs = qsa.make_segments([(i, 1, 4 * n + 3, 0) for i, n in enumerate(lengths)])
+    T = len(lengths)
+    sc = rows.cuda().contiguous()
+    sel = torch.full((T, S), -7, dtype=torch.int32, device="cuda")
+    nsel = torch.full((T,), -7, dtype=torch.int32, device="cuda")
+    ws = torch.empty(max(1, qsa.workspace_size(cfg, segs, T, qsa.QSA_OP_SELECT)), dtype=torch.uint8, device="cuda")
+    qsa.select_fallbacks()
+    qsa.qsa_select_topk(cfg, segs, T, sc, sc.shape[1], sel, nsel, ws)
+    torch.cuda.synchronize()
+    fallbacks = qsa.select_fallbacks()
+    if tie_levels == 2:
+        assert fallbacks > 0
+    rc = oracle.config_from_shape(cfg_sh)
+    sel_c, nsel_c = sel.cpu().numpy(), nsel.cpu().numpy()
+    for i, n in enumerate(lengths):
+        ref, rn = oracle.select(rc, rows[i, :n].double().numpy(), 4 * n + 3)
+        assert int(nsel_c[i]) == rn, i
+        np.testing.assert_array_equal(sel_c[i], ref, err_msg=f"row {i} length {n}")
+
+
 # --------------------------------------------------------------------------- stage: attention
 @pytest.mark.parametrize("name,over,every", [
     ("tiny_fp32", {}, 1),
