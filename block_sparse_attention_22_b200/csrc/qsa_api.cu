@@ -13,6 +13,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <functional>
 #include <vector>
 
 #include "qsa_internal.cuh"
@@ -303,19 +304,32 @@ struct FusedBufs {
 
 qsa_status_t run_fused_select(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
                               const qsa_segment_t* segs, int n, const void* q_idx, const float* w,
-                              const FusedBufs& f, int32_t* sel, int32_t* nsel, cudaStream_t st) {
+                              const FusedBufs& f, int32_t* sel, int32_t* nsel, cudaStream_t st,
+                              const std::function<qsa_status_t()>& after_filter = nullptr) {
   constexpr int kStride = topk::kFusedStride;
   CUtensorMap tm_s, tm;
   if (!make_khat_map(&tm_s, c, cache, kStride) || !make_khat_map(&tm, c, cache, 1)) return QSA_ERR_CUDA;
+  // prefill-like segments on 64-query index tiles, decode-like ones on 4-query tiles
+  std::vector<qsa_segment_t> wide, narrow;
+  for (int i = 0; i < n; ++i) (segs[i].q_len >= 16 ? wide : narrow).push_back(segs[i]);
+  auto index_pass = [&](const IndexTcArgs& a, const CUtensorMap& m) -> qsa_status_t {
+    qsa_status_t r = for_each_table(
+        wide.data(), (int)wide.size(),
+        [&](const qsa_segment_t& s) { return index_tc_units<64>(s.q_len, s.pos0, g.r, a.stride); },
+        [&](const SegTable& t) { return launch_index_tc<64>(g, t, m, a, st); });
+    if (r != QSA_OK) return r;
+    return for_each_table(
+        narrow.data(), (int)narrow.size(),
+        [&](const qsa_segment_t& s) { return index_tc_units<4>(s.q_len, s.pos0, g.r, a.stride); },
+        [&](const SegTable& t) { return launch_index_tc<4>(g, t, m, a, st); });
+  };
   IndexTcArgs a{};
   a.q_idx = (const __nv_bfloat16*)q_idx;
   a.w = w;
   a.scores = f.samples;
   a.ld = f.ld_s;
   a.stride = kStride;
-  qsa_status_t r = for_each_table(
-      segs, n, [&](const qsa_segment_t& s) { return index_tc_units<64>(s.q_len, s.pos0, g.r, kStride); },
-      [&](const SegTable& t) { return launch_index_tc<64>(g, t, tm_s, a, st); });
+  qsa_status_t r = index_pass(a, tm_s);
   if (r != QSA_OK) return r;
   FusedSelArgs fa;
   memset(&fa, 0, sizeof fa);
@@ -331,12 +345,19 @@ qsa_status_t run_fused_select(const Geo& g, const qsa_config_t* c, const qsa_cac
   fa.q_idx = (const __nv_bfloat16*)q_idx;
   fa.w = w;
   fa.khat = (const __nv_bfloat16*)cache->khat;
+  // many rows: a 4-warp CTA per row, six per SM; few rows: 32 warps per row
+  const bool many = seg_rows(segs, n) >= 4 * kNumSms;
   const int ctas = 6 * sm_count();
   auto rows = [](const qsa_segment_t& s) { return (int64_t)s.q_len; };
-  r = for_each_table(segs, n, rows, [&](const SegTable& t) {
-    count_launch();
-    return launch_chained(topk_tau_kernel, dim3(std::min(t.item0[t.n], ctas)), dim3(topk::THREADS), 0, st, g, t, fa);
-  });
+  auto per_row = [&](auto kernel_many, auto kernel_few) {
+    return for_each_table(segs, n, rows, [&](const SegTable& t) {
+      count_launch();
+      const int items = t.item0[t.n];
+      return many ? launch_chained(kernel_many, dim3(std::min(items, ctas)), dim3(topk::THREADS), 0, st, g, t, fa)
+                  : launch_chained(kernel_few, dim3(items), dim3(topk::kWideThreads), 0, st, g, t, fa);
+    });
+  };
+  r = per_row(topk_tau_kernel<topk::THREADS>, topk_tau_kernel<topk::kWideThreads>);
   if (r != QSA_OK) return r;
   a.scores = nullptr;
   a.ld = 0;
@@ -346,14 +367,9 @@ qsa_status_t run_fused_select(const Geo& g, const qsa_config_t* c, const qsa_cac
   a.cand_idx = f.cand_idx;
   a.cand_cnt = f.cand_cnt;
   a.cand_cap = topk::CAP;
-  r = for_each_table(
-      segs, n, [&](const qsa_segment_t& s) { return index_tc_units<64>(s.q_len, s.pos0, g.r, 1); },
-      [&](const SegTable& t) { return launch_index_tc<64>(g, t, tm, a, st); });
-  if (r != QSA_OK) return r;
-  return for_each_table(segs, n, rows, [&](const SegTable& t) {
-    count_launch();
-    return launch_chained(topk_cand_kernel, dim3(std::min(t.item0[t.n], ctas)), dim3(topk::THREADS), 0, st, g, t, fa);
-  });
+  if ((r = index_pass(a, tm)) != QSA_OK) return r;
+  if (after_filter && (r = after_filter()) != QSA_OK) return r;
+  return per_row(topk_cand_kernel<topk::THREADS>, topk_cand_kernel<topk::kWideThreads>);
 }
 
 qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const float* scores,
@@ -557,14 +573,20 @@ qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* ca
 }
 
 // ------------------------------------------------------------------ forward workspace
-// In the low-memory forward, prefill-like segments (64-query index tiles) of
-// the bf16 path select through the fused path; the others (decode-like, or
-// fp32), and every segment of the default forward, through the score matrix.
-bool fused_segment(const qsa_segment_t& s, bool tc, bool lowmem) { return lowmem && tc && s.q_len >= 16; }
+// Segments that select through the fused path (no score rows): in the
+// low-memory forward, the bf16 prefill-like segments (64-query index tiles).
+// Decode-like segments keep their score rows in both forwards: their rows are
+// few, and for them the sample pass, the thresholds and the candidate
+// selection took longer than the split selection they replace (1M-context
+// decode step 0.164 ms against 0.144 ms).
+bool fused_segment(const qsa_segment_t& s, bool tc, bool lowmem, int r) {
+  (void)r;
+  return lowmem && tc && s.q_len >= 16;
+}
 
-void split_fused(const qsa_segment_t* segs, int n, bool tc, bool lowmem, std::vector<qsa_segment_t>& fused,
+void split_fused(const qsa_segment_t* segs, int n, bool tc, bool lowmem, int r, std::vector<qsa_segment_t>& fused,
                  std::vector<qsa_segment_t>& plain) {
-  for (int i = 0; i < n; ++i) (fused_segment(segs[i], tc, lowmem) ? fused : plain).push_back(segs[i]);
+  for (int i = 0; i < n; ++i) (fused_segment(segs[i], tc, lowmem, r) ? fused : plain).push_back(segs[i]);
 }
 
 struct FwdLayout {
@@ -575,7 +597,7 @@ struct FwdLayout {
 
 FwdLayout fwd_layout(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens, bool tc, bool lowmem) {
   std::vector<qsa_segment_t> fused, plain;
-  split_fused(segs, n, tc, lowmem, fused, plain);
+  split_fused(segs, n, tc, lowmem, g.r, fused, plain);
   FwdLayout L;
   L.ld = std::max<int64_t>(4, cdiv(seg_max_blocks(plain.data(), (int)plain.size(), g.r), 4) * 4);
   const int64_t nb_f = seg_max_blocks(fused.data(), (int)fused.size(), g.r);
@@ -760,7 +782,7 @@ qsa_status_t forward_impl(const qsa_config_t* cfg, const qsa_cache_t* cache, con
     nsel = (int32_t*)(ws + L.nsel);
   }
   std::vector<qsa_segment_t> fused, plain;
-  split_fused(segs, n_segs, cfg->dtype == QSA_DTYPE_BF16, lowmem, fused, plain);
+  split_fused(segs, n_segs, cfg->dtype == QSA_DTYPE_BF16, lowmem, g.r, fused, plain);
   // 1. pool the blocks each segment completes
   std::vector<int32_t> slots;
   std::vector<int64_t> b0, b1;
@@ -773,26 +795,36 @@ qsa_status_t forward_impl(const qsa_config_t* cfg, const qsa_cache_t* cache, con
     own_blocks_only &= ((int64_t)segs[i].pos0 + segs[i].q_len - 1) / cfg->r <= segs[i].pos0 / cfg->r;
   }
   const int n_plain = (int)plain.size();
+  auto compress = [&](bool late) {
+    return run_compress(g, cfg, cache, slots.data(), b0.data(), b1.data(), (int)slots.size(), st, late);
+  };
+  bool pooled = false;
   if (own_blocks_only) {
-    // decode-like batch (no prefill-like segment completes no block): the
-    // indexer reads no block pooled now, so the pooling runs alongside it
-    // (its exit still waits for the indexer)
-    if ((s = run_index(g, cfg, cache, plain.data(), n_plain, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
-    s = run_compress(g, cfg, cache, slots.data(), b0.data(), b1.data(), (int)slots.size(), st, true);
-    if (s != QSA_OK) return s;
+    // decode-like batch: no query scores a block pooled now, so the pooling
+    // runs alongside the indexer (its exit still waits for the indexer)
+    if (n_plain > 0) {
+      if ((s = run_index(g, cfg, cache, plain.data(), n_plain, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
+      if ((s = compress(true)) != QSA_OK) return s;
+      pooled = true;
+    }
   } else {
-    s = run_compress(g, cfg, cache, slots.data(), b0.data(), b1.data(), (int)slots.size(), st);
-    if (s != QSA_OK) return s;
+    if ((s = compress(false)) != QSA_OK) return s;
+    pooled = true;
     // 2. indexer scores of the plain segments
     if ((s = run_index(g, cfg, cache, plain.data(), n_plain, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
   }
-  // 2-3. fused scoring and selection of the prefill-like segments
+  // 2-3. fused scoring and selection (alongside the filtered scoring pass, the
+  // pooling of a decode-like batch that has not run yet)
   if (!fused.empty()) {
     const FusedBufs f{(float*)(ws + L.samples), L.ld_s, (float*)(ws + L.tau), (float*)(ws + L.ckey),
                       (int32_t*)(ws + L.cidx), (int32_t*)(ws + L.cnt)};
-    if ((s = run_fused_select(g, cfg, cache, fused.data(), (int)fused.size(), q_idx, w, f, sel, nsel, st)) != QSA_OK)
-      return s;
+    std::function<qsa_status_t()> hook;
+    if (!pooled) hook = [&]() { return compress(true); };
+    s = run_fused_select(g, cfg, cache, fused.data(), (int)fused.size(), q_idx, w, f, sel, nsel, st, hook);
+    if (s != QSA_OK) return s;
+    pooled = true;
   }
+  if (!pooled && (s = compress(true)) != QSA_OK) return s;
   // 3. selection of the plain segments, 4. attention
   if (n_plain > 0 &&
       (s = run_select(g, plain.data(), n_plain, scores, L.ld, sel, nsel, ws + L.topk, L.attn - L.topk, st)) != QSA_OK)

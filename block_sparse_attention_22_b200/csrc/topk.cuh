@@ -1328,11 +1328,14 @@ __device__ __forceinline__ FusedRow fused_row(const Geo& g, const SegTable& st, 
   return r;
 }
 
-__global__ void __launch_bounds__(topk::THREADS, 6) topk_tau_kernel(Geo g, SegTable st, FusedSelArgs a) {
+// NT threads per row: 128 when rows are many (six CTAs per SM), 1024 when
+// they are few (decode).
+template <int NT>
+__global__ void __launch_bounds__(NT, NT >= 512 ? 1 : 6) topk_tau_kernel(Geo g, SegTable st, FusedSelArgs a) {
   using namespace topk;
   pdl_wait();
   pdl_trigger();
-  __shared__ TopkShared<topk::THREADS> sh;
+  __shared__ TopkShared<NT> sh;
   const int n_items = st.item0[st.n];
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const FusedRow r = fused_row(g, st, item);
@@ -1386,11 +1389,12 @@ struct ComputedRow {
   __device__ __forceinline__ uint32_t index(int i) const { return (uint32_t)i; }
 };
 
-__global__ void __launch_bounds__(topk::THREADS, 6) topk_cand_kernel(Geo g, SegTable st, FusedSelArgs a) {
+template <int NT>
+__global__ void __launch_bounds__(NT, NT >= 512 ? 1 : 6) topk_cand_kernel(Geo g, SegTable st, FusedSelArgs a) {
   using namespace topk;
   pdl_wait();
   pdl_trigger();
-  __shared__ TopkShared<topk::THREADS> sh;
+  __shared__ TopkShared<NT> sh;
   const int n_items = st.item0[st.n];
   const int S = g.S, K = S - 1;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
@@ -1408,10 +1412,10 @@ __global__ void __launch_bounds__(topk::THREADS, 6) topk_cand_kernel(Geo g, SegT
     const int nc = a.cand_cnt[r.tok];
     __syncthreads();
     if (nc >= K && nc <= CAP) {
-      // at most CAP/THREADS per thread: CAPL own slots, the rest (<= OVF in all) in overflow
+      // at most CAP/NT per thread: CAPL own slots, the rest (<= OVF in all) in overflow
       int cnt = 0;
       const int64_t base = r.tok * (int64_t)CAP;
-      for (int i = threadIdx.x; i < nc; i += THREADS)
+      for (int i = threadIdx.x; i < nc; i += NT)
         cand_append(score_key(a.cand_score[base + i]), (uint32_t)a.cand_idx[base + i], cnt, sh);
       __syncthreads();
       select_candidates(cnt, K, sh);
@@ -1420,7 +1424,7 @@ __global__ void __launch_bounds__(topk::THREADS, 6) topk_cand_kernel(Geo g, SegT
       float* qt = reinterpret_cast<float*>(sh.cbuf);        // unused by the streamed selection
       const int DI = g.DI, half = g.rope_half;
       const __nv_bfloat16* qr = a.q_idx + r.tok * 4 * (int64_t)DI;
-      for (int e = threadIdx.x; e < 4 * DI; e += THREADS) {
+      for (int e = threadIdx.x; e < 4 * DI; e += NT) {
         const int h = e / DI, d = e - h * DI;
         float v = __bfloat162float(qr[e]);
         if (d < 2 * half) {

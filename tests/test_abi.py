@@ -113,8 +113,10 @@ def test_workspace_sizes_are_host_only_and_grow_with_the_batch():
     sh32 = synth.Shape(dtype="f32")
     b32 = qsa.workspace_size(qsa.make_config(sh32), big, 131072, qsa.QSA_OP_FORWARD_LOWMEM)
     assert b32 >= 131072 * 32767 * 4
+    # decode-like rows keep their score rows in both forwards
     dec_fwd = qsa.make_segments([(i, 1, (1 << 20) - 1, i) for i in range(8)])
-    assert qsa.workspace_size(cfg, dec_fwd, 8, qsa.QSA_OP_FORWARD_LOWMEM) >= 8 * 262143 * 4
+    for op in (qsa.QSA_OP_FORWARD, qsa.QSA_OP_FORWARD_LOWMEM):
+        assert qsa.workspace_size(cfg, dec_fwd, 8, op) >= 8 * 262143 * 4
     assert qsa.workspace_size(cfg, small, 1024, qsa.QSA_OP_COMPRESS) == 0
     dec = qsa.make_segments([(i, 1, (1 << 20) - 1, i) for i in range(8)])
     assert qsa.workspace_size(cfg, dec, 8, qsa.QSA_OP_SELECT) > 0     # few long rows are split

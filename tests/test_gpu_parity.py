@@ -204,6 +204,8 @@ def test_attention_parity_on_oracle_selection(name, over, every):
     ("prefill_8k", dict(n=2500, n_seqs=2), 7, 0.99),
     ("decode_256k", dict(ctx=20001, n_seqs=4), 1, 0.99),
     ("spec_decode_1m", dict(ctx=20001, n_seqs=3), 1, 0.99),     # 4 queries share a k^ stream
+    ("decode_256k", dict(ctx=140001, n_seqs=3), 1, 0.99),      # rows past 32K blocks: split selection
+    ("spec_decode_1m", dict(ctx=140001, n_seqs=2), 1, 0.99),
     ("mixed_1m", dict(ctx=16384, n_decode=3, chunk=300, chunk_pos0=5001), 3, 0.99),
 ])
 def test_forward_parity_small(name, over, every, min_exact):
