@@ -549,6 +549,15 @@ def traffic_record(kernel: str, alg_bytes: float):
     return None
 
 
+def bench_config(name: str, wl: synth.Workload, ws: int) -> dict:
+    """The workload description both arms print."""
+    return {"workload": name, "batch": len(wl.segments), "seq_len": wl.segments[0].q_len,
+            "budget_tokens": wl.shape.budget_tokens, "heads": wl.shape.n_heads, "kv_groups": wl.shape.n_groups,
+            "head_dim": wl.shape.head_dim, "idx_heads": wl.shape.idx_heads, "idx_dim": wl.shape.idx_dim,
+            "parallelism": f"replicas x{ws}",
+            "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)"}
+
+
 def run_reference(args):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -568,7 +577,7 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": wl.n_tokens / val * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": args.workload, "tokens_per_step": wl.n_tokens},
+            "config": bench_config(args.workload, wl, ws),
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -668,12 +677,7 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": m["fused_ms"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": wl.shape.dtype, "data": "synthetic",
-                "config": {"workload": args.workload, "batch": len(wl.segments), "seq_len": wl.segments[0].q_len,
-                           "budget_tokens": wl.shape.budget_tokens, "heads": wl.shape.n_heads,
-                           "kv_groups": wl.shape.n_groups, "head_dim": wl.shape.head_dim,
-                           "idx_heads": wl.shape.idx_heads, "idx_dim": wl.shape.idx_dim,
-                           "parallelism": f"replicas x{ws}",
-                           "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)"},
+                "config": bench_config(args.workload, wl, ws),
                 "roofline": roofline, "stages": m["stages"], "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": m["launches"], "clocks": m["clocks"], "lowmem_forward": lowmem}
         line.update(extra)
