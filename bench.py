@@ -466,10 +466,13 @@ def measure(prep: Prepared, steps, warmup, ws, flush, peaks, clocks=None):
 def measure_backward(name, steps, warmup, ws, flush, peaks):
     """qsa_sparse_attn_bwd on one workload: the forward runs once for o, lse and
     the selection; each timed step zeroes dk/dv (outside the events) and runs the
-    backward.  Algorithmic work: five dot products of head_dim per (head, kept
-    key) -- scores, dp, and the dq, dk, dv contributions -- on CUDA cores, so the
-    roofline is the fp32 FMA peak from the unit count and clock (148 SMs x 128
-    lanes x 2 flop x 1.965 GHz)."""
+    backward.  Algorithmic work per (query, group, kept key): five dot products
+    of head_dim per head (scores, dp, and the dq, dk, dv contributions), the K
+    and V rows read (2 x 256 x 2 B) and the dK and dV rows accumulated (read and
+    written: 2 x 2 x 256 x 4 B).  bf16 runs on tensor cores and streams that
+    traffic: roofline against the HBM copy peak (tensor fraction alongside);
+    fp32 runs on CUDA cores: roofline against the fp32 FMA peak from the unit
+    count and clock (148 SMs x 128 lanes x 2 flop x 1.965 GHz)."""
     wl = synth.make_workload(name)
     prep = Prepared(wl)
     prep.forward()
@@ -508,13 +511,23 @@ def measure_backward(name, steps, warmup, ws, flush, peaks):
     pos = wl.token_positions().double()
     keys = float((torch.clamp(torch.floor(pos / sh.r) + 1, max=sh.budget_blocks) * sh.r).sum().item())
     flops = 10.0 * sh.head_dim * sh.n_heads * keys
-    peak = 148 * 128 * 2 * 1.965e9 / 1e12
     tflops = flops / (ms * 1e-3) / 1e12
+    D, H, G = sh.head_dim, sh.n_heads, sh.n_groups
     del prep
     torch.cuda.empty_cache()
-    return {"workload": name, "ms_per_step": ms, "tokens_per_s": job_throughput(T, ms, ws),
-            "roofline": {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
-                         "frac": tflops / peak, "peak_source": "fp32 FMA lanes x clock (148 x 128 x 2 x 1.965 GHz)"}}
+    out = {"workload": name, "ms_per_step": ms, "tokens_per_s": job_throughput(T, ms, ws)}
+    if sh.dtype == "bf16":
+        nbytes = keys * G * (2 * D * 2 + 2 * 2 * D * 4) + T * H * (3 * D * 2 + D * 4 + 4)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes,
+                           "peak_source": peaks["source"], "tflops": tflops,
+                           "tensor_frac": tflops / peaks["bf16_tflops"]}
+    else:
+        peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        out["roofline"] = {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                           "peak_source": "fp32 FMA lanes x clock (148 x 128 x 2 x 1.965 GHz)"}
+    return out
 
 
 KERNEL_SOURCES = {

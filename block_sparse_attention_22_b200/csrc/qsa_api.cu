@@ -21,6 +21,7 @@
 #include "index_simt.cuh"
 #include "topk.cuh"
 #include "attn_bwd.cuh"
+#include "attn_bwd_tc.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "index_tc.cuh"
@@ -716,10 +717,30 @@ QSA_API qsa_status_t qsa_sparse_attn_bwd(const qsa_config_t* cfg, const qsa_cach
       !aligned16(dv) || !aligned16(cache->k) || !aligned16(cache->v))
     return QSA_ERR_INVALID_ARG;
   const Geo g = make_geo(cfg, cache);
-  AttnBwdArgs a{q, o, lse, dout, cache->k, cache->v, sel, nsel, dq, dk, dv};
-  const size_t smem = attn_bwd_smem();
   const bool bf = cfg->dtype == QSA_DTYPE_BF16;
   cudaStream_t st = (cudaStream_t)stream;
+  if (bf) {
+    // tensor cores: one CTA per SM, persistent over (query, group) units
+    CUtensorMap tq, tdo;
+    if (!make_map_bf16(&tq, q, kHeadDim, (uint64_t)n_tokens * g.H, 64, (uint32_t)g.hpg) ||
+        !make_map_bf16(&tdo, dout, kHeadDim, (uint64_t)n_tokens * g.H, 64, (uint32_t)g.hpg))
+      return QSA_ERR_CUDA;
+    AttnBwdTcArgs ta{o, lse, dout, cache->k, cache->v, sel, nsel, dq, dk, dv, 0};
+    const int smem_tc = tc_bwd::kSmemBytes;
+    cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_tc);
+    const int sms = sm_count();
+    return for_each_table(
+        segs, n_segs, [&](const qsa_segment_t& sg) { return (int64_t)sg.q_len; },
+        [&](const SegTable& t) {
+          ta.units_per_group = t.item0[t.n];
+          const int64_t units = ta.units_per_group * g.G;
+          count_launch();
+          return launch_chained(attn_bwd_tc_kernel, dim3((unsigned)std::min<int64_t>(units, sms)),
+                                dim3(tc_bwd::kThreads), smem_tc, st, tq, tdo, g, t, ta);
+        });
+  }
+  AttnBwdArgs a{q, o, lse, dout, cache->k, cache->v, sel, nsel, dq, dk, dv};
+  const size_t smem = attn_bwd_smem();
   if (bf)
     cudaFuncSetAttribute(attn_bwd_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   else

@@ -44,6 +44,7 @@ def _check(name, got, ref, dtype):
 @pytest.mark.parametrize("name,over", [
     ("tiny_fp32", {}),
     ("prefill_8k", dict(n=600, n_seqs=1)),
+    ("prefill_8k", dict(n=1200, n_seqs=2)),     # tensor-core path: several units per SM, 10 chunks
     ("decode_256k", dict(ctx=20001, n_seqs=3)),
 ])
 def test_backward_matches_oracle_gradients(name, over):
@@ -88,13 +89,14 @@ def test_backward_matches_oracle_gradients(name, over):
         assert torch.count_nonzero(dk[s, :, fill:]) == 0 and torch.count_nonzero(dv[s, :, fill:]) == 0
 
 
-def test_backward_accumulates_key_gradients():
-    wl = synth.make_workload("tiny_fp32")
+@pytest.mark.parametrize("name,over", [("tiny_fp32", {}), ("prefill_8k", dict(n=600, n_seqs=1))])
+def test_backward_accumulates_key_gradients(name, over):
+    wl = synth.make_workload(name, **over)
     x = {k: v.cuda() for k, v in synth.make_inputs(wl).items()}
     sh = wl.shape
     fwd = gpu_forward(wl, x)
     T = wl.n_tokens
-    dout = torch.ones((T, sh.n_heads, sh.head_dim), device="cuda")
+    dout = torch.ones((T, sh.n_heads, sh.head_dim), device="cuda").to(sh.torch_dtype)
     cfg, cache, _ = gpu_prepare_cache(wl, x)
     segs = segments_of(wl)
     dq = torch.empty((T, sh.n_heads, sh.head_dim), device="cuda")
