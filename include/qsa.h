@@ -198,7 +198,9 @@ qsa_status_t qsa_sparse_attn_fwd(const qsa_config_t* cfg, const qsa_cache_t* cac
  * laid out like cache->k / cache->v ([n_slots][n_kv_groups][n_cap][head_dim]),
  * ACCUMULATED into (fp32 atomic adds, so the order of additions and the last
  * bits vary from run to run): zero them before the first call of a step.
- * The indexer and the selection have no gradient here.
+ * The indexer and the selection have no gradient here.  bf16 runs on the
+ * tensor cores with P and the probability gradients rounded to bf16 for the
+ * products (as the forward rounds P); fp32 runs on CUDA cores in fp32.
  */
 qsa_status_t qsa_sparse_attn_bwd(const qsa_config_t* cfg, const qsa_cache_t* cache,
                                  const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
