@@ -137,7 +137,8 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
 
     Keyword overrides allow reduced sizes of the same recipe for parity tests:
     n (prefill length), n_seqs, ctx (decode context), chunk (prefill chunk
-    length), chunk_pos0, n_decode.
+    length), chunk_pos0, n_decode; `shape` (Shape fields) for prefill_8k and
+    the decode workloads.
     """
     rng = torch.Generator().manual_seed(1000 + (seed if seed is not None else 0))
     if name == "tiny_fp32":
@@ -167,7 +168,7 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
         return Workload(name, sh, [Segment(0, 0, n)], 1, _round_cap(n, sh.r), [n], [0], needles,
                         seed if seed is not None else 2)
     if name in ("decode_256k", "decode_1m"):
-        sh = Shape()
+        sh = Shape(**over.get("shape", {}))
         big = name == "decode_1m"
         ctx = over.get("ctx", (1 << 20) if big else 262144)
         n_seqs = over.get("n_seqs", 8 if big else 32)
@@ -182,7 +183,7 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
         return Workload(name, sh, segs, n_seqs, _round_cap(ctx, sh.r), [ctx] * n_seqs, cached, needles,
                         seed if seed is not None else (6 if big else 3))
     if name == "spec_decode_1m":
-        sh = Shape()
+        sh = Shape(**over.get("shape", {}))
         ctx = over.get("ctx", 1 << 20)
         n_seqs = over.get("n_seqs", 8)
         q_len = over.get("q_len", 4)

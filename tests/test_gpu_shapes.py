@@ -76,3 +76,18 @@ def test_backward_parity_on_layer_shapes(shape):
         assert np.isfinite(got).all(), name
         assert err.max() <= 1e-2 * scale, (name, float(err.max()), scale)
         assert err.mean() <= 1e-3 * scale, (name, float(err.mean()), scale)
+
+
+@pytest.mark.parametrize("name,shape", [
+    ("decode_256k", dict(n_heads=32, n_groups=2)),
+    ("decode_256k", dict(idx_dim=64)),
+    ("spec_decode_1m", dict(n_heads=8, n_groups=4)),
+], ids=lambda x: x if isinstance(x, str) else "-".join(f"{k}{v}" for k, v in x.items()))
+def test_decode_parity_on_layer_shapes(name, shape):
+    """Decode-like segments: 4-query index tiles, the few-rows selection and
+    split-K attention with its combine, on the same shape variants."""
+    wl = synth.make_workload(name, ctx=20001, n_seqs=3, shape=shape)
+    x = {k: v.cuda() for k, v in synth.make_inputs(wl).items()}
+    run = gpu_forward(wl, x)
+    res = compare_forward(wl, x, run, range(wl.n_tokens))
+    assert res["n"] == wl.n_tokens
