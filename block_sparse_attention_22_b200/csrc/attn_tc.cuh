@@ -13,11 +13,15 @@
 // K-major layout the MMA reads (8-row atoms are filled by two blocks).
 //
 // Two-phase softmax per unit: every chunk's S^T goes to its own TMEM buffer
-// (16 x 16 columns), the exact per-head maximum is taken once over all of
-// them, then P = exp2(S - max) is written chunk by chunk and P.V accumulates
-// straight into a TMEM output buffer.  K slots are therefore freed as soon
-// as their MMA has run, V slots as soon as their P is written, and the load
-// stream waits on the softmax only between units.  Loads and MMAs walk one
+// (16 x 16 columns), the per-head maximum is taken over all of them but the
+// last, then P = exp2(S - max) is written chunk by chunk and P.V accumulates
+// straight into a TMEM output buffer.  The last chunk's maximum is folded in
+// before the third P chunk: it replaces the running one only when it exceeds
+// it by more than 8 (log2 units), and then O and the row sums so far are
+// rescaled once in TMEM (softmax is shift invariant; P stays below 2^8).  So
+// a unit's first P.V products need not wait for its last S.  K slots are
+// freed as soon as their MMA has run, V slots as soon as their P is written,
+// and the load stream waits on the softmax only between units.  Loads and MMAs walk one
 // item sequence, K(0..n-1) then V(0..n-1) per unit; an item is two 32 KiB
 // half-slots (128 keys x 128 dims) of a 6-slot ring.
 //
@@ -394,8 +398,10 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
           if (row >= 0 && row <= u.t) vbits |= 1u << c;
         }
       }
-      // phase 1: exact per-head maximum over every chunk
-      for (int c = 0; c < u.nchunks; ++c) {
+      // phase 1: per-head maximum over every chunk but the last, so that the
+      // first P chunks need not wait for the last S (folded in below)
+      const int n_pre = u.nchunks > 1 ? u.nchunks - 1 : u.nchunks;
+      for (int c = 0; c < n_pre; ++c) {
         mbar_wait(&ctl.s_full[c], (sbits >> c) & 1u, abort_flag);
         tc_fence_after();
         float s[kHH];
@@ -420,7 +426,65 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
                      fmaxf(ctl.red[0][2][h0 + h], ctl.red[0][3][h0 + h]));
       // phase 2: P = exp2(S - max) per chunk, written as the B operand of P.V
       const int slab = li >> 6, kin = li & 63;
+      const int fold_at = u.nchunks > 1 ? min(2, u.nchunks - 1) : -1;
+      const int ob_u = (int)(uc & 1);                   // this unit's O buffer
       for (int c = 0; c < u.nchunks; ++c, ++gp) {
+        if (c == fold_at) {
+          // the last chunk's maximum: while it exceeds the running one by at
+          // most 8 (log2 units) the running one stands -- softmax is shift
+          // invariant and P stays below 2^8; beyond that, O and l of the
+          // chunks already weighted are rescaled once
+          const int cl = u.nchunks - 1;
+          mbar_wait(&ctl.s_full[cl], (sbits >> cl) & 1u, abort_flag);
+          tc_fence_after();
+          float sl[kHH];
+          tmem_ld8(lane_addr + cl * kN + h0, sl);
+          tmem_wait_ld();
+          float ml[kHH];
+#pragma unroll
+          for (int h = 0; h < kHH; ++h) ml[h] = ((vbits >> cl) & 1u) ? sl[h] * scale_log2 : -INFINITY;
+#pragma unroll
+          for (int off = 16; off; off >>= 1)
+#pragma unroll
+            for (int h = 0; h < kHH; ++h) ml[h] = fmaxf(ml[h], __shfl_xor_sync(0xffffffffu, ml[h], off));
+          if (lane == 0)
+#pragma unroll
+            for (int h = 0; h < kHH; ++h) ctl.red[1][quad][h0 + h] = ml[h];
+          named_bar_sync(1, nthr);
+          float f[kHH];
+          bool any = false;                             // uniform across the warp (same heads)
+#pragma unroll
+          for (int h = 0; h < kHH; ++h) {
+            const float mf = fmaxf(fmaxf(ctl.red[1][0][h0 + h], ctl.red[1][1][h0 + h]),
+                                   fmaxf(ctl.red[1][2][h0 + h], ctl.red[1][3][h0 + h]));
+            f[h] = 1.f;
+            if (mf > m[h] + 8.f) {
+              f[h] = m[h] == -INFINITY ? 0.f : exp2f(m[h] - mf);
+              m[h] = mf;
+              any = true;
+            }
+          }
+          if (any) {
+            // O holds chunks 0..c-1: wait for the last of their P.V products
+            const int64_t gprev = gp - 1;
+            mbar_wait(&ctl.p_free[gprev & 1], (uint32_t)((gprev >> 1) & 1), abort_flag);
+            tc_fence_after();
+            float o0[kHH], o1[kHH];
+            tmem_ld8(lane_addr + kTmemO + ob_u * 32 + h0, o0);
+            tmem_ld8(lane_addr + kTmemO + ob_u * 32 + kN + h0, o1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < kHH; ++h) {
+              o0[h] *= f[h];
+              o1[h] *= f[h];
+              l[h] *= f[h];
+            }
+            tmem_st8(lane_addr + kTmemO + ob_u * 32 + h0, o0);
+            tmem_st8(lane_addr + kTmemO + ob_u * 32 + kN + h0, o1);
+            tmem_wait_st();
+            tc_fence_before();
+          }
+        }
         float s[kHH];
         tmem_ld8(lane_addr + c * kN + h0, s);
         tmem_wait_ld();
