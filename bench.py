@@ -18,6 +18,17 @@ launching stream, max over ranks.  With torchrun and N > 1 every rank runs
 an independent replica of the workload on its own GPU (the method has no
 cross-GPU exchange): scaling is weak.
 
+Besides the main line's device-timed step the JSON line carries: "stages"
+(each public entry point timed alone) and the attention "roofline" (gathered
+bytes over the attention stage, DRAM traffic from the committed ncu record);
+"e2e" (the step through qsa_forward with every input copied from pinned host
+memory and the output copied back inside the timed region, as 8 chunked-
+prefill calls whose copies overlap the neighbouring chunks' compute; output
+checked equal to one call); "lowmem_forward" (the same step through
+qsa_forward_lowmem, with both workspace sizes); "decode_1m" / "mixed_1m";
+"attn_backward" (qsa_sparse_attn_bwd on a 2 x 8192-token prefill);
+"cpu_baseline" (the oracle on a bounded sample); "gpu_launches"; "clocks".
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qsa|reference]
 """
 from __future__ import annotations
