@@ -27,6 +27,9 @@ prefill calls whose copies overlap the neighbouring chunks' compute; output
 checked equal to one call); "lowmem_forward" (the same step through
 qsa_forward_lowmem, with both workspace sizes); "decode_1m" / "mixed_1m";
 "attn_backward" (qsa_sparse_attn_bwd on a 2 x 8192-token prefill);
+"attn_union" (the attention of prefill_128k_local, whose indexer queries drift
+along the sequence, on union tiles of neighbouring queries beside the
+per-query path);
 "cpu_baseline" (the oracle on a bounded sample); "gpu_launches"; "clocks".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qsa|reference]
@@ -541,6 +544,97 @@ def measure_backward(name, steps, warmup, ws, flush, peaks):
     return out
 
 
+def union_lengths(sel: torch.Tensor, nsel: torch.Tensor, segl, mq: int) -> torch.Tensor:
+    """Distinct kept blocks of every tile of mq consecutive queries of a segment
+    (computed here with a sort, independently of the library's union lists)."""
+    out = []
+    S = sel.shape[1]
+    cols = torch.arange(S, device=sel.device)
+    for off, q_len, _, _ in segl:
+        s = sel[off:off + q_len].clone()
+        s[cols[None, :] >= nsel[off:off + q_len, None]] = -1
+        pad = (-q_len) % mq
+        if pad:
+            s = torch.cat([s, torch.full((pad, S), -1, dtype=s.dtype, device=s.device)])
+        s = torch.sort(s.view(-1, mq * S), dim=1).values
+        new = torch.ones_like(s, dtype=torch.bool)
+        new[:, 1:] = s[:, 1:] != s[:, :-1]
+        out.append((new & (s >= 0)).sum(1))
+    return torch.cat(out)
+
+
+def measure_union(name, steps, warmup, ws, flush, peaks, n=None):
+    """The attention stage of one workload on union tiles
+    (qsa_sparse_attn_fwd_union) beside the per-query path (qsa_sparse_attn_fwd),
+    both over the selection the forward made, L2 flushed before every step.
+    Algorithmic bytes of the union path: per tile and KV group the union's K and
+    V rows (2 x r x head_dim x 2 B per block), plus Q read and O written
+    (H x head_dim x 2 B each per query), lse, the sel rows read and the union
+    lists written and read (8 B per entry, twice).  `n`: a shorter prefill of the
+    same recipe (profiles)."""
+    wl = synth.make_workload(name, **({"n": n} if n else {}))
+    prep = Prepared(wl)
+    prep.forward()
+    torch.cuda.synchronize()
+    sh, x, T = prep.sh, prep.x, prep.T
+    mq = min(32, 128 // (sh.n_heads // sh.n_groups))
+    o_ref = prep.o.clone()
+    o_u = torch.empty_like(prep.o)
+    lse_u = torch.empty_like(prep.lse)
+    ws_u = torch.empty(max(1, qsa.workspace_size(prep.cfg, prep.segs, T, qsa.QSA_OP_ATTN_UNION)),
+                       dtype=torch.uint8, device="cuda")
+    st = torch.cuda.current_stream()
+
+    def per_query():
+        prep.stage(3)
+
+    def union():
+        qsa.qsa_sparse_attn_fwd_union(prep.cfg, prep.cache, prep.segs, T, x["q"], prep.sel, prep.nsel, o_u, lse_u,
+                                      ws_u)
+
+    def time_of(fn):
+        for _ in range(warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            fn()
+            e1.record(st)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        return max_over_ranks(tot / steps, ws)
+
+    n0 = qsa.launch_count()
+    ms_u = time_of(union)
+    launches = (qsa.launch_count() - n0) // (steps + warmup)
+    ms_q = time_of(per_query)
+    diff = float((o_u.float() - o_ref.float()).abs().max().item())
+    lens = union_lengths(prep.sel, prep.nsel, prep.segl, mq).double()
+    el = 2
+    D, H, G = sh.head_dim, sh.n_heads, sh.n_groups
+    blocks_u = float(lens.sum().item())
+    blocks_q = float(prep.nsel.double().sum().item())
+    gathered_u = blocks_u * G * sh.r * D * el * 2
+    gathered_q = blocks_q * G * sh.r * D * el * 2
+    nbytes = gathered_u + T * H * D * el * 2 + T * H * 4 + T * sh.budget_blocks * 4 + blocks_u * 16
+    gbs = nbytes / (ms_u * 1e-3) / 1e9
+    out = {"workload": name, "drift": wl.drift, "tile_queries": mq, "ms_union": ms_u, "ms_per_query": ms_q,
+           "speedup": ms_q / ms_u, "tokens_per_s_union": job_throughput(T, ms_u, ws),
+           "union_blocks_per_tile": blocks_u / len(lens), "kept_blocks_per_query": blocks_q / T,
+           "gathered_bytes_union": gathered_u, "gathered_bytes_per_query": gathered_q,
+           "max_abs_diff_vs_per_query": diff, "gpu_launches_per_call": launches,
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes, "peak_source": peaks["source"]}}
+    del prep
+    torch.cuda.empty_cache()
+    return out
+
+
 KERNEL_SOURCES = {
     "attn": ["attn_tc.cuh", "sm100.cuh", "qsa_internal.cuh"],
     "index": ["index_tc.cuh", "sm100.cuh", "qsa_internal.cuh"],
@@ -619,6 +713,9 @@ def main():
                     help="comma-separated extra workloads reported beside the main line; 'none' to skip")
     ap.add_argument("--bwd-workload", default="prefill_8k",
                     help="workload of the attention-backward measurement; 'none' to skip")
+    ap.add_argument("--union-workload", default="prefill_128k_local",
+                    help="attention on union tiles beside the per-query path ('none' to skip)")
+    ap.add_argument("--union-n", type=int, default=0, help="query tokens of the union workload (0: its own)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-lowmem", action="store_true", help="skip the low-memory forward line")
@@ -693,6 +790,10 @@ def main():
         extra[name] = d
         del prep2
         torch.cuda.empty_cache()
+
+    if args.union_workload != "none":
+        extra["attn_union"] = measure_union(args.union_workload, args.steps, args.warmup, ws, flush, peaks,
+                                            args.union_n or None)
 
     if args.bwd_workload != "none":
         extra["attn_backward"] = measure_backward(args.bwd_workload, args.steps, args.warmup, ws, flush, peaks)

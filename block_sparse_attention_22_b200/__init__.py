@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(HERE, "libqsa.so")
 
 QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA, QSA_ERR_TIMEOUT = range(6)
 QSA_DTYPE_F32, QSA_DTYPE_BF16 = 0, 1
-QSA_OP_COMPRESS, QSA_OP_INDEX, QSA_OP_SELECT, QSA_OP_ATTN, QSA_OP_FORWARD, QSA_OP_FORWARD_LOWMEM = range(6)
+(QSA_OP_COMPRESS, QSA_OP_INDEX, QSA_OP_SELECT, QSA_OP_ATTN, QSA_OP_FORWARD, QSA_OP_FORWARD_LOWMEM,
+ QSA_OP_ATTN_UNION) = range(7)
 
 
 class qsa_config_t(ctypes.Structure):
@@ -59,6 +60,7 @@ def _load():
         "qsa_index_scores": [C, K, S, I32, I32, P, P, P, I64, P],
         "qsa_select_topk": [C, S, I32, I32, P, I64, P, P, P, SZ, P],
         "qsa_sparse_attn_fwd": [C, K, S, I32, I32, P, P, P, P, P, P, SZ, P],
+        "qsa_sparse_attn_fwd_union": [C, K, S, I32, I32, P, P, P, P, P, P, SZ, P],
         "qsa_sparse_attn_bwd": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, P, P],
         "qsa_forward": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, SZ, P],
         "qsa_forward_lowmem": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, SZ, P],
@@ -174,6 +176,18 @@ def qsa_sparse_attn_fwd(cfg, cache, segs, n_tokens, q, sel, nsel, o, lse=None, w
     _check(get_lib().qsa_sparse_attn_fwd(ctypes.byref(cfg), ctypes.byref(cache), arr, n, n_tokens, _ptr(q),
                                    _ptr(sel), _ptr(nsel), _ptr(o), _ptr(lse), _ptr(workspace), ws_bytes,
                                    _stream(stream)), "qsa_sparse_attn_fwd")
+
+
+def qsa_sparse_attn_fwd_union(cfg, cache, segs, n_tokens, q, sel, nsel, o, lse=None, workspace=None,
+                              stream=None):
+    """qsa_sparse_attn_fwd on tiles of neighbouring queries that gather the union
+    of their kept blocks once (workspace: QSA_OP_ATTN_UNION; bf16 only)."""
+    arr, n = segs
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(get_lib().qsa_sparse_attn_fwd_union(ctypes.byref(cfg), ctypes.byref(cache), arr, n, n_tokens,
+                                               _ptr(q), _ptr(sel), _ptr(nsel), _ptr(o), _ptr(lse),
+                                               _ptr(workspace), ws_bytes, _stream(stream)),
+           "qsa_sparse_attn_fwd_union")
 
 
 def qsa_sparse_attn_bwd(cfg, cache, segs, n_tokens, q, o, lse, dout, sel, nsel, dq, dk, dv, stream=None):

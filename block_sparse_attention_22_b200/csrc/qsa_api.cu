@@ -24,6 +24,7 @@
 #include "attn_bwd_tc.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "attn_union_tc.cuh"
 #include "index_tc.cuh"
 
 #include <cudaTypedefs.h>
@@ -573,6 +574,104 @@ qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* ca
       });
 }
 
+// ------------------------------------------------------------------ union-tile attention
+// Query tokens per union tile: as many as fill the 128 query rows of an MMA
+// tile with one group's heads, at most the 32 bits of a member mask.
+int union_mq(const Geo& g) { return std::min(tc_union::kMaxMembers, 128 / g.hpg); }
+
+struct UnionPlan {
+  int mq;
+  int64_t tiles;
+  int64_t cap;               // union entries per tile
+  size_t off_blk, off_mask, ws;
+};
+
+UnionPlan union_plan(const Geo& g, const qsa_segment_t* segs, int n) {
+  UnionPlan p;
+  p.mq = union_mq(g);
+  p.cap = (int64_t)p.mq * g.S;
+  p.tiles = 0;
+  for (int i = 0; i < n; ++i)
+    if (segs[i].q_len > 0) p.tiles += union_tiles(segs[i].q_len, p.mq);
+  p.off_blk = align_up((size_t)p.tiles * 4, 256);
+  p.off_mask = p.off_blk + align_up((size_t)p.tiles * p.cap * 4, 256);
+  p.ws = p.tiles > 0 ? p.off_mask + align_up((size_t)p.tiles * p.cap * 4, 256) : 0;
+  return p;
+}
+
+// q as [T][H][256] bf16: boxes of 64 dims x hpg heads x mq tokens, 128-byte
+// swizzle, tokens past T read as zero.
+bool make_q_tile_map(CUtensorMap* m, const void* q, int64_t n_tokens, const Geo& g, int mq) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)g.H, (cuuint64_t)n_tokens};
+  cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)g.H * kHeadDim * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)g.hpg, (cuuint32_t)mq};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+qsa_status_t run_attn_union(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens,
+                            const qsa_cache_t* cache, const void* q, const int32_t* sel, const int32_t* nsel,
+                            void* o, float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const UnionPlan p = union_plan(g, segs, n);
+  if (p.ws > 0 && (!ws || ws_bytes < p.ws)) return QSA_ERR_WORKSPACE;
+  // the union build holds a bitmap of the context's blocks and its prefix in shared memory
+  const int64_t max_words = cdiv(seg_max_blocks(segs, n, g.r) + 1, 32);
+  if (((size_t)2 * max_words + (size_t)p.cap) * 4 > (size_t)227 * 1024) return QSA_ERR_UNSUPPORTED;
+  CUtensorMap tq;
+  if (!make_q_tile_map(&tq, q, n_tokens, g, p.mq)) return QSA_ERR_CUDA;
+  UnionBuildArgs ba;
+  memset(&ba, 0, sizeof ba);
+  ba.sel = sel;
+  ba.nsel = nsel;
+  ba.ulen = (int32_t*)ws;
+  ba.ublk = (int32_t*)((char*)ws + p.off_blk);
+  ba.umask = (uint32_t*)((char*)ws + p.off_mask);
+  ba.cap = p.cap;
+  ba.mq = p.mq;
+  AttnUnionArgs ta;
+  memset(&ta, 0, sizeof ta);
+  ta.k = cache->k;
+  ta.v = cache->v;
+  ta.ulen = ba.ulen;
+  ta.ublk = ba.ublk;
+  ta.umask = ba.umask;
+  ta.cap = p.cap;
+  ta.mq = p.mq;
+  ta.o = o;
+  ta.lse = lse;
+  cudaFuncSetAttribute(attn_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_union::kSmemBytes);
+  const int sms = sm_count();
+  int64_t tile_base = 0;
+  return for_each_table(
+      segs, n, [&](const qsa_segment_t& s) { return union_tiles(s.q_len, p.mq); },
+      [&](const SegTable& t) -> cudaError_t {
+        const int64_t tiles = t.item0[t.n];
+        int64_t nb = 1;
+        for (int i = 0; i < t.n; ++i) nb = std::max<int64_t>(nb, ((int64_t)t.pos0[i] + t.q_len[i] - 1) / g.r + 1);
+        ba.words = (int)cdiv(nb, 32);
+        ba.tile_base = tile_base;
+        const size_t smem = ((size_t)2 * ba.words + (size_t)p.cap) * 4;
+        if (cudaFuncSetAttribute(union_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+          return cudaErrorInvalidValue;
+        count_launch();
+        union_build_kernel<<<dim3((unsigned)tiles), dim3(tc_union::kBuildThreads), smem, st>>>(g, t, ba);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        ta.tiles = tiles;
+        ta.tile_base = tile_base;
+        const int grid = (int)std::min<int64_t>(tiles * g.G, sms);
+        count_launch();
+        attn_union_kernel<<<dim3(grid), dim3(tc_attn::kThreads), tc_union::kSmemBytes, st>>>(tq, g, t, ta);
+        tile_base += tiles;
+        return cudaGetLastError();
+      });
+}
+
 // ------------------------------------------------------------------ forward workspace
 // Segments that select through the fused path (no score rows): in the
 // low-memory forward, the bf16 prefill-like segments (64-query index tiles).
@@ -701,6 +800,25 @@ QSA_API qsa_status_t qsa_sparse_attn_fwd(const qsa_config_t* cfg, const qsa_cach
                   (cudaStream_t)stream);
 }
 
+QSA_API qsa_status_t qsa_sparse_attn_fwd_union(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                               const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                                               const void* q, const int32_t* sel, const int32_t* nsel,
+                                               void* o, float* lse, void* workspace, size_t ws_bytes,
+                                               void* stream) {
+  qsa_status_t s = check_cfg(cfg);
+  if (s != QSA_OK) return s;
+  if ((s = check_cache(cfg, cache)) != QSA_OK) return s;
+  if ((s = check_segments(segs, n_segs, n_tokens, cache, 0)) != QSA_OK) return s;
+  if (cfg->dtype != QSA_DTYPE_BF16) return QSA_ERR_UNSUPPORTED;
+  if (seg_rows(segs, n_segs) == 0) return QSA_OK;
+  if (!q || !sel || !nsel || !o || !cache->k || !cache->v || !aligned16(q) || !aligned16(o) ||
+      !aligned16(cache->k) || !aligned16(cache->v) || !aligned16(sel))
+    return QSA_ERR_INVALID_ARG;
+  const Geo g = make_geo(cfg, cache);
+  return run_attn_union(g, segs, n_segs, n_tokens, cache, q, sel, nsel, o, lse, workspace, ws_bytes,
+                        (cudaStream_t)stream);
+}
+
 QSA_API qsa_status_t qsa_sparse_attn_bwd(const qsa_config_t* cfg, const qsa_cache_t* cache,
                                          const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
                                          const void* q, const void* o, const float* lse, const void* dout,
@@ -769,6 +887,7 @@ QSA_API size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* 
     case QSA_OP_FORWARD: return fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16, false).total;
     case QSA_OP_FORWARD_LOWMEM:
       return fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16, true).total;
+    case QSA_OP_ATTN_UNION: return union_plan(g, segs, n_segs).ws;
   }
   return SIZE_MAX;
 }

@@ -24,9 +24,19 @@ kv-channels 256, rotary 0.25 at base 1e7; design report, QSA item: r=4, a
   chunk_128k    one 4096-query prefill chunk at [126976, 131072) of a
                 131072-token sequence whose prefix is cached (a ~1 GB case
                 whose K/V still exceeds L2; used for kernel profiles)
+  prefill_128k_local  prefill_128k with indexer queries that drift slowly
+                along the sequence (below), so neighbouring tokens keep
+                mostly the same blocks
 
 Distributions: q, k, v, indexer q and indexer k ~ N(0, 1) drawn in fp32 and
 rounded once to the I/O dtype; head weights w ~ U(0, 1) in fp32.
+
+Locality (`drift` rho > 0, an input made to have it, not a property the pages
+state): along each segment's tokens the indexer queries follow a stationary
+AR(1) process, q_idx[t] = rho q_idx[t-1] + sqrt(1 - rho^2) e[t] with e ~ N(0,1)
+(so every q_idx[t] is still N(0,1)), and the head weights a convex one,
+w[t] = rho w[t-1] + (1 - rho) u[t] with u ~ U(0,1).  prefill_128k_local uses
+rho = 0.99.
 
 Needles ("key = scaled copy of query"): for a target query t* of cache slot s
 and a block b* < floor(t*/r), the r indexer-key rows of b* are set to
@@ -89,6 +99,7 @@ class Workload:
     cached_blocks: List[int]           # k^ blocks already pooled before the step
     needles: List[Tuple[int, int, int]] = field(default_factory=list)  # (slot, t*, b*)
     seed: int = 0
+    drift: float = 0.0                 # AR(1) coefficient of the indexer queries along a segment
 
     @property
     def n_tokens(self) -> int:
@@ -155,8 +166,8 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
         for s in range(n_seqs):
             needles += _needles_per_window(rng, s, 0, n, 4, sh.r)
         return Workload(name, sh, segs, n_seqs, _round_cap(n, sh.r), [n] * n_seqs, [0] * n_seqs, needles,
-                        seed if seed is not None else 1)
-    if name == "prefill_128k":
+                        seed if seed is not None else 1, over.get("drift", 0.0))
+    if name in ("prefill_128k", "prefill_128k_local"):
         sh = Shape()
         n = over.get("n", 131072)
         every = over.get("every", 8192)
@@ -165,8 +176,9 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
             t = every * i + every - 1
             b = int(torch.randint(0, t // sh.r, (1,), generator=rng))
             needles.append((0, t, b))
+        drift = over.get("drift", 0.99 if name == "prefill_128k_local" else 0.0)
         return Workload(name, sh, [Segment(0, 0, n)], 1, _round_cap(n, sh.r), [n], [0], needles,
-                        seed if seed is not None else 2)
+                        seed if seed is not None else 2, drift)
     if name in ("decode_256k", "decode_1m"):
         sh = Shape(**over.get("shape", {}))
         big = name == "decode_1m"
@@ -237,6 +249,32 @@ def _randn(shape, gen, device, dtype, chunk_elems=1 << 28):
     return out
 
 
+def _ar1_(x: torch.Tensor, rho: float, innov: float, block: int = 256) -> None:
+    """In place along dim 0: y[0] = x[0], y[t] = rho y[t-1] + innov x[t]
+    (fp32 carry, one rounding to x's dtype), evaluated block by block as
+    y[s:s+L] = A (innov x[s:s+L]) + rho^(1..L) y[s-1] with A[i,j] = rho^(i-j)."""
+    n = x.shape[0]
+    if n < 2 or rho == 0.0:
+        return
+    flat = x.view(n, -1)
+    i = torch.arange(block, dtype=torch.float64, device=x.device)
+    d = i[:, None] - i[None, :]
+    A = torch.where(d >= 0, rho ** d.clamp(min=0), torch.zeros_like(d)).float()
+    pw = (rho ** (i + 1)).float()
+    prev = None
+    for s in range(0, n, block):
+        e = flat[s:s + block].float()
+        L = e.shape[0]
+        inn = innov * e
+        if prev is None:
+            inn[0] = e[0]
+            y = A[:L, :L] @ inn
+        else:
+            y = A[:L, :L] @ inn + pw[:L, None] * prev
+        flat[s:s + L] = y.to(x.dtype)
+        prev = y[-1]
+
+
 def make_inputs(wl: Workload, device="cpu") -> Dict[str, torch.Tensor]:
     """Draw every input tensor of the workload on `device` (seeded).
 
@@ -261,9 +299,14 @@ def make_inputs(wl: Workload, device="cpu") -> Dict[str, torch.Tensor]:
         for g in range(sh.n_groups):
             k[s, g, :f] = _randn((f, sh.head_dim), gen, dev, dt)
             v[s, g, :f] = _randn((f, sh.head_dim), gen, dev, dt)
-    # needles
     offs = wl.token_offsets()
-    rho = sh.rope_dims
+    if wl.drift > 0:
+        rho = wl.drift
+        for o0, seg in zip(offs, wl.segments):
+            _ar1_(q_idx[o0:o0 + seg.q_len], rho, (1.0 - rho * rho) ** 0.5)
+            _ar1_(w[o0:o0 + seg.q_len], rho, 1.0 - rho)
+    # needles
+    n_rot = sh.rope_dims
     for (slot, t, b) in wl.needles:
         tok = None
         for si, seg in enumerate(wl.segments):
@@ -272,7 +315,7 @@ def make_inputs(wl: Workload, device="cpu") -> Dict[str, torch.Tensor]:
         if tok is None:
             continue
         u = (w[tok].unsqueeze(1) * q_idx[tok].float()).sum(0)
-        u[:rho] = 0
+        u[:n_rot] = 0
         k_idx[slot, b * sh.r:(b + 1) * sh.r] = u.to(dt)
         for g in range(sh.n_groups):
             k[slot, g, b * sh.r:(b + 1) * sh.r] = q[tok, 0]

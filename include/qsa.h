@@ -119,7 +119,8 @@ typedef enum {
   QSA_OP_SELECT = 2,
   QSA_OP_ATTN = 3,
   QSA_OP_FORWARD = 4,
-  QSA_OP_FORWARD_LOWMEM = 5
+  QSA_OP_FORWARD_LOWMEM = 5,
+  QSA_OP_ATTN_UNION = 6
 } qsa_op_t;
 
 /*
@@ -183,6 +184,29 @@ qsa_status_t qsa_sparse_attn_fwd(const qsa_config_t* cfg, const qsa_cache_t* cac
                                  const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
                                  const void* q, const int32_t* sel, const int32_t* nsel, void* o,
                                  float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * qsa_sparse_attn_fwd computed on tiles of neighbouring queries (the same o
+ * and lse, up to the rounding of P to bf16 against a different reference
+ * maximum).  Miles docs section 1: each query attends only its kept tokens;
+ * neighbouring tokens whose indexer queries are close keep mostly the same
+ * blocks.  Each segment is cut into tiles of mq = min(32, 128 / heads per
+ * group) consecutive query tokens; a tile gathers the ascending union of its
+ * members' kept blocks once per KV group, and a per-block member mask plus
+ * each member's causal limit give every query exactly its own key set J.
+ * Gathered K/V bytes per query fall by the tile's sharing factor (mq x 512
+ * blocks / union length); with no sharing they equal the per-query path's.
+ * Arguments, layouts and errors as qsa_sparse_attn_fwd; in addition every
+ * sel row must hold distinct blocks (qsa_select_topk writes them so).
+ * bf16 only (QSA_ERR_UNSUPPORTED otherwise).  workspace >=
+ * qsa_workspace_size(..., QSA_OP_ATTN_UNION) bytes (the union lists and
+ * masks: about 8 * mq * budget_tokens / r bytes per tile); contents on entry
+ * are ignored.
+ */
+qsa_status_t qsa_sparse_attn_fwd_union(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                       const qsa_segment_t* segs, int32_t n_segs, int32_t n_tokens,
+                                       const void* q, const int32_t* sel, const int32_t* nsel, void* o,
+                                       float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Backward of qsa_sparse_attn_fwd (Miles docs section 1: the QSA attention

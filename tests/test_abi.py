@@ -132,3 +132,33 @@ def test_status_strings_and_version():
     assert qsa.status_string(qsa.QSA_OK) == "ok"
     assert "workspace" in qsa.status_string(qsa.QSA_ERR_WORKSPACE)
     assert qsa.version() >= 100
+
+
+def _call_union(cfg, cache, segs, T=16, ws_bytes=1 << 40, **kw):
+    L = qsa.get_lib()
+    args = dict(q=16, o=16, lse=None, sel=16, nsel=16, ws=16)
+    args.update(kw)
+    return L.qsa_sparse_attn_fwd_union(ctypes.byref(cfg), ctypes.byref(cache), segs[0], segs[1], T, args["q"],
+                                       args["sel"], args["nsel"], args["o"], args["lse"], args["ws"], ws_bytes,
+                                       None)
+
+
+def test_union_attention_host_checks_and_workspace():
+    """The union-tile attention: tiles of min(32, 128 / heads per group) query
+    tokens per segment, one length word plus a block and a mask word per
+    union entry (tile size x budget blocks) per tile; bf16 only."""
+    sh, cfg, segs, cache = _setup()
+    big = qsa.make_segments([(0, 131072, 0, 0)])
+    tiles = -(-131072 // 10)                     # 12 heads per group -> 10 queries per tile
+    ws = qsa.workspace_size(cfg, big, 131072, qsa.QSA_OP_ATTN_UNION)
+    assert tiles * (4 + 2 * 10 * 512 * 4) <= ws < tiles * (4 + 2 * 10 * 512 * 4) + 1024
+    mha = qsa.make_config(synth.Shape(n_heads=16, n_groups=16))
+    assert qsa.workspace_size(mha, big, 131072, qsa.QSA_OP_ATTN_UNION) >= (131072 // 32) * 2 * 32 * 512 * 4
+    ragged = qsa.make_segments([(0, 11, 0, 0), (11, 1, 50, 1)])
+    assert qsa.workspace_size(cfg, ragged, 12, qsa.QSA_OP_ATTN_UNION) >= 3 * (4 + 2 * 10 * 512 * 4)
+    assert _call_union(cfg, cache, segs, ws_bytes=10) == qsa.QSA_ERR_WORKSPACE
+    assert _call_union(cfg, cache, segs, q=18) == qsa.QSA_ERR_INVALID_ARG
+    assert _call_union(cfg, cache, segs, sel=None) == qsa.QSA_ERR_INVALID_ARG
+    assert _call_union(cfg, cache, qsa.make_segments([(0, 0, 100, 0)]), T=0, ws=None, ws_bytes=0) == qsa.QSA_OK
+    f32 = qsa.make_config(synth.Shape(dtype="f32"))
+    assert _call_union(f32, cache, segs) == qsa.QSA_ERR_UNSUPPORTED
