@@ -27,12 +27,15 @@
 //     below 2^8 in between).
 //
 // Roles follow attn_tc.cuh (20 warps, warp w on sub-partition w % 4): nine
-// cp.async producers gather K(c), V(c) chunk by chunk into a 4-slot ring of
-// 32 KiB slots (64 keys x 256 dims, 128-byte swizzled K-major); warp 0
-// issues the MMAs; eight softmax warps, two per TMEM lane quadrant, own one
-// query row each (TMEM lane) and 32 of a chunk's 64 keys; idle warp 12 loads
-// each unit's Q tile with one 3-D TMA box per 64-dim slab.  Every mbarrier
-// wait is bounded; a timeout records an error and the CTA drains and returns.
+// cp.async producers gather the chunks' K and V into a 7-slot ring of 32 KiB
+// slots (64 keys x 256 dims, 128-byte swizzled K-major) in the order the
+// MMAs consume them (K0, K1, V0, K2, V1, ...); warp 0 issues the MMAs; eight
+// softmax warps, two per TMEM lane quadrant, own one query row each (TMEM
+// lane) and 32 of a chunk's 64 keys.  Q and P live in tensor memory as the A
+// operands of their MMAs (bf16 pairs per 32-bit column): the softmax warps
+// write each unit's Q rows there, and P over the first half of its chunk's S
+// columns, which leaves shared memory to the K/V ring.  Every mbarrier wait
+// is bounded; a timeout records an error and the CTA drains and returns.
 #pragma once
 #include "qsa_internal.cuh"
 #include "sm100.cuh"
@@ -43,17 +46,14 @@ namespace tc_union {
 constexpr int kMaxMembers = 32;            // bits of a union mask
 constexpr int kBlk = 16;                   // union blocks per chunk
 constexpr int kKeys = 64;                  // keys per chunk
-constexpr int kSlots = 4;                  // ring slots: one chunk's K or V each
+constexpr int kSlots = 7;                  // ring slots: one chunk's K or V each
 constexpr int kSlotBytes = 32768;          // 64 keys x 256 dims, 4 slabs of 8 KiB
-constexpr int kQBytes = 65536;             // 128 rows x 256 dims, 4 slabs of 16 KiB
-constexpr int kPBytes = 16384;             // 128 rows x 64 keys
-constexpr int kOffQ = kSlots * kSlotBytes;                 // 131072
-constexpr int kOffP = kOffQ + kQBytes;                     // 196608
-constexpr int kOffBar = kOffP + 2 * kPBytes;               // 229376
+constexpr int kOffBar = kSlots * kSlotBytes;               // 229376
 constexpr int kCtlBytes = 1280;
 constexpr int kSmemBytes = kOffBar + kCtlBytes + 1024;     // + alignment slack: 231680
-constexpr uint32_t kTmemCols = 512;        // S: 2 x 64 columns at 0; O: 256 columns at 256
-constexpr uint32_t kTmemO = 256;
+constexpr uint32_t kTmemCols = 512;        // S (then P over its first 32): 2 x 64 columns at 0
+constexpr uint32_t kTmemQ = 128;           // Q: 128 rows x 256 dims as 128 columns of bf16 pairs
+constexpr uint32_t kTmemO = 256;           // O: 256 columns
 constexpr uint32_t kIdescS = sm100::idesc_bf16(128, kKeys, false, false);
 constexpr uint32_t kIdescPV = sm100::idesc_bf16(128, 256, false, true);
 constexpr int kBuildThreads = 256;
@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(tc_union::kBuildThreads)
 }
 
 struct AttnUnionArgs {
+  const void* q;            // bf16 [T][H][D]
   const void* k;            // bf16 [n_slots][G][n_cap][D]
   const void* v;
   const int32_t* ulen;
@@ -201,6 +202,15 @@ struct AttnUnionCtl {
   int abort;
 };
 static_assert(sizeof(AttnUnionCtl) <= tc_union::kCtlBytes, "control block");
+
+// Ring position of chunk c's K (kind 0) or V (kind 1) within a unit of n
+// chunks: K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1) -- the order in
+// which the MMAs consume them, so slots free in ring order and each V chunk
+// arrives one chunk later than with K(c), V(c) adjacent.
+__device__ __forceinline__ int union_item(int c, int kind, int n) {
+  if (kind == 0) return c == 0 ? 0 : 2 * c - 1;
+  return c == n - 1 ? 2 * n - 1 : 2 * c + 2;
+}
 
 struct UnionUnit {
   TileInfo ti;
@@ -233,12 +243,48 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
-         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]: A (M=128 rows, 16-bit pairs along the
+// columns) read from tensor memory.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u));
+}
+
+// 32 lanes x 32-bit, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// 2^x by the MUFU instruction (inputs here are <= 8 or -inf; results below
+// 2^-126 flush to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Warp-uniform wait that suspends lane 0 in the barrier probe (no issue
+// slots spent while the phase is open).
+__device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = sm100::mbar_wait_sleep(bar, parity, abort_flag) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 __global__ void __launch_bounds__(tc_attn::kThreads, 1)
-    attn_union_kernel(const __grid_constant__ CUtensorMap tm_q, Geo g, SegTable st, AttnUnionArgs a) {
+    attn_union_kernel(Geo g, SegTable st, AttnUnionArgs a) {
   using namespace tc_union;
   using namespace sm100;
   using tc_attn::kProducers;
@@ -264,19 +310,14 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       mbar_init(&ctl.p_full[i], kSoftmaxWarps);
       mbar_init(&ctl.p_free[i], 1);
     }
-    mbar_init(&ctl.q_full, 1);
+    mbar_init(&ctl.q_full, kSoftmaxWarps);
     mbar_init(&ctl.q_empty, 1);
     mbar_init(&ctl.o_full, 1);
     mbar_init(&ctl.o_free, kSoftmaxWarps);
     mbar_init(&ctl.mma_done, 1);
     ctl.abort = 0;
     fence_mbar_init();
-    prefetch_tmap(&tm_q);
   }
-  // rows mq*hpg..127 of the Q tile are never loaded and must read as zero
-  for (int i = threadIdx.x; i < kQBytes / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(smem + kOffQ)[i] = make_uint4(0, 0, 0, 0);
-  fence_proxy_async_smem();
   if (role == tc_attn::kRoleMma) {
     tmem_alloc(&ctl.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -289,7 +330,7 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
   if (role == tc_attn::kRoleProducer) {
     // ============================================================ producers
     const int pw = ridx;                         // copies union blocks pw and pw + 9 of each chunk
-    int64_t item = 0;                            // ring items issued so far: K(c), V(c) per chunk
+    int64_t item = 0;                            // ring items issued so far (two per chunk)
     bool ok = true;
     const int r = (lane >> 3) & 3, jc = lane & 7;   // row of a block and 16-byte piece of a 128-byte line
     for (int64_t w = blockIdx.x; w < n_units && ok; w += gridDim.x) {
@@ -300,15 +341,19 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       const __nv_bfloat16* kg = (const __nv_bfloat16*)a.k + kv_off;
       const __nv_bfloat16* vg = (const __nv_bfloat16*)a.v + kv_off;
       const int32_t* ub = a.ublk + u.tile * a.cap;
-      for (int c = 0; c < u.nchunks && ok; ++c) {
+      const int n = u.nchunks;
+      for (int j = 0; j < 2 * n && ok; ++j, ++item) {
+        // the chunk and tensor of ring position j (inverse of union_item)
+        const int kind = (j == 0) ? 0 : (j == 2 * n - 1) ? 1 : (j & 1) ? 0 : 1;
+        const int c = (j == 0) ? 0 : (j == 2 * n - 1) ? n - 1 : (j & 1) ? (j + 1) / 2 : j / 2 - 1;
         int64_t myrow = -1;                      // lane i < 2: cache row of block pw + 9 i
         if (lane < 2 && pw + kProducers * lane < kBlk) {
           const int pos = c * kBlk + pw + kProducers * lane;
           if (pos < u.len) myrow = (int64_t)ub[pos] * 4;       // entries checked by the union build
         }
-        for (int kind = 0; kind < 2 && ok; ++kind, ++item) {
+        {
           const int slot = (int)(item % kSlots);
-          if (!(ok = warp_wait(&ctl.slot_empty[slot], (uint32_t)(((item / kSlots) & 1) ^ 1), abort_flag)))
+          if (!(ok = warp_wait_sleep(&ctl.slot_empty[slot], (uint32_t)(((item / kSlots) & 1) ^ 1), abort_flag)))
             break;
           const __nv_bfloat16* base = kind == 0 ? kg : vg;
           const uint32_t dst0 = smem_u32(smem + slot * kSlotBytes);
@@ -329,51 +374,30 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       }
     }
     cp_async_wait_all();                         // no copy of this warp outlives the CTA
-  } else if (role == tc_attn::kRoleIdle) {
-    // ============================================================ Q tiles (warp 12)
-    if (warp == 12) {
-      int64_t uc = 0;
-      for (int64_t w = blockIdx.x; w < n_units; w += gridDim.x) {
-        if (warp_aborted(abort_flag)) break;
-        const UnionUnit u = union_unit(st, a, w);
-        if (u.nchunks == 0) continue;
-        if (!warp_wait(&ctl.q_empty, (uint32_t)((uc & 1) ^ 1), abort_flag)) break;
-        if (lane == 0) {
-          const uint32_t box = (uint32_t)(a.mq * g.hpg * 128);
-          mbar_expect_tx(&ctl.q_full, 4 * box);
-          for (int s = 0; s < 4; ++s)
-            tma_load_3d(smem + kOffQ + s * 16384, &tm_q, 64 * s, u.grp * g.hpg, (int32_t)u.ti.tok0, &ctl.q_full);
-        }
-        __syncwarp();
-        ++uc;
-      }
-    }
   } else if (role == tc_attn::kRoleMma) {
     // ============================================================ MMA issuer
     // Per unit: S(0); then S(c), P.V(c-1) for c = 1..n-1; then P.V(n-1).
     int64_t gc = 0, uc = 0;                      // chunks and units so far
     const uint32_t sb = smem_u32(smem);
     bool ok = true;
-    auto pv = [&](int64_t x, int cx, bool first, bool last) -> bool {
+    auto pv = [&](int64_t x, int cx, int n) -> bool {
       const int pb = (int)(x & 1);
-      if (!warp_wait(&ctl.p_full[pb], (uint32_t)((x >> 1) & 1), abort_flag)) return false;
-      if (first && !warp_wait(&ctl.o_free, (uint32_t)((uc & 1) ^ 1), abort_flag)) return false;
-      const int64_t it = 2 * x + 1;
+      if (!warp_wait_sleep(&ctl.p_full[pb], (uint32_t)((x >> 1) & 1), abort_flag)) return false;
+      if (cx == 0 && !warp_wait_sleep(&ctl.o_free, (uint32_t)((uc & 1) ^ 1), abort_flag)) return false;
+      const int64_t it = 2 * gc + union_item(cx, 1, n);
       const int slot = (int)(it % kSlots);
-      if (!warp_wait(&ctl.slot_full[slot], (uint32_t)((it / kSlots) & 1), abort_flag)) return false;
+      if (!warp_wait_sleep(&ctl.slot_full[slot], (uint32_t)((it / kSlots) & 1), abort_flag)) return false;
       tc_fence_after();
       if (lane == 0) {
         fence_proxy_async_smem();
-        const uint32_t p_addr = sb + kOffP + pb * kPBytes;
         const uint32_t v_addr = sb + slot * kSlotBytes;
-        for (int kk = 0; kk < 4; ++kk) {                 // 4 k-steps of 16 keys
-          const uint64_t da = desc_sw128(p_addr + kk * 32, 16, 1024);
+        for (int kk = 0; kk < 4; ++kk) {                 // 4 k-steps of 16 keys; P: 8 columns of bf16 pairs each
           const uint64_t db = desc_sw128(v_addr + kk * 2048, 8192, 1024);
-          umma_bf16(tmem + kTmemO, da, db, kIdescPV, (cx | kk) != 0);
+          umma_bf16_ts(tmem + kTmemO, tmem + pb * kKeys + kk * 8, db, kIdescPV, (cx | kk) != 0);
         }
         umma_commit(&ctl.slot_empty[slot]);
         umma_commit(&ctl.p_free[pb]);
-        if (last) umma_commit(&ctl.o_full);
+        if (cx == n - 1) umma_commit(&ctl.o_full);
       }
       __syncwarp();
       return true;
@@ -382,34 +406,33 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       if (warp_aborted(abort_flag)) break;
       const UnionUnit u = union_unit(st, a, w);
       if (u.nchunks == 0) continue;
-      if (!(ok = warp_wait(&ctl.q_full, (uint32_t)(uc & 1), abort_flag))) break;
-      const uint32_t q_addr = sb + kOffQ;
-      for (int c = 0; c < u.nchunks && ok; ++c) {
+      if (!(ok = warp_wait_sleep(&ctl.q_full, (uint32_t)(uc & 1), abort_flag))) break;
+      const int n = u.nchunks;
+      for (int c = 0; c < n && ok; ++c) {
         const int64_t x = gc + c;
         const int b = (int)(x & 1);
-        if (!(ok = warp_wait(&ctl.s_free[b], (uint32_t)(((x >> 1) & 1) ^ 1), abort_flag))) break;
-        const int64_t it = 2 * x;
+        if (!(ok = warp_wait_sleep(&ctl.s_free[b], (uint32_t)(((x >> 1) & 1) ^ 1), abort_flag))) break;
+        const int64_t it = 2 * gc + union_item(c, 0, n);
         const int slot = (int)(it % kSlots);
-        if (!(ok = warp_wait(&ctl.slot_full[slot], (uint32_t)((it / kSlots) & 1), abort_flag))) break;
+        if (!(ok = warp_wait_sleep(&ctl.slot_full[slot], (uint32_t)((it / kSlots) & 1), abort_flag))) break;
         tc_fence_after();
         if (lane == 0) {
           fence_proxy_async_smem();
           const uint32_t k_addr = sb + slot * kSlotBytes;
-          for (int kk = 0; kk < 16; ++kk) {             // 16 k-steps of 16 dims
+          for (int kk = 0; kk < 16; ++kk) {             // 16 k-steps of 16 dims; Q: 8 columns each
             const int slab = kk >> 2, sub = kk & 3;
-            const uint64_t da = desc_sw128(q_addr + slab * 16384 + sub * 32, 16, 1024);
             const uint64_t db = desc_sw128(k_addr + slab * 8192 + sub * 32, 16, 1024);
-            umma_bf16(tmem + b * kKeys, da, db, kIdescS, kk != 0);
+            umma_bf16_ts(tmem + b * kKeys, tmem + kTmemQ + kk * 8, db, kIdescS, kk != 0);
           }
           umma_commit(&ctl.slot_empty[slot]);
           umma_commit(&ctl.s_full[b]);
           if (c == u.nchunks - 1) umma_commit(&ctl.q_empty);
         }
         __syncwarp();
-        if (c > 0) ok = pv(x - 1, c - 1, c == 1, false);
+        if (c > 0) ok = pv(x - 1, c - 1, n);
       }
       if (!ok) break;
-      ok = pv(gc + u.nchunks - 1, u.nchunks - 1, u.nchunks == 1, true);
+      ok = pv(gc + n - 1, n - 1, n);
       gc += u.nchunks;
       ++uc;
     }
@@ -440,6 +463,29 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       const uint32_t own_rows = (2u << (uint32_t)(t & 3)) - 1u;
       const int32_t* ub = a.ublk + u.tile * a.cap;
       const uint32_t* um = a.umask + u.tile * a.cap;
+      // this unit's Q rows into TMEM, the A operand of S (bf16 pairs as they
+      // lie in memory): row li = member qi, head hh; this thread dims
+      // 128 half .. +127; rows of no member are zero.  The previous unit's
+      // last S products have finished first.
+      mbar_wait_sleep(&ctl.q_empty, (uint32_t)((uc & 1) ^ 1), abort_flag);
+      {
+        const uint4* qrow = reinterpret_cast<const uint4*>(
+            (const __nv_bfloat16*)a.q + ((u.ti.tok0 + qi) * g.H + (int64_t)u.grp * g.hpg + hh) * kHeadDim + half * 128);
+        tc_fence_after();
+#pragma unroll
+        for (int piece = 0; piece < 4; ++piece) {
+          uint4 x[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) x[j] = active ? qrow[piece * 4 + j] : make_uint4(0, 0, 0, 0);
+          const uint32_t v[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
+                                  x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
+          tmem_st16u(lane_addr + kTmemQ + half * 64 + piece * 16, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl.q_full);
+      }
       float m = -INFINITY, l = 0.f;
       // this thread's 8 union entries of a chunk (blocks and member masks),
       // loaded one chunk ahead: entries c*16 + 8 half .. +7 (inside the
@@ -472,9 +518,9 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
           }
         }
         if (c + 1 < u.nchunks) fetch(c + 1);
-        mbar_wait(&ctl.s_full[b], (uint32_t)((gc >> 1) & 1), abort_flag);
+        mbar_wait_sleep(&ctl.s_full[b], (uint32_t)((gc >> 1) & 1), abort_flag);
         tc_fence_after();
-        float s[32];
+        float s[32];                             // raw scores; keys this row does not attend: -inf
         {
           float s0[16], s1[16];
           tmem_ld16(lane_addr + b * kKeys + half * 32, s0);
@@ -482,18 +528,14 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            s[i] = s0[i] * tau2;
-            s[16 + i] = s1[i] * tau2;
+            s[i] = ((vbits >> i) & 1u) ? s0[i] : -INFINITY;
+            s[16 + i] = ((vbits >> (16 + i)) & 1u) ? s1[i] : -INFINITY;
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl.s_free[b]);
         float pm = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if ((vbits >> i) & 1u) pm = fmaxf(pm, s[i]);
-        ctl.red[li][half] = pm;
+        for (int i = 0; i < 32; ++i) pm = fmaxf(pm, s[i]);
+        ctl.red[li][half] = pm * tau2;
         named_bar_sync(1 + quad, 64);
         const float mc = fmaxf(ctl.red[li][0], ctl.red[li][1]);
         named_bar_sync(1 + quad, 64);            // both read before the next chunk writes
@@ -510,7 +552,7 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
         if (__any_sync(0xffffffffu, need)) {
           // O holds chunks 0..c-1 (c >= 1 here): wait for the last of their P.V products
           const int64_t xp = gc - 1;
-          mbar_wait(&ctl.p_free[xp & 1], (uint32_t)((xp >> 1) & 1), abort_flag);
+          mbar_wait_sleep(&ctl.p_free[xp & 1], (uint32_t)((xp >> 1) & 1), abort_flag);
           tc_fence_after();
 #pragma unroll 1
           for (int piece = 0; piece < 8; ++piece) {
@@ -525,32 +567,34 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
           tmem_wait_st();
           tc_fence_before();
         }
+        // P = 2^(tau2 s - m): -inf scores give 0; a row with no attended key yet keeps m = -inf
+        const float mb = m == -INFINITY ? 0.f : m;
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ((vbits >> (2 * i)) & 1u) ? exp2f(s[2 * i] - m) : 0.f;
-          const float p1 = ((vbits >> (2 * i + 1)) & 1u) ? exp2f(s[2 * i + 1] - m) : 0.f;
+          const float p0 = ex2_approx(fmaf(s[2 * i], tau2, -mb));
+          const float p1 = ex2_approx(fmaf(s[2 * i + 1], tau2, -mb));
           l += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
-        mbar_wait(&ctl.p_free[b], (uint32_t)(((gc >> 1) & 1) ^ 1), abort_flag);
-        {
-          unsigned char* prow = smem + kOffP + b * kPBytes + li * 128;
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(prow + (((half * 4 + j) ^ (li & 7)) << 4)) =
-                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        }
-        fence_proxy_async_smem();
+        // P over the first 32 of this chunk's 64 S columns: both warps of the
+        // row have read S (the exchange above), and P.V(c-2), the last reader
+        // of these columns, ran before S(c) in the MMA order
+        tmem_st16u(lane_addr + b * kKeys + half * 16, pk);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl.p_full[b]);
+        if (lane == 0) {
+          mbar_arrive(&ctl.s_free[b]);
+          mbar_arrive(&ctl.p_full[b]);
+        }
       }
       // the row's denominator: both warps' partial sums
       ctl.red[li][half] = l;
       named_bar_sync(1 + quad, 64);
       const float lt = ctl.red[li][0] + ctl.red[li][1];
       named_bar_sync(1 + quad, 64);
-      mbar_wait(&ctl.o_full, (uint32_t)(uc & 1), abort_flag);
+      mbar_wait_sleep(&ctl.o_full, (uint32_t)(uc & 1), abort_flag);
       tc_fence_after();
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       __nv_bfloat16* orow = (__nv_bfloat16*)a.o +

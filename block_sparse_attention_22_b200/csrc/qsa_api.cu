@@ -599,20 +599,6 @@ UnionPlan union_plan(const Geo& g, const qsa_segment_t* segs, int n) {
   return p;
 }
 
-// q as [T][H][256] bf16: boxes of 64 dims x hpg heads x mq tokens, 128-byte
-// swizzle, tokens past T read as zero.
-bool make_q_tile_map(CUtensorMap* m, const void* q, int64_t n_tokens, const Geo& g, int mq) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)g.H, (cuuint64_t)n_tokens};
-  cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)g.H * kHeadDim * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)g.hpg, (cuuint32_t)mq};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 qsa_status_t run_attn_union(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens,
                             const qsa_cache_t* cache, const void* q, const int32_t* sel, const int32_t* nsel,
                             void* o, float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -621,8 +607,7 @@ qsa_status_t run_attn_union(const Geo& g, const qsa_segment_t* segs, int n, int3
   // the union build holds a bitmap of the context's blocks and its prefix in shared memory
   const int64_t max_words = cdiv(seg_max_blocks(segs, n, g.r) + 1, 32);
   if (((size_t)2 * max_words + (size_t)p.cap) * 4 > (size_t)227 * 1024) return QSA_ERR_UNSUPPORTED;
-  CUtensorMap tq;
-  if (!make_q_tile_map(&tq, q, n_tokens, g, p.mq)) return QSA_ERR_CUDA;
+  (void)n_tokens;
   UnionBuildArgs ba;
   memset(&ba, 0, sizeof ba);
   ba.sel = sel;
@@ -634,6 +619,7 @@ qsa_status_t run_attn_union(const Geo& g, const qsa_segment_t* segs, int n, int3
   ba.mq = p.mq;
   AttnUnionArgs ta;
   memset(&ta, 0, sizeof ta);
+  ta.q = q;
   ta.k = cache->k;
   ta.v = cache->v;
   ta.ulen = ba.ulen;
@@ -666,7 +652,7 @@ qsa_status_t run_attn_union(const Geo& g, const qsa_segment_t* segs, int n, int3
         ta.tile_base = tile_base;
         const int grid = (int)std::min<int64_t>(tiles * g.G, sms);
         count_launch();
-        attn_union_kernel<<<dim3(grid), dim3(tc_attn::kThreads), tc_union::kSmemBytes, st>>>(tq, g, t, ta);
+        attn_union_kernel<<<dim3(grid), dim3(tc_attn::kThreads), tc_union::kSmemBytes, st>>>(g, t, ta);
         tile_base += tiles;
         return cudaGetLastError();
       });
