@@ -194,7 +194,7 @@ struct AttnUnionCtl {
   uint64_t slot_empty[tc_union::kSlots];
   uint64_t q_full, q_empty;
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2], p_free[2];
+  uint64_t p_full[2], p_free[2];   // P of a chunk written / its P.V finished (a rescale of O waits on it)
   uint64_t o_full, o_free;
   uint64_t mma_done;
   float red[128][2];        // a row's partial maximum / sum from each of its two softmax warps
