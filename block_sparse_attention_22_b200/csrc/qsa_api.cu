@@ -599,15 +599,14 @@ UnionPlan union_plan(const Geo& g, const qsa_segment_t* segs, int n) {
   return p;
 }
 
-qsa_status_t run_attn_union(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens,
-                            const qsa_cache_t* cache, const void* q, const int32_t* sel, const int32_t* nsel,
-                            void* o, float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
+qsa_status_t run_attn_union(const Geo& g, const qsa_segment_t* segs, int n, const qsa_cache_t* cache,
+                            const void* q, const int32_t* sel, const int32_t* nsel, void* o, float* lse,
+                            void* ws, size_t ws_bytes, cudaStream_t st) {
   const UnionPlan p = union_plan(g, segs, n);
   if (p.ws > 0 && (!ws || ws_bytes < p.ws)) return QSA_ERR_WORKSPACE;
   // the union build holds a bitmap of the context's blocks and its prefix in shared memory
   const int64_t max_words = cdiv(seg_max_blocks(segs, n, g.r) + 1, 32);
   if (((size_t)2 * max_words + (size_t)p.cap) * 4 > (size_t)227 * 1024) return QSA_ERR_UNSUPPORTED;
-  (void)n_tokens;
   UnionBuildArgs ba;
   memset(&ba, 0, sizeof ba);
   ba.sel = sel;
@@ -801,7 +800,7 @@ QSA_API qsa_status_t qsa_sparse_attn_fwd_union(const qsa_config_t* cfg, const qs
       !aligned16(cache->k) || !aligned16(cache->v) || !aligned16(sel))
     return QSA_ERR_INVALID_ARG;
   const Geo g = make_geo(cfg, cache);
-  return run_attn_union(g, segs, n_segs, n_tokens, cache, q, sel, nsel, o, lse, workspace, ws_bytes,
+  return run_attn_union(g, segs, n_segs, cache, q, sel, nsel, o, lse, workspace, ws_bytes,
                         (cudaStream_t)stream);
 }
 
