@@ -342,15 +342,32 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       const __nv_bfloat16* vg = (const __nv_bfloat16*)a.v + kv_off;
       const int32_t* ub = a.ublk + u.tile * a.cap;
       const int n = u.nchunks;
-      for (int j = 0; j < 2 * n && ok; ++j, ++item) {
-        // the chunk and tensor of ring position j (inverse of union_item)
-        const int kind = (j == 0) ? 0 : (j == 2 * n - 1) ? 1 : (j & 1) ? 0 : 1;
-        const int c = (j == 0) ? 0 : (j == 2 * n - 1) ? n - 1 : (j & 1) ? (j + 1) / 2 : j / 2 - 1;
-        int64_t myrow = -1;                      // lane i < 2: cache row of block pw + 9 i
+      // the chunk and tensor of ring position j (inverse of union_item)
+      auto chunk_of = [&](int j) -> int {
+        return (j == 0) ? 0 : (j == 2 * n - 1) ? n - 1 : (j & 1) ? (j + 1) / 2 : j / 2 - 1;
+      };
+      // lane i < 2: cache row of union block pw + 9 i of chunk c (entries checked by the union build)
+      auto rows_of = [&](int c) -> int64_t {
+        int64_t row = -1;
         if (lane < 2 && pw + kProducers * lane < kBlk) {
           const int pos = c * kBlk + pw + kProducers * lane;
-          if (pos < u.len) myrow = (int64_t)ub[pos] * 4;       // entries checked by the union build
+          if (pos < u.len) row = (int64_t)ub[pos] * 4;
         }
+        return row;
+      };
+      // the union entries are prefetched into L1 four ring positions ahead, so
+      // that their load does not hold up each position's copies
+      auto prefetch_rows = [&](int c) {
+        if (lane < 2 && pw + kProducers * lane < kBlk) {
+          const int pos = c * kBlk + pw + kProducers * lane;
+          if (pos < u.len) asm volatile("prefetch.global.L1 [%0];" ::"l"(ub + pos));
+        }
+      };
+      for (int j = 0; j < 4 && j < 2 * n; ++j) prefetch_rows(chunk_of(j));
+      for (int j = 0; j < 2 * n && ok; ++j, ++item) {
+        const int kind = (j == 0) ? 0 : (j == 2 * n - 1) ? 1 : (j & 1) ? 0 : 1;
+        if (j + 4 < 2 * n) prefetch_rows(chunk_of(j + 4));
+        const int64_t myrow = rows_of(chunk_of(j));
         {
           const int slot = (int)(item % kSlots);
           if (!(ok = warp_wait_sleep(&ctl.slot_empty[slot], (uint32_t)(((item / kSlots) & 1) ^ 1), abort_flag)))
