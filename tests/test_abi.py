@@ -162,3 +162,16 @@ def test_union_attention_host_checks_and_workspace():
     assert _call_union(cfg, cache, qsa.make_segments([(0, 0, 100, 0)]), T=0, ws=None, ws_bytes=0) == qsa.QSA_OK
     f32 = qsa.make_config(synth.Shape(dtype="f32"))
     assert _call_union(f32, cache, segs) == qsa.QSA_ERR_UNSUPPORTED
+
+
+def test_missing_library_fails_loudly():
+    """No fallback: without the built library every entry point raises."""
+    import subprocess
+    import sys
+    code = ("import block_sparse_attention_22_b200 as q\n"
+            "q.LIB_PATH = q.LIB_PATH + '.absent'\n"
+            "q.qsa_device_status()\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "not built" in r.stderr
