@@ -66,8 +66,15 @@ _C = ctypes.POINTER(RefConfig)
 def _lib(acc="f64"):
     name = "libqsa_oracle.so" if acc == "f64" else "libqsa_oracle_f32.so"
     if name not in _LIBS:
-        _build.build()
-        lib = ctypes.CDLL(os.path.join(HERE, name))
+        # QSA_ORACLE_LIB / QSA_ORACLE_LIB_F32: another build of qsa_oracle.c (the
+        # planted-mistake tests load deliberately wrong builds through these)
+        override = os.environ.get("QSA_ORACLE_LIB" if acc == "f64" else "QSA_ORACLE_LIB_F32")
+        if override:
+            path = override
+        else:
+            _build.build()
+            path = os.path.join(HERE, name)
+        lib = ctypes.CDLL(path)
         lib.qsa_ref_round_bf16.argtypes = [ctypes.c_double]
         lib.qsa_ref_round_bf16.restype = ctypes.c_double
         lib.qsa_ref_rope_theta.argtypes = [_C, ctypes.c_int]
