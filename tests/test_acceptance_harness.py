@@ -34,7 +34,6 @@ def test_exact_selection_is_accepted():
 def test_swap_inside_the_tie_band_is_accepted():
     _, s, sel, n, t = _row()
     s = s.copy()
-    kept = [int(b) for b in sel[:n - 1]]
     order = np.lexsort((np.arange(len(s)), -s))
     last_kept, first_out = int(order[S - 2]), int(order[S - 1])
     s[first_out] = s[last_kept]                   # a tie between the last kept and the first dropped block
