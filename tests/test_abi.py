@@ -175,3 +175,24 @@ def test_missing_library_fails_loudly():
                        capture_output=True, text=True, timeout=300)
     assert r.returncode != 0
     assert "not built" in r.stderr
+
+
+def test_product_never_reaches_the_oracle():
+    """The library and its binding neither import, load nor link the oracle."""
+    import ast
+    pkg = os.path.join(ROOT, "block_sparse_attention_22_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            tree = ast.parse(open(os.path.join(pkg, fn)).read())
+            for node in ast.walk(tree):
+                if isinstance(node, (ast.Import, ast.ImportFrom)):
+                    names = [a.name for a in node.names] + [getattr(node, "module", None) or ""]
+                    assert not any("oracle" in n for n in names), (fn, names)
+    csrc = os.path.join(pkg, "csrc")
+    for fn in os.listdir(csrc):
+        src = open(os.path.join(csrc, fn)).read()
+        assert "qsa_oracle" not in src and "qsa_ref_" not in src, fn
+    deps = os.popen(f"ldd {qsa.LIB_PATH}").read()
+    assert "oracle" not in deps
+    syms = os.popen(f"nm -D {qsa.LIB_PATH}").read()
+    assert "qsa_ref_" not in syms
