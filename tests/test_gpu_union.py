@@ -140,3 +140,19 @@ def test_tiles_with_hand_made_selections():
     sel, nsel = sel.cuda(), nsel.cuda()
     o, lse = union_attn(wl, x, sel, nsel)
     oracle_check(wl, x, sel, nsel, o, lse, list(range(T)), "hand-made")
+
+
+def test_union_attention_over_several_launch_tables():
+    """More than 128 segments (several launches sharing one workspace through
+    their tile offsets), out of slot order, with 1- to 3-query segments."""
+    sh = synth.Shape()
+    n_seq, ctx = 150, 700
+    wl = synth.Workload("many", sh, [], n_seq, 1024, [ctx] * n_seq, [0] * n_seq, [], 11)
+    wl.segments = [synth.Segment(s, ctx - 3 - (s % 3), 1 + (s % 3)) for s in reversed(range(n_seq))]
+    wl.cached_blocks = [sg.pos0 // 4 for sg in sorted(wl.segments, key=lambda sg: sg.slot)]
+    x = {k: v.cuda() for k, v in synth.make_inputs(wl).items()}
+    run = gpu_forward(wl, x)
+    o, lse = union_attn(wl, x, run.sel, run.nsel)
+    oracle_check(wl, x, run.sel, run.nsel, o, lse, list(range(0, wl.n_tokens, 7)), "many segments")
+    check_outputs(to_np(o), to_np(run.o).astype(np.float64), to_np(lse), to_np(run.lse).astype(np.float64),
+                  "bf16", "many segments vs per-query")
