@@ -18,6 +18,8 @@ kv-channels 256, rotary 0.25 at base 1e7; design report, QSA item: r=4, a
                 prefill chunk at [942080, 946176) of a 90%-cached sequence
   decode_1m     the decode part of mixed_1m alone: 8 sequences x 1 decode
                 query against a 1048576-token cache
+  mixed_1m_tail mixed_1m with the prefill chunk at the end of its sequence,
+                [1044480, 1048576)
   spec_decode_1m  8 sequences x 4 consecutive query tokens (a speculative
                 decode step) at the end of a 1048576-token cache; the 4
                 queries of a sequence share one stream of its k^
@@ -207,12 +209,12 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
         cached = [(ctx - q_len) // sh.r] * n_seqs
         return Workload(name, sh, segs, n_seqs, _round_cap(ctx, sh.r), [ctx] * n_seqs, cached, needles,
                         seed if seed is not None else 7)
-    if name == "mixed_1m":
+    if name in ("mixed_1m", "mixed_1m_tail"):
         sh = Shape()
         ctx = over.get("ctx", 1 << 20)
         n_dec = over.get("n_decode", 8)
         chunk = over.get("chunk", 4096)
-        pos0 = over.get("chunk_pos0", 942080)
+        pos0 = over.get("chunk_pos0", ctx - chunk if name == "mixed_1m_tail" else 942080)
         segs = [Segment(s, ctx - 1, 1) for s in range(n_dec)]
         segs.append(Segment(n_dec, pos0, chunk))
         needles = []

@@ -52,3 +52,14 @@ def test_drift_leaves_every_other_tensor_and_the_default_inputs_unchanged():
     local = synth.make_workload("prefill_128k_local")
     assert local.drift == 0.99 and synth.make_workload("prefill_128k").drift == 0.0
     assert [s.q_len for s in local.segments] == [131072]
+
+
+def test_mixed_tail_variant_puts_the_chunk_at_the_end_of_its_sequence():
+    tail = synth.make_workload("mixed_1m_tail")
+    base = synth.make_workload("mixed_1m")
+    assert [(s.slot, s.pos0, s.q_len) for s in tail.segments[:8]] == \
+        [(s.slot, s.pos0, s.q_len) for s in base.segments[:8]]
+    chunk = tail.segments[8]
+    assert (chunk.pos0, chunk.q_len) == ((1 << 20) - 4096, 4096)
+    assert tail.fill[8] == 1 << 20 and tail.cached_blocks[8] == chunk.pos0 // 4
+    assert (base.segments[8].pos0, base.fill[8]) == (942080, 946176)
