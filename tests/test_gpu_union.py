@@ -8,8 +8,9 @@ section 1).  Cases: inputs with and without locality (drifting indexer
 queries), ragged tiles at segment ends, decode and speculative-decode
 segments (tiles of 1 and 4 queries), tiles whose union spans the whole
 context (hundreds of 64-key chunks, so the running maximum moves and O is
-rescaled), and layer shapes that fill 128, 96, 64 and 32 query rows of a tile.
-Tolerances are the forward's (bf16 I/O).
+rescaled), layer shapes that fill 128, 96, 64 and 32 query rows of a tile,
+hand-made selections, and more than 128 segments (several launches sharing
+one workspace).  Tolerances are the forward's (bf16 I/O).
 """
 import numpy as np
 import pytest
