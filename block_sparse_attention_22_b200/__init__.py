@@ -15,7 +15,8 @@ from typing import Iterable, Optional, Sequence
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libqsa.so")
 
-QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA, QSA_ERR_TIMEOUT = range(6)
+(QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA, QSA_ERR_TIMEOUT,
+ QSA_ERR_BAD_INDEX) = range(7)
 QSA_DTYPE_F32, QSA_DTYPE_BF16 = 0, 1
 (QSA_OP_COMPRESS, QSA_OP_INDEX, QSA_OP_SELECT, QSA_OP_ATTN, QSA_OP_FORWARD, QSA_OP_FORWARD_LOWMEM,
  QSA_OP_ATTN_UNION) = range(7)

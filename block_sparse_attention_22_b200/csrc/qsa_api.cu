@@ -999,6 +999,7 @@ QSA_API qsa_status_t qsa_device_status(void* stream) {
     return QSA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return QSA_ERR_CUDA;
   if (h == kErrWaitTimeout) return QSA_ERR_TIMEOUT;
+  if (h == kErrBadIndex) return QSA_ERR_BAD_INDEX;
   if (h != kErrNone) return QSA_ERR_CUDA;
   return QSA_OK;
 }
@@ -1032,6 +1033,7 @@ QSA_API const char* qsa_status_string(qsa_status_t status) {
     case QSA_ERR_WORKSPACE: return "workspace missing or too small";
     case QSA_ERR_CUDA: return "CUDA error";
     case QSA_ERR_TIMEOUT: return "device-side wait timed out";
+    case QSA_ERR_BAD_INDEX: return "selection entry out of range (skipped)";
   }
   return "unknown status";
 }
@@ -1056,18 +1058,49 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxDevices];
+unsigned long long g_scratch_ctx[kMaxDevices];
+
+// Process-unique id of the current context (cuCtxGetId, through the
+// runtime's driver entry points), or 0 if the driver cannot tell.  A device
+// reset replaces the context, and with it the id.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of g_select_scratch on the current device.  In host code
 // the array's name only stands for a host-side shadow, so the address is
-// looked up once per device, with that device current, and cached.
+// looked up once per device and context, with that device current, and
+// cached; a new context on the device (after a device reset) looks it up
+// again.
 qsa_status_t select_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QSA_ERR_CUDA;
+  // 0 until the runtime has made the device's context current on this thread:
+  // then the address is looked up again, which also binds the context
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || ctx == 0 || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || !p) return QSA_ERR_CUDA;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();
   }
   *out = g_scratch_ptr[dev];
   return QSA_OK;

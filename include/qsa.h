@@ -46,8 +46,10 @@
  *     All work is enqueued on it in order; a call returns before it runs.
  *   - Host-checkable errors return QSA_ERR_INVALID_ARG / QSA_ERR_UNSUPPORTED /
  *     QSA_ERR_WORKSPACE before anything is enqueued.  A failed launch returns
- *     QSA_ERR_CUDA.  Device-side faults of bounded waits are reported by
- *     qsa_device_status().  A call with no query tokens is a no-op (QSA_OK).
+ *     QSA_ERR_CUDA.  Device-side faults of bounded waits, and selection
+ *     entries outside [0, n_cap/r) that an attention kernel skipped, are
+ *     reported by qsa_device_status().  A call with no query tokens is a
+ *     no-op (QSA_OK).
  *   - Supported shapes: r == 4, head_dim == 256, n_q_heads/n_kv_groups <= 16,
  *     idx_heads == 4, idx_dim in {64, 128}, budget_tokens a multiple of r with
  *     budget_tokens/r <= 512.
@@ -75,7 +77,9 @@ typedef enum {
   QSA_ERR_UNSUPPORTED = 2,  /* valid configuration the kernels do not implement      */
   QSA_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than qsa_workspace_size()     */
   QSA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed             */
-  QSA_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (qsa_device_status)  */
+  QSA_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (qsa_device_status)  */
+  QSA_ERR_BAD_INDEX = 6     /* a caller-supplied sel entry was out of range and skipped
+                               (qsa_device_status)                                     */
 } qsa_status_t;
 
 typedef enum { QSA_DTYPE_F32 = 0, QSA_DTYPE_BF16 = 1 } qsa_dtype_t;
@@ -297,7 +301,9 @@ qsa_status_t qsa_forward_lowmem(const qsa_config_t* cfg, const qsa_cache_t* cach
  *
  * The first call on a device looks up the array's device address (a CUDA
  * runtime query, once per device, with that device current); make that first
- * call before any stream capture on the device.  All calls on a device share
+ * call before any stream capture on the device.  After a device reset the
+ * first call in the new context looks it up again, so the same rule applies
+ * to it.  All calls on a device share
  * the one array and it keeps the last call's contents: calls that can
  * overlap on the GPU (other streams without ordering between them) race on
  * it; calls ordered on one stream do not.
@@ -313,8 +319,13 @@ qsa_status_t qsa_select_topk_noalloc(const qsa_config_t* cfg, const qsa_segment_
 size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* segs, int32_t n_segs,
                           int32_t n_tokens, qsa_op_t op);
 
-/* Reads and clears the current device's error word written by bounded
- * device-side waits; synchronises `stream`.  QSA_OK if no wait gave up. */
+/* Reads and clears the current device's error word; synchronises `stream`.
+ * QSA_OK if nothing was recorded; QSA_ERR_TIMEOUT if a bounded device-side
+ * wait gave up; QSA_ERR_BAD_INDEX if an attention kernel (forward, union or
+ * backward) met a sel entry other than the -1 padding outside
+ * [0, n_cap/r): such an entry is skipped (it contributes no key) and the
+ * rest of the row is attended as usual.  The first error recorded since the
+ * last call wins. */
 qsa_status_t qsa_device_status(void* stream);
 
 /* Reads into *count and clears the number of query rows whose selection took
