@@ -30,7 +30,13 @@ qsa_forward_lowmem, with both workspace sizes); "decode_1m" / "mixed_1m";
 "attn_union" (the attention of prefill_128k_local, whose indexer queries drift
 along the sequence, on union tiles of neighbouring queries beside the
 per-query path);
-"cpu_baseline" (the oracle on a bounded sample); "gpu_launches"; "clocks".
+"cpu_baseline" (the oracle on a bounded sample); "gpu_launches"; "clocks";
+"tensor_roofline" (the step's flops over its time against the bf16 peak, the
+index stage alone, and the attainable step time).  Side lines "decode_256k"
+and "prefill_8k" (the 256K-context decode batch and the 2 x 8K prefill) carry
+their own CPU oracle timing.  Each side line's "hbm_roofline" counts the
+algorithmic bytes only (no score round trip), with the bytes the
+score-matrix path actually moves beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qsa|reference]
 """
@@ -146,15 +152,38 @@ class Prepared:
         self.sel = torch.empty((T, sh.budget_blocks), dtype=torch.int32, device="cuda")
         self.nsel = torch.empty((T,), dtype=torch.int32, device="cuda")
         self.ld = max(4, math.ceil(max((p + n - 1) // sh.r for _, n, p, _ in self.segl) / 4) * 4)
-        self.ws = torch.empty(max(1, qsa.workspace_size(self.cfg, self.segs, T, qsa.QSA_OP_FORWARD)),
-                              dtype=torch.uint8, device="cuda")
-        self.scores = torch.empty((T, self.ld), dtype=torch.float32, device="cuda")
-        self.ws_sel = torch.empty(max(1, qsa.workspace_size(self.cfg, self.segs, T, qsa.QSA_OP_SELECT)),
-                                  dtype=torch.uint8, device="cuda")
-        self.ws_attn = torch.empty(max(1, qsa.workspace_size(self.cfg, self.segs, T, qsa.QSA_OP_ATTN)),
-                                   dtype=torch.uint8, device="cuda")
-        self.ranges = [(s.slot, s.pos0 // sh.r, (s.pos0 + s.q_len) // sh.r) for s in wl.segments]
-        self.ws_low = None
+        self.ranges = step_ranges(wl)
+        self._bufs = {}
+
+    # workspaces and the score matrix, allocated on first use (a profiling run of
+    # one stage holds only what that stage needs)
+    def _ws(self, op):
+        if op not in self._bufs:
+            self._bufs[op] = torch.empty(max(1, qsa.workspace_size(self.cfg, self.segs, self.T, op)),
+                                         dtype=torch.uint8, device="cuda")
+        return self._bufs[op]
+
+    @property
+    def ws(self):
+        return self._ws(qsa.QSA_OP_FORWARD)
+
+    @property
+    def ws_low(self):
+        return self._ws(qsa.QSA_OP_FORWARD_LOWMEM)
+
+    @property
+    def ws_sel(self):
+        return self._ws(qsa.QSA_OP_SELECT)
+
+    @property
+    def ws_attn(self):
+        return self._ws(qsa.QSA_OP_ATTN)
+
+    @property
+    def scores(self):
+        if "scores" not in self._bufs:
+            self._bufs["scores"] = torch.empty((self.T, self.ld), dtype=torch.float32, device="cuda")
+        return self._bufs["scores"]
 
     def workspace_bytes(self, lowmem: bool) -> int:
         op = qsa.QSA_OP_FORWARD_LOWMEM if lowmem else qsa.QSA_OP_FORWARD
@@ -163,8 +192,6 @@ class Prepared:
     def forward(self, lowmem: bool = False):
         x = self.x
         if lowmem:
-            if self.ws_low is None:
-                self.ws_low = torch.empty(max(1, self.workspace_bytes(True)), dtype=torch.uint8, device="cuda")
             qsa.qsa_forward_lowmem(self.cfg, self.cache, self.segs, self.T, x["q"], x["q_idx"], x["w"], self.o,
                                    self.lse, self.sel, self.nsel, self.ws_low)
         else:
@@ -185,35 +212,56 @@ class Prepared:
             qsa.qsa_sparse_attn_fwd(self.cfg, self.cache, self.segs, self.T, x["q"], self.sel, self.nsel, self.o,
                                     self.lse, self.ws_attn)
 
-    # ---------------------------------------------------------------- algorithmic work
     def work(self):
-        """Algorithmic bytes / flops of each stage for this batch (what QSA must touch)."""
-        sh, wl = self.sh, self.wl
-        pos = wl.token_positions().double()
-        bt = torch.floor(pos / sh.r)
-        nsel = torch.clamp(bt + 1, max=sh.budget_blocks)
-        el = 2 if sh.dtype == "bf16" else 4
-        D, H, G, DI, HI = sh.head_dim, sh.n_heads, sh.n_groups, sh.idx_dim, sh.idx_heads
-        n_new_blocks = sum(b1 - b0 for _, b0, b1 in self.ranges)
-        comp_bytes = n_new_blocks * (sh.r + 1) * DI * el
-        cand = bt.sum().item()
-        idx_flops = 2.0 * HI * DI * cand
-        # scores: score writes + query rows; k^ of prefill-like segments (64-query tiles) is
-        # L2-resident, while decode-like segments (< 16 queries, 4-query tiles) stream their
-        # sequence's k^ from HBM once per tile of 4 consecutive queries
-        idx_bytes = cand * 4 + self.T * HI * (DI * el + 4)
-        for s in wl.segments:
-            if s.q_len < 16:
-                for q0 in range(0, s.q_len, 4):
-                    t_last = s.pos0 + min(q0 + 4, s.q_len) - 1
-                    idx_bytes += (t_last // sh.r) * DI * el
-        sel_bytes = cand * 4 + self.T * (sh.budget_blocks + 1) * 4
-        gathered = float((nsel * sh.r).sum().item()) * G * D * el * 2
-        attn_bytes = gathered + self.T * H * D * el * 2 + self.T * H * 4 + self.T * (sh.budget_blocks + 1) * 4
-        attn_flops = 4.0 * H * D * float((nsel * sh.r).sum().item())
-        return dict(compress=dict(bytes=comp_bytes), index=dict(bytes=idx_bytes, flops=idx_flops),
-                    select=dict(bytes=sel_bytes), attn=dict(bytes=attn_bytes, flops=attn_flops,
-                                                            gathered_bytes=gathered))
+        return algorithmic_work(self.wl)
+
+
+def step_ranges(wl: synth.Workload):
+    """(slot, first block, end block) of the blocks each segment completes."""
+    r = wl.shape.r
+    return [(s.slot, s.pos0 // r, (s.pos0 + s.q_len) // r) for s in wl.segments]
+
+
+def algorithmic_work(wl: synth.Workload):
+    """Algorithmic bytes / flops of each stage for this batch (what QSA must touch)."""
+    sh = wl.shape
+    T = wl.n_tokens
+    pos = wl.token_positions().double()
+    bt = torch.floor(pos / sh.r)
+    nsel = torch.clamp(bt + 1, max=sh.budget_blocks)
+    el = 2 if sh.dtype == "bf16" else 4
+    D, H, G, DI, HI = sh.head_dim, sh.n_heads, sh.n_groups, sh.idx_dim, sh.idx_heads
+    n_new_blocks = sum(b1 - b0 for _, b0, b1 in step_ranges(wl))
+    comp_bytes = n_new_blocks * (sh.r + 1) * DI * el
+    cand = bt.sum().item()
+    idx_flops = 2.0 * HI * DI * cand
+    # scores: score writes + query rows; k^ of prefill-like segments (64-query tiles) is
+    # L2-resident, while decode-like segments (< 16 queries, 4-query tiles) stream their
+    # sequence's k^ from HBM once per tile of 4 consecutive queries
+    idx_q = T * HI * (DI * el + 4)
+    idx_khat = 0.0
+    for s in wl.segments:
+        if s.q_len < 16:
+            for q0 in range(0, s.q_len, 4):
+                t_last = s.pos0 + min(q0 + 4, s.q_len) - 1
+                idx_khat += (t_last // sh.r) * DI * el
+    score_bytes = cand * 4                     # the fp32 score matrix, written once and read once
+    idx_bytes = score_bytes + idx_q + idx_khat
+    sel_out = T * (sh.budget_blocks + 1) * 4
+    sel_bytes = score_bytes + sel_out
+    gathered = float((nsel * sh.r).sum().item()) * G * D * el * 2
+    attn_bytes = gathered + T * H * D * el * 2 + T * H * 4 + T * (sh.budget_blocks + 1) * 4
+    attn_flops = 4.0 * H * D * float((nsel * sh.r).sum().item())
+    # what the method must touch (no score round trip; the selection's algorithmic
+    # bytes are 0 when it is fused with the scoring): pooling, the k^ stream of
+    # decode-like queries, query rows, kept K/V rows, q/o/lse and sel
+    alg = comp_bytes + idx_q + idx_khat + sel_out + attn_bytes
+    return dict(compress=dict(bytes=comp_bytes),
+                index=dict(bytes=idx_bytes, flops=idx_flops, khat_bytes=idx_khat, query_bytes=idx_q,
+                           score_bytes=score_bytes),
+                select=dict(bytes=sel_bytes), attn=dict(bytes=attn_bytes, flops=attn_flops, gathered_bytes=gathered),
+                algorithmic_bytes=alg, actual_bytes=comp_bytes + idx_bytes + sel_bytes + attn_bytes,
+                flops=idx_flops + attn_flops)
 
 
 class L2Flush:
@@ -355,23 +403,38 @@ def e2e_prefill(prep: Prepared, steps: int, warmup: int, n_chunks: int = 8):
 
 
 # ------------------------------------------------------------------ CPU oracle
-def oracle_sample(wl: synth.Workload, x, target_s: float = 10.0):
+def oracle_sample(wl: synth.Workload, x, target_s: float = 10.0, max_slots: int = 0, phase: float = 0.0):
     """Time the CPU oracle on a stratified sample of the workload's queries and
     extrapolate to the whole batch (per-query work grows linearly with the
-    position, so evenly spaced positions give an unbiased mean).  Returns
-    (tokens/s, threads, description)."""
+    position, so evenly spaced positions give an unbiased mean; `phase` in
+    [0, 1) shifts the evenly spaced picks).  With max_slots > 0 only that many
+    cache slots are timed (evenly spaced) and the estimate is scaled by the
+    query count of all slots (for batches of like sequences whose caches
+    would not all fit in host memory).  Returns (tokens/s, threads,
+    description)."""
     import oracle
     sh = wl.shape
     cfg = oracle.config_from_shape(sh)
     threads = len(os.sched_getaffinity(0))
     pos_all = wl.token_positions().numpy()
-    slots_all = wl.token_slots().numpy()
     f = lambda t: t.float().cpu().numpy()
     # per slot: pooled-key cost once (all blocks the queries need), then queries
     total_s, n_done, desc = 0.0, 0, []
     seg_rows = {}
     for off, s in zip(wl.token_offsets(), wl.segments):
         seg_rows.setdefault(s.slot, []).extend(range(off, off + s.q_len))
+    all_rows = sum(len(r) for r in seg_rows.values())
+    if max_slots and len(seg_rows) > max_slots:
+        keys = sorted(seg_rows)
+        keep = [keys[i] for i in np.linspace(0, len(keys) - 1, max_slots).astype(int)]
+        seg_rows = {k: seg_rows[k] for k in keep}
+    timed_rows = sum(len(r) for r in seg_rows.values())
+
+    def picks(rows, n):
+        if n >= len(rows):
+            return rows
+        return rows[np.minimum(len(rows) - 1, ((np.arange(n) + phase) * len(rows) / n).astype(int))]
+
     budget_per_slot = target_s / max(1, len(seg_rows))
     est_total = 0.0
     for slot, rows in seg_rows.items():
@@ -391,7 +454,7 @@ def oracle_sample(wl: synth.Workload, x, target_s: float = 10.0):
         oracle.forward(cfg, f(x["q"][pick]), f(x["q_idx"][pick]), f(x["w"][pick]), pos_all[pick], k_idx, k, v)
         t_cal = time.perf_counter() - t0
         n_s = int(min(len(rows), max(n_cal, n_cal * budget_per_slot / max(t_cal, 1e-3))))
-        pick = rows[np.linspace(0, len(rows) - 1, n_s).astype(int)]
+        pick = picks(rows, n_s)
         t0 = time.perf_counter()
         oracle.forward(cfg, f(x["q"][pick]), f(x["q_idx"][pick]), f(x["w"][pick]), pos_all[pick], k_idx, k, v)
         t_s = time.perf_counter() - t0
@@ -403,10 +466,15 @@ def oracle_sample(wl: synth.Workload, x, target_s: float = 10.0):
         est_total += t_comp + per_query * len(rows)
         total_s += t_s + t_comp
         n_done += n_s
-        desc.append(f"slot {slot}: {n_s} of {len(rows)} queries at evenly spaced positions")
+        desc.append(f"slot {slot}: {n_s} of {len(rows)} queries" +
+                    (" (all)" if n_s == len(rows) else " at evenly spaced positions"))
+    est_total *= all_rows / timed_rows
     tokens = wl.n_tokens
-    return tokens / est_total, threads, "; ".join(desc) + f"; {total_s:.1f} s of oracle wall time, " \
-        f"extrapolated by query count (pooling of the step's new blocks timed in full)"
+    slots_note = (f"{len(seg_rows)} of {len(set(s.slot for s in wl.segments))} sequences timed; "
+                  if timed_rows < all_rows else "")
+    return tokens / est_total, threads, slots_note + "; ".join(desc) + \
+        f"; {total_s:.1f} s of oracle wall time, extrapolated by query count (pooling of the step's new " \
+        f"blocks timed in full)"
 
 
 # ------------------------------------------------------------------ main
@@ -533,10 +601,13 @@ def measure_backward(name, steps, warmup, ws, flush, peaks):
     if sh.dtype == "bf16":
         nbytes = keys * G * (2 * D * 2 + 2 * 2 * D * 4) + T * H * (3 * D * 2 + D * 4 + 4)
         gbs = nbytes / (ms * 1e-3) / 1e9
-        out["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        out["roofline"] = {"bound": "gather (L2/HBM)", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                            "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes,
                            "peak_source": peaks["source"], "tflops": tflops,
-                           "tensor_frac": tflops / peaks["bf16_tflops"]}
+                           "tensor_frac": tflops / peaks["bf16_tflops"],
+                           "basis": "kept K/V rows read and dK/dV rows read and written, as logical bytes over "
+                                    "the HBM copy peak; the two sequences' K/V and dK/dV (about 100 MB) stay "
+                                    "in L2, so DRAM moves a small part of it"}
     else:
         peak = 148 * 128 * 2 * 1.965e9 / 1e12
         out["roofline"] = {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
@@ -628,8 +699,10 @@ def measure_union(name, steps, warmup, ws, flush, peaks, n=None):
            "union_blocks_per_tile": blocks_u / len(lens), "kept_blocks_per_query": blocks_q / T,
            "gathered_bytes_union": gathered_u, "gathered_bytes_per_query": gathered_q,
            "max_abs_diff_vs_per_query": diff, "gpu_launches_per_call": launches,
-           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes, "peak_source": peaks["source"]}}
+           "roofline": {"bound": "gather (L2/HBM)", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": nbytes, "peak_source": peaks["source"],
+                        "basis": "union K/V rows gathered once per tile and group, as logical bytes over the "
+                                 "HBM copy peak; neighbouring tiles share blocks, so most gathers hit L2"}}
     del prep
     torch.cuda.empty_cache()
     return out
@@ -667,6 +740,135 @@ def traffic_record(kernel: str, alg_bytes: float):
     return None
 
 
+def attention_roofline(work, attn_ms: float, peaks) -> dict:
+    """Roofline of the dominant kernel, the sparse attention.  Its algorithmic
+    bytes are the kept K/V rows gathered at zero reuse (2 x r x head_dim x 2 B
+    per kept block and KV group) plus q, o, lse and sel.  Part of that gather is
+    served from L2 (a group's K/V is about the size of L2), so the fraction of
+    the HBM copy peak can pass 1; the DRAM bytes of the committed ncu record
+    (scaled to this launch) give the fraction DRAM actually moved."""
+    nbytes = work["attn"]["bytes"]
+    achieved = nbytes / (attn_ms * 1e-3) / 1e9
+    traffic = traffic_record("attn", nbytes)
+    r = {"kernel": "sparse attention (attn stage)", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peaks["source"],
+         "bytes_per_launch": nbytes,
+         "basis": "gathered K/V bytes at zero reuse, partly served from L2 (not all HBM traffic)",
+         "tensor_frac": work["attn"]["flops"] / (attn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+    if traffic is not None:
+        r["dram_gbs"] = traffic / (attn_ms * 1e-3) / 1e9
+        r["dram_frac"] = r["dram_gbs"] / peaks["hbm_gbs"]
+    return r
+
+
+def step_tensor_roofline(work, step_ms: float, stage_ms, peaks) -> dict:
+    """The whole step's algorithmic flops (indexer and attention contractions)
+    over its device time, against the bf16 tensor peak: the literal figure for
+    the prefill target.  Beside it: the index stage alone (the one dense
+    contraction, k^ L2-resident) and the attainable step time, the sum over the
+    stages of max(flops / tensor peak, algorithmic bytes / HBM peak), where the
+    attention's bytes are its zero-reuse gather and the selection's are 0 (it
+    can be fused with the scoring)."""
+    tp, bw = peaks["bf16_tflops"] * 1e12, peaks["hbm_gbs"] * 1e9
+    flops = work["flops"]
+    achieved = flops / (step_ms * 1e-3) / 1e12
+    idx_ms = stage_ms[1]
+    att = [work["compress"]["bytes"] / bw,
+           max(work["index"]["flops"] / tp, (work["index"]["khat_bytes"] + work["index"]["query_bytes"]) / bw),
+           0.0,
+           max(work["attn"]["flops"] / tp, work["attn"]["bytes"] / bw)]
+    attainable_ms = sum(att) * 1e3
+    return {"flops_per_step": flops, "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": achieved / peaks["bf16_tflops"], "peak_source": peaks["source"],
+            "index_stage": {"ms": idx_ms, "flops": work["index"]["flops"],
+                            "achieved": work["index"]["flops"] / (idx_ms * 1e-3) / 1e12,
+                            "frac": work["index"]["flops"] / (idx_ms * 1e-3) / tp},
+            "attainable": {"ms_per_step": attainable_ms, "stage_ms": [a * 1e3 for a in att],
+                           "frac": attainable_ms / step_ms,
+                           "basis": "per stage max(flops / bf16 peak, algorithmic bytes / HBM peak); "
+                                    "attention bytes = zero-reuse gather; selection fused (0)"}}
+
+
+def side_line(name: str, args, ws: int, rank: int, flush, peaks) -> dict:
+    """One more workload's step beside the main line: device time, per-stage
+    times, the step's roofline on its algorithmic bytes (no score round trip)
+    and flops, the actual bytes the score-matrix path moves, and (rank 0, one
+    GPU) the CPU oracle on a bounded sample."""
+    wl2 = synth.make_workload(name)
+    prep2 = Prepared(wl2)
+    m2 = measure(prep2, args.steps, args.warmup, ws, flush, peaks)
+    w2 = m2["work"]
+    ms = m2["fused_ms"]
+    d = {"workload": name, "ms_per_step": ms, "tokens_per_step": wl2.n_tokens,
+         "tokens_per_s": job_throughput(wl2.n_tokens, ms, ws), "stages": m2["stages"], "gpu_launches": m2["launches"]}
+    alg, act = w2["algorithmic_bytes"], w2["actual_bytes"]
+    d["hbm_roofline"] = {"bytes_per_step": alg, "achieved_gbs": alg / (ms * 1e-3) / 1e9,
+                         "frac": alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+                         "peak_source": peaks["source"],
+                         "basis": "algorithmic bytes: pooling, k^ stream, query rows, kept K/V (zero reuse), "
+                                  "q/o/lse, sel; no score round trip",
+                         "actual_bytes_per_step": act,
+                         "actual_frac": act / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    d["tensor_roofline"] = {"flops_per_step": w2["flops"], "achieved": w2["flops"] / (ms * 1e-3) / 1e12,
+                            "frac": w2["flops"] / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                            "peak": peaks["bf16_tflops"]}
+    if rank == 0 and ws == 1 and not args.no_cpu and args.side_cpu_seconds > 0 and name in ORACLE_SIDE:
+        v, threads, desc = oracle_sample(wl2, prep2.x, args.side_cpu_seconds, max_slots=ORACLE_SIDE[name])
+        d["cpu_oracle"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
+    del prep2
+    torch.cuda.empty_cache()
+    return d
+
+
+# side lines with an oracle timing, and how many of their sequences it times
+# (each 256K-context sequence's K/V is 1 GiB in the oracle's fp32)
+ORACLE_SIDE = {"prefill_8k": 0, "decode_256k": 2}
+
+
+def parse_overrides(text: str) -> dict:
+    """'n_seqs=2,ctx=262144' -> {'n_seqs': 2, 'ctx': 262144} (integer or float values)."""
+    out = {}
+    for kv in [t for t in text.split(",") if t]:
+        k, v = kv.split("=")
+        out[k.strip()] = float(v) if "." in v else int(v)
+    return out
+
+
+def profile_stage(prep: Prepared, args, flush, peaks) -> int:
+    """One stage's public entry point alone, --warmup + --steps times, L2 flushed
+    before each; the stages before it run once, untimed, for its inputs."""
+    i = ["compress", "index", "select", "attn"].index(args.profile_stage)
+    for j in range(i):
+        prep.stage(j)
+    st = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        prep.stage(i)
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        prep.stage(i)
+        e1.record(st)
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    ms = tot / args.steps
+    w = prep.work()[args.profile_stage]
+    out = {"profile_stage": args.profile_stage, "workload": args.workload, "overrides": args.wl, "ms": ms}
+    if "bytes" in w:
+        out["algorithmic_bytes"] = w["bytes"]
+        out["gbs"] = w["bytes"] / (ms * 1e-3) / 1e9
+        out["hbm_frac"] = out["gbs"] / peaks["hbm_gbs"]
+    if "flops" in w:
+        out["tflops"] = w["flops"] / (ms * 1e-3) / 1e12
+        out["tensor_frac"] = out["tflops"] / peaks["bf16_tflops"]
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def bench_config(name: str, wl: synth.Workload, ws: int) -> dict:
     """The workload description both arms print."""
     return {"workload": name, "batch": len(wl.segments), "seq_len": wl.segments[0].q_len,
@@ -683,14 +885,22 @@ def run_reference(args):
         return 0
     wl = synth.make_workload(args.workload)
     x = synth.make_inputs(wl, device="cuda" if torch.cuda.is_available() else "cpu")
-    vals = []
+    # warm-up steps: a short sample each; timed steps: the time budget split over
+    # the steps, each on evenly spaced queries at its own phase, so that together
+    # they cover more distinct queries than the cpu_baseline leg's sample
+    for i in range(args.warmup):
+        oracle_sample(wl, x, target_s=0.5, phase=0.5)
+    est = []
     desc = ""
     threads = 0
-    for i in range(args.warmup + args.steps):
-        v, threads, desc = oracle_sample(wl, x, target_s=args.cpu_seconds / max(1, args.steps + args.warmup))
-        if i >= args.warmup:
-            vals.append(v)
-    val = statistics.mean(vals)
+    per_step = max(1.0, args.ref_seconds / max(1, args.steps))
+    for i in range(args.steps):
+        v, threads, d = oracle_sample(wl, x, target_s=per_step, phase=(i + 0.5) / args.steps)
+        est.append(wl.n_tokens / v)
+        desc = d
+    val = wl.n_tokens / statistics.mean(est)
+    desc = f"{args.steps} timed steps of about {per_step:.1f} s each, each a different evenly spaced query " \
+           f"sample; the last: {desc}"
     line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": wl.n_tokens / val * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -709,8 +919,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["qsa", "reference"], default="qsa")
     ap.add_argument("--workload", default="prefill_128k")
-    ap.add_argument("--decode-workload", default="decode_1m,mixed_1m",
+    ap.add_argument("--decode-workload", default="decode_1m,mixed_1m,decode_256k,prefill_8k",
                     help="comma-separated extra workloads reported beside the main line; 'none' to skip")
+    ap.add_argument("--side-cpu-seconds", type=float, default=8.0,
+                    help="oracle time budget of each side line's CPU timing (0: none)")
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="oracle time budget of the reference arm's timed steps, all together")
     ap.add_argument("--bwd-workload", default="prefill_8k",
                     help="workload of the attention-backward measurement; 'none' to skip")
     ap.add_argument("--union-workload", default="prefill_128k_local",
@@ -720,6 +934,11 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-lowmem", action="store_true", help="skip the low-memory forward line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--wl", default="",
+                    help="size overrides of --workload's recipe, e.g. n_seqs=2,ctx=262144 (profiling cases)")
+    ap.add_argument("--profile-stage", choices=["compress", "index", "select", "attn"], default=None,
+                    help="run one stage's entry point --warmup + --steps times on --workload and print its "
+                         "mean device time (the earlier stages run once, untimed); for ncu captures")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -729,20 +948,18 @@ def main():
     ws, rank = dist_setup()
     peaks = load_peaks()
     flush = L2Flush()
-    wl = synth.make_workload(args.workload)
+    wl = synth.make_workload(args.workload, **parse_overrides(args.wl))
     prep = Prepared(wl)
+    if args.profile_stage:
+        return profile_stage(prep, args, flush, peaks)
     clocks = ClockSampler(torch.cuda.current_device())
     m = measure(prep, args.steps, args.warmup, ws, flush, peaks, clocks)
     tokens = wl.n_tokens
     value = job_throughput(tokens, m["fused_ms"], ws)
 
     work = m["work"]
-    attn_ms = m["stage_ms"][3]
-    achieved = work["attn"]["bytes"] / (attn_ms * 1e-3) / 1e9
-    roofline = {"kernel": "sparse attention (attn stage)", "bound": "hbm", "achieved": achieved,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                "traffic": traffic_record("attn", work["attn"]["bytes"]), "peak_source": peaks["source"],
-                "bytes_per_launch": work["attn"]["bytes"]}
+    roofline = attention_roofline(work, m["stage_ms"][3], peaks)
+    tensor_roofline = step_tensor_roofline(work, m["fused_ms"], m["stage_ms"], peaks)
 
     e2e = None
     if not args.no_e2e:
@@ -774,22 +991,7 @@ def main():
 
     extra = {}
     for name in [n for n in args.decode_workload.split(",") if n and n != "none"]:
-        wl2 = synth.make_workload(name)
-        prep2 = Prepared(wl2)
-        m2 = measure(prep2, args.steps, args.warmup, ws, flush, peaks)
-        w2 = m2["work"]
-        dec_tokens = wl2.n_tokens
-        d = {"workload": name, "ms_per_step": m2["fused_ms"], "tokens_per_step": dec_tokens,
-             "tokens_per_s": job_throughput(dec_tokens, m2["fused_ms"], ws), "stages": m2["stages"],
-             "gpu_launches": m2["launches"]}
-        tot_bytes = sum(w2[k]["bytes"] for k in ("compress", "index", "select", "attn"))
-        # whole fused step against HBM: every byte QSA must touch, over the step's device time
-        d["hbm_roofline"] = {"bytes_per_step": tot_bytes,
-                             "achieved_gbs": tot_bytes / (m2["fused_ms"] * 1e-3) / 1e9}
-        d["hbm_roofline"]["frac"] = d["hbm_roofline"]["achieved_gbs"] / peaks["hbm_gbs"]
-        extra[name] = d
-        del prep2
-        torch.cuda.empty_cache()
+        extra[name] = side_line(name, args, ws, rank, flush, peaks)
 
     if args.union_workload != "none":
         extra["attn_union"] = measure_union(args.union_workload, args.steps, args.warmup, ws, flush, peaks,
@@ -803,7 +1005,8 @@ def main():
                 "warmup": args.warmup, "ms_per_step": m["fused_ms"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": wl.shape.dtype, "data": "synthetic",
                 "config": bench_config(args.workload, wl, ws),
-                "roofline": roofline, "stages": m["stages"], "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "tensor_roofline": tensor_roofline, "stages": m["stages"],
+                "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": m["launches"], "clocks": m["clocks"], "lowmem_forward": lowmem}
         line.update(extra)
         print(json.dumps(line), flush=True)

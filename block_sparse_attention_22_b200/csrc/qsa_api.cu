@@ -158,18 +158,37 @@ int sm_count();
 
 // ------------------------------------------------------------------ selection plan
 struct TopkPlan {
-  int chunk;
-  int max_ch;      // chunks per row in the workspace (1: no split rows)
   bool wide;       // few rows: one wide CTA per row
+  bool hist;       // few long rows: 4096-score chunks sharing a row histogram
   size_t ws;
+  size_t zero;     // leading workspace bytes to clear before the launches
 };
 
+// Workspace of the few-long-rows selection, per token row: a record of
+// counters and the histogram (cleared first), a list of S-1 indices and a
+// list of CAP key/index pairs.
+struct TopkHistLayout {
+  size_t rec, hist, sure, key, idx, zero, total;
+};
+
+TopkHistLayout topk_hist_layout(int64_t T) {
+  TopkHistLayout L;
+  L.rec = 0;
+  L.hist = (size_t)T * topk::kRecWords * 4;
+  L.zero = align_up(L.hist + (size_t)T * topk::kHistBins * 4, 256);
+  L.sure = L.zero;
+  L.key = L.sure + align_up((size_t)T * topk::KMAX * 4, 256);
+  L.idx = L.key + align_up((size_t)T * topk::CAP * 4, 256);
+  L.total = L.idx + align_up((size_t)T * topk::CAP * 4, 256);
+  return L;
+}
+
 // Many rows: one 4-warp CTA per row.  Few rows (too few to fill the GPU with
-// 4-warp CTAs): one 32-warp CTA per row while rows are short, else a split
-// into chunks (one 16-warp CTA each) that share a sampled row threshold,
-// then a merge (one 32-warp CTA per row).
+// 4-warp CTAs): one 32-warp CTA per row while rows are short, else 4096-score
+// chunks sharing a histogram of the row's top key bits, in three launches:
+// histograms, filter, final selection (one CTA per row).
 TopkPlan topk_plan(const Geo& g, const qsa_segment_t* segs, int n) {
-  TopkPlan p{topk::kChunkLarge, 1, false, 0};
+  TopkPlan p{false, false, 0, 0};
   const int64_t nblk = seg_max_blocks(segs, n, g.r);
   const int64_t rows = seg_rows(segs, n);
   if (nblk + 1 <= g.S || rows >= 4 * kNumSms) return p;
@@ -177,12 +196,12 @@ TopkPlan topk_plan(const Geo& g, const qsa_segment_t* segs, int n) {
     p.wide = true;
     return p;
   }
-  p.chunk = (int)std::max<int64_t>(topk::kChunkSmall, cdiv(nblk, 32));
-  p.max_ch = (int)cdiv(nblk, p.chunk);
+  p.hist = true;
   int64_t T = 0;
   for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
-  const size_t K = (size_t)(g.S - 1);
-  p.ws = align_up((size_t)T * p.max_ch * K * 4, 256) * 2 + align_up((size_t)T * p.max_ch * 4, 256);
+  const TopkHistLayout L = topk_hist_layout(T);
+  p.zero = L.zero;
+  p.ws = L.total;
   return p;
 }
 
@@ -385,18 +404,18 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
   a.ld = ld;
   a.sel = sel;
   a.nsel = nsel;
-  a.chunk = p.chunk;
-  a.max_ch = p.max_ch;
-  if (p.max_ch > 1) {
+  a.chunk = topk::kHistChunk;
+  if (p.hist) {
     int64_t T = 0;
     for (int i = 0; i < n; ++i) T = std::max<int64_t>(T, (int64_t)segs[i].q_offset + segs[i].q_len);
-    const size_t K = (size_t)(g.S - 1);
+    const TopkHistLayout L = topk_hist_layout(T);
     char* base = (char*)ws;
-    a.cand_key = (uint32_t*)base;
-    base += align_up((size_t)T * p.max_ch * K * 4, 256);
-    a.cand_idx = (int32_t*)base;
-    base += align_up((size_t)T * p.max_ch * K * 4, 256);
-    a.cand_cnt = (int32_t*)base;
+    a.hrec = (int32_t*)(base + L.rec);
+    a.hhist = (uint32_t*)(base + L.hist);
+    a.hsure = (int32_t*)(base + L.sure);
+    a.hkey = (uint32_t*)(base + L.key);
+    a.hidx = (int32_t*)(base + L.idx);
+    if (cudaMemsetAsync(ws, 0, L.zero, st) != cudaSuccess) return QSA_ERR_CUDA;
   }
   const size_t smem_c = 0;
   if (p.wide) {
@@ -408,23 +427,27 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
           return launch_chained(topk_wide_kernel, dim3(t.item0[t.n]), dim3(topk::kWideThreads), topk::kWideRingBytes, st, g, t, a);
         });
   }
-  if (p.max_ch > 1) {
-    qsa_status_t r = for_each_table(
+  if (p.hist) {
+    return for_each_table(
         segs, n,
         [&](const qsa_segment_t& s) {
           const int64_t nb = ((int64_t)s.pos0 + s.q_len - 1) / g.r;
-          return (int64_t)s.q_len * std::max<int64_t>(1, cdiv(nb, p.chunk));
+          return (int64_t)s.q_len * std::max<int64_t>(1, cdiv(nb, topk::kHistChunk));
         },
         [&](const SegTable& t) {
           count_launch();
-          return launch_chained(topk_split_kernel, dim3(t.item0[t.n]), dim3(topk::kSplitThreads), 0, st, g, t, a);
-        });
-    if (r != QSA_OK) return r;
-    return for_each_table(
-        segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
-        [&](const SegTable& t) {
+          cudaError_t e = launch_chained(topk_hist_kernel, dim3(t.item0[t.n]), dim3(topk::kHistThreads), 0, st, g,
+                                         t, a);
+          if (e != cudaSuccess) return e;
           count_launch();
-          return launch_chained(topk_merge_kernel, dim3(t.item0[t.n]), dim3(topk::kWideThreads), 0, st, g, t, a);
+          e = launch_chained(topk_hfilter_kernel, dim3(t.item0[t.n]), dim3(topk::kHistThreads), 0, st, g, t, a);
+          if (e != cudaSuccess) return e;
+          SegTable rt = t;                                   // one item per row
+          rt.item0[0] = 0;
+          for (int i = 0; i < t.n; ++i) rt.item0[i + 1] = rt.item0[i] + t.q_len[i];
+          count_launch();
+          return launch_chained(topk_hfinal_kernel, dim3(rt.item0[rt.n]), dim3(topk::kWideThreads), 0, st, g, rt,
+                                a);
         });
   }
   (void)smem_c;
@@ -761,7 +784,6 @@ QSA_API qsa_status_t qsa_select_topk(const qsa_config_t* cfg, const qsa_segment_
   if (!scores || !sel || !nsel || !aligned16(sel)) return QSA_ERR_INVALID_ARG;
   const int64_t nblk = seg_max_blocks(segs, n_segs, cfg->r);
   if (ld_scores < std::max<int64_t>(1, nblk)) return QSA_ERR_INVALID_ARG;
-  if (nblk > (int64_t)topk::kChunkLarge * 32) return QSA_ERR_UNSUPPORTED;
   const Geo g = make_geo(cfg, nullptr);
   return run_select(g, segs, n_segs, scores, ld_scores, sel, nsel, workspace, ws_bytes,
                     (cudaStream_t)stream);
@@ -894,8 +916,6 @@ qsa_status_t forward_impl(const qsa_config_t* cfg, const qsa_cache_t* cache, con
       !aligned16(cache->v) || !aligned16(cache->k_idx) || !aligned16(cache->khat))
     return QSA_ERR_INVALID_ARG;
   if ((sel == nullptr) != (nsel == nullptr) || (sel && !aligned16(sel))) return QSA_ERR_INVALID_ARG;
-  const int64_t nblk = seg_max_blocks(segs, n_segs, cfg->r);
-  if (nblk > (int64_t)topk::kChunkLarge * 32) return QSA_ERR_UNSUPPORTED;
   const Geo g = make_geo(cfg, cache);
   const FwdLayout L = fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16, lowmem);
   if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return QSA_ERR_WORKSPACE;
@@ -1119,7 +1139,6 @@ QSA_API qsa_status_t qsa_select_topk_noalloc(const qsa_config_t* cfg, const qsa_
   if (!scores || !sel || !nsel || !aligned16(sel)) return QSA_ERR_INVALID_ARG;
   const int64_t nblk = seg_max_blocks(segs, n_segs, cfg->r);
   if (ld_scores < std::max<int64_t>(1, nblk)) return QSA_ERR_INVALID_ARG;
-  if (nblk > (int64_t)topk::kChunkLarge * 32) return QSA_ERR_UNSUPPORTED;
   const Geo g = make_geo(cfg, nullptr);
   if (topk_plan(g, segs, n_segs).ws > (size_t)QSA_NOALLOC_SCRATCH_BYTES) return QSA_ERR_WORKSPACE;
   void* scratch = nullptr;

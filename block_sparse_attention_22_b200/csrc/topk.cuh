@@ -8,9 +8,10 @@
 //
 // Many rows: one warp per row (topk_rows_kernel, below), with the rows it
 // leaves selected by a 4-warp CTA each (~35 KB of shared memory, six CTAs per
-// SM); 32 warps per row when rows are few and at most 32K blocks long; split
-// chunks and a merge for few longer rows.  The CTA-level selection of one
-// row (topk_select) runs as follows.  Scores are compared as 32-bit keys
+// SM); 32 warps per row when rows are few and at most 32K blocks long; for
+// few longer rows, 4096-score chunks sharing an exact histogram of the row
+// (topk_hist_kernel, topk_hfilter_kernel, topk_hfinal_kernel).  The
+// CTA-level selection of one row (topk_select) runs as follows.  Scores are compared as 32-bit keys
 // whose unsigned order is the float order.  For a row of n candidates and
 // K = S-1:
 //   1. threshold: m = n/16 keys (1024 .. 8192, in runs of 8 neighbours spread
@@ -33,11 +34,7 @@
 // If the sampled threshold admits fewer than K or more than CAP elements, an
 // exact fallback runs: a radix select streamed over the whole row (four
 // passes), then one ordered pass that keeps everything above T and the
-// lowest-indexed elements equal to T.  Longer rows, when few, are split into
-// 16K-block chunks: the 16-warp CTA of each chunk derives the row's sampled
-// threshold (all chunks of a row agree on it) and writes the chunk's
-// elements at or above it, and a 32-warp merge runs steps 3-4 on the union
-// (or the exact fallback).
+// lowest-indexed elements equal to T.
 #pragma once
 #include "qsa_internal.cuh"
 #include "sm100.cuh"
@@ -55,14 +52,17 @@ constexpr int kMinSamples = 1024;
 constexpr int kMaxSamples = kBufWords;
 constexpr int kSampleGroup = 8;            // samples are runs of 8 neighbours (one 32-byte sector)
 constexpr int kSampleTarget = 1536;        // expected elements at or above the sampled threshold
-constexpr int kChunkLarge = 1 << 30;       // no split
-constexpr int kChunkSmall = 16384;         // chunk of a split row
 constexpr int kWideMaxBlocks = 32768;      // few rows up to this long: one wide CTA per row
-constexpr int kSplitThreads = 512;         // CTA of a split-row chunk
-constexpr int kMaxSplitChunks = 64;        // chunks per split row (the plan uses 32)
 constexpr int kWideStages = 8;             // cp.async slots per thread of the wide CTA
 constexpr int kWideRingBytes = kWideStages * kWideThreads * 16;
 constexpr int kFusedStride = 16;          // fused prefill selection: one sampled block in 16
+// few long rows: an exact histogram of the top key bits, then a filter
+constexpr int kHistBits = 12;              // sign, 8 exponent and 3 mantissa bits of the score
+constexpr int kHistBins = 1 << kHistBits;
+constexpr int kHistShift = 32 - kHistBits;
+constexpr int kHistChunk = 4096;           // scores per CTA
+constexpr int kHistThreads = 256;
+constexpr int kHistPer = kHistChunk / (4 * kHistThreads);   // 16-byte groups per thread
 }
 
 // Per-CTA-size constants: each thread owns CAPL candidate slots.
@@ -75,7 +75,7 @@ struct TopkCfg {
 };
 
 template <int NT>
-struct TopkShared {
+struct alignas(16) TopkShared {
   uint32_t hist[topk::NBINS];
   uint32_t cbuf[topk::kBufWords];          // candidates | sample | bitmap
   uint32_t kept[topk::KMAX];               // kept indices / final sorted list
@@ -651,11 +651,13 @@ struct TopkArgs {
   int64_t ld;
   int32_t* sel;
   int32_t* nsel;
-  uint32_t* cand_key;   // [T][max_ch][S-1]   (split rows only)
-  int32_t* cand_idx;    // [T][max_ch][S-1]
-  int32_t* cand_cnt;    // [T][max_ch]
-  int chunk;            // candidates per chunk
-  int max_ch;           // chunks per row in the workspace layout
+  int chunk;            // scores per chunk CTA (few long rows)
+  // few long rows (histogram path); hrec and hhist start zeroed
+  int32_t* hrec;        // [T][kRecWords] list counters and the row's threshold bin
+  uint32_t* hhist;      // [T][kHistBins] row histograms of the top key bits
+  int32_t* hsure;       // [T][KMAX] elements above the threshold bin
+  uint32_t* hkey;       // [T][CAP] keys of the threshold bin's elements
+  int32_t* hidx;        // [T][CAP] their block indices
 };
 
 // Puts sh.kept[0..K) (distinct indices in [lo, hi)) in ascending order.  A
@@ -682,28 +684,37 @@ __device__ void topk_sort_kept(TopkShared<NT>& sh, int K, int64_t lo, int64_t hi
     atomicOr(&bm[off >> 5], 1u << (off & 31));
   }
   __syncthreads();
-  const int wpt = (nw + NT - 1) / NT;         // words per thread, contiguous
-  const int w0 = min(nw, (int)threadIdx.x * wpt), w1 = min(nw, w0 + wpt);
+  // warp w owns the words [beg, end); its lanes read 32 consecutive words at
+  // a time (no bank conflicts) and a warp scan of their popcounts places
+  // each word's set bits
+  constexpr int WARPS = TopkCfg<NT>::WARPS;
+  const int per = (int)cdiv(cdiv(nw, WARPS), 32) * 32;
+  const int beg = min(nw, warp * per), end = min(nw, beg + per);
   int cnt = 0;
-  for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
-  int incl = cnt;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += v;
-  }
-  if (lane == 31) sh.warp_a[warp] = incl;
+  for (int w = beg + lane; w < end; w += 32) cnt += __popc(bm[w]);
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (lane == 0) sh.warp_a[warp] = cnt;
   __syncthreads();
-  int pos = incl - cnt;
-  for (int w = 0; w < warp; ++w) pos += sh.warp_a[w];
-  for (int w = w0; w < w1; ++w) {
-    uint32_t bits = bm[w];
+  int run = 0;
+  for (int w = 0; w < warp; ++w) run += sh.warp_a[w];
+  for (int w0 = beg; w0 < end; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t bits = w < end ? bm[w] : 0u;
+    const int c = __popc(bits);
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int pos = run + incl - c;
     while (bits) {
       const int b = __ffs(bits) - 1;
       bits &= bits - 1u;
       if (pos < KMAX) sh.kept[pos] = (uint32_t)(lo + ((int64_t)w << 5) + b);
       ++pos;
     }
+    run += __shfl_sync(0xffffffffu, incl, 31);
   }
   __syncthreads();
 }
@@ -714,76 +725,6 @@ __device__ void topk_write_final(TopkShared<NT>& sh, int K, int S, int64_t bt, i
   topk_sort_kept(sh, K, 0, bt);
   for (int i = threadIdx.x; i < S; i += blockDim.x)
     sel_row[i] = i < K ? (int32_t)sh.kept[i] : (i == K ? (int32_t)bt : -1);
-}
-
-// One row, or one chunk of a split row.
-struct TopkItem {
-  int64_t tok, bt, c0;
-  int n, c, n_ch_row;
-  bool all;            // every block in reach is kept (short context)
-  bool skip;           // nothing to do for this item
-};
-
-__device__ __forceinline__ TopkItem topk_item(const Geo& g, const SegTable& st, const TopkArgs& a, int item) {
-  TopkItem it;
-  const int si = find_segment(st, item);
-  const int local = item - st.item0[si];
-  const int64_t pos0 = st.pos0[si];
-  const int q_len = st.q_len[si];
-  const int64_t nb_seg = cdiv((pos0 + q_len - 1) / g.r, a.chunk);
-  const int n_ch_seg = (int)(nb_seg > 1 ? nb_seg : 1);
-  const int j = local / n_ch_seg;
-  it.c = local - j * n_ch_seg;
-  it.tok = st.q_offset[si] + j;
-  it.bt = (pos0 + j) / g.r;
-  it.all = it.bt + 1 <= g.S;
-  it.n_ch_row = it.all ? 1 : (int)cdiv(it.bt, a.chunk);
-  it.c0 = (int64_t)it.c * a.chunk;
-  it.n = it.all ? 0 : (int)((it.bt - it.c0) < a.chunk ? (it.bt - it.c0) : a.chunk);
-  it.skip = it.all ? it.c != 0 : it.c >= it.n_ch_row;
-  return it;
-}
-
-// A chunk of a split row: every chunk element at or above the row's sampled
-// threshold (computed by each chunk's CTA from the same sample, so all agree)
-// is written out, up to K per chunk (more marks the chunk as overflowed with
-// a count of -1).
-template <int NT>
-__device__ void topk_chunk_row_threshold(const Geo& g, const TopkArgs& a, const TopkItem& it, TopkShared<NT>& sh) {
-  using namespace topk;
-  const int K = g.S - 1;
-  if (threadIdx.x == 0) {
-    sh.n_kept = 0;
-    sh.n_ovf = 0;
-  }
-  const RowSrc row{a.scores + it.tok * a.ld, nullptr, nullptr, 0};
-  // every chunk CTA of the row repeats this: a smaller sample with a larger
-  // target (about 2048 of the row, 32 sampled above it) keeps it short, and
-  // the chunk lists (K each) and the merge buffer (CAP) hold that many
-  const uint32_t tkey = sampled_threshold(row, (int)it.bt, sh, 4096, 2048);
-  __syncthreads();
-  int cnt = 0;
-  filter_scores(a.scores + it.tok * a.ld + it.c0, it.c0, it.n, key_to_float(tkey), cnt, sh);
-  __syncthreads();
-  const int own = min(cnt, TopkCfg<NT>::CAPL);
-  int own_total;
-  const int pos = block_exscan(own, &own_total, sh);
-  const int n_ovf = sh.n_ovf;
-  const int nc = own_total + n_ovf;
-  const int64_t base = (it.tok * a.max_ch + it.c) * (int64_t)K;
-  if (nc > K || n_ovf > OVF) {
-    if (threadIdx.x == 0) a.cand_cnt[it.tok * a.max_ch + it.c] = -1;
-    return;
-  }
-  for (int s = 0; s < own; ++s) {
-    a.cand_key[base + pos + s] = sh.lkey()[s * NT + threadIdx.x];
-    a.cand_idx[base + pos + s] = (int32_t)sh.lidx()[s * NT + threadIdx.x];
-  }
-  for (int o = threadIdx.x; o < n_ovf; o += NT) {
-    a.cand_key[base + own_total + o] = sh.okey()[o];
-    a.cand_idx[base + own_total + o] = (int32_t)sh.oidx()[o];
-  }
-  if (threadIdx.x == 0) a.cand_cnt[it.tok * a.max_ch + it.c] = nc;
 }
 
 // Few rows, each up to kWideMaxBlocks blocks: one CTA of kWideThreads per
@@ -812,102 +753,254 @@ __global__ void __launch_bounds__(topk::kWideThreads, 1) topk_wide_kernel(Geo g,
   if (threadIdx.x == 0) a.nsel[tok] = S;
 }
 
-// Few long rows: one CTA of kSplitThreads per (row, chunk).  Rows of a
-// single chunk are selected in place; chunks of longer rows write their
-// elements at or above the row's sampled threshold for the merge.
-__global__ void __launch_bounds__(topk::kSplitThreads) topk_split_kernel(Geo g, SegTable st, TopkArgs a) {
+// One chunk of a row (few long rows).
+struct TopkItem {
+  int64_t tok, bt, c0;
+  int n, c, n_ch_row;
+  bool all;            // every block in reach is kept (short context)
+  bool skip;           // nothing to do for this item
+};
+
+__device__ __forceinline__ TopkItem topk_item(const Geo& g, const SegTable& st, const TopkArgs& a, int item) {
+  TopkItem it;
+  const int si = find_segment(st, item);
+  const int local = item - st.item0[si];
+  const int64_t pos0 = st.pos0[si];
+  const int q_len = st.q_len[si];
+  const int64_t nb_seg = cdiv((pos0 + q_len - 1) / g.r, a.chunk);
+  const int n_ch_seg = (int)(nb_seg > 1 ? nb_seg : 1);
+  const int j = local / n_ch_seg;
+  it.c = local - j * n_ch_seg;
+  it.tok = st.q_offset[si] + j;
+  it.bt = (pos0 + j) / g.r;
+  it.all = it.bt + 1 <= g.S;
+  it.n_ch_row = it.all ? 1 : (int)cdiv(it.bt, a.chunk);
+  it.c0 = (int64_t)it.c * a.chunk;
+  it.n = it.all ? 0 : (int)((it.bt - it.c0) < a.chunk ? (it.bt - it.c0) : a.chunk);
+  it.skip = it.all ? it.c != 0 : it.c >= it.n_ch_row;
+  return it;
+}
+
+// Few long rows (decode: a handful of rows of 32K to millions of blocks).
+// Three launches, each a stage of the whole batch:
+//   topk_hist_kernel (one CTA per 4096-score chunk of a row): the chunk's
+//     histogram of the top 12 key bits, added into the row's histogram;
+//   topk_hfilter_kernel (one CTA per chunk): the bin B of the row's (S-1)-th
+//     largest key (from the row's histogram, found by every chunk CTA while
+//     its chunk loads), then the chunk's elements in bins above B ("sure":
+//     all kept) and in B ("tied bin") appended to the row's two lists, each
+//     CTA reserving its ranges with one atomic per list;
+//   topk_hfinal_kernel (one CTA of kWideThreads per row): the sure elements
+//     and the best (key desc, index asc) of the tied bin (a radix select
+//     over the bin), ordered through a bitmap of the row.  A tied bin larger
+//     than its list sends the row to the exact streamed fallback.
+// Per token row the workspace holds a record (two list counters, cleared by
+// the launcher with the histogram; B and the counts), the histogram, the
+// sure list (S-1 entries) and the tied-bin list (CAP pairs).
+namespace topk {
+enum : int { kRecSure = 0, kRecTie, kRecBin, kRecAbove, kRecCount, kRecWords = 8 };
+
+// The chunk's scores, kHistPer 16-byte groups per thread (coalesced), in
+// registers; elements past n read as -inf and are flagged invalid.
+struct HistChunk {
+  float v[kHistPer * 4];
+  __device__ __forceinline__ void load(const float* row, int n) {
+    const bool vec = ((uintptr_t)row & 15) == 0;
+#pragma unroll
+    for (int k = 0; k < kHistPer; ++k) {
+      const int i = (k * kHistThreads + (int)threadIdx.x) * 4;
+      if (vec && i + 4 <= n) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(row + i));
+        v[4 * k] = x.x;
+        v[4 * k + 1] = x.y;
+        v[4 * k + 2] = x.z;
+        v[4 * k + 3] = x.w;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[4 * k + j] = i + j < n ? __ldcg(row + i + j) : -INFINITY;
+      }
+    }
+  }
+  __device__ __forceinline__ static int index(int e) {       // element e of this thread
+    return ((e >> 2) * kHistThreads + (int)threadIdx.x) * 4 + (e & 3);
+  }
+};
+
+// The bin of the row histogram h (kHistBins words in shared memory) that
+// holds the k-th largest element: *bin, *above = elements in higher bins,
+// *count = elements in that bin.  Warp w holds bins [w P, w P + P), P =
+// kHistBins / warps, read 32 consecutive words at a time.  Ends with a
+// barrier.
+template <int NT>
+__device__ void hist_row_locate(const uint32_t* h, int k, uint32_t* bin, int* above, int* count,
+                                TopkShared<NT>& sh) {
+  constexpr int WARPS = TopkCfg<NT>::WARPS;
+  constexpr int P = kHistBins / WARPS;
+  constexpr int STEPS = P / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int mine = 0;
+#pragma unroll
+  for (int j = 0; j < STEPS; ++j) mine += (int)h[warp * P + 32 * j + lane];
+  const int wsum = __reduce_add_sync(0xffffffffu, mine);
+  if (lane == 0) sh.warp_a[warp] = wsum;
+  __syncthreads();
+  int higher = 0;
+  for (int w = warp + 1; w < WARPS; ++w) higher += sh.warp_a[w];
+  if (higher < k && k <= higher + wsum) {       // this warp's bins hold it: walk its steps down
+    int run = higher;
+    for (int j = STEPS - 1; j >= 0; --j) {
+      const int c = (int)h[warp * P + 32 * j + lane];
+      const int step = __reduce_add_sync(0xffffffffu, c);
+      if (run + step >= k) {
+        int suf = c;                           // this and higher lanes of the step
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_down_sync(0xffffffffu, suf, off);
+          if (lane + off < 32) suf += v;
+        }
+        const int ex = run + suf - c;
+        if (ex < k && k <= ex + c) {
+          sh.sel_digit = (uint32_t)(warp * P + 32 * j + lane);
+          sh.sel_above = ex;
+          sh.sel_count = c;
+        }
+        break;
+      }
+      run += step;
+    }
+  }
+  __syncthreads();
+  *bin = sh.sel_digit;
+  *above = sh.sel_above;
+  *count = sh.sel_count;
+  __syncthreads();
+}
+}  // namespace topk
+
+__global__ void __launch_bounds__(topk::kHistThreads) topk_hist_kernel(Geo g, SegTable st, TopkArgs a) {
   using namespace topk;
   pdl_wait();
   pdl_trigger();
-  __shared__ TopkShared<topk::kSplitThreads> sh;
+  __shared__ uint32_t hist[kHistBins];
+  const TopkItem it = topk_item(g, st, a, blockIdx.x);
+  if (it.skip || it.all) return;
+  for (int b = threadIdx.x; b < kHistBins; b += kHistThreads) hist[b] = 0u;
+  HistChunk ch;
+  ch.load(a.scores + it.tok * a.ld + it.c0, it.n);
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < kHistPer * 4; ++e)
+    if (HistChunk::index(e) < it.n) atomicAdd(&hist[score_key(ch.v[e]) >> kHistShift], 1u);
+  __syncthreads();
+  uint32_t* gh = a.hhist + it.tok * kHistBins;
+  for (int b = threadIdx.x; b < kHistBins; b += kHistThreads) {
+    const uint32_t c = hist[b];
+    if (c) atomicAdd(&gh[b], c);
+  }
+}
+
+__global__ void __launch_bounds__(topk::kHistThreads, 4) topk_hfilter_kernel(Geo g, SegTable st, TopkArgs a) {
+  using namespace topk;
+  constexpr int NT = kHistThreads;
+  constexpr int E = kHistPer * 4;
+  pdl_wait();
+  pdl_trigger();
+  __shared__ TopkShared<NT> sh;
+  __shared__ int s_base_sure, s_base_tie;
   const int S = g.S, K = S - 1;
   const TopkItem it = topk_item(g, st, a, blockIdx.x);
   if (it.skip) return;
   int32_t* sel_row = a.sel + it.tok * S;
   if (it.all) {
-    for (int i = threadIdx.x; i < S; i += blockDim.x) sel_row[i] = (i <= it.bt) ? i : -1;
+    for (int i = threadIdx.x; i < S; i += NT) sel_row[i] = (i <= it.bt) ? i : -1;
     if (threadIdx.x == 0) a.nsel[it.tok] = (int32_t)(it.bt + 1);
     return;
   }
-  if (it.n_ch_row > 1) {
-    topk_chunk_row_threshold(g, a, it, sh);
-    return;
+  HistChunk ch;
+  ch.load(a.scores + it.tok * a.ld + it.c0, it.n);          // in flight while the threshold is found
+  uint32_t* h = sh.cbuf;
+  const uint32_t* gh = a.hhist + it.tok * kHistBins;
+  for (int b = threadIdx.x; b < kHistBins; b += NT) h[b] = __ldcg(gh + b);
+  __syncthreads();
+  uint32_t B;
+  int above, count;
+  hist_row_locate(h, K, &B, &above, &count, sh);
+  int32_t* rec = a.hrec + it.tok * kRecWords;
+  if (it.c == 0 && threadIdx.x == 0) {
+    rec[kRecBin] = (int32_t)B;
+    rec[kRecAbove] = above;
+    rec[kRecCount] = count;
   }
-  const RowSrc src{a.scores + it.tok * a.ld, nullptr, nullptr, 0};
-  topk_select(src, it.n, K, sh);
-  topk_write_final(sh, K, S, it.bt, sel_row);
-  if (threadIdx.x == 0) a.nsel[it.tok] = S;
+  if (count > CAP) return;                                  // the final kernel falls back
+  uint32_t is_sure = 0u, is_tie = 0u;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const uint32_t bin = score_key(ch.v[e]) >> kHistShift;
+    const bool in = HistChunk::index(e) < it.n;
+    is_sure |= (uint32_t)(in && bin > B) << e;
+    is_tie |= (uint32_t)(in && bin == B) << e;
+  }
+  int tot_sure, tot_tie;
+  const int ex_sure = block_exscan(__popc(is_sure), &tot_sure, sh);
+  const int ex_tie = block_exscan(__popc(is_tie), &tot_tie, sh);
+  if (threadIdx.x == 0) {
+    s_base_sure = tot_sure ? atomicAdd(rec + kRecSure, tot_sure) : 0;
+    s_base_tie = tot_tie ? atomicAdd(rec + kRecTie, tot_tie) : 0;
+  }
+  __syncthreads();
+  int32_t* sure = a.hsure + it.tok * KMAX;
+  uint32_t* tkey = a.hkey + it.tok * CAP;
+  int32_t* tidx = a.hidx + it.tok * CAP;
+  int ps = s_base_sure + ex_sure, pt = s_base_tie + ex_tie;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = HistChunk::index(e);
+    if ((is_sure >> e) & 1u) {
+      if (ps < KMAX) sure[ps] = (int32_t)(it.c0 + i);
+      ++ps;
+    } else if ((is_tie >> e) & 1u) {
+      if (pt < CAP) {
+        tkey[pt] = score_key(ch.v[e]);
+        tidx[pt] = (int32_t)(it.c0 + i);
+      }
+      ++pt;
+    }
+  }
 }
 
-// Merge of split rows (one CTA of kWideThreads per row): the union of the
-// chunk lists (every chunk element at or above the row's threshold) holds
-// every element of the row at or above the K-th largest once it has at
-// least K elements, so the exact selection runs on the union.  A chunk that
-// overflowed, a union smaller than K or larger than the candidate buffer
-// sends the row to the exact streamed fallback over its scores.
-__global__ void __launch_bounds__(topk::kWideThreads, 1) topk_merge_kernel(Geo g, SegTable st, TopkArgs a) {
+// One CTA per row: the sure elements, then the best K - above of the tied bin.
+__global__ void __launch_bounds__(topk::kWideThreads, 1) topk_hfinal_kernel(Geo g, SegTable st, TopkArgs a) {
   using namespace topk;
+  constexpr int NT = kWideThreads;
   pdl_wait();
   pdl_trigger();
-  constexpr int NT = kWideThreads;
   __shared__ TopkShared<NT> sh;
-  __shared__ int start[kMaxSplitChunks + 1];
-  __shared__ int bad;
   const int S = g.S, K = S - 1;
   const int item = blockIdx.x;
   const int si = find_segment(st, item);
   const int j = item - st.item0[si];
   const int64_t tok = st.q_offset[si] + j;
-  const int64_t t = st.pos0[si] + j;
-  const int64_t bt = t / g.r;
-  if (bt + 1 <= S) return;
-  const int n_ch_row = (int)cdiv(bt, a.chunk);
-  if (n_ch_row <= 1) return;
-  if (threadIdx.x < 32) {
-    // chunk list offsets (n_ch_row <= kMaxSplitChunks)
-    const int lane = threadIdx.x;
-    int run = 0, neg = 0;
-    for (int c0 = 0; c0 < n_ch_row; c0 += 32) {
-      const int c = c0 + lane;
-      const int v = c < n_ch_row ? a.cand_cnt[tok * a.max_ch + c] : 0;
-      neg |= v < 0;
-      int incl = v < 0 ? 0 : v;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += u;
-      }
-      if (c < n_ch_row) start[c + 1] = run + incl;
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    neg = __any_sync(0xffffffffu, neg);
-    if (lane == 0) {
-      start[0] = 0;
-      bad = neg;
-      sh.n_kept = 0;
-      sh.n_ovf = 0;
-    }
+  const int64_t bt = (st.pos0[si] + j) / g.r;
+  if (bt + 1 <= S) return;                                  // written by the filter kernel
+  const int32_t* rec = a.hrec + tok * kRecWords;
+  const int above = __ldcg(rec + kRecAbove), count = __ldcg(rec + kRecCount);
+  if (threadIdx.x == 0) {
+    sh.n_kept = 0;
+    sh.n_ovf = 0;
   }
   __syncthreads();
-  const int total = start[n_ch_row];
-  if (bad || total < K || total > CAP) {
+  if (count <= CAP) {
+    int cnt = 0;
+    for (int i = threadIdx.x; i < count; i += NT)
+      cand_append(__ldcg(a.hkey + tok * CAP + i), (uint32_t)__ldcg(a.hidx + tok * CAP + i), cnt, sh);
+    for (int i = threadIdx.x; i < above; i += NT) sh.kept[i] = (uint32_t)__ldcg(a.hsure + tok * KMAX + i);
+    if (threadIdx.x == 0) sh.n_kept = above;
+    __syncthreads();
+    select_candidates(cnt, K - above, sh);
+  } else {
     const RowSrc row{a.scores + tok * a.ld, nullptr, nullptr, 0};
     count_fallback();
     select_streamed(row, (int)bt, K, sh);
-  } else {
-    int cnt = 0;
-    const int64_t row_base = tok * a.max_ch * (int64_t)K;
-    for (int i = threadIdx.x; i < total; i += NT) {
-      int lo = 0, hi = n_ch_row - 1;            // chunk c with start[c] <= i < start[c+1]
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (start[mid] <= i) lo = mid; else hi = mid - 1;
-      }
-      const int64_t e = row_base + (int64_t)lo * K + (i - start[lo]);
-      cand_append(a.cand_key[e], (uint32_t)a.cand_idx[e], cnt, sh);
-    }
-    __syncthreads();
-    select_candidates(cnt, K, sh);
   }
   topk_write_final(sh, K, S, bt, a.sel + tok * S);
   if (threadIdx.x == 0) a.nsel[tok] = S;

@@ -291,13 +291,14 @@ qsa_status_t qsa_forward_lowmem(const qsa_config_t* cfg, const qsa_cache_t* cach
  * convenience, not part of the method.
  *
  * Same arguments, results and errors as qsa_select_topk, minus the
- * workspace.  Rows long enough to be split (beyond 32K candidate blocks,
- * in a batch of few rows) keep their per-chunk candidates in a device array
- * built into the library, QSA_NOALLOC_SCRATCH_BYTES (16 MiB)
- * per device, held by every GPU that loads the library until the process
- * exits.  A batch whose selection needs more than that (see
- * qsa_workspace_size(..., QSA_OP_SELECT)) returns QSA_ERR_WORKSPACE and
- * enqueues nothing.  Nothing is allocated or freed.
+ * workspace.  Rows beyond 32K candidate blocks, in a batch of few rows,
+ * keep their row histograms, counters and candidate lists (48 KiB per token
+ * row) in a device array built into the library,
+ * QSA_NOALLOC_SCRATCH_BYTES (16 MiB) per device, held by every GPU that
+ * loads the library until the process exits; each call clears the part it
+ * uses with cudaMemsetAsync on `stream`.  A batch whose selection needs more
+ * than that (see qsa_workspace_size(..., QSA_OP_SELECT)) returns
+ * QSA_ERR_WORKSPACE and enqueues nothing.  Nothing is allocated or freed.
  *
  * The first call on a device looks up the array's device address (a CUDA
  * runtime query, once per device, with that device current); make that first

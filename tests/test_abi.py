@@ -119,7 +119,7 @@ def test_workspace_sizes_are_host_only_and_grow_with_the_batch():
         assert qsa.workspace_size(cfg, dec_fwd, 8, op) >= 8 * 262143 * 4
     assert qsa.workspace_size(cfg, small, 1024, qsa.QSA_OP_COMPRESS) == 0
     dec = qsa.make_segments([(i, 1, (1 << 20) - 1, i) for i in range(8)])
-    assert qsa.workspace_size(cfg, dec, 8, qsa.QSA_OP_SELECT) > 0     # few long rows are split
+    assert qsa.workspace_size(cfg, dec, 8, qsa.QSA_OP_SELECT) > 0     # few long rows: row histograms
     assert qsa.workspace_size(cfg, dec, 8, qsa.QSA_OP_ATTN) > 0       # few units: split-K
     dec2 = qsa.make_segments([(i, 1, (1 << 21) - 1, i) for i in range(8)])
     short = qsa.make_segments([(i, 1, 100000, i) for i in range(8)])

@@ -45,3 +45,36 @@ def test_union_lengths_match_sets_on_ragged_batches():
 def test_job_throughput_counts_every_rank():
     assert bench.job_throughput(1000, 2.0, 1) == 500000.0
     assert bench.job_throughput(1000, 2.0, 4) == 2000000.0
+
+
+def test_algorithmic_work_matches_the_per_unit_figures():
+    """The bench's algorithmic work against the per-unit figures of the method:
+    a 1M-context decode query streams its sequence's k^ (262143 blocks x 128
+    dims x 2 B = 67.1 MB) and gathers 512 kept blocks of K and V in both groups
+    (4.19 MB); the 128K prefill does 2.20 TFLOP of indexer and 6.54 TFLOP of
+    attention contractions and gathers 545 GB at zero reuse."""
+    from block_sparse_attention_22_b200 import synth
+    w = bench.algorithmic_work(synth.make_workload("decode_1m"))
+    assert w["index"]["khat_bytes"] == 8 * 262143 * 128 * 2
+    assert w["attn"]["gathered_bytes"] == 8 * 512 * 4 * 2 * 256 * 2 * 2
+    per_query = w["algorithmic_bytes"] / 8
+    assert 71.3e6 < per_query < 71.5e6, per_query
+    assert w["actual_bytes"] - w["algorithmic_bytes"] == 2 * w["index"]["score_bytes"]
+    p = bench.algorithmic_work(synth.make_workload("prefill_128k"))
+    assert abs(p["index"]["flops"] - 2.20e12) < 0.01e12
+    assert abs(p["attn"]["flops"] - 6.54e12) < 0.01e12
+    assert abs(p["attn"]["gathered_bytes"] - 545.5e9) < 0.5e9
+    assert p["index"]["khat_bytes"] == 0            # a prefill's k^ is L2-resident
+
+
+def test_step_tensor_roofline_arithmetic():
+    work = {"flops": 8.0e12, "compress": {"bytes": 1e6},
+            "index": {"flops": 2.0e12, "khat_bytes": 0.0, "query_bytes": 1e6},
+            "attn": {"flops": 6.0e12, "bytes": 500e9}}
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0, "source": "test"}
+    r = bench.step_tensor_roofline(work, 80.0, [0.1, 4.0, 5.0, 70.0], peaks)
+    assert abs(r["achieved"] - 100.0) < 1e-9          # 8e12 flop / 80 ms
+    assert abs(r["frac"] - 0.1) < 1e-12
+    assert abs(r["index_stage"]["frac"] - 0.5) < 1e-12
+    # attainable: 1e6/5e12 + 2e12/1e15 + 0 + 500e9/5e12 seconds
+    assert abs(r["attainable"]["ms_per_step"] - (0.0002 + 2.0 + 100.0)) < 1e-9

@@ -31,9 +31,14 @@ def _cuda_inputs(wl, gen_device="cpu"):
 
 
 # --------------------------------------------------------------------------- stage: pooling
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_compress_keys_bit_exact_including_large_positions(dtype):
-    sh = synth.Shape(dtype=dtype, idx_dim=128 if dtype == "bf16" else 64)
+@pytest.mark.parametrize("dtype,idx_dim,rope_fraction", [
+    ("bf16", 128, 0.25), ("f32", 64, 0.25), ("bf16", 64, 0.25), ("f32", 128, 0.25),
+    ("bf16", 128, 0.3),      # 19 rotated pairs: a pair's partner sits in another 16-byte chunk
+    ("f32", 64, 0.3),        # 9 pairs
+    ("f32", 64, 1.0),        # every dim rotates
+])
+def test_compress_keys_bit_exact_including_large_positions(dtype, idx_dim, rope_fraction):
+    sh = synth.Shape(dtype=dtype, idx_dim=idx_dim, rope_fraction=rope_fraction)
     n_cap = 1 << 20
     g = torch.Generator().manual_seed(5)
     k_idx = torch.randn((1, n_cap, sh.idx_dim), generator=g).to(sh.torch_dtype).cuda()
@@ -96,9 +101,10 @@ def _score_rows(seed, lengths, tie_levels=None):
     ([1, 3, 511, 512, 513, 600, 2047, 2048, 4096, 32767], None),
     ([600, 3000, 32767], 3),
     ([20000, 32768, 3000], None),         # few rows: one wide CTA per row
-    ([32769, 40000, 65535], None),        # few long rows: chunks sharing a row threshold + merge
+    ([32769, 40000, 65535], None),        # few long rows: 4096-score chunks sharing a row histogram
     ([65535, 262143], 5),
-    ([300001, 70000], 2),                 # ties everywhere: chunk overflow, exact fallback
+    ([300001, 70000], 2),                 # ties everywhere: candidate list too long, exact fallback
+    ([40961, 4097, 4096, 8191, 600, 511, 1], None),   # one-element last chunks, single-chunk rows, short rows
 ])
 def test_select_topk_matches_oracle_on_seeded_rows(lengths, ties):
     S = 512
@@ -121,6 +127,64 @@ def test_select_topk_matches_oracle_on_seeded_rows(lengths, ties):
         ref, rn = oracle.select(rc, rows[i, :n].double().numpy(), t)
         assert int(nsel[i]) == rn
         np.testing.assert_array_equal(sel[i].cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("case", ["odd_ld", "negative", "needles", "one_hot", "dense_bin", "mid_bin", "tied_bin"])
+def test_select_few_long_rows_edge_cases(case):
+    """The few-long-rows path (a row histogram of the top 12 key bits, then a
+    filter at the bin holding the 511th largest): rows whose start is not
+    16-byte aligned (odd row pitch), negative scores, a few dominant needles
+    far above the rest, a row that is zero but for one element, scores
+    packed into a narrow range so that the threshold bin holds thousands of
+    elements (near and over the candidate list's capacity: the exact
+    fallback), a threshold bin of about 2000 elements (radix select over the
+    bin), and 600 equal scores in the threshold bin of which the lowest
+    indices must win (selection by counting)."""
+    S = 512
+    cfg_sh = synth.Shape()
+    cfg = qsa.make_config(cfg_sh)
+    lengths = [65535, 100003, 40000, 262143]
+    g = torch.Generator().manual_seed(23)
+    ld = max(lengths) + (1 if case == "odd_ld" else 0)
+    rows = torch.randn((len(lengths), ld), generator=g) * 7
+    if case != "negative":
+        rows = rows.abs()
+    if case == "needles":
+        for i, n in enumerate(lengths):
+            rows[i, torch.randint(0, n, (40,), generator=g)] = 1e6 + torch.arange(40).float()
+    if case == "one_hot":
+        rows.zero_()
+        rows[:, 12345] = 1.0
+    if case == "dense_bin":
+        rows = 100.0 + torch.rand((len(lengths), ld), generator=g) * 0.5   # one bin of the top bits holds ~all
+        rows[0] = 100.0 + torch.rand((ld,), generator=g) * 12.5 * 8        # ~5000 per bin near the top: fits or not
+    if case in ("mid_bin", "tied_bin"):
+        rows = torch.rand((len(lengths), ld), generator=g)                 # below the threshold bin
+        for i, n in enumerate(lengths):
+            pos = torch.randperm(n, generator=g)
+            rows[i, pos[:300]] = 200.0 + torch.rand(300, generator=g) * 50   # 300 above the bin
+            if case == "mid_bin":
+                rows[i, pos[300:2300]] = 96.0 + torch.rand(2000, generator=g) * 7.9   # one bin of the top bits
+            else:
+                rows[i, pos[300:900]] = 100.0                                  # 600 equal keys, 211 kept
+    segs = qsa.make_segments([(i, 1, 4 * n + 3, 0) for i, n in enumerate(lengths)])
+    T = len(lengths)
+    sc = rows.cuda().contiguous()
+    sel = torch.full((T, S), -7, dtype=torch.int32, device="cuda")
+    nsel = torch.full((T,), -7, dtype=torch.int32, device="cuda")
+    ws = torch.empty(max(1, qsa.workspace_size(cfg, segs, T, qsa.QSA_OP_SELECT)), dtype=torch.uint8, device="cuda")
+    qsa.qsa_select_topk(cfg, segs, T, sc, ld, sel, nsel, ws)
+    torch.cuda.synchronize()
+    rc = oracle.config_from_shape(cfg_sh)
+    for i, n in enumerate(lengths):
+        ref, rn = oracle.select(rc, rows[i, :n].double().numpy(), 4 * n + 3)
+        assert int(nsel[i]) == rn
+        np.testing.assert_array_equal(sel[i].cpu().numpy(), ref, err_msg=f"{case} row {i}")
+    # the same call again on the same workspace: the histograms and counters restart from zero
+    sel2 = torch.full((T, S), -7, dtype=torch.int32, device="cuda")
+    qsa.qsa_select_topk(cfg, segs, T, sc, ld, sel2, nsel, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(sel, sel2)
 
 
 @pytest.mark.parametrize("tie_levels", [None, 2, 1000])
@@ -204,7 +268,7 @@ def test_attention_parity_on_oracle_selection(name, over, every):
     ("prefill_8k", dict(n=2500, n_seqs=2), 7, 0.99),
     ("decode_256k", dict(ctx=20001, n_seqs=4), 1, 0.99),
     ("spec_decode_1m", dict(ctx=20001, n_seqs=3), 1, 0.99),     # 4 queries share a k^ stream
-    ("decode_256k", dict(ctx=140001, n_seqs=3), 1, 0.99),      # rows past 32K blocks: split selection
+    ("decode_256k", dict(ctx=140001, n_seqs=3), 1, 0.99),      # rows past 32K blocks: histogram selection
     ("spec_decode_1m", dict(ctx=140001, n_seqs=2), 1, 0.99),
     ("mixed_1m", dict(ctx=16384, n_decode=3, chunk=300, chunk_pos0=5001), 3, 0.99),
 ])

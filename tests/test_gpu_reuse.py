@@ -41,7 +41,7 @@ def test_second_layer_attends_with_the_first_layers_selection(name, over, every)
     n0 = qsa.launch_count()
     qsa.qsa_sparse_attn_fwd(cfg, cache2, segs, T, x2["q"], run1.sel, run1.nsel, o, lse, ws)
     torch.cuda.synchronize()
-    assert qsa.launch_count() - n0 <= 2                        # attention (+ split merge): no index/select
+    assert qsa.launch_count() - n0 <= 2                        # attention (+ split-K combine): no index/select
     rc = oracle.config_from_shape(sh)
     pos = wl.token_positions().numpy()
     slots = wl.token_slots().numpy()

@@ -1,5 +1,5 @@
 """qsa_select_topk_noalloc: the selection entry point for callers that cannot
-allocate device memory (its split-row scratch is a static device array in the
+allocate device memory (its few-long-rows scratch is a static device array in the
 library).  It must give the same selection as qsa_select_topk with a caller
 workspace, call after call.  Selections are integer results, so the
 comparison is exact, as in the other selection tests.
@@ -42,8 +42,9 @@ def test_noalloc_selection_matches_workspace_entry_point_on_consecutive_calls():
     sh = synth.Shape()
     cfg = qsa.make_config(sh)
     S = sh.budget_blocks
-    # long rows (when rows are few) are split into chunks whose candidates use
-    # the scratch; the short row takes the in-place path
+    # few long rows: their histograms, counters and candidate lists live in
+    # the scratch (cleared at the start of every call); the short row keeps
+    # every block
     lengths = [300001, 65535, 300, 40000, 524287]
     segs = qsa.make_segments([(i, 1, 4 * n + 3, 0) for i, n in enumerate(lengths)])
     T = len(lengths)
@@ -65,7 +66,7 @@ def test_noalloc_selection_matches_workspace_entry_point_on_consecutive_calls():
 def test_noalloc_rejects_a_batch_larger_than_its_scratch():
     sh = synth.Shape()
     cfg = qsa.make_config(sh)
-    T = 500         # 500 decode rows at 2M context, split into 32 chunks each: ~65 MB of candidates
+    T = 500         # 500 decode rows at 2M context: 48 KiB of histogram and candidate list each
     segs = qsa.make_segments([(i, 1, (1 << 21) - 1, 0) for i in range(T)])
     assert qsa.workspace_size(cfg, segs, T, qsa.QSA_OP_SELECT) > (16 << 20)
     scores = torch.zeros((1, 1), device="cuda")   # never read: rejected before any launch
