@@ -154,6 +154,7 @@ class Prepared:
         self.ld = max(4, math.ceil(max((p + n - 1) // sh.r for _, n, p, _ in self.segl) / 4) * 4)
         self.ranges = step_ranges(wl)
         self._bufs = {}
+        self.prefixes = qsa.make_prefixes(wl.prefix) if wl.prefix else None
 
     # workspaces and the score matrix, allocated on first use (a profiling run of
     # one stage holds only what that stage needs)
@@ -191,7 +192,11 @@ class Prepared:
 
     def forward(self, lowmem: bool = False):
         x = self.x
-        if lowmem:
+        if self.wl.prefix:
+            qsa.qsa_forward_prefixed(self.cfg, self.cache, self.segs, self.prefixes, self.T, x["q"], x["q_idx"],
+                                     x["w"], self.o, self.lse, self.sel, self.nsel,
+                                     self._ws(qsa.QSA_OP_FORWARD_PREFIXED))
+        elif lowmem:
             qsa.qsa_forward_lowmem(self.cfg, self.cache, self.segs, self.T, x["q"], x["q_idx"], x["w"], self.o,
                                    self.lse, self.sel, self.nsel, self.ws_low)
         else:
@@ -240,11 +245,17 @@ def algorithmic_work(wl: synth.Workload):
     # sequence's k^ from HBM once per tile of 4 consecutive queries
     idx_q = T * HI * (DI * el + 4)
     idx_khat = 0.0
-    for s in wl.segments:
+    shared = {}
+    for i, s in enumerate(wl.segments):
+        pb = wl.prefix[i][1] if wl.prefix else 0
+        if pb > 0:                      # its own blocks here; the prefix's once per 16 sharing queries, below
+            shared[wl.prefix[i]] = shared.get(wl.prefix[i], 0) + s.q_len
         if s.q_len < 16:
             for q0 in range(0, s.q_len, 4):
                 t_last = s.pos0 + min(q0 + 4, s.q_len) - 1
-                idx_khat += (t_last // sh.r) * DI * el
+                idx_khat += (t_last // sh.r - pb) * DI * el
+    for (_, pb), m in shared.items():
+        idx_khat += math.ceil(m / 16) * pb * DI * el
     score_bytes = cand * 4                     # the fp32 score matrix, written once and read once
     idx_bytes = score_bytes + idx_q + idx_khat
     sel_out = T * (sh.budget_blocks + 1) * 4
@@ -526,12 +537,14 @@ def measure(prep: Prepared, steps, warmup, ws, flush, peaks, clocks=None):
     barrier(ws)
     fused_ms = sum(p[0] for p in per) / steps
     fused_ms = max_over_ranks(fused_ms, ws)
-    per_s, launches_s = timed(prep, steps, max(1, warmup // 2), flush, staged=True)
-    barrier(ws)
-    stage_ms = [sum(p[i] for p in per_s) / steps for i in range(4)]
     work = prep.work()
     names = ["compress", "index", "select", "attn"]
     stages = {}
+    if prep.wl.prefix:          # the per-stage entry points take no shared prefixes: the fused step only
+        return dict(fused_ms=fused_ms, stage_ms=None, stages=None, work=work, launches=launches, clocks=clk)
+    per_s, launches_s = timed(prep, steps, max(1, warmup // 2), flush, staged=True)
+    barrier(ws)
+    stage_ms = [sum(p[i] for p in per_s) / steps for i in range(4)]
     for n, ms in zip(names, stage_ms):
         d = {"ms": ms}
         if "bytes" in work[n]:
@@ -809,6 +822,13 @@ def side_line(name: str, args, ws: int, rank: int, flush, peaks) -> dict:
                                   "q/o/lse, sel; no score round trip",
                          "actual_bytes_per_step": act,
                          "actual_frac": act / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    if wl2.prefix:
+        import dataclasses
+        alone = algorithmic_work(dataclasses.replace(wl2, prefix=[]))["index"]["khat_bytes"]
+        d["shared_prefix"] = {"khat_bytes_per_step": w2["index"]["khat_bytes"],
+                              "khat_bytes_if_unshared": alone,
+                              "khat_cut": alone / max(1.0, w2["index"]["khat_bytes"]),
+                              "prefix_blocks": wl2.prefix[0][1], "sequences": len(wl2.segments)}
     d["tensor_roofline"] = {"flops_per_step": w2["flops"], "achieved": w2["flops"] / (ms * 1e-3) / 1e12,
                             "frac": w2["flops"] / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                             "peak": peaks["bf16_tflops"]}
@@ -919,7 +939,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["qsa", "reference"], default="qsa")
     ap.add_argument("--workload", default="prefill_128k")
-    ap.add_argument("--decode-workload", default="decode_1m,mixed_1m,decode_256k,prefill_8k",
+    ap.add_argument("--decode-workload", default="decode_1m,mixed_1m,decode_256k,prefill_8k,shared_prefix_1m",
                     help="comma-separated extra workloads reported beside the main line; 'none' to skip")
     ap.add_argument("--side-cpu-seconds", type=float, default=8.0,
                     help="oracle time budget of each side line's CPU timing (0: none)")

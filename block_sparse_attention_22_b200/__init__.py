@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(HERE, "libqsa.so")
  QSA_ERR_BAD_INDEX) = range(7)
 QSA_DTYPE_F32, QSA_DTYPE_BF16 = 0, 1
 (QSA_OP_COMPRESS, QSA_OP_INDEX, QSA_OP_SELECT, QSA_OP_ATTN, QSA_OP_FORWARD, QSA_OP_FORWARD_LOWMEM,
- QSA_OP_ATTN_UNION) = range(7)
+ QSA_OP_ATTN_UNION, QSA_OP_FORWARD_PREFIXED) = range(8)
 
 
 class qsa_config_t(ctypes.Structure):
@@ -34,6 +34,10 @@ class qsa_config_t(ctypes.Structure):
 class qsa_segment_t(ctypes.Structure):
     _fields_ = [("q_offset", ctypes.c_int32), ("q_len", ctypes.c_int32),
                 ("pos0", ctypes.c_int32), ("slot", ctypes.c_int32)]
+
+
+class qsa_prefix_t(ctypes.Structure):
+    _fields_ = [("slot", ctypes.c_int32), ("blocks", ctypes.c_int32)]
 
 
 class qsa_cache_t(ctypes.Structure):
@@ -65,6 +69,7 @@ def _load():
         "qsa_sparse_attn_bwd": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, P, P],
         "qsa_forward": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, SZ, P],
         "qsa_forward_lowmem": [C, K, S, I32, I32, P, P, P, P, P, P, P, P, SZ, P],
+        "qsa_forward_prefixed": [C, K, S, ctypes.POINTER(qsa_prefix_t), I32, I32, P, P, P, P, P, P, P, P, SZ, P],
         "qsa_device_status": [P],
         "qsa_select_fallbacks": [P, ctypes.POINTER(ctypes.c_int64)],
         "qsa_selftest_wait_timeout": [P],
@@ -117,6 +122,15 @@ def make_segments(segs: Iterable[Sequence[int]]):
     for i, (off, n, p0, slot) in enumerate(segs):
         arr[i] = qsa_segment_t(off, n, p0, slot)
     return arr, len(segs)
+
+
+def make_prefixes(prefixes: Iterable[Sequence[int]]):
+    """Array of qsa_prefix_t from (slot, blocks) pairs, one per segment."""
+    prefixes = list(prefixes)
+    arr = (qsa_prefix_t * max(1, len(prefixes)))()
+    for i, (slot, blocks) in enumerate(prefixes):
+        arr[i] = qsa_prefix_t(slot, blocks)
+    return arr
 
 
 def _ptr(t) -> Optional[int]:
@@ -217,6 +231,18 @@ def qsa_forward_lowmem(cfg, cache, segs, n_tokens, q, q_idx, w, o, lse=None, sel
     _check(get_lib().qsa_forward_lowmem(ctypes.byref(cfg), ctypes.byref(cache), arr, n, n_tokens, _ptr(q),
                                         _ptr(q_idx), _ptr(w), _ptr(o), _ptr(lse), _ptr(sel), _ptr(nsel),
                                         _ptr(workspace), ws_bytes, _stream(stream)), "qsa_forward_lowmem")
+
+
+def qsa_forward_prefixed(cfg, cache, segs, prefixes, n_tokens, q, q_idx, w, o, lse=None, sel=None, nsel=None,
+                         workspace=None, stream=None):
+    """qsa_forward for sequences that share cached prefixes: prefixes is the
+    make_prefixes() array, one (slot, blocks) per segment (workspace:
+    QSA_OP_FORWARD_PREFIXED)."""
+    arr, n = segs
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(get_lib().qsa_forward_prefixed(ctypes.byref(cfg), ctypes.byref(cache), arr, prefixes, n, n_tokens,
+                                          _ptr(q), _ptr(q_idx), _ptr(w), _ptr(o), _ptr(lse), _ptr(sel), _ptr(nsel),
+                                          _ptr(workspace), ws_bytes, _stream(stream)), "qsa_forward_prefixed")
 
 
 def qsa_device_status(stream=None):

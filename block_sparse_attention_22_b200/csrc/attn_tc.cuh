@@ -109,6 +109,8 @@ struct TcUnit {
   int64_t tok;
   int64_t t;
   int64_t slot;
+  int64_t pslot;   // slot of the blocks below pblk (a shared prefix)
+  int pblk;
   int grp;
   int split;
   int blk_begin;   // first position in the sel row
@@ -138,6 +140,8 @@ __device__ __forceinline__ TcUnit tc_unit(const Geo& g, const SegTable& st, cons
   u.tok = st.q_offset[si] + j;
   u.t = (int64_t)st.pos0[si] + j;
   u.slot = st.slot[si];
+  u.pslot = st.pslot[si];
+  u.pblk = st.pblk[si];
   const int nsel = min(max(a.nsel[u.tok], 0), g.S);
   u.blk_begin = u.split * a.blocks_per_split;
   u.blk_end = min(nsel, u.blk_begin + a.blocks_per_split);
@@ -246,6 +250,10 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       ++uc;
       const __nv_bfloat16* kg = (const __nv_bfloat16*)a.k + (u.slot * g.G + u.grp) * g.n_cap * kHeadDim;
       const __nv_bfloat16* vg = (const __nv_bfloat16*)a.v + (u.slot * g.G + u.grp) * g.n_cap * kHeadDim;
+      // rows below the shared prefix's end come from its slot
+      const __nv_bfloat16* kp = (const __nv_bfloat16*)a.k + (u.pslot * g.G + u.grp) * g.n_cap * kHeadDim;
+      const __nv_bfloat16* vp = (const __nv_bfloat16*)a.v + (u.pslot * g.G + u.grp) * g.n_cap * kHeadDim;
+      const int64_t prow_end = (int64_t)u.pblk * g.r;
       const int32_t* selrow = a.sel + u.tok * g.S;
       // cache rows of this warp's kept blocks pw + 9 i of a chunk (lane i < 4)
       auto rows_of = [&](int cc) -> int64_t {
@@ -260,6 +268,7 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
         for (int c = 0; c < u.nchunks && ok; ++c) {
           const int64_t myrow = rows_of(c);
           const __nv_bfloat16* base = kind == 0 ? kg : vg;
+          const __nv_bfloat16* pbase = kind == 0 ? kp : vp;
           for (int h = 0; h < 2 && ok; ++h) {
             const int64_t hs = hs_next++;
             const int slot = (int)(hs % kSlots);
@@ -272,7 +281,8 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
               const int64_t row = __shfl_sync(0xffffffffu, myrow, bq);
               const int line = 4 * b + r;
               const uint32_t dst = dst0 + line * 128 + ((jc ^ (line & 7)) << 4);
-              const __nv_bfloat16* src = base + 128 * h + 8 * jc + (row >= 0 ? (row + r) * kHeadDim : 0);
+              const __nv_bfloat16* src = (row < prow_end ? pbase : base) + 128 * h + 8 * jc +
+                                         (row >= 0 ? (row + r) * kHeadDim : 0);
               const uint32_t nb = row >= 0 ? 16u : 0u;
               cp_async16(dst, src, nb);                       // dims 128h + 8jc .. +8
               cp_async16(dst + 16384, src + 64, nb);          // dims 128h + 64 + 8jc .. +8

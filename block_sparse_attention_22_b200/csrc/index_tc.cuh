@@ -84,6 +84,10 @@ struct IndexTcArgs {
   int32_t* cand_idx;            // [T][cand_cap]
   int32_t* cand_cnt;            // [T], zero on entry
   int cand_cap;
+  // queries already rotated (q_idx holds q~ rows): the query tile skips the
+  // rotation; row_map (or null): score row of query row i is row_map[i]
+  int prerotated;
+  const int32_t* row_map;
 };
 
 struct IndexTcCtl {
@@ -130,10 +134,17 @@ __host__ __device__ inline int64_t floor_sum(int64_t n, int64_t m, int64_t a, in
 // k^ tiles scored by query tile qt of a segment (the blocks its last query
 // scores, floor(t_last / r), in tiles of 128 scored rows; with stride s a row
 // is every s-th block, so a tile spans 128 s blocks).
+// The segment's scored blocks are [blk_lo, limit): tiles start at tile
+// floor(blk_lo / 128 s); limit = blk_cap when > 0, else the causal limit
+// (every query of a capped segment scores the same blocks).  First blocks
+// past 0 and caps are for the decode-like tiles (NQ < 64) only.
 template <int NQ>
-__host__ __device__ inline int index_qtile_tiles(int64_t pos0, int q_len, int qt, int r, int stride) {
+__host__ __device__ inline int index_qtile_tiles(int64_t pos0, int q_len, int qt, int r, int stride, int blk_lo = 0,
+                                                 int blk_cap = 0) {
+  const int64_t P = (int64_t)tc_index::kTileRows * stride;
   const int64_t t_last = pos0 + (int64_t)min(NQ * (qt + 1), q_len) - 1;
-  return (int)cdiv(t_last / r, (int64_t)tc_index::kTileRows * stride);
+  const int64_t n = cdiv(blk_cap > 0 ? (int64_t)blk_cap : t_last / r, P) - blk_lo / P;
+  return n > 0 ? (int)n : 0;
 }
 
 // Balancing weight of a query tile's prologue (building its rotated B tile),
@@ -147,19 +158,25 @@ constexpr int index_prologue_units() { return NQ >= 64 ? 6 : 2; }
 // 0..J-1 of a segment, where with P = 128 s blocks per tile the k^ tiles of
 // full query tile j are
 //   ceil(floor((pos0 + NQ j + NQ - 1) / r) / P) = floor((pos0 + NQ - 1 + (P-1) r + NQ j) / (P r)).
+// With a first block, every full query tile has floor(blk_lo / P) tiles
+// fewer (its causal limit is at least blk_lo: its queries lie past the
+// blocks it skips); with a cap, every query tile has the same count.
 template <int NQ>
-__host__ __device__ inline int64_t index_units_before(int64_t pos0, int J, int r, int stride) {
+__host__ __device__ inline int64_t index_units_before(int64_t pos0, int J, int r, int stride, int blk_lo = 0,
+                                                      int blk_cap = 0) {
   const int64_t P = (int64_t)tc_index::kTileRows * stride;
-  return floor_sum(J, P * r, NQ, pos0 + NQ - 1 + (P - 1) * r) + (int64_t)index_prologue_units<NQ>() * J;
+  const int64_t W = index_prologue_units<NQ>();
+  if (blk_cap > 0) return (int64_t)J * (index_qtile_tiles<NQ>(pos0, NQ, 0, r, stride, blk_lo, blk_cap) + W);
+  return floor_sum(J, P * r, NQ, pos0 + NQ - 1 + (P - 1) * r) - (int64_t)(blk_lo / P) * J + W * J;
 }
 
 // All work units of a segment.
 template <int NQ>
-inline int64_t index_tc_units(int q_len, int64_t pos0, int r, int stride = 1) {
+inline int64_t index_tc_units(int q_len, int64_t pos0, int r, int stride = 1, int blk_lo = 0, int blk_cap = 0) {
   if (q_len <= 0) return 0;
   const int nqt = (int)cdiv(q_len, NQ);
-  return index_units_before<NQ>(pos0, nqt - 1, r, stride) + index_prologue_units<NQ>() +
-         index_qtile_tiles<NQ>(pos0, q_len, nqt - 1, r, stride);
+  return index_units_before<NQ>(pos0, nqt - 1, r, stride, blk_lo, blk_cap) + index_prologue_units<NQ>() +
+         index_qtile_tiles<NQ>(pos0, q_len, nqt - 1, r, stride, blk_lo, blk_cap);
 }
 
 // Position in the flat sequence of work units: per segment, per query tile,
@@ -180,7 +197,8 @@ __device__ __forceinline__ void index_skip(const Geo& g, const SegTable& st, int
       c.qt = 0;
       ++c.si;
     }
-    c.nt = index_qtile_tiles<NQ>(st.pos0[c.si], st.q_len[c.si], c.qt, g.r, stride);
+    c.nt = index_qtile_tiles<NQ>(st.pos0[c.si], st.q_len[c.si], c.qt, g.r, stride, st.blk_lo[c.si],
+                                 st.blk_cap[c.si]);
     c.left -= index_prologue_units<NQ>();
   }
 }
@@ -195,14 +213,15 @@ __device__ __forceinline__ void index_seek(const Geo& g, const SegTable& st, int
   const int64_t local = L - st.item0[c.si];
   const int64_t pos0 = st.pos0[c.si];
   const int nqt = (int)cdiv(st.q_len[c.si], NQ);
+  const int blo = st.blk_lo[c.si], bcap = st.blk_cap[c.si];
   int lo = 0, hi = nqt - 1;                       // largest J with units_before(J) <= local
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (index_units_before<NQ>(pos0, mid, g.r, stride) <= local) lo = mid; else hi = mid - 1;
+    if (index_units_before<NQ>(pos0, mid, g.r, stride, blo, bcap) <= local) lo = mid; else hi = mid - 1;
   }
   c.qt = lo;
-  const int64_t o = local - index_units_before<NQ>(pos0, lo, g.r, stride);
-  c.nt = index_qtile_tiles<NQ>(pos0, st.q_len[c.si], lo, g.r, stride);
+  const int64_t o = local - index_units_before<NQ>(pos0, lo, g.r, stride, blo, bcap);
+  c.nt = index_qtile_tiles<NQ>(pos0, st.q_len[c.si], lo, g.r, stride, blo, bcap);
   if (o < W) {                                    // the slice starts inside the prologue weight
     c.left -= W - o;
     c.tile = 0;
@@ -275,7 +294,8 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
         if (!mbar_wait(&ctl.a_empty[s], (uint32_t)(((i / C::kStages) & 1) ^ 1), abort_flag)) break;
         mbar_expect_tx(&ctl.a_full[s], (uint32_t)(kTileRows * g.DI * 2));
         // tensor map [slot][scored row][dim]: rows past the slot's last read as zero
-        const int32_t y = (int32_t)((int64_t)cur.tile * kTileRows);
+        const int64_t lo_tile = NQ < 64 ? (int64_t)st.blk_lo[cur.si] / ((int64_t)kTileRows * a.stride) : 0;
+        const int32_t y = (int32_t)((lo_tile + cur.tile) * kTileRows);
         for (int slab = 0; slab < g.DI / 64; ++slab)
           tma_load_3d(smem + s * C::kABytes + slab * 16384, &tm_khat, 64 * slab, y, st.slot[cur.si], &ctl.a_full[s]);
       }
@@ -331,6 +351,7 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
 
     int64_t tok0 = 0, t_first = 0;
     int nq = 0;
+    int blo = 0, row0 = 0;                          // the segment's first scored block, and its tile row
     for (int i = 0; cur.left > 0; ++i, index_advance<NQ>(g, st, a.stride, cur)) {
       if (i == 0 || cur.tile == 0) {
         // ---------------------------------------------- new query tile
@@ -338,6 +359,10 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
         tok0 = st.q_offset[cur.si] + q0;
         t_first = (int64_t)st.pos0[cur.si] + q0;
         nq = min(NQ, st.q_len[cur.si] - q0);
+        if constexpr (NQ < 64) {                    // first blocks past 0: decode-like tiles only
+          blo = st.blk_lo[cur.si];
+          row0 = blo / (kTileRows * a.stride) * kTileRows;
+        }
         named_bar_sync(1, C::kEpiThreads);          // every share is done with the previous w, cos/sin
         for (int k = et; k < nq * half; k += C::kEpiThreads) {
           const int q = k / half, p = k - q * half;
@@ -348,6 +373,9 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
         for (int k = et; k < NQ * 4; k += C::kEpiThreads) ws[k] = (k >> 2) < nq ? a.w[tok0 * 4 + k] : 0.f;
         if (a.tau)
           for (int k = et; k < NQ; k += C::kEpiThreads) taus[k] = k < nq ? a.tau[tok0 + k] : __int_as_float(0x7fffffff);
+        else if (NQ == 16 && a.row_map)     // score mode: the tau area holds the score rows
+          for (int k = et; k < NQ; k += C::kEpiThreads)
+            reinterpret_cast<int32_t*>(taus)[k] = k < nq ? a.row_map[tok0 + k] : 0;
         named_bar_sync(1, C::kEpiThreads);
         // rotated queries: row n = q*4 + h of the B tile (K-major, 128-byte swizzle).
         // The accumulators of the previous query tile were all observed full,
@@ -367,7 +395,9 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
           const int n = task / chunks, j = task - n * chunks;
           const int q = n >> 2;
           uint4 out = raw[k];
-          if (hc > 0) {
+          if (NQ == 16 && a.prerotated) {
+            // q~ rows as given (the shared-prefix tiles)
+          } else if (hc > 0) {
             // partner chunk of a rotated pair: j + hc for first halves, j - hc for second halves
             const int src = j < hc ? lane + hc : (j < 2 * hc ? lane - hc : lane);
             uint4 pr;
@@ -435,13 +465,27 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.acc_free[ab]);  // values are in registers: the MMA may reuse it
 
-      const int64_t b0 = (int64_t)cur.tile * kTileRows;   // first scored row of the tile
+      const int64_t b0 = row0 + (int64_t)cur.tile * kTileRows;   // first scored row of the tile
       const int bl = quad * 32 + lane;                // scored row within the tile
       const int qb = cq * kQ;                         // first query of this share
       const int64_t t0 = t_first + qb;
       const int64_t blk = (b0 + bl) * a.stride;       // the pooled block of this row
-      // block blk is a candidate of the query at t iff (blk + 1) r <= t
-      const int64_t lim = t0 - (blk + 1) * g.r;
+      // block blk is a candidate of the query at t iff blk >= blk_lo and
+      // (blk + 1) r <= t (lim + qq >= 0); in a capped segment (the 16-query
+      // tiles of shared prefixes) iff blk < blk_cap instead
+      int64_t lim = t0 - (blk + 1) * g.r;
+      bool tile_in = ((b0 + kTileRows - 1) * a.stride + 1) * g.r <= t0;
+      if constexpr (NQ < 64) {
+        if (blk < blo) lim = -(int64_t)1 << 40;
+        tile_in = tile_in && b0 * a.stride >= blo;
+      }
+      if constexpr (NQ == 16) {
+        const int bcap = st.blk_cap[cur.si];
+        if (bcap > 0) {
+          lim = blk < bcap ? (int64_t)1 << 40 : -(int64_t)1 << 40;
+          tile_in = (b0 + kTileRows - 1) * a.stride < bcap;
+        }
+      }
       const float4* w4 = reinterpret_cast<const float4*>(ws) + qb;
       float sc[kQ];
 #pragma unroll
@@ -460,7 +504,7 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
         // trips of a tile overlap), then the hits of each query are stored at
         // consecutive positions
         static_assert(kQ <= 32, "one lane per query of the share");
-        const bool full = qb + kQ <= nq && ((b0 + kTileRows - 1) * a.stride + 1) * g.r <= t0;
+        const bool full = qb + kQ <= nq && tile_in;
         uint32_t hits = 0, my_m = 0;
 #pragma unroll
         for (int qq = 0; qq < kQ; ++qq) {
@@ -484,10 +528,15 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
             pi[pos] = (int32_t)blk;
           }
         }
+      } else if (NQ == 16 && a.row_map) {
+        const int32_t* rows = reinterpret_cast<const int32_t*>(taus) + qb;
+#pragma unroll
+        for (int qq = 0; qq < kQ; ++qq)
+          if (qb + qq < nq && lim + qq >= 0) a.scores[(int64_t)rows[qq] * a.ld + b0 + bl] = sc[qq];
       } else {
         const int64_t ld = a.ld;
         float* p = a.scores + (tok0 + qb) * ld + b0 + bl;
-        if (qb + kQ <= nq && ((b0 + kTileRows - 1) * a.stride + 1) * g.r <= t0) {
+        if (qb + kQ <= nq && tile_in) {
           // every block of the tile is a candidate of every query of the share
 #pragma unroll
           for (int qq = 0; qq < kQ; ++qq, p += ld) *p = sc[qq];

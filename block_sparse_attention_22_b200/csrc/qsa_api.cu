@@ -26,6 +26,7 @@
 #include "attn_tc.cuh"
 #include "attn_union_tc.cuh"
 #include "index_tc.cuh"
+#include "prefix.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -115,9 +116,11 @@ int64_t seg_rows(const qsa_segment_t* segs, int n) {
 }
 
 // Calls launch(table) for batches of at most kMaxSegs non-empty segments;
-// items(seg) gives each segment's work-item count.
+// items(seg) gives each segment's work-item count; extra (or null) the
+// segments' SegExtra fields.
 template <typename Items, typename Launch>
-qsa_status_t for_each_table(const qsa_segment_t* segs, int n_segs, Items items, Launch launch) {
+qsa_status_t for_each_table(const qsa_segment_t* segs, int n_segs, Items items, Launch launch,
+                            const SegExtra* extra = nullptr) {
   SegTable st;
   memset(&st, 0, sizeof st);
   auto flush = [&]() -> qsa_status_t {
@@ -141,6 +144,11 @@ qsa_status_t for_each_table(const qsa_segment_t* segs, int n_segs, Items items, 
     st.q_len[st.n] = s.q_len;
     st.pos0[st.n] = s.pos0;
     st.slot[st.n] = s.slot;
+    const SegExtra e = extra ? extra[i] : SegExtra{0, 0, 0, 0};
+    st.blk_lo[st.n] = e.blk_lo;
+    st.blk_cap[st.n] = e.blk_cap;
+    st.pslot[st.n] = e.pslot;
+    st.pblk[st.n] = e.pblk;
     if (st.n == 0) st.item0[0] = 0;
     st.item0[st.n + 1] = st.item0[st.n] + (int32_t)it;
     st.n++;
@@ -281,7 +289,7 @@ cudaError_t launch_index_tc(const Geo& g, const SegTable& t, const CUtensorMap& 
 
 qsa_status_t run_index(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
                        const qsa_segment_t* segs, int n, const void* q_idx, const float* w,
-                       float* scores, int64_t ld, cudaStream_t st) {
+                       float* scores, int64_t ld, cudaStream_t st, const SegExtra* extra = nullptr) {
   if (c->dtype == QSA_DTYPE_BF16) {
     CUtensorMap tm;
     if (!make_khat_map(&tm, c, cache, 1)) return QSA_ERR_CUDA;
@@ -293,16 +301,27 @@ qsa_status_t run_index(const Geo& g, const qsa_config_t* c, const qsa_cache_t* c
     a.stride = 1;
     // prefill-like segments on 64-query tiles, decode-like ones on 4-query tiles
     std::vector<qsa_segment_t> wide, narrow;
-    for (int i = 0; i < n; ++i) (segs[i].q_len >= 16 ? wide : narrow).push_back(segs[i]);
+    std::vector<SegExtra> xw, xn;
+    for (int i = 0; i < n; ++i) {
+      const bool wd = segs[i].q_len >= 16;
+      (wd ? wide : narrow).push_back(segs[i]);
+      (wd ? xw : xn).push_back(extra ? extra[i] : SegExtra{0, 0, 0, 0});
+    }
     qsa_status_t r = for_each_table(
         wide.data(), (int)wide.size(),
-        [&](const qsa_segment_t& s) { return index_tc_units<64>(s.q_len, s.pos0, g.r); },
-        [&](const SegTable& t) { return launch_index_tc<64>(g, t, tm, a, st); });
+        [&](const qsa_segment_t& s) {
+          const SegExtra& e = xw[&s - wide.data()];
+          return index_tc_units<64>(s.q_len, s.pos0, g.r, 1, e.blk_lo, e.blk_cap);
+        },
+        [&](const SegTable& t) { return launch_index_tc<64>(g, t, tm, a, st); }, xw.data());
     if (r != QSA_OK) return r;
     return for_each_table(
         narrow.data(), (int)narrow.size(),
-        [&](const qsa_segment_t& s) { return index_tc_units<4>(s.q_len, s.pos0, g.r); },
-        [&](const SegTable& t) { return launch_index_tc<4>(g, t, tm, a, st); });
+        [&](const qsa_segment_t& s) {
+          const SegExtra& e = xn[&s - narrow.data()];
+          return index_tc_units<4>(s.q_len, s.pos0, g.r, 1, e.blk_lo, e.blk_cap);
+        },
+        [&](const SegTable& t) { return launch_index_tc<4>(g, t, tm, a, st); }, xn.data());
   }
   size_t smem = sizeof(float) * (simt_index::QT * g.HI * g.DI + simt_index::QT * g.HI);
   if (smem > 48 * 1024)
@@ -524,7 +543,7 @@ int sm_count() {
 qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
                       const qsa_segment_t* segs, int n, int32_t n_tokens, const void* q, const int32_t* sel,
                       const int32_t* nsel, void* o, float* lse, void* ws, size_t ws_bytes,
-                      cudaStream_t st) {
+                      cudaStream_t st, const SegExtra* extra = nullptr) {
   const bool bf = c->dtype == QSA_DTYPE_BF16;
   const AttnPlan p = attn_plan(g, segs, n, bf);
   if (p.ws > 0 && (!ws || ws_bytes < p.ws)) return QSA_ERR_WORKSPACE;
@@ -572,7 +591,8 @@ qsa_status_t run_attn(const Geo& g, const qsa_config_t* c, const qsa_cache_t* ca
           const int grid = (int)std::min<int64_t>(units, sms);
           count_launch();
           return launch_chained(attn_tc_kernel, dim3(grid), dim3(tc_attn::kThreads), smem, st, tq, g, t, ta);
-        });
+        },
+        extra);
   } else {
     const size_t smem = attn_simt_smem();
     cudaFuncSetAttribute(attn_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -700,10 +720,11 @@ void split_fused(const qsa_segment_t* segs, int n, bool tc, bool lowmem, int r, 
 struct FwdLayout {
   int64_t ld;      // score rows of the plain segments
   int64_t ld_s;    // sample rows of the fused segments
-  size_t scores, sel, nsel, topk, attn, samples, tau, cnt, ckey, cidx, total;
+  size_t scores, sel, nsel, topk, attn, samples, tau, cnt, ckey, cidx, qrot, wrot, rmap, total;
 };
 
-FwdLayout fwd_layout(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens, bool tc, bool lowmem) {
+FwdLayout fwd_layout(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_tokens, bool tc, bool lowmem,
+                     bool prefixed = false) {
   std::vector<qsa_segment_t> fused, plain;
   split_fused(segs, n, tc, lowmem, g.r, fused, plain);
   FwdLayout L;
@@ -728,8 +749,82 @@ FwdLayout fwd_layout(const Geo& g, const qsa_segment_t* segs, int n, int32_t n_t
   L.cnt = take(f ? T * 4 : 0);
   L.ckey = take(f ? T * topk::CAP * 4 : 0);
   L.cidx = take(f ? T * topk::CAP * 4 : 0);
+  // shared prefixes: the sharing queries' rotated rows, head weights and score rows
+  L.qrot = take(prefixed ? T * 4 * g.DI * 2 : 0);
+  L.wrot = take(prefixed ? T * 16 : 0);
+  L.rmap = take(prefixed ? T * 4 : 0);
   L.total = off;
   return L;
+}
+
+// Scores of the queries that share a cached prefix, over the prefix's blocks:
+// the sequences with the same (prefix slot, length) form one capped segment
+// of the indexer over that slot (up to 16 queries per k^ stream), whose
+// queries were rotated at their own positions into workspace rows.
+qsa_status_t run_index_shared(const Geo& g, const qsa_config_t* c, const qsa_cache_t* cache,
+                              const qsa_segment_t* segs, const qsa_prefix_t* prefix, int n, const void* q_idx,
+                              const float* w, float* scores, int64_t ld, __nv_bfloat16* q_rot, float* w_rot,
+                              int32_t* row_map, cudaStream_t st) {
+  // members of each (slot, blocks) group, in segment order
+  std::vector<std::pair<std::pair<int, int>, std::vector<int>>> groups;
+  for (int i = 0; i < n; ++i) {
+    if (segs[i].q_len <= 0 || prefix[i].blocks <= 0) continue;
+    const std::pair<int, int> key{prefix[i].slot, prefix[i].blocks};
+    auto it = std::find_if(groups.begin(), groups.end(), [&](const auto& gr) { return gr.first == key; });
+    if (it == groups.end()) {
+      groups.push_back({key, {}});
+      it = groups.end() - 1;
+    }
+    it->second.push_back(i);
+  }
+  if (groups.empty()) return QSA_OK;
+  // 1. rotated rows: virtual row v = the v-th member query, group by group
+  std::vector<qsa_segment_t> members, shared;
+  std::vector<SegExtra> xs;
+  int32_t v0 = 0;
+  for (const auto& gr : groups) {
+    int32_t m = 0;
+    for (int i : gr.second) {
+      members.push_back(segs[i]);
+      m += segs[i].q_len;
+    }
+    // one capped segment per group: rows [v0, v0 + m) of the rotated buffers
+    shared.push_back(qsa_segment_t{v0, m, gr.first.second * g.r, gr.first.first});
+    xs.push_back(SegExtra{0, gr.first.second, 0, 0});
+    v0 += m;
+  }
+  PrefixRotArgs ra{(const __nv_bfloat16*)q_idx, w, q_rot, w_rot, row_map};
+  int32_t vbase = 0;
+  qsa_status_t r = for_each_table(
+      members.data(), (int)members.size(), [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
+      [&](const SegTable& t) {
+        PrefixRotArgs at = ra;                          // rows of this table start at vbase
+        at.q_rot = q_rot + (int64_t)vbase * 4 * g.DI;
+        at.w_rot = w_rot + (int64_t)vbase * 4;
+        at.row_map = row_map + vbase;
+        vbase += t.item0[t.n];
+        count_launch();
+        return launch_chained(prefix_rotate_kernel, dim3((unsigned)t.item0[t.n] * 4), dim3(128), 0, st, g, t, at);
+      });
+  if (r != QSA_OK) return r;
+  // 2. the capped segments over the prefix slots
+  CUtensorMap tm;
+  if (!make_khat_map(&tm, c, cache, 1)) return QSA_ERR_CUDA;
+  IndexTcArgs a{};
+  a.q_idx = q_rot;
+  a.w = w_rot;
+  a.scores = scores;
+  a.ld = ld;
+  a.stride = 1;
+  a.prerotated = 1;
+  a.row_map = row_map;
+  return for_each_table(
+      shared.data(), (int)shared.size(),
+      [&](const qsa_segment_t& s) {
+        const SegExtra& e = xs[&s - shared.data()];
+        return index_tc_units<16>(s.q_len, s.pos0, g.r, 1, e.blk_lo, e.blk_cap);
+      },
+      [&](const SegTable& t) { return launch_index_tc<16>(g, t, tm, a, st); }, xs.data());
 }
 
 }  // namespace
@@ -895,16 +990,34 @@ QSA_API size_t qsa_workspace_size(const qsa_config_t* cfg, const qsa_segment_t* 
     case QSA_OP_FORWARD_LOWMEM:
       return fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16, true).total;
     case QSA_OP_ATTN_UNION: return union_plan(g, segs, n_segs).ws;
+    case QSA_OP_FORWARD_PREFIXED:
+      return fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16, false, true).total;
   }
   return SIZE_MAX;
 }
 
 namespace qsa {
 namespace {
+// Checks of the shared-prefix table: every segment that shares a prefix
+// lies wholly past it, in a cache that holds it.
+qsa_status_t check_prefix(const qsa_config_t* cfg, const qsa_cache_t* cache, const qsa_segment_t* segs,
+                          const qsa_prefix_t* prefix, int32_t n_segs) {
+  if (n_segs > 0 && !prefix) return QSA_ERR_INVALID_ARG;
+  for (int i = 0; i < n_segs; ++i) {
+    const qsa_prefix_t& p = prefix[i];
+    if (p.blocks < 0) return QSA_ERR_INVALID_ARG;
+    if (p.blocks == 0 || segs[i].q_len <= 0) continue;
+    if (p.slot < 0 || p.slot >= cache->n_slots) return QSA_ERR_INVALID_ARG;
+    if ((int64_t)p.blocks * cfg->r > segs[i].pos0 || (int64_t)p.blocks * cfg->r > cache->n_cap)
+      return QSA_ERR_INVALID_ARG;
+  }
+  return QSA_OK;
+}
+
 qsa_status_t forward_impl(const qsa_config_t* cfg, const qsa_cache_t* cache, const qsa_segment_t* segs,
                           int32_t n_segs, int32_t n_tokens, const void* q, const void* q_idx, const float* w,
                           void* o, float* lse, int32_t* sel, int32_t* nsel, void* workspace, size_t ws_bytes,
-                          void* stream, bool lowmem) {
+                          void* stream, bool lowmem, const qsa_prefix_t* prefix = nullptr) {
   qsa_status_t s = check_cfg(cfg);
   if (s != QSA_OK) return s;
   if ((s = check_cache(cfg, cache)) != QSA_OK) return s;
@@ -916,8 +1029,19 @@ qsa_status_t forward_impl(const qsa_config_t* cfg, const qsa_cache_t* cache, con
       !aligned16(cache->v) || !aligned16(cache->k_idx) || !aligned16(cache->khat))
     return QSA_ERR_INVALID_ARG;
   if ((sel == nullptr) != (nsel == nullptr) || (sel && !aligned16(sel))) return QSA_ERR_INVALID_ARG;
+  std::vector<SegExtra> extra;
+  if (prefix) {
+    if ((s = check_prefix(cfg, cache, segs, prefix, n_segs)) != QSA_OK) return s;
+    if (cfg->dtype != QSA_DTYPE_BF16 || lowmem) return QSA_ERR_UNSUPPORTED;
+    for (int i = 0; i < n_segs; ++i)                       // decode-like segments only (< 16 queries)
+      if (prefix[i].blocks > 0 && segs[i].q_len >= 16) return QSA_ERR_UNSUPPORTED;
+    for (int i = 0; i < n_segs; ++i) {
+      const int32_t P = segs[i].q_len > 0 ? prefix[i].blocks : 0;
+      extra.push_back(SegExtra{P, 0, P > 0 ? prefix[i].slot : 0, P});
+    }
+  }
   const Geo g = make_geo(cfg, cache);
-  const FwdLayout L = fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16, lowmem);
+  const FwdLayout L = fwd_layout(g, segs, n_segs, n_tokens, cfg->dtype == QSA_DTYPE_BF16, lowmem, prefix != nullptr);
   if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return QSA_ERR_WORKSPACE;
   cudaStream_t st = (cudaStream_t)stream;
   char* ws = (char*)workspace;
@@ -943,20 +1067,28 @@ qsa_status_t forward_impl(const qsa_config_t* cfg, const qsa_cache_t* cache, con
   auto compress = [&](bool late) {
     return run_compress(g, cfg, cache, slots.data(), b0.data(), b1.data(), (int)slots.size(), st, late);
   };
+  // 2. indexer scores of the plain segments (with shared prefixes: each
+  // sequence's own blocks, then the prefixes' blocks shared by their queries)
+  const SegExtra* xp = prefix ? extra.data() : nullptr;   // plain == segs when prefixes are given
+  auto index = [&]() -> qsa_status_t {
+    qsa_status_t r = run_index(g, cfg, cache, plain.data(), n_plain, q_idx, w, scores, L.ld, st, xp);
+    if (r != QSA_OK || !prefix) return r;
+    return run_index_shared(g, cfg, cache, segs, prefix, n_segs, q_idx, w, scores, L.ld,
+                            (__nv_bfloat16*)(ws + L.qrot), (float*)(ws + L.wrot), (int32_t*)(ws + L.rmap), st);
+  };
   bool pooled = false;
   if (own_blocks_only) {
     // decode-like batch: no query scores a block pooled now, so the pooling
     // runs alongside the indexer (its exit still waits for the indexer)
     if (n_plain > 0) {
-      if ((s = run_index(g, cfg, cache, plain.data(), n_plain, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
+      if ((s = index()) != QSA_OK) return s;
       if ((s = compress(true)) != QSA_OK) return s;
       pooled = true;
     }
   } else {
     if ((s = compress(false)) != QSA_OK) return s;
     pooled = true;
-    // 2. indexer scores of the plain segments
-    if ((s = run_index(g, cfg, cache, plain.data(), n_plain, q_idx, w, scores, L.ld, st)) != QSA_OK) return s;
+    if ((s = index()) != QSA_OK) return s;
   }
   // 2-3. fused scoring and selection (alongside the filtered scoring pass, the
   // pooling of a decode-like batch that has not run yet)
@@ -974,7 +1106,8 @@ qsa_status_t forward_impl(const qsa_config_t* cfg, const qsa_cache_t* cache, con
   if (n_plain > 0 &&
       (s = run_select(g, plain.data(), n_plain, scores, L.ld, sel, nsel, ws + L.topk, L.attn - L.topk, st)) != QSA_OK)
     return s;
-  return run_attn(g, cfg, cache, segs, n_segs, n_tokens, q, sel, nsel, o, lse, ws + L.attn, L.samples - L.attn, st);
+  return run_attn(g, cfg, cache, segs, n_segs, n_tokens, q, sel, nsel, o, lse, ws + L.attn, L.samples - L.attn, st,
+                  xp);
 }
 }  // namespace
 }  // namespace qsa
@@ -986,6 +1119,16 @@ QSA_API qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cac
                                  size_t ws_bytes, void* stream) {
   return forward_impl(cfg, cache, segs, n_segs, n_tokens, q, q_idx, w, o, lse, sel, nsel, workspace, ws_bytes,
                       stream, false);
+}
+
+QSA_API qsa_status_t qsa_forward_prefixed(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                          const qsa_segment_t* segs, const qsa_prefix_t* prefix, int32_t n_segs,
+                                          int32_t n_tokens, const void* q, const void* q_idx, const float* w,
+                                          void* o, float* lse, int32_t* sel, int32_t* nsel, void* workspace,
+                                          size_t ws_bytes, void* stream) {
+  if (n_segs > 0 && !prefix) return QSA_ERR_INVALID_ARG;
+  return forward_impl(cfg, cache, segs, n_segs, n_tokens, q, q_idx, w, o, lse, sel, nsel, workspace, ws_bytes,
+                      stream, false, prefix);
 }
 
 QSA_API qsa_status_t qsa_forward_lowmem(const qsa_config_t* cfg, const qsa_cache_t* cache,

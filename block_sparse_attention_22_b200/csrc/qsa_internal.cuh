@@ -39,6 +39,10 @@ struct Geo {
 
 // Segment table of one launch, with a prefix sum of the work items each
 // segment contributes (the kernel maps blockIdx to a segment by bisection).
+// blk_lo / blk_cap restrict the blocks the indexer scores for the segment's
+// queries to [blk_lo, limit), limit = blk_cap when > 0, else the causal
+// limit floor(t/r); pslot / pblk: the segment's blocks below pblk live in
+// cache slot pslot (a prefix shared with other sequences), the rest in slot.
 struct SegTable {
   int32_t n;
   int32_t q_offset[kMaxSegs];
@@ -46,6 +50,15 @@ struct SegTable {
   int32_t pos0[kMaxSegs];
   int32_t slot[kMaxSegs];
   int32_t item0[kMaxSegs + 1];
+  int32_t blk_lo[kMaxSegs];
+  int32_t blk_cap[kMaxSegs];
+  int32_t pslot[kMaxSegs];
+  int32_t pblk[kMaxSegs];
+};
+
+// Per-segment fields of SegTable beyond qsa_segment_t (all zero by default).
+struct SegExtra {
+  int32_t blk_lo, blk_cap, pslot, pblk;
 };
 
 __device__ __forceinline__ int find_segment(const SegTable& st, int item) {

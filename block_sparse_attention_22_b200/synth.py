@@ -26,6 +26,11 @@ kv-channels 256, rotary 0.25 at base 1e7; design report, QSA item: r=4, a
   chunk_128k    one 4096-query prefill chunk at [126976, 131072) of a
                 131072-token sequence whose prefix is cached (a ~1 GB case
                 whose K/V still exceeds L2; used for kernel profiles)
+  shared_prefix_1m  8 sequences x 1 decode query at 1048576-token context
+                that share a cached prefix of 943716 tokens (90 %): the
+                prefix lives once in its own cache slot, each sequence's
+                suffix in its slot; 4 needles per sequence in the prefix and
+                4 in its suffix
   prefill_128k_local  prefill_128k with indexer queries that drift slowly
                 along the sequence (below), so neighbouring tokens keep
                 mostly the same blocks
@@ -102,6 +107,10 @@ class Workload:
     needles: List[Tuple[int, int, int]] = field(default_factory=list)  # (slot, t*, b*)
     seed: int = 0
     drift: float = 0.0                 # AR(1) coefficient of the indexer queries along a segment
+    # per segment (prefix slot, prefix blocks), or empty: blocks below the
+    # prefix's end live in the prefix slot; the segment's slot holds the rest
+    prefix: List[Tuple[int, int]] = field(default_factory=list)
+    start: List[int] = field(default_factory=list)   # first present row of each slot (default 0)
 
     @property
     def n_tokens(self) -> int:
@@ -196,6 +205,24 @@ def make_workload(name: str, seed: Optional[int] = None, **over) -> Workload:
         cached = [(ctx - 1) // sh.r] * n_seqs
         return Workload(name, sh, segs, n_seqs, _round_cap(ctx, sh.r), [ctx] * n_seqs, cached, needles,
                         seed if seed is not None else (6 if big else 3))
+    if name == "shared_prefix_1m":
+        sh = Shape(**over.get("shape", {}))
+        ctx = over.get("ctx", 1 << 20)
+        n_seqs = over.get("n_seqs", 8)
+        q_len = over.get("q_len", 1)
+        p_tok = over.get("prefix", int(0.9 * ctx) // sh.r * sh.r)
+        P = p_tok // sh.r
+        pslot = n_seqs
+        segs = [Segment(s, ctx - q_len, q_len) for s in range(n_seqs)]
+        needles = []
+        for s in range(n_seqs):
+            t = ctx - 1
+            needles += [(s, t, b) for b in _distinct_blocks(rng, P, 4)]
+            needles += [(s, t, P + b) for b in _distinct_blocks(rng, (ctx - 1) // sh.r - P - (q_len - 1), 4)]
+        cached = [(ctx - q_len) // sh.r] * n_seqs + [P]
+        return Workload(name, sh, segs, n_seqs + 1, _round_cap(ctx, sh.r), [ctx] * n_seqs + [p_tok], cached,
+                        needles, seed if seed is not None else 9, prefix=[(pslot, P)] * n_seqs,
+                        start=[p_tok] * n_seqs + [0])
     if name == "spec_decode_1m":
         sh = Shape(**over.get("shape", {}))
         ctx = over.get("ctx", 1 << 20)
@@ -297,10 +324,11 @@ def make_inputs(wl: Workload, device="cpu") -> Dict[str, torch.Tensor]:
     v = torch.zeros_like(k)
     for s in range(wl.n_slots):
         f = wl.fill[s]
-        k_idx[s, :f] = _randn((f, sh.idx_dim), gen, dev, dt)
+        f0 = wl.start[s] if wl.start else 0
+        k_idx[s, f0:f] = _randn((f - f0, sh.idx_dim), gen, dev, dt)
         for g in range(sh.n_groups):
-            k[s, g, :f] = _randn((f, sh.head_dim), gen, dev, dt)
-            v[s, g, :f] = _randn((f, sh.head_dim), gen, dev, dt)
+            k[s, g, f0:f] = _randn((f - f0, sh.head_dim), gen, dev, dt)
+            v[s, g, f0:f] = _randn((f - f0, sh.head_dim), gen, dev, dt)
     offs = wl.token_offsets()
     if wl.drift > 0:
         rho = wl.drift
@@ -318,9 +346,14 @@ def make_inputs(wl: Workload, device="cpu") -> Dict[str, torch.Tensor]:
             continue
         u = (w[tok].unsqueeze(1) * q_idx[tok].float()).sum(0)
         u[:n_rot] = 0
-        k_idx[slot, b * sh.r:(b + 1) * sh.r] = u.to(dt)
+        dst = slot
+        if wl.prefix:                          # a needle in a shared prefix lives in the prefix's slot
+            ps, pb = wl.prefix[[sg.slot for sg in wl.segments].index(slot)]
+            if b < pb:
+                dst = ps
+        k_idx[dst, b * sh.r:(b + 1) * sh.r] = u.to(dt)
         for g in range(sh.n_groups):
-            k[slot, g, b * sh.r:(b + 1) * sh.r] = q[tok, 0]
+            k[dst, g, b * sh.r:(b + 1) * sh.r] = q[tok, 0]
     return {"q": q, "q_idx": q_idx, "w": w, "k_idx": k_idx, "k": k, "v": v}
 
 
@@ -330,3 +363,18 @@ def describe(wl: Workload) -> dict:
     d.pop("needles")
     d["n_needles"] = len(wl.needles)
     return d
+
+
+def sequence_cache(wl: Workload, x: Dict[str, torch.Tensor], slot: int, fill: int):
+    """A sequence's whole cache rows [0, fill) (k_idx [fill, dI], k and v
+    [G, fill, D]): with a shared prefix, its first rows come from the prefix's
+    slot and the rest from the sequence's slot."""
+    k_idx, k, v = x["k_idx"][slot, :fill], x["k"][slot, :, :fill], x["v"][slot, :, :fill]
+    if wl.prefix:
+        ps, pb = wl.prefix[[sg.slot for sg in wl.segments].index(slot)]
+        n = min(fill, pb * wl.shape.r)
+        if n > 0:
+            k_idx = torch.cat([x["k_idx"][ps, :n], k_idx[n:]])
+            k = torch.cat([x["k"][ps, :, :n], k[:, n:]], dim=1)
+            v = torch.cat([x["v"][ps, :, :n], v[:, n:]], dim=1)
+    return k_idx, k, v

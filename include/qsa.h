@@ -124,8 +124,20 @@ typedef enum {
   QSA_OP_ATTN = 3,
   QSA_OP_FORWARD = 4,
   QSA_OP_FORWARD_LOWMEM = 5,
-  QSA_OP_ATTN_UNION = 6
+  QSA_OP_ATTN_UNION = 6,
+  QSA_OP_FORWARD_PREFIXED = 7
 } qsa_op_t;
+
+/* A cached prefix that a segment's sequence shares with other sequences:
+ * its first `blocks` micro-blocks (blocks*r tokens) live in cache slot
+ * `slot` (k_idx, khat, K, V), once for all the sequences that use it; the
+ * rest of the sequence lives in the segment's own slot, at the same absolute
+ * positions (positions below blocks*r of the own slot are never read).
+ * blocks == 0: the segment shares nothing. */
+typedef struct {
+  int32_t slot;
+  int32_t blocks;
+} qsa_prefix_t;
 
 /*
  * Key pooling + block position encoding (design report, QSA item: keys are
@@ -254,6 +266,30 @@ qsa_status_t qsa_forward(const qsa_config_t* cfg, const qsa_cache_t* cache,
                          const void* q, const void* q_idx, const float* w, void* o, float* lse,
                          int32_t* sel, int32_t* nsel, void* workspace, size_t ws_bytes,
                          void* stream);
+
+/*
+ * qsa_forward for sequences that share cached prefixes (the release article's
+ * section "GDN+QSA" quotes its 1M-context throughput at a 90 % prefix-cache
+ * hit: many requests on one cached prefix).  prefix: host array [n_segs];
+ * segment i's sequence is prefix[i] followed by its own slot (see
+ * qsa_prefix_t).  Results are those of qsa_forward on each sequence's whole
+ * cache.  The queries of all segments with the same (slot, blocks) are
+ * scored over the prefix's blocks together, up to 16 queries per pass over
+ * the prefix's pooled keys (in qsa_forward every decode query streams its
+ * own); each segment's own blocks are scored from its slot; the attention
+ * reads kept prefix blocks from the prefix's slot.
+ * Requires bf16 I/O, and segments with blocks > 0 of fewer than 16 queries
+ * (decode and speculative decode; QSA_ERR_UNSUPPORTED otherwise), and for
+ * every segment with blocks > 0: 0 <= slot < n_slots and blocks*r <= pos0
+ * (all of its queries past the prefix; QSA_ERR_INVALID_ARG otherwise).  The prefix's blocks must
+ * already be pooled in its slot's khat.  workspace >= qsa_workspace_size(...,
+ * QSA_OP_FORWARD_PREFIXED).
+ */
+qsa_status_t qsa_forward_prefixed(const qsa_config_t* cfg, const qsa_cache_t* cache,
+                                  const qsa_segment_t* segs, const qsa_prefix_t* prefix, int32_t n_segs,
+                                  int32_t n_tokens, const void* q, const void* q_idx, const float* w,
+                                  void* o, float* lse, int32_t* sel, int32_t* nsel, void* workspace,
+                                  size_t ws_bytes, void* stream);
 
 /*
  * qsa_forward without the score matrix, for callers short of device memory.

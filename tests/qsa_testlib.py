@@ -59,6 +59,8 @@ def gpu_prepare_cache(wl: synth.Workload, x: Dict[str, torch.Tensor]):
 
 
 def gpu_forward(wl: synth.Workload, x: Dict[str, torch.Tensor], lowmem: bool = False) -> GpuRun:
+    """One forward call over the workload (qsa_forward_prefixed when it has
+    shared prefixes)."""
     sh = wl.shape
     cfg, cache, khat = gpu_prepare_cache(wl, x)
     segs = segments_of(wl)
@@ -67,6 +69,14 @@ def gpu_forward(wl: synth.Workload, x: Dict[str, torch.Tensor], lowmem: bool = F
     lse = torch.full((T, sh.n_heads), float("nan"), dtype=torch.float32, device="cuda")
     sel = torch.full((T, sh.budget_blocks), -7, dtype=torch.int32, device="cuda")
     nsel = torch.full((T,), -7, dtype=torch.int32, device="cuda")
+    if wl.prefix:
+        ws = torch.empty(max(1, qsa.workspace_size(cfg, segs, T, qsa.QSA_OP_FORWARD_PREFIXED)), dtype=torch.uint8,
+                         device="cuda")
+        qsa.qsa_forward_prefixed(cfg, cache, segs, qsa.make_prefixes(wl.prefix), T, x["q"], x["q_idx"], x["w"], o,
+                                 lse, sel, nsel, ws)
+        torch.cuda.synchronize()
+        qsa.qsa_device_status()
+        return GpuRun(o, lse, sel, nsel, khat)
     op = qsa.QSA_OP_FORWARD_LOWMEM if lowmem else qsa.QSA_OP_FORWARD
     ws = torch.empty(max(1, qsa.workspace_size(cfg, segs, T, op)), dtype=torch.uint8, device="cuda")
     fwd = qsa.qsa_forward_lowmem if lowmem else qsa.qsa_forward
@@ -87,9 +97,10 @@ class OracleSeq:
         self.cfg = oracle.config_from_shape(wl.shape)
         self.r = wl.shape.r
         fill = wl.fill[slot]
-        self.k_idx = to_np(x["k_idx"][slot, :fill])
-        self.k = to_np(x["k"][slot, :, :fill])
-        self.v = to_np(x["v"][slot, :, :fill])
+        k_idx, k, v = synth.sequence_cache(wl, x, slot, fill)     # with a shared prefix: its rows first
+        self.k_idx = to_np(k_idx)
+        self.k = to_np(k)
+        self.v = to_np(v)
         self.khat = oracle.compress_keys(self.cfg, self.k_idx, 0, fill // self.r)
 
     def attend(self, q, t, sel, nsel):

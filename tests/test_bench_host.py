@@ -78,3 +78,18 @@ def test_step_tensor_roofline_arithmetic():
     assert abs(r["index_stage"]["frac"] - 0.5) < 1e-12
     # attainable: 1e6/5e12 + 2e12/1e15 + 0 + 500e9/5e12 seconds
     assert abs(r["attainable"]["ms_per_step"] - (0.0002 + 2.0 + 100.0)) < 1e-9
+
+
+def test_shared_prefix_work_counts_the_prefix_once():
+    """8 decode queries on a 943716-token shared prefix: the prefix's pooled
+    keys are streamed once (8 sharing queries fit one 16-query tile), each
+    sequence's own blocks once per sequence."""
+    import dataclasses
+    from block_sparse_attention_22_b200 import synth
+    wl = synth.make_workload("shared_prefix_1m")
+    P = wl.prefix[0][1]
+    own = ((1 << 20) - 1) // 4 - P
+    w = bench.algorithmic_work(wl)
+    assert w["index"]["khat_bytes"] == (P + 8 * own) * 128 * 2
+    alone = bench.algorithmic_work(dataclasses.replace(wl, prefix=[]))
+    assert alone["index"]["khat_bytes"] == 8 * (((1 << 20) - 1) // 4) * 128 * 2
