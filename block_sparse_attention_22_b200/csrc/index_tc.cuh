@@ -364,7 +364,8 @@ __global__ void __launch_bounds__(IndexTcCfg<NQ>::kThreads, 1)
           row0 = blo / (kTileRows * a.stride) * kTileRows;
         }
         named_bar_sync(1, C::kEpiThreads);          // every share is done with the previous w, cos/sin
-        for (int k = et; k < nq * half; k += C::kEpiThreads) {
+        const bool rotate = !(NQ == 16 && a.prerotated);
+        for (int k = et; rotate && k < nq * half; k += C::kEpiThreads) {
           const int q = k / half, p = k - q * half;
           float c, sn;
           rope_cs(g, t_first + q, p, c, sn);
