@@ -978,8 +978,10 @@ def main():
     value = job_throughput(tokens, m["fused_ms"], ws)
 
     work = m["work"]
-    roofline = attention_roofline(work, m["stage_ms"][3], peaks)
-    tensor_roofline = step_tensor_roofline(work, m["fused_ms"], m["stage_ms"], peaks)
+    roofline = tensor_roofline = None
+    if m["stage_ms"] is not None:    # (a shared-prefix workload has no per-stage times)
+        roofline = attention_roofline(work, m["stage_ms"][3], peaks)
+        tensor_roofline = step_tensor_roofline(work, m["fused_ms"], m["stage_ms"], peaks)
 
     e2e = None
     if not args.no_e2e:

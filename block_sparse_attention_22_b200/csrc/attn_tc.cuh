@@ -250,17 +250,22 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
       ++uc;
       const __nv_bfloat16* kg = (const __nv_bfloat16*)a.k + (u.slot * g.G + u.grp) * g.n_cap * kHeadDim;
       const __nv_bfloat16* vg = (const __nv_bfloat16*)a.v + (u.slot * g.G + u.grp) * g.n_cap * kHeadDim;
-      // rows below the shared prefix's end come from its slot
-      const __nv_bfloat16* kp = (const __nv_bfloat16*)a.k + (u.pslot * g.G + u.grp) * g.n_cap * kHeadDim;
-      const __nv_bfloat16* vp = (const __nv_bfloat16*)a.v + (u.pslot * g.G + u.grp) * g.n_cap * kHeadDim;
+      // rows below a shared prefix's end live in the prefix's slot: their
+      // offset from the unit's own base shifts by whole slots
       const int64_t prow_end = (int64_t)u.pblk * g.r;
+      const int64_t pshift = (u.pslot - u.slot) * g.G * g.n_cap;
       const int32_t* selrow = a.sel + u.tok * g.S;
-      // cache rows of this warp's kept blocks pw + 9 i of a chunk (lane i < 4)
+      // rows (from the unit's own K/V base) of this warp's kept blocks pw + 9 i
+      // of a chunk (lane i < 4); kNoRow for padding and rejected entries
+      constexpr int64_t kNoRow = INT64_MIN / 2;
       auto rows_of = [&](int cc) -> int64_t {
-        int64_t row = -1;
+        int64_t row = kNoRow;
         if (lane < 4 && cc < u.nchunks && pw + kProducers * lane < kBlk) {
           const int pos = u.blk_begin + cc * kBlk + pw + kProducers * lane;
-          if (pos < u.blk_end) row = block_row(selrow[pos], 0, g);
+          if (pos < u.blk_end) {
+            const int64_t br = block_row(selrow[pos], 0, g);
+            if (br >= 0) row = br < prow_end ? br + pshift : br;
+          }
         }
         return row;
       };
@@ -268,7 +273,6 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
         for (int c = 0; c < u.nchunks && ok; ++c) {
           const int64_t myrow = rows_of(c);
           const __nv_bfloat16* base = kind == 0 ? kg : vg;
-          const __nv_bfloat16* pbase = kind == 0 ? kp : vp;
           for (int h = 0; h < 2 && ok; ++h) {
             const int64_t hs = hs_next++;
             const int slot = (int)(hs % kSlots);
@@ -281,9 +285,8 @@ __global__ void __launch_bounds__(tc_attn::kThreads, 1)
               const int64_t row = __shfl_sync(0xffffffffu, myrow, bq);
               const int line = 4 * b + r;
               const uint32_t dst = dst0 + line * 128 + ((jc ^ (line & 7)) << 4);
-              const __nv_bfloat16* src = (row < prow_end ? pbase : base) + 128 * h + 8 * jc +
-                                         (row >= 0 ? (row + r) * kHeadDim : 0);
-              const uint32_t nb = row >= 0 ? 16u : 0u;
+              const __nv_bfloat16* src = base + 128 * h + 8 * jc + (row != kNoRow ? (row + r) * kHeadDim : 0);
+              const uint32_t nb = row != kNoRow ? 16u : 0u;
               cp_async16(dst, src, nb);                       // dims 128h + 8jc .. +8
               cp_async16(dst + 16384, src + 64, nb);          // dims 128h + 64 + 8jc .. +8
             }
