@@ -1207,13 +1207,14 @@ QSA_API int64_t qsa_launch_count(void) { return (int64_t)launch_counter().load()
 
 // ------------------------------------------------------------------ allocation-free selection
 // Top-k selection for callers that cannot allocate device memory: the
-// split-row candidate buffers live in this file-scope device array instead
-// of a caller workspace.  Every device that loads the library holds the
-// array until the process exits.  All calls on a device share it, so calls
-// whose work overlaps on the GPU (different streams, no ordering) race on
-// it; calls on one stream are ordered and safe.  Nothing in it needs to start
-// at zero: every candidate count the merge pass reads is written first by
-// the chunk pass of the same call.
+// few-long-rows buffers (per token row a record of counters, the row
+// histogram and two candidate lists) live in this file-scope device array
+// instead of a caller workspace.  Every device that loads the library holds
+// the array until the process exits.  All calls on a device share it, so
+// calls whose work overlaps on the GPU (different streams, no ordering) race
+// on it; calls on one stream are ordered and safe.  What must start at zero
+// (the counters and histograms) is cleared by each call, on its stream,
+// before its kernels run.
 static __device__ __align__(256) unsigned char g_select_scratch[QSA_NOALLOC_SCRATCH_BYTES];
 
 namespace qsa {
