@@ -183,7 +183,7 @@ TopkHistLayout topk_hist_layout(int64_t T) {
   TopkHistLayout L;
   L.rec = 0;
   L.hist = (size_t)T * topk::kRecWords * 4;
-  L.zero = align_up(L.hist + (size_t)T * topk::kHistBins * 4, 256);
+  L.zero = align_up(L.hist + (size_t)T * (topk::kHistBins + topk::kCoarseBins) * 4, 256);
   L.sure = L.zero;
   L.key = L.sure + align_up((size_t)T * topk::KMAX * 4, 256);
   L.idx = L.key + align_up((size_t)T * topk::CAP * 4, 256);

@@ -60,6 +60,7 @@ constexpr int kFusedStride = 16;          // fused prefill selection: one sample
 constexpr int kHistBits = 12;              // sign, 8 exponent and 3 mantissa bits of the score
 constexpr int kHistBins = 1 << kHistBits;
 constexpr int kHistShift = 32 - kHistBits;
+constexpr int kCoarseBins = 256;           // the top 8 key bits: 16 fine bins each
 constexpr int kHistChunk = 4096;           // scores per CTA
 constexpr int kHistThreads = 256;
 constexpr int kHistPer = kHistChunk / (4 * kHistThreads);   // 16-byte groups per thread
@@ -654,7 +655,7 @@ struct TopkArgs {
   int chunk;            // scores per chunk CTA (few long rows)
   // few long rows (histogram path); hrec and hhist start zeroed
   int32_t* hrec;        // [T][kRecWords] list counters and the row's threshold bin
-  uint32_t* hhist;      // [T][kHistBins] row histograms of the top key bits
+  uint32_t* hhist;      // [T][kHistBins + kCoarseBins] row histograms of the top 12 and 8 key bits
   int32_t* hsure;       // [T][KMAX] elements above the threshold bin
   uint32_t* hkey;       // [T][CAP] keys of the threshold bin's elements
   int32_t* hidx;        // [T][CAP] their block indices
@@ -784,9 +785,11 @@ __device__ __forceinline__ TopkItem topk_item(const Geo& g, const SegTable& st, 
 // Few long rows (decode: a handful of rows of 32K to millions of blocks).
 // Three launches, each a stage of the whole batch:
 //   topk_hist_kernel (one CTA per 4096-score chunk of a row): the chunk's
-//     histogram of the top 12 key bits, added into the row's histogram;
+//     histogram of the top 12 key bits, added into the row's histogram, and
+//     its sums over 16 bins (the top 8 bits) into the row's coarse one;
 //   topk_hfilter_kernel (one CTA per chunk): the bin B of the row's (S-1)-th
-//     largest key (from the row's histogram, found by every chunk CTA while
+//     largest key (from the row's coarse histogram of the top 8 key bits,
+//     then the 16 fine bins of one coarse bin, found by every chunk CTA while
 //     its chunk loads), then the chunk's elements in bins above B ("sure":
 //     all kept) and in B ("tied bin") appended to the row's two lists, each
 //     CTA reserving its ranges with one atomic per list;
@@ -826,47 +829,48 @@ struct HistChunk {
   }
 };
 
-// The bin of the row histogram h (kHistBins words in shared memory) that
-// holds the k-th largest element: *bin, *above = elements in higher bins,
-// *count = elements in that bin.  Warp w holds bins [w P, w P + P), P =
-// kHistBins / warps, read 32 consecutive words at a time.  Ends with a
-// barrier.
+// The fine bin of a row histogram gh (kHistBins fine bins, then kCoarseBins
+// coarse bins, in global memory) that holds the k-th largest element: first
+// the coarse bin from the 256 coarse counts (one per thread), then, by warp 0,
+// the fine bin among that coarse bin's 16.  *bin, *above = elements in
+// higher fine bins, *count = elements in that bin.  Ends with a barrier.
 template <int NT>
-__device__ void hist_row_locate(const uint32_t* h, int k, uint32_t* bin, int* above, int* count,
+__device__ void hist_row_locate(const uint32_t* gh, int k, uint32_t* bin, int* above, int* count,
                                 TopkShared<NT>& sh) {
+  static_assert(NT == kCoarseBins, "one coarse bin per thread");
   constexpr int WARPS = TopkCfg<NT>::WARPS;
-  constexpr int P = kHistBins / WARPS;
-  constexpr int STEPS = P / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int mine = 0;
+  const int c = (int)__ldcg(gh + kHistBins + threadIdx.x);
+  int suf = c;                                   // this and higher lanes of the warp
 #pragma unroll
-  for (int j = 0; j < STEPS; ++j) mine += (int)h[warp * P + 32 * j + lane];
-  const int wsum = __reduce_add_sync(0xffffffffu, mine);
-  if (lane == 0) sh.warp_a[warp] = wsum;
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_down_sync(0xffffffffu, suf, off);
+    if (lane + off < 32) suf += v;
+  }
+  if (lane == 0) sh.warp_a[warp] = suf;
   __syncthreads();
   int higher = 0;
   for (int w = warp + 1; w < WARPS; ++w) higher += sh.warp_a[w];
-  if (higher < k && k <= higher + wsum) {       // this warp's bins hold it: walk its steps down
-    int run = higher;
-    for (int j = STEPS - 1; j >= 0; --j) {
-      const int c = (int)h[warp * P + 32 * j + lane];
-      const int step = __reduce_add_sync(0xffffffffu, c);
-      if (run + step >= k) {
-        int suf = c;                           // this and higher lanes of the step
+  const int ex = higher + suf - c;               // elements in higher coarse bins
+  if (ex < k && k <= ex + c) {
+    sh.sel_digit = threadIdx.x;
+    sh.sel_above = ex;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int cb = (int)sh.sel_digit, cab = sh.sel_above;
+    const int f = lane < 16 ? (int)__ldcg(gh + cb * 16 + lane) : 0;
+    int fs = f;                                  // fine bins >= this one, within the coarse bin
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int v = __shfl_down_sync(0xffffffffu, suf, off);
-          if (lane + off < 32) suf += v;
-        }
-        const int ex = run + suf - c;
-        if (ex < k && k <= ex + c) {
-          sh.sel_digit = (uint32_t)(warp * P + 32 * j + lane);
-          sh.sel_above = ex;
-          sh.sel_count = c;
-        }
-        break;
-      }
-      run += step;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_down_sync(0xffffffffu, fs, off);
+      if (lane + off < 32) fs += v;
+    }
+    const int fex = cab + fs - f;
+    if (lane < 16 && fex < k && k <= fex + f) {
+      sh.sel_digit = (uint32_t)(cb * 16 + lane);
+      sh.sel_above = fex;
+      sh.sel_count = f;
     }
   }
   __syncthreads();
@@ -892,11 +896,17 @@ __global__ void __launch_bounds__(topk::kHistThreads) topk_hist_kernel(Geo g, Se
   for (int e = 0; e < kHistPer * 4; ++e)
     if (HistChunk::index(e) < it.n) atomicAdd(&hist[score_key(ch.v[e]) >> kHistShift], 1u);
   __syncthreads();
-  uint32_t* gh = a.hhist + it.tok * kHistBins;
+  uint32_t* gh = a.hhist + it.tok * (kHistBins + kCoarseBins);
   for (int b = threadIdx.x; b < kHistBins; b += kHistThreads) {
     const uint32_t c = hist[b];
     if (c) atomicAdd(&gh[b], c);
   }
+  // coarse bin t: fine bins [16 t, 16 t + 16)
+  static_assert(kHistThreads == kCoarseBins, "one coarse bin per thread");
+  uint32_t cs = 0u;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) cs += hist[threadIdx.x * 16 + ((j + threadIdx.x) & 15)];
+  if (cs) atomicAdd(&gh[kHistBins + threadIdx.x], cs);
 }
 
 __global__ void __launch_bounds__(topk::kHistThreads, 4) topk_hfilter_kernel(Geo g, SegTable st, TopkArgs a) {
@@ -918,13 +928,9 @@ __global__ void __launch_bounds__(topk::kHistThreads, 4) topk_hfilter_kernel(Geo
   }
   HistChunk ch;
   ch.load(a.scores + it.tok * a.ld + it.c0, it.n);          // in flight while the threshold is found
-  uint32_t* h = sh.cbuf;
-  const uint32_t* gh = a.hhist + it.tok * kHistBins;
-  for (int b = threadIdx.x; b < kHistBins; b += NT) h[b] = __ldcg(gh + b);
-  __syncthreads();
   uint32_t B;
   int above, count;
-  hist_row_locate(h, K, &B, &above, &count, sh);
+  hist_row_locate(a.hhist + it.tok * (kHistBins + kCoarseBins), K, &B, &above, &count, sh);
   int32_t* rec = a.hrec + it.tok * kRecWords;
   if (it.c == 0 && threadIdx.x == 0) {
     rec[kRecBin] = (int32_t)B;
