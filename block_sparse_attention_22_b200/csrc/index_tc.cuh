@@ -51,7 +51,7 @@ constexpr int kMaxRopeHalf = 32;           // rotated pairs per vector (rope_dim
 template <int NQ>
 struct IndexTcCfg {
   static constexpr int N = 4 * NQ;                         // MMA N = queries x 4 heads
-  static constexpr int kEpiWarps = NQ >= 64 ? 8 : 4;       // 2 per TMEM lane quadrant for prefill
+  static constexpr int kEpiWarps = NQ >= 16 ? 8 : 4;       // 2 per TMEM lane quadrant for 16+ queries
   static constexpr int kEpiThreads = 32 * kEpiWarps;
   static constexpr int kThreads = 64 + kEpiThreads;
   static constexpr int kColsPerWarp = N / (kEpiWarps / 4);  // 64 (16 queries) or 16 (4 queries)
