@@ -822,6 +822,11 @@ def side_line(name: str, args, ws: int, rank: int, flush, peaks) -> dict:
                                   "q/o/lse, sel; no score round trip",
                          "actual_bytes_per_step": act,
                          "actual_frac": act / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    if wl2.n_tokens <= 64:
+        # the same step captured once in a CUDA graph and replayed (a decode loop's usual form)
+        gr = graph_replay(prep2, args.steps, args.warmup, flush, ws)
+        gr["hbm_frac"] = alg / (gr["ms_per_step"] * 1e-3) / 1e9 / peaks["hbm_gbs"]
+        d["graph_replay"] = gr
     if wl2.prefix:
         import dataclasses
         alone = algorithmic_work(dataclasses.replace(wl2, prefix=[]))["index"]["khat_bytes"]
@@ -838,6 +843,40 @@ def side_line(name: str, args, ws: int, rank: int, flush, peaks) -> dict:
     del prep2
     torch.cuda.empty_cache()
     return d
+
+
+def graph_replay(prep: Prepared, steps: int, warmup: int, flush, ws: int) -> dict:
+    """Device time of the workload's forward captured in a CUDA graph and
+    replayed (L2 flushed before each replay), and whether a replay's output
+    equals a direct call's."""
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        prep.forward()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        prep.forward()
+    for _ in range(warmup):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    o = prep.o.clone()
+    prep.forward()
+    torch.cuda.synchronize()
+    same = bool(torch.equal(o, prep.o))
+    del graph
+    ms = max_over_ranks(tot / steps, ws)
+    return {"ms_per_step": ms, "tokens_per_s": job_throughput(prep.T, ms, ws), "output_matches_direct_call": same}
 
 
 # side lines with an oracle timing, and how many of their sequences it times
