@@ -838,7 +838,8 @@ def side_line(name: str, args, ws: int, rank: int, flush, peaks) -> dict:
                             "frac": w2["flops"] / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                             "peak": peaks["bf16_tflops"]}
     if rank == 0 and ws == 1 and not args.no_cpu and args.side_cpu_seconds > 0 and name in ORACLE_SIDE:
-        v, threads, desc = oracle_sample(wl2, prep2.x, args.side_cpu_seconds, max_slots=ORACLE_SIDE[name])
+        slots, budget = ORACLE_SIDE[name]
+        v, threads, desc = oracle_sample(wl2, prep2.x, args.side_cpu_seconds * budget, max_slots=slots)
         d["cpu_oracle"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
     del prep2
     torch.cuda.empty_cache()
@@ -879,9 +880,10 @@ def graph_replay(prep: Prepared, steps: int, warmup: int, flush, ws: int) -> dic
     return {"ms_per_step": ms, "tokens_per_s": job_throughput(prep.T, ms, ws), "output_matches_direct_call": same}
 
 
-# side lines with an oracle timing, and how many of their sequences it times
-# (each 256K-context sequence's K/V is 1 GiB in the oracle's fp32)
-ORACLE_SIDE = {"prefill_8k": 0, "decode_256k": 2}
+# side lines with an oracle timing: (sequences it times, 0 = all; time budget in
+# units of --side-cpu-seconds).  Each 256K-context sequence's K/V is 1 GiB in the
+# oracle's fp32; the 8K prefill's budget covers all of its queries on 16 cores.
+ORACLE_SIDE = {"tiny_fp32": (0, 1.0), "prefill_8k": (0, 6.0), "decode_256k": (8, 1.0)}
 
 
 def parse_overrides(text: str) -> dict:
@@ -978,7 +980,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["qsa", "reference"], default="qsa")
     ap.add_argument("--workload", default="prefill_128k")
-    ap.add_argument("--decode-workload", default="decode_1m,mixed_1m,decode_256k,prefill_8k,shared_prefix_1m",
+    ap.add_argument("--decode-workload", default="decode_1m,mixed_1m,decode_256k,prefill_8k,tiny_fp32,shared_prefix_1m",
                     help="comma-separated extra workloads reported beside the main line; 'none' to skip")
     ap.add_argument("--side-cpu-seconds", type=float, default=8.0,
                     help="oracle time budget of each side line's CPU timing (0: none)")
