@@ -470,7 +470,7 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
         });
   }
   (void)smem_c;
-  // many rows: one warp per row (five 4-warp CTAs per SM), then a CTA-level
+  // many rows: one warp per row (topk_w::CTAS 4-warp CTAs per SM), then a CTA-level
   // selection of the rows it left (long rows, sampled thresholds that
   // missed).  Plain launches: chained, the pair ran 1.7x slower (the
   // dependent's CTAs, resident early, held the SMs the other grid needed).
@@ -478,9 +478,11 @@ qsa_status_t run_select(const Geo& g, const qsa_segment_t* segs, int n, const fl
       segs, n, [&](const qsa_segment_t& s) { return (int64_t)s.q_len; },
       [&](const SegTable& t) {
         const int rows = t.item0[t.n];
-        const int grid = std::min((int)cdiv(rows, topk_w::WARPS), 5 * sm_count());
+        const int grid = std::min((int)cdiv(rows, topk_w::WARPS), topk_w::CTAS * sm_count());
+        constexpr int smem_rows = (int)(topk_w::WARPS * sizeof(WarpRowShared));
+        cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_rows);
         count_launch();
-        topk_rows_kernel<<<dim3(grid), dim3(topk_w::THREADS), 0, st>>>(g, t, a);
+        topk_rows_kernel<<<dim3(grid), dim3(topk_w::THREADS), smem_rows, st>>>(g, t, a);
         count_launch();
         topk_rows_fallback_kernel<<<dim3(std::min(rows, 6 * sm_count())), dim3(topk::THREADS), 0, st>>>(g, t, a);
         return cudaGetLastError();

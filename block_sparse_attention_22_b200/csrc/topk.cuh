@@ -1015,17 +1015,23 @@ __global__ void __launch_bounds__(topk::kWideThreads, 1) topk_hfinal_kernel(Geo 
 // ---------------------------------------------------------------- many rows: one warp per row
 // The 4-warp CTA per row above spends most of a row in barrier-separated
 // phases with no loads in flight.  Here each warp selects its own row with
-// warp-synchronous steps only, so an SM has 20 rows in flight (4 warps x 5
-// CTAs) whose load phases overlap each other's selection phases:
+// warp-synchronous steps only, so an SM has 24 rows in flight (4 warps x 6
+// CTAs) whose load phases overlap each other's selection phases.  The number
+// of rows in flight sets the speed: each row is a chain of dependent steps,
+// and its loads go through cp.async (16-byte loads into registers stalled in
+// the L1 miss path at about 2 TB/s over all SMs, however many were in flight).
 //   1. rows of at most CAPW candidates take them all; longer rows take the
 //      lower edge of the 16-bit bucket of the rank-th largest of m = n/16
-//      sampled keys (runs of 8 neighbours), rank chosen so that about TARGET
-//      elements of the row are expected at or above it;
-//   2. filter: 16-byte loads, U in flight per lane; the lanes' hits are
-//      compacted into the warp's list by a warp prefix sum;
+//      sampled keys (runs of 8 neighbours on 16-byte boundaries, copied to
+//      shared memory all at once), rank chosen so that about TARGET elements
+//      of the row are expected at or above it;
+//   2. filter: the row streams through a ring of RS slots of 32 x U 16-byte
+//      pieces per warp; the lanes' hits are compacted into the warp's list by
+//      a warp prefix sum, in ascending block order;
 //   3. if the list holds K..CAPW elements: exact radix select (8-bit digits
 //      below the common high bits, then lowest indices among the ties);
-//   4. ordering through a bitmap of the row.
+//   4. the kept elements, read from the list in its order, are already in
+//      ascending block order.
 // A row whose list holds fewer than K or more than CAPW elements is marked
 // (nsel = -1) and selected exactly by topk_rows_fallback_kernel.  Rows of
 // more than 64K blocks are marked -2 and left to that kernel's 4-warp CTAs:
@@ -1034,18 +1040,30 @@ namespace topk_w {
 constexpr int WARPS = 4;
 constexpr int THREADS = 32 * WARPS;
 constexpr int CAPW = 1024;                 // candidates a row may collect
-constexpr int BUFW = 2 * CAPW;             // keys | indices; reused for the sample and the bitmap
+constexpr int BUFW = 2 * CAPW;             // sample keys held in shared memory
 constexpr int TARGET = 768;                // expected elements at or above the sampled threshold
 constexpr int MIN_S = 512;
 constexpr int MAX_S = 16384;               // samples beyond BUFW are re-read from the row each pass
-constexpr int U = 4;                       // 16-byte loads in flight per lane
-constexpr int64_t kMaxRowBlocks = (int64_t)BUFW * 32;   // the bitmap of the row fits the buffer
+constexpr int U = 2;                       // 16-byte loads in flight per lane (at most 4: a byte each)
+constexpr int RS = 2;                      // ring slots of U x 32 16-byte pieces per warp
+constexpr int CTAS = 6;                    // resident CTAs per SM (shared memory, 80 registers)
+constexpr int64_t kMaxRowBlocks = 65536;   // longer rows go to 4-warp CTAs; 16-bit candidate indices
+static_assert(U <= 4, "a packed count holds one byte per load row");
 }
 
-struct WarpRowShared {
+// Per warp: the sample keys (step 1) share their space with the filter's
+// ring and the candidate list (steps 2-4).  Candidate indices are below
+// kMaxRowBlocks = 2^16, so 16 bits hold them.
+struct alignas(16) WarpRowShared {
   uint32_t hist[topk::NBINS];
-  uint32_t buf[topk_w::BUFW];
-  uint32_t kept[topk::KMAX];
+  union {
+    uint32_t sample[topk_w::BUFW];
+    struct {
+      float4 ring[topk_w::RS][topk_w::U * 32];
+      uint32_t key[topk_w::CAPW];
+      uint16_t idx[topk_w::CAPW];
+    } f;
+  };
 };
 
 // Bin holding the k-th largest counted value: each lane owns 8 consecutive
@@ -1145,16 +1163,17 @@ __device__ uint32_t warp_radix(int n, int k, Val val, Ok ok, int* above, int* eq
   return prefix;
 }
 
-__global__ void __launch_bounds__(topk_w::THREADS, 5) topk_rows_kernel(Geo g, SegTable st, TopkArgs a) {
+__global__ void __launch_bounds__(topk_w::THREADS, topk_w::CTAS) topk_rows_kernel(Geo g, SegTable st, TopkArgs a) {
   using namespace topk;
   using namespace topk_w;
   pdl_wait();
   pdl_trigger();
-  __shared__ WarpRowShared shw[WARPS];
+  extern __shared__ __align__(16) unsigned char topk_rows_smem[];
+  WarpRowShared* shw = reinterpret_cast<WarpRowShared*>(topk_rows_smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WarpRowShared& sh = shw[warp];
-  uint32_t* ckey = sh.buf;
-  uint32_t* cidx = sh.buf + CAPW;
+  uint32_t* ckey = sh.f.key;
+  uint16_t* cidx = sh.f.idx;
   const int n_items = st.item0[st.n];
   const int S = g.S, K = S - 1;
   const uint32_t below = (1u << lane) - 1u;
@@ -1175,84 +1194,120 @@ __global__ void __launch_bounds__(topk_w::THREADS, 5) topk_rows_kernel(Geo g, Se
     }
     const int n = (int)bt;
     const float* row = a.scores + tok * a.ld;
+    // the row as a ragged head, nvec 16-byte pieces and a ragged tail
+    const int head = min(n, (int)(((16 - ((uintptr_t)row & 15)) & 15) / 4));
+    const int nvec = (n - head) / 4;
+    const int tail0 = head + nvec * 4;
+    const float4* v4 = reinterpret_cast<const float4*>(row + head);
     // 1. threshold
     uint32_t tkey = 0u;
     if (n > CAPW) {
       const int m0 = n / 16 < MIN_S ? MIN_S : (n / 16 > MAX_S ? MAX_S : n / 16);
       const int groups = m0 / kSampleGroup;
       const int m = groups * kSampleGroup;
-      // sample s: element gi*(n-8)/(groups-1) + j of group gi = s/8 (< n)
-      auto sample = [&](int s_i) -> uint32_t {
-        const int gi = s_i / kSampleGroup, jj = s_i - gi * kSampleGroup;
-        return score_key(row[(int64_t)gi * (n - kSampleGroup) / (groups - 1) + jj]);
-      };
+      // group gi: the 8 elements of pieces q, q+1 with q = gi*(nvec-2)/(groups-1)
+      // (nvec >= 255 here; gi < 2048 and nvec <= 16384 keep the product below 2^25)
+      const uint32_t qspan = (uint32_t)(nvec - 2), den = (uint32_t)(groups - 1);
       const int rank = max(1, (int)((int64_t)m * TARGET / n));
       int ab, eq;
       if (m <= BUFW) {
-        for (int s_i = lane; s_i < m; s_i += 32) sh.buf[s_i] = sample(s_i);
+        // every lane's groups in flight at once: two 16-byte copies each
+        for (int gi = lane; gi < groups; gi += 32) {
+          const uint32_t q = (uint32_t)gi * qspan / den;
+          sm100::cp_async16(sm100::smem_u32(sh.sample + gi * kSampleGroup), v4 + q, 16);
+          sm100::cp_async16(sm100::smem_u32(sh.sample + gi * kSampleGroup + 4), v4 + q + 1, 16);
+        }
+        sm100::cp_async_wait_all();
         __syncwarp();
         tkey = warp_radix(
-            m, rank, [&](int i) { return sh.buf[i]; }, [](int) { return true; }, &ab, &eq, sh.hist, 2);
+            m, rank, [&](int i) { return score_key(__uint_as_float(sh.sample[i])); }, [](int) { return true; }, &ab,
+            &eq, sh.hist, 2);
       } else {
+        auto sample = [&](int s_i) -> uint32_t {
+          const uint32_t gi = (uint32_t)s_i / kSampleGroup, jj = (uint32_t)s_i % kSampleGroup;
+          return score_key(row[head + 4 * (gi * qspan / den) + jj]);
+        };
         tkey = warp_radix(m, rank, sample, [](int) { return true; }, &ab, &eq, sh.hist, 2);
       }
       __syncwarp();
     }
     const float tau = key_to_float(tkey);
-    // 2. filter into the warp's list
+    // 2. filter into the warp's list in ascending block order: the ragged
+    // head, then per iteration U rows of 32 16-byte loads (byte u of a packed
+    // count holds row u's hits, so one warp scan gives every row's offsets),
+    // then the ragged tail
     int nc = 0;                                   // warp-uniform count (may exceed CAPW)
-    const int head = min(n, (int)(((16 - ((uintptr_t)row & 15)) & 15) / 4));
-    const int nvec = (n - head) / 4;
-    const int tail0 = head + nvec * 4;
-    {
-      // ragged ends: at most 3 + 3 elements, one per lane
-      const int e = lane < head ? lane : (lane >= 4 && lane < 4 + n - tail0 ? tail0 + lane - 4 : -1);
+    auto append_one = [&](int e) {                // one element per lane, e < 0: none
       const float v = e >= 0 ? row[e] : 0.f;
       const bool hit = e >= 0 && v >= tau;
-      const uint32_t m = __ballot_sync(0xffffffffu, hit);
-      const int pos = nc + __popc(m & below);
+      const uint32_t mb = __ballot_sync(0xffffffffu, hit);
+      const int pos = nc + __popc(mb & below);
       if (hit && pos < CAPW) {
         ckey[pos] = score_key(v);
-        cidx[pos] = (uint32_t)e;
+        cidx[pos] = (uint16_t)e;
       }
-      nc += __popc(m);
-    }
-    const float4* v4 = reinterpret_cast<const float4*>(row + head);
-    for (int b = 0; b < nvec; b += 32 * U) {
+      nc += __popc(mb);
+    };
+    append_one(lane < head ? lane : -1);
+    const int iters = (nvec + 32 * U - 1) / (32 * U);
+    // iteration `it` of the row through ring slot it % RS: each lane copies
+    // its own U pieces and later reads back only those (no warp barrier)
+    auto issue = [&](int it) {
+      float4* slot = sh.f.ring[it % RS];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int vi = it * 32 * U + u * 32 + lane;
+        if (vi < nvec) sm100::cp_async16(sm100::smem_u32(slot + u * 32 + lane), v4 + vi, 16);
+      }
+      sm100::cp_async_commit();
+    };
+#pragma unroll
+    for (int k = 0; k < RS - 1; ++k) issue(k);
+    for (int it = 0; it < iters; ++it) {
+      const int b = it * 32 * U;
+      issue(it + RS - 1);                         // the slot read in the previous iteration
+      sm100::cp_async_wait<RS - 1>();             // this lane's pieces of iteration `it` have landed
       float4 x[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int vi = b + u * 32 + lane;
-        x[u] = vi < nvec ? __ldcs(v4 + vi) : make_float4(NAN, NAN, NAN, NAN);   // NaN never passes
+        x[u] = vi < nvec ? sh.f.ring[it % RS][u * 32 + lane] : make_float4(NAN, NAN, NAN, NAN);   // NaN never passes
       }
-      int cnt = 0;
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        cnt += (x[u].x >= tau) + (x[u].y >= tau) + (x[u].z >= tau) + (x[u].w >= tau);
-      int incl = cnt;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += t;
-      }
-      int o = nc + incl - cnt;
+      uint32_t hm[U];                             // the lane's hits in piece u, a bit per element
+      uint32_t packed = 0u;                       // a byte per row: at most 4 x 32 = 128
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const uint32_t i0 = (uint32_t)(head + 4 * (b + u * 32 + lane));
-        const float c4[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c4[c] >= tau) {
-            if (o < CAPW) {
-              ckey[o] = score_key(c4[c]);
-              cidx[o] = i0 + c;
-            }
-            ++o;
-          }
-        }
+        hm[u] = (uint32_t)(x[u].x >= tau) | (uint32_t)(x[u].y >= tau) << 1 | (uint32_t)(x[u].z >= tau) << 2 |
+                (uint32_t)(x[u].w >= tau) << 3;
+        packed |= (uint32_t)__popc(hm[u]) << (8 * u);
       }
-      nc += __shfl_sync(0xffffffffu, incl, 31);
+      uint32_t incl = packed;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+      }
+      const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+      const uint32_t excl = incl - packed;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        int o = nc + (int)((excl >> (8 * u)) & 255u);
+        const uint32_t i0 = (uint32_t)(head + 4 * (b + u * 32 + lane));
+        // one trip per hit of the lane (few pass the threshold), in element order
+        for (uint32_t bits = hm[u]; bits; bits &= bits - 1u) {
+          const int c = __ffs(bits) - 1;
+          const float v = c == 0 ? x[u].x : c == 1 ? x[u].y : c == 2 ? x[u].z : x[u].w;
+          if (o < CAPW) {
+            ckey[o] = score_key(v);
+            cidx[o] = (uint16_t)(i0 + c);
+          }
+          ++o;
+        }
+        nc += (int)((tot >> (8 * u)) & 255u);
+      }
     }
+    sm100::cp_async_wait_all();
+    append_one(lane < n - tail0 ? tail0 + lane : -1);
     __syncwarp();
     if (nc < K || nc > CAPW) {
       if (lane == 0) {
@@ -1270,46 +1325,18 @@ __global__ void __launch_bounds__(topk_w::THREADS, 5) topk_rows_kernel(Geo g, Se
     if (need < equal) {
       int a2, e2;
       imax = ~warp_radix(
-          nc, need, [&](int i) { return ~cidx[i]; }, [&](int i) { return ckey[i] == T; }, &a2, &e2, sh.hist);
+          nc, need, [&](int i) { return ~(uint32_t)cidx[i]; }, [&](int i) { return ckey[i] == T; }, &a2, &e2, sh.hist);
     }
+    // 4. the list is in ascending block order, so the kept candidates are
+    // written in order as they are found, then the own block
     int nk = 0;
     for (int b = 0; b < nc; b += 32) {
       const int i = b + lane;
-      const bool take = i < nc && (ckey[i] > T || (ckey[i] == T && cidx[i] <= imax));
-      const uint32_t m = __ballot_sync(0xffffffffu, take);
-      const int pos = nk + __popc(m & below);
-      if (take && pos < KMAX) sh.kept[pos] = cidx[i];
-      nk += __popc(m);
-    }
-    __syncwarp();
-    // 4. ascending order, the own block, padding
-    {
-      uint32_t* bm = sh.buf;                      // the candidates are no longer needed
-      const int nw = (int)((bt + 31) >> 5);
-      for (int w = lane; w < nw; w += 32) bm[w] = 0u;
-      __syncwarp();
-      for (int i = lane; i < K; i += 32) atomicOr(&bm[sh.kept[i] >> 5], 1u << (sh.kept[i] & 31));
-      __syncwarp();
-      const int wpl = (nw + 31) / 32;
-      const int w0 = min(nw, lane * wpl), w1 = min(nw, w0 + wpl);
-      int cnt = 0;
-      for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
-      int incl = cnt;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += t;
-      }
-      int pos = incl - cnt;
-      for (int w = w0; w < w1; ++w) {
-        uint32_t bits = bm[w];
-        while (bits) {
-          const int bb = __ffs(bits) - 1;
-          bits &= bits - 1u;
-          if (pos < K) sel_row[pos] = (int32_t)(w * 32 + bb);
-          ++pos;
-        }
-      }
+      const bool take = i < nc && (ckey[i] > T || (ckey[i] == T && (uint32_t)cidx[i] <= imax));
+      const uint32_t mb = __ballot_sync(0xffffffffu, take);
+      const int pos = nk + __popc(mb & below);
+      if (take && pos < K) sel_row[pos] = (int32_t)cidx[i];
+      nk += __popc(mb);
     }
     for (int i = K + lane; i < S; i += 32) sel_row[i] = i == K ? (int32_t)bt : -1;
     if (lane == 0) a.nsel[tok] = S;
