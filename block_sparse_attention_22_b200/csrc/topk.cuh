@@ -1049,6 +1049,8 @@ constexpr int RS = 2;                      // ring slots of U x 32 16-byte piece
 constexpr int CTAS = 6;                    // resident CTAs per SM (shared memory, 80 registers)
 constexpr int64_t kMaxRowBlocks = 65536;   // longer rows go to 4-warp CTAs; 16-bit candidate indices
 static_assert(U <= 4, "a packed count holds one byte per load row");
+static_assert(kMaxRowBlocks <= 65536, "candidate indices are held in 16 bits");
+static_assert(RS * U * 32 * 16 + CAPW * 6 <= BUFW * 4, "the ring and the candidates fit the sample space");
 }
 
 // Per warp: the sample keys (step 1) share their space with the filter's
