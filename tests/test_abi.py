@@ -88,6 +88,38 @@ def test_bad_segments_pointers_and_workspace_are_rejected_on_host():
     assert _call_forward(cfg, bad_cache, segs) == qsa.QSA_ERR_INVALID_ARG
 
 
+def _call_prefixed(cfg, cache, segs, prefixes, T, ws_bytes=1 << 40, **kw):
+    L = qsa.get_lib()
+    args = dict(q=16, q_idx=16, w=16, o=16, ws=16)
+    args.update(kw)
+    return L.qsa_forward_prefixed(ctypes.byref(cfg), ctypes.byref(cache), segs[0], prefixes, segs[1], T, args["q"],
+                                  args["q_idx"], args["w"], args["o"], None, None, None, args["ws"], ws_bytes, None)
+
+
+def test_prefix_arguments_are_checked_on_host():
+    """qsa_forward_prefixed: a prefix's slot, length (at most the query's
+    position, in blocks) and the decode-only rule are checked before any
+    CUDA call; a valid table passes every check and stops at the workspace."""
+    sh = synth.Shape()
+    cfg = qsa.make_config(sh)
+    cache = qsa.qsa_cache_t(16, 16, 16, 16, 3, 4096)       # 3 slots of 4096 tokens (fake addresses)
+    segs = qsa.make_segments([(0, 1, 2000, 0), (1, 1, 3000, 1)])
+    ok = qsa.make_prefixes([(2, 400), (2, 400)])
+    assert _call_prefixed(cfg, cache, segs, ok, 2, ws_bytes=10) == qsa.QSA_ERR_WORKSPACE
+    for bad in ([(3, 400), (2, 400)],      # slot past the cache
+                [(-1, 400), (2, 400)],     # negative slot
+                [(2, -1), (2, 400)],       # negative length
+                [(2, 501), (2, 400)]):     # 501 blocks = 2004 tokens > position 2000
+        assert _call_prefixed(cfg, cache, segs, qsa.make_prefixes(bad), 2) == qsa.QSA_ERR_INVALID_ARG, bad
+    assert _call_prefixed(cfg, cache, segs, None, 2) == qsa.QSA_ERR_INVALID_ARG       # no prefix table
+    no_share = qsa.make_prefixes([(0, 0), (0, 0)])                                  # nothing shared: plain forward
+    assert _call_prefixed(cfg, cache, segs, no_share, 2, ws_bytes=10) == qsa.QSA_ERR_WORKSPACE
+    long_seg = qsa.make_segments([(0, 16, 2000, 0), (16, 1, 3000, 1)])
+    assert _call_prefixed(cfg, cache, long_seg, ok, 17) == qsa.QSA_ERR_UNSUPPORTED     # 16 queries on a prefix
+    f32 = qsa.make_config(synth.Shape(dtype="f32"))
+    assert _call_prefixed(f32, cache, segs, ok, 2) == qsa.QSA_ERR_UNSUPPORTED
+
+
 def test_empty_batches_are_noops_without_touching_the_device():
     sh, cfg, segs, cache = _setup()
     empty = qsa.make_segments([(0, 0, 100, 0)])
