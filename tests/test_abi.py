@@ -120,6 +120,26 @@ def test_prefix_arguments_are_checked_on_host():
     assert _call_prefixed(f32, cache, segs, ok, 2) == qsa.QSA_ERR_UNSUPPORTED
 
 
+def test_noalloc_selection_checks_run_before_the_scratch_lookup():
+    """qsa_select_topk_noalloc rejects bad arguments and a batch whose
+    selection needs more than its fixed scratch before it looks the scratch
+    up or launches anything (fake pointers, never dereferenced)."""
+    cfg = qsa.make_config(synth.Shape())
+    L = qsa.get_lib()
+
+    def call(segs, T, scores=16, ld=524288, sel=16, nsel=16):
+        return L.qsa_select_topk_noalloc(ctypes.byref(cfg), segs[0], segs[1], T, scores, ld, sel, nsel, None)
+
+    big = qsa.make_segments([(i, 1, (1 << 21) - 1, 0) for i in range(500)])   # 48 KiB of scratch per row
+    assert qsa.workspace_size(cfg, big, 500, qsa.QSA_OP_SELECT) > (16 << 20)
+    assert call(big, 500) == qsa.QSA_ERR_WORKSPACE
+    small = qsa.make_segments([(0, 1, 40003, 0)])                              # 10000 candidate blocks
+    assert call(small, 1, ld=9999) == qsa.QSA_ERR_INVALID_ARG                 # row pitch below the row
+    assert call(small, 1, sel=18) == qsa.QSA_ERR_INVALID_ARG                  # misaligned sel
+    assert call(small, 1, scores=None) == qsa.QSA_ERR_INVALID_ARG
+    assert call(qsa.make_segments([]), 0) == qsa.QSA_OK                        # empty batch: nothing to do
+
+
 def test_empty_batches_are_noops_without_touching_the_device():
     sh, cfg, segs, cache = _setup()
     empty = qsa.make_segments([(0, 0, 100, 0)])
