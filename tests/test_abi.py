@@ -140,6 +140,26 @@ def test_noalloc_selection_checks_run_before_the_scratch_lookup():
     assert call(qsa.make_segments([]), 0) == qsa.QSA_OK                        # empty batch: nothing to do
 
 
+def test_backward_arguments_are_checked_on_host():
+    """qsa_sparse_attn_bwd rejects missing or misaligned buffers and bad
+    segments before any CUDA call; an empty batch is a no-op."""
+    sh, cfg, segs, cache = _setup()
+    L = qsa.get_lib()
+
+    def call(segs, T=16, **kw):
+        a = dict(q=16, o=16, lse=16, dout=16, sel=16, nsel=16, dq=16, dk=16, dv=16)
+        a.update(kw)
+        return L.qsa_sparse_attn_bwd(ctypes.byref(cfg), ctypes.byref(cache), segs[0], segs[1], T, a["q"], a["o"],
+                                     a["lse"], a["dout"], a["sel"], a["nsel"], a["dq"], a["dk"], a["dv"], None)
+
+    for name in ("q", "o", "lse", "dout", "sel", "nsel", "dq", "dk", "dv"):
+        assert call(segs, **{name: None}) == qsa.QSA_ERR_INVALID_ARG, name
+    for name in ("q", "o", "dout", "dq", "dk", "dv"):
+        assert call(segs, **{name: 24}) == qsa.QSA_ERR_INVALID_ARG, name          # not 16-byte aligned
+    assert call(qsa.make_segments([(0, 16, 1020, 0)])) == qsa.QSA_ERR_INVALID_ARG   # past the cache
+    assert call(qsa.make_segments([]), T=0) == qsa.QSA_OK
+
+
 def test_empty_batches_are_noops_without_touching_the_device():
     sh, cfg, segs, cache = _setup()
     empty = qsa.make_segments([(0, 0, 100, 0)])
