@@ -160,6 +160,61 @@ def test_backward_arguments_are_checked_on_host():
     assert call(qsa.make_segments([]), T=0) == qsa.QSA_OK
 
 
+def test_stage_entry_points_check_arguments_on_host():
+    """The four stage entry points and the low-memory forward reject bad
+    ranges, missing or misaligned buffers and short score rows before any
+    CUDA call (fake pointers, never dereferenced)."""
+    sh, cfg, segs, cache = _setup()           # 16 queries at positions 100..115: up to 28 candidate blocks
+    L = qsa.get_lib()
+
+    def compress(slots, b0, b1, n=None):
+        n = len(slots) if n is None else n
+        return L.qsa_compress_keys(ctypes.byref(cfg), ctypes.byref(cache), (ctypes.c_int32 * 2)(*slots),
+                                   (ctypes.c_int64 * 2)(*b0), (ctypes.c_int64 * 2)(*b1), n, None)
+
+    assert compress([0], [0], [0], n=-1) == qsa.QSA_ERR_INVALID_ARG
+    assert compress([1], [0], [4]) == qsa.QSA_ERR_INVALID_ARG        # slot past the cache
+    assert compress([0], [5], [4]) == qsa.QSA_ERR_INVALID_ARG        # end before begin
+    assert compress([0], [0], [257]) == qsa.QSA_ERR_INVALID_ARG      # past 1024 / r blocks
+    assert compress([], [], []) == qsa.QSA_OK
+    assert L.qsa_compress_keys(ctypes.byref(cfg), ctypes.byref(cache), None, None, None, 1, None) == \
+        qsa.QSA_ERR_INVALID_ARG
+
+    def index(q_idx=16, w=16, scores=16, ld=28):
+        return L.qsa_index_scores(ctypes.byref(cfg), ctypes.byref(cache), segs[0], segs[1], 16, q_idx, w, scores,
+                                  ld, None)
+
+    assert index(q_idx=None) == qsa.QSA_ERR_INVALID_ARG
+    assert index(scores=20) == qsa.QSA_ERR_INVALID_ARG               # not 16-byte aligned
+    assert index(ld=27) == qsa.QSA_ERR_INVALID_ARG                   # row pitch below 28 blocks
+
+    def select(scores=16, ld=28, sel=16, nsel=16):
+        return L.qsa_select_topk(ctypes.byref(cfg), segs[0], segs[1], 16, scores, ld, sel, nsel, 16, 1 << 40, None)
+
+    assert select(scores=None) == qsa.QSA_ERR_INVALID_ARG
+    assert select(sel=20) == qsa.QSA_ERR_INVALID_ARG
+    assert select(nsel=None) == qsa.QSA_ERR_INVALID_ARG
+    assert select(ld=27) == qsa.QSA_ERR_INVALID_ARG
+
+    def attend(q=16, sel=16, nsel=16, o=16):
+        return L.qsa_sparse_attn_fwd(ctypes.byref(cfg), ctypes.byref(cache), segs[0], segs[1], 16, q, sel, nsel, o,
+                                     None, 16, 1 << 40, None)
+
+    assert attend(q=24) == qsa.QSA_ERR_INVALID_ARG
+    assert attend(sel=None) == qsa.QSA_ERR_INVALID_ARG
+    assert attend(o=None) == qsa.QSA_ERR_INVALID_ARG
+
+    def lowmem(**kw):
+        a = dict(q=16, q_idx=16, w=16, o=16)
+        a.update(kw)
+        return L.qsa_forward_lowmem(ctypes.byref(cfg), ctypes.byref(cache), segs[0], segs[1], 16, a["q"], a["q_idx"],
+                                    a["w"], a["o"], None, None, None, 16, 10, None)
+
+    assert lowmem(q_idx=None) == qsa.QSA_ERR_INVALID_ARG
+    assert lowmem(w=20) == qsa.QSA_ERR_INVALID_ARG
+    assert lowmem() == qsa.QSA_ERR_WORKSPACE                          # valid arguments, 10-byte workspace
+
+
 def test_empty_batches_are_noops_without_touching_the_device():
     sh, cfg, segs, cache = _setup()
     empty = qsa.make_segments([(0, 0, 100, 0)])
